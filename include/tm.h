@@ -1,0 +1,217 @@
+/*
+ * tm.h -- C ABI of libtm: tile-routed FP16/INT8 fused prefill attention for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (TileMix, Lattice paper page, abstract): the Lq x Lk score
+ * matrix of scaled-dot-product attention is cut into hardware-aligned
+ * tile_m x tile_n score tiles; one routing bit per (query tile, group of g
+ * adjacent key tiles), packed into a compact bitmask, sends the group's scores
+ * through an FP16 or an INT8 QK^T; both routes feed one online-softmax state
+ * and one P.V accumulation; every legal group is computed, so no visible
+ * query-key pair is dropped; grouped-query attention, variable-length batches
+ * and INT8 key/value caches are supported.  With no bitmask the call is plain
+ * fused attention (MLX PR "Nax Refactor", attention tables: fp16, GQA,
+ * causal).
+ *
+ * Conventions shared by every call
+ *  - Tensors are token-major [T, H, d] ("THD"): element (t, h, c) is at
+ *    data[t * stride_t + h * stride_h + c]; the innermost dimension is
+ *    contiguous; strides are in elements.  d is 64 or 128.
+ *  - Pointers are device pointers unless the argument name ends in _host.
+ *    The caller owns every buffer.  The library allocates no device memory;
+ *    it keeps only a per-process table of kernel attributes.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t / CUstream passed
+ *    as void*, NULL = legacy default stream) and never synchronises, except
+ *    tm_get_device_error.
+ *  - Arguments are validated on the host before any launch; a rejected call
+ *    launches nothing and returns TM_ERR_INVALID_ARG or TM_ERR_UNSUPPORTED.
+ *    A failed launch returns TM_ERR_CUDA (tm_last_cuda_error() gives the CUDA
+ *    code).  Conditions only the device can see (a sequence longer than
+ *    max_seqlen; a pipeline wait that exceeded its time limit) are recorded
+ *    in a device error word read by tm_get_device_error.
+ *  - Variable-length batches: cu_seqlens is a device int32 array [batch + 1],
+ *    non-decreasing, cu_seqlens[0] = 0; sequence b holds rows
+ *    cu_seqlens[b] .. cu_seqlens[b+1]-1 of BOTH Q and K/V (self-attention
+ *    prefill), so Lq = Lk = its length.  max_seqlen must be >= every length.
+ *    With cu_seqlens == NULL there is one sequence, Lq = q->T, Lk = k->T,
+ *    and batch / max_seqlen are ignored.
+ *  - Tiles restart at every sequence.  Query tile I of sequence b is global
+ *    query tile I_glob = (number of query tiles of sequences < b) + I; key
+ *    tiles are numbered the same way with tile_n.
+ *  - Causal masking is bottom-right aligned: key j is visible to query i iff
+ *    j < Lk and j <= i + Lk - Lq.  A query row with no visible key is 0.
+ */
+#ifndef TM_H_
+#define TM_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TM_OK = 0,
+  TM_ERR_INVALID_ARG = 1,  /* bad pointer, shape, stride, alignment or length */
+  TM_ERR_UNSUPPORTED = 2,  /* valid request outside what is built (d, tiles) */
+  TM_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  TM_ERR_TIMEOUT = 4       /* a device pipeline wait exceeded its limit */
+} tm_status;
+
+/* How a tensor's INT8 scales are laid out (field tm_tensor.scale_kind). */
+typedef enum {
+  TM_SCALE_NONE = 0,
+  TM_SCALE_TILE = 1,   /* fp32 [n_tiles, H]: one scale per (tile, head), written by tm_quantize_qk */
+  TM_SCALE_TOKEN = 2   /* fp16 [T, H]: one scale per (token, head), an INT8 K/V cache */
+} tm_scale_kind;
+
+/* One attention operand or output, [T, H, d].
+ *  data     fp16 values with strides stride_t / stride_h (elements); for an
+ *           INT8 cache operand (scale_kind == TM_SCALE_TOKEN) data is NULL.
+ *  codes    int8 values, dense [T, H, d] (stride_t = H*d, stride_h = d), or NULL.
+ *  scales   see scale_kind, or NULL.
+ * Alignment: data and codes 16-byte aligned; stride_t and stride_h multiples
+ * of 8 elements; scales 4-byte (fp32) or 2-byte (fp16) aligned. */
+typedef struct {
+  void* data;
+  int64_t T, H, d;
+  int64_t stride_t, stride_h;
+  const int8_t* codes;
+  const void* scales;
+  int32_t scale_kind;
+} tm_tensor;
+
+/* ---------------------------------------------------------------------------
+ * tm_quantize_qk -- per-tile symmetric INT8 quantisation of Q and K.
+ *
+ * TileMix abstract: the INT8 route computes scores from INT8 codes.  The
+ * per-tile rule (symmetric absmax / 127) is the one this library fixes:
+ *   amax = max |x| over the tile's rows x d of one head (tiles of tile_m rows
+ *          for Q, tile_n rows for K, restarting at every sequence);
+ *   s    = fl32(amax / 127)                  (IEEE fp32 division)
+ *   code = clamp(rne(fl32(x / s)), -127, 127), and all codes 0 when s == 0.
+ * q: fp16 [Tq, Hq, d] (its codes/scales fields are ignored); q_codes: int8
+ * dense [Tq, Hq, d]; q_scales: fp32 [n_qtiles, Hq].  Same for k with tile_n
+ * into k_codes [Tk, Hkv, d] / k_scales [n_ktiles, Hkv]; k may be NULL (Q only;
+ * used with an INT8 K/V cache).  Code rows outside every sequence are not
+ * written.  tile_m, tile_n in {64, 128}.
+ * Results are bit-identical to the definition above (no contraction of the
+ * division, round-to-nearest-even conversion).
+ * ------------------------------------------------------------------------- */
+tm_status tm_quantize_qk(const tm_tensor* q, const tm_tensor* k,
+                         int8_t* q_codes, float* q_scales,
+                         int8_t* k_codes, float* k_scales,
+                         const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen,
+                         int32_t tile_m, int32_t tile_n, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Routing bitmask layout (TileMix abstract: "compact bitmasks", one bit per
+ * query tile x key-tile group, "each routing bit govern[s] multiple adjacent
+ * key tiles").
+ *   word  bitmask[h * mask_head_stride + I_glob * W + G / 32], bit G % 32;
+ *   G = J / g is the group of key tile J;  bit 1 = INT8, 0 = FP16;
+ *   W = tm_mask_words(max Lk, tile_n, g) = ceil(ceil(ceil(Lk/tile_n)/g)/32).
+ * Bits of groups with no visible pair for the query tile are ignored.
+ * A per-head mask has mask_head_stride = n_qtiles * W; 0 shares one plane.
+ * ------------------------------------------------------------------------- */
+int32_t tm_mask_words(int64_t max_lk, int32_t tile_n, int32_t g);
+
+/* Number of tiles of `tile` rows over a batch: sum_b ceil(len_b / tile) from
+ * a HOST copy of cu_seqlens, or ceil(L / tile) when cu_seqlens_host == NULL.
+ * Returns -1 on invalid arguments. */
+int64_t tm_count_tiles(const int32_t* cu_seqlens_host, int32_t batch, int64_t L, int32_t tile);
+
+/* ---------------------------------------------------------------------------
+ * tm_build_mask -- seeded routing bitmask on the device.
+ *
+ * The pages say only that routing is decided per tile group at inference
+ * time without training.  This builder draws an independent Bernoulli(p)
+ * per group: for head h (0..Hq-1), query tile I_glob, group G that is legal
+ * (holds a visible pair for the tile) and not forced,
+ *   u   = (splitmix64(seed XOR (h * 2^40 + I_glob * 2^20 + G)) >> 11) * 2^-53
+ *   bit = (u < p)
+ * where splitmix64(x) is the SplitMix64 output function applied to
+ * x + 0x9E3779B97F4A7C15.  Forced groups are 0: with force_diag the group that
+ * holds the query tile's last visible key tile, with force_sink group 0.
+ * Illegal groups and padding bits are 0.  Writes the n_qtiles * W words of
+ * every head plane h at bitmask + h * mask_head_stride, where n_qtiles =
+ * tm_count_tiles(cu_seqlens_host, batch, Lq, tile_m) and W = tm_mask_words(
+ * max Lk, tile_n, g); mask_head_stride >= n_qtiles * W is the caller's
+ * contract (checked on the host when cu_seqlens == NULL).
+ * Lq, Lk: lengths when cu_seqlens == NULL; max_seqlen: bound when not.
+ * Hq < 2^24, n_qtiles < 2^20, groups < 2^20; 0 <= p <= 1.
+ * ------------------------------------------------------------------------- */
+tm_status tm_build_mask(uint32_t* bitmask, int32_t Hq,
+                        const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen,
+                        int64_t Lq, int64_t Lk, int32_t tile_m, int32_t tile_n, int32_t g,
+                        int32_t causal, double p, uint64_t seed,
+                        int32_t force_diag, int32_t force_sink, int64_t mask_head_stride,
+                        void* stream);
+
+/* Same bits computed on the host (bitmask_host and cu_seqlens_host are host
+ * pointers), written with mask_head_stride = n_qtiles * W; bit-identical to
+ * tm_build_mask. */
+tm_status tm_build_mask_host(uint32_t* bitmask_host, int32_t Hq,
+                             const int32_t* cu_seqlens_host, int32_t batch,
+                             int64_t Lq, int64_t Lk, int32_t tile_m, int32_t tile_n, int32_t g,
+                             int32_t causal, double p, uint64_t seed,
+                             int32_t force_diag, int32_t force_sink);
+
+/* Host statistics of a host bitmask: n_vis = visible query-key pairs summed
+ * over heads and sequences; e8 = those in INT8-routed tiles.  The realised
+ * INT8 fraction is e8 / n_vis.  bitmask_host may be NULL (e8 = 0). */
+tm_status tm_route_stats(const uint32_t* bitmask_host, int64_t mask_head_stride, int32_t Hq,
+                         const int32_t* cu_seqlens_host, int32_t batch,
+                         int64_t Lq, int64_t Lk, int32_t tile_m, int32_t tile_n, int32_t g,
+                         int32_t causal, double* n_vis, double* e8);
+
+/* ---------------------------------------------------------------------------
+ * tm_attn_fwd -- fused tile-routed attention forward (prefill).
+ *
+ * For every sequence, query head h (KV head h / (Hq / Hkv)) and visible pair
+ * (i, j) in query tile I_glob and key tile J:
+ *   FP16 route: S_ij = sigma * q_i . k_j                 (fp16 operands)
+ *   INT8 route: S_ij = sigma * s_q * s_k * (cq_i . ck_j) (int8 operands,
+ *               exact int32 sum; s_q = q tile scale, s_k = k tile scale or,
+ *               for an INT8 cache, the scale of key j)
+ *   sigma = 1/sqrt(d); route = bit of group J / g (always FP16 when bitmask
+ *   is NULL); out_i = fp16( sum_j softmax_j(S_i.) v_j ) with P rounded to fp16
+ *   for the P.V product, fp32 accumulation and fp32 row sums.
+ *
+ * q:   fp16 data [Tq, Hq, d]; when bitmask != NULL also codes and
+ *      TM_SCALE_TILE scales (from tm_quantize_qk with the same tile_m).
+ * k,v: either fp16 data [Tk, Hkv, d] (k also with codes + TM_SCALE_TILE scales
+ *      from tm_quantize_qk with tile_n when bitmask != NULL), or an INT8 cache:
+ *      data NULL, codes + TM_SCALE_TOKEN scales, for BOTH k and v.  The cache
+ *      is dequantised to fp16 (fp16(code * scale)) in shared memory for FP16
+ *      groups and for all of V; INT8 groups use the K codes directly.
+ * out: fp16 data [Tq, Hq, d]; every row of every sequence is written.
+ * bitmask / mask_head_stride: see the layout above; NULL = all FP16.
+ * tile_m in {64, 128}; tile_n in {64, 128}; g >= 1; d in {64, 128};
+ * Hq % Hkv == 0; the INT8 cache requires d == 128 and tile_n == 128.
+ * ------------------------------------------------------------------------- */
+tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                      const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen,
+                      const uint32_t* bitmask, int64_t mask_head_stride,
+                      int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal, void* stream);
+
+/* Reads and clears the device error word after synchronising `stream`.
+ * Returns TM_OK, TM_ERR_TIMEOUT (a pipeline wait gave up; the output of the
+ * affected call is unspecified) or TM_ERR_INVALID_ARG (a sequence exceeded
+ * max_seqlen; its extra tiles were not computed). */
+tm_status tm_get_device_error(void* stream);
+
+/* Static description of a status code. */
+const char* tm_status_string(tm_status s);
+
+/* CUDA error code of the last TM_ERR_CUDA returned on this thread (0 if none). */
+int32_t tm_last_cuda_error(void);
+
+/* Library version, "major.minor.patch". */
+const char* tm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TM_H_ */

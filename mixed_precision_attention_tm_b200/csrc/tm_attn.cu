@@ -1,0 +1,548 @@
+// tm_attn.cu -- fused tile-routed FP16/INT8 attention forward (tm_attn_fwd).
+//
+// TileMix (Lattice paper page), abstract: score tiles, one routing bit per
+// (query tile, group of g key tiles), FP16 or INT8 score computation per
+// group, both routes updating one online-softmax state; all legal groups are
+// computed; GQA, variable-length batches and INT8 K/V caches.  The all-FP16
+// case is fused SDPA as benchmarked in the MLX PR "Nax Refactor" tables.
+//
+// Kernel design (sm_100a, one CTA per (query tile, sequence, head)):
+//   warp 4      TMA producer: Q (fp16, and int8 codes when the row has INT8
+//               groups) once; per key tile either the fp16 K tile or the int8
+//               K-code tile, chosen by the routing bit, plus the fp16 V tile,
+//               into 2-stage rings of 128B-swizzled shared memory.
+//   warp 5      tcgen05 issuer (one thread): S_j = Q K_j^T with kind::f16
+//               (fp32 accumulate) or kind::i8 (s32 accumulate) into TMEM
+//               (double-buffered S), then O += P_{j-1} V_{j-1} with P read
+//               from TMEM (kind::f16, fp32 accumulate in TMEM).
+//   warps 0-3   softmax, one query row per thread (TMEM lane = row): S row
+//               from TMEM, int32 -> fp32 and dequantisation by
+//               s_q * s_k * sigma for INT8 tiles, causal / ragged masking,
+//               online max / sum with a lazy rescale of O (only when the row
+//               max grows by more than 2^8), P rounded to fp16 and written back
+//               over S in TMEM, and the final O / l epilogue.
+// Every mbarrier wait is bounded (tm_device.cuh).
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "tm_device.cuh"
+#include "tm_host.h"
+
+namespace tmk {
+namespace {
+
+template <int D, int BN>
+struct Cfg {
+  static constexpr int BM = 128;                 // MMA rows (query tile of 128, or 64 + unused)
+  static constexpr int NK = 2, NV = 2;           // ring depths
+  static constexpr int Q16_HALF = BM * 128;      // bytes of one 64-column fp16 slab of Q
+  static constexpr int KV16_HALF = BN * 128;     // bytes of one 64-column fp16 slab of K / V
+  static constexpr int Q16_BYTES = BM * D * 2;
+  static constexpr int Q8_BYTES = BM * D;
+  static constexpr int K_STAGE = BN * D * 2;
+  static constexpr int V_STAGE = BN * D * 2;
+  static constexpr int OFF_Q16 = 0;
+  static constexpr int OFF_Q8 = OFF_Q16 + Q16_BYTES;
+  static constexpr int OFF_K = OFF_Q8 + Q8_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * K_STAGE;
+  static constexpr int OFF_BAR = OFF_V + NV * V_STAGE;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;   // + alignment slack
+  static constexpr uint32_t TMEM_COLS = (2 * BN + D <= 256) ? 256u : 512u;
+  static constexpr uint32_t O_COL = 2 * BN;
+  static constexpr uint32_t IDESC_S16 = idesc_f16(BM, BN, false);
+  static constexpr uint32_t IDESC_S8 = idesc_i8(BM, BN);
+  static constexpr uint32_t IDESC_PV = idesc_f16(BM, D, true);
+  static constexpr uint32_t Q8_SWZ = (D == 128) ? kSwizzle128 : kSwizzle64;
+  static constexpr uint32_t Q8_SBO = (D == 128) ? 1024u : 512u;
+};
+
+// Barrier slots (uint64 each) inside the barrier block.
+enum {
+  B_QFULL = 0,
+  B_KFULL = 1,   // +NK
+  B_KEMPTY = 3,  // +NK
+  B_VFULL = 5,   // +NV
+  B_VEMPTY = 7,  // +NV
+  B_SFULL = 9,   // +2
+  B_PFULL = 11,  // +2
+  B_ODONE = 13,
+  B_DRAIN = 14,
+  B_COUNT = 15
+};
+
+struct Params {
+  __half* out;
+  int64_t out_st, out_sh;
+  const float* q_scales;   // [n_qtiles, Hq]
+  const float* k_scales;   // [n_ktiles, Hkv]
+  const uint32_t* bitmask;
+  int64_t mask_hs;
+  int W;
+  const int32_t* cu;
+  int64_t Lq, Lk;          // lengths without cu_seqlens
+  int Hq, Hkv, tile_m, g, causal, n_qt_max, batch;
+  float scale_log2;        // sigma * log2(e)
+  DevErr err;
+};
+
+__device__ __forceinline__ bool route_int8(const uint32_t* row, int g, int j) {
+  if (row == nullptr) return false;
+  const int G = j / g;
+  return (__ldg(row + (G >> 5)) >> (G & 31)) & 1u;
+}
+
+template <int D, int BN>
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmQ8,
+                    const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmK8,
+                    const __grid_constant__ CUtensorMap tmV16, const Params p) {
+  using C = Cfg<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_s + pad;
+  const uint32_t sQ16 = sbase + C::OFF_Q16;
+  const uint32_t sQ8 = sbase + C::OFF_Q8;
+  const uint32_t sK = sbase + C::OFF_K;
+  const uint32_t sV = sbase + C::OFF_V;
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * B_COUNT + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: heaviest query tiles first (causal), heads fastest
+  const int h = blockIdx.x % p.Hq;
+  const int t1 = blockIdx.x / p.Hq;
+  const int b = t1 % p.batch;
+  const int I = p.n_qt_max - 1 - t1 / p.batch;
+  const SeqInfo sq = seq_info(p.cu, b, p.Lq, p.tile_m);
+  const int64_t Lq = sq.len;
+  const int64_t Lk = p.cu ? sq.len : p.Lk;
+  const int64_t kstart = p.cu ? sq.start : 0;
+  if (p.cu != nullptr && I == 0 && threadIdx.x == 0 &&
+      Lq > static_cast<int64_t>(p.n_qt_max) * p.tile_m)
+    dev_error(p.err, TM_DEVERR_SEQLEN);
+  if (static_cast<int64_t>(I) * p.tile_m >= Lq) return;   // whole CTA: no setup done yet
+
+  const int rows_valid = static_cast<int>(min(static_cast<int64_t>(p.tile_m), Lq - static_cast<int64_t>(I) * p.tile_m));
+  const int64_t i_last = static_cast<int64_t>(I) * p.tile_m + rows_valid - 1;
+  int64_t jmax = Lk - 1;
+  if (p.causal) jmax = min(jmax, i_last + Lk - Lq);
+  const int nJ = (Lk <= 0 || jmax < 0) ? 0 : static_cast<int>(jmax / BN + 1);
+  const int64_t ig = sq.tile_base + I;
+  const int hk = h / (p.Hq / p.Hkv);
+  const uint32_t* mrow = p.bitmask ? p.bitmask + static_cast<int64_t>(h) * p.mask_hs + ig * p.W : nullptr;
+  const int64_t qrow0 = sq.start + static_cast<int64_t>(I) * p.tile_m;
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    for (int s = 0; s < C::NK; ++s) { mbar_init(bar(B_KFULL + s), 1); mbar_init(bar(B_KEMPTY + s), 1); }
+    for (int s = 0; s < C::NV; ++s) { mbar_init(bar(B_VFULL + s), 1); mbar_init(bar(B_VEMPTY + s), 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(bar(B_SFULL + s), 1); mbar_init(bar(B_PFULL + s), 128); }
+    mbar_init(bar(B_ODONE), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmQ16);
+    prefetch_tmap(&tmK16);
+    prefetch_tmap(&tmV16);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ======================= TMA producer =======================
+    if (lane == 0 && nJ > 0) {
+      bool any8 = false;
+      if (mrow != nullptr)
+        for (int w = 0; w < p.W; ++w) any8 |= (__ldg(mrow + w) != 0u);
+      mbar_arrive_expect_tx(bar(B_QFULL), C::Q16_BYTES + (any8 ? C::Q8_BYTES : 0));
+#pragma unroll
+      for (int hh = 0; hh < D / 64; ++hh)
+        tma_load_3d(sQ16 + hh * C::Q16_HALF, &tmQ16, bar(B_QFULL), hh * 64, h, static_cast<int32_t>(qrow0));
+      if (any8) tma_load_3d(sQ8, &tmQ8, bar(B_QFULL), 0, h, static_cast<int32_t>(qrow0));
+      int nk_issued = 0, nv_issued = 0;
+      for (int j = 0; j < nJ; ++j) {
+        const bool i8 = route_int8(mrow, p.g, j);
+        const int32_t krow = static_cast<int32_t>(kstart + static_cast<int64_t>(j) * BN);
+        const int ks = j % C::NK, kn = j / C::NK;
+        if (kn > 0 && !mbar_wait(bar(B_KEMPTY + ks), (kn - 1) & 1, p.err, abort_flag)) break;
+        const uint32_t kdst = sK + ks * C::K_STAGE;
+        if (i8) {
+          mbar_arrive_expect_tx(bar(B_KFULL + ks), BN * D);
+          tma_load_3d(kdst, &tmK8, bar(B_KFULL + ks), 0, hk, krow);
+        } else {
+          mbar_arrive_expect_tx(bar(B_KFULL + ks), BN * D * 2);
+#pragma unroll
+          for (int hh = 0; hh < D / 64; ++hh)
+            tma_load_3d(kdst + hh * C::KV16_HALF, &tmK16, bar(B_KFULL + ks), hh * 64, hk, krow);
+        }
+        ++nk_issued;
+        const int vs = j % C::NV, vn = j / C::NV;
+        if (vn > 0 && !mbar_wait(bar(B_VEMPTY + vs), (vn - 1) & 1, p.err, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(B_VFULL + vs), BN * D * 2);
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d(sV + vs * C::V_STAGE + hh * C::KV16_HALF, &tmV16, bar(B_VFULL + vs), hh * 64, hk, krow);
+        ++nv_issued;
+      }
+      // Drain: every issued copy has landed before the CTA may exit.
+      volatile int never = 0;
+      mbar_wait(bar(B_QFULL), 0, p.err, &never);
+      for (int s = 0; s < C::NK; ++s) {
+        const int cnt = nk_issued > s ? (nk_issued - 1 - s) / C::NK + 1 : 0;
+        if (cnt > 0) mbar_wait(bar(B_KFULL + s), (cnt - 1) & 1, p.err, &never);
+      }
+      for (int s = 0; s < C::NV; ++s) {
+        const int cnt = nv_issued > s ? (nv_issued - 1 - s) / C::NV + 1 : 0;
+        if (cnt > 0) mbar_wait(bar(B_VFULL + s), (cnt - 1) & 1, p.err, &never);
+      }
+    }
+  } else if (warp == 5) {
+    // ======================= tcgen05 issuer =======================
+    if (lane == 0 && nJ > 0) {
+      bool ok = mbar_wait(bar(B_QFULL), 0, p.err, abort_flag);
+      tc_fence_after();
+      auto issue_pv = [&](int t) -> bool {
+        if (!mbar_wait(bar(B_PFULL + (t & 1)), (t >> 1) & 1, p.err, abort_flag)) return false;
+        const int vs = t % C::NV;
+        if (!mbar_wait(bar(B_VFULL + vs), (t / C::NV) & 1, p.err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t a_tmem = tmem + static_cast<uint32_t>(t & 1) * BN;
+        const uint32_t vbase = sV + vs * C::V_STAGE;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bdesc = smem_desc(vbase + kk * 2048, C::KV16_HALF, 1024, kSwizzle128);
+          mma_f16_ts(tmem + C::O_COL, a_tmem + kk * 8, bdesc, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(bar(B_ODONE));
+        tc_commit(bar(B_VEMPTY + vs));
+        return true;
+      };
+      for (int j = 0; ok && j < nJ; ++j) {
+        const bool i8 = route_int8(mrow, p.g, j);
+        const int ks = j % C::NK;
+        if (!mbar_wait(bar(B_KFULL + ks), (j / C::NK) & 1, p.err, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
+        const uint32_t kbase = sK + ks * C::K_STAGE;
+        if (i8) {
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk) {
+            const uint64_t ad = smem_desc(sQ8 + kk * 32, 16, C::Q8_SBO, C::Q8_SWZ);
+            const uint64_t bd = smem_desc(kbase + kk * 32, 16, C::Q8_SBO, C::Q8_SWZ);
+            mma_i8_ss(d_tmem, ad, bd, C::IDESC_S8, kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 0u + (kk & 3) * 32;
+            const uint64_t ad = smem_desc(sQ16 + (kk >> 2) * C::Q16_HALF + off, 16, 1024, kSwizzle128);
+            const uint64_t bd = smem_desc(kbase + (kk >> 2) * C::KV16_HALF + off, 16, 1024, kSwizzle128);
+            mma_f16_ss(d_tmem, ad, bd, C::IDESC_S16, kk > 0 ? 1u : 0u);
+          }
+        }
+        tc_commit(bar(B_SFULL + (j & 1)));
+        tc_commit(bar(B_KEMPTY + ks));
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) issue_pv(nJ - 1);
+      // Drain: all issued tcgen05 work completes before TMEM is released.
+      tc_commit(bar(B_DRAIN));
+      volatile int never = 0;
+      mbar_wait(bar(B_DRAIN), 0, p.err, &never);
+    }
+  } else {
+    // ======================= softmax (warps 0-3) =======================
+    const int r = threadIdx.x;                       // query row in the tile = TMEM lane
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const bool row_ok = r < rows_valid;
+    const int64_t i_row = static_cast<int64_t>(I) * p.tile_m + r;
+    int64_t lim = -1;                                // last visible key of this row
+    if (row_ok) lim = p.causal ? min(Lk - 1, i_row + Lk - Lq) : Lk - 1;
+    float c8_row = 0.f;
+    if (mrow != nullptr) c8_row = __ldg(p.q_scales + ig * p.Hq + h) * p.scale_log2;
+    const SeqInfo sk = seq_info(p.cu, b, p.Lk, BN);  // key-tile numbering of this sequence
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nJ; ++j) {
+      const bool i8 = route_int8(mrow, p.g, j);
+      float c = p.scale_log2;
+      if (i8) c = c8_row * __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk);
+      if (!mbar_wait(bar(B_SFULL + (j & 1)), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      __syncwarp();
+      float x[BN];
+      {
+        uint32_t u[32];
+#pragma unroll
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          tmem_ld32(lane_addr + static_cast<uint32_t>(j & 1) * BN + cc * 32, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (i8) x[cc * 32 + e] = __int_as_float(static_cast<int>(u[e]) + 0x4B400000) - 12582912.0f;
+            else x[cc * 32 + e] = __uint_as_float(u[e]);
+          }
+        }
+      }
+      const int64_t nv64 = lim - static_cast<int64_t>(j) * BN + 1;
+      const int nv = nv64 <= 0 ? 0 : (nv64 >= BN ? BN : static_cast<int>(nv64));
+      const bool full = __all_sync(0xffffffffu, nv == BN);   // warp-uniform fast path
+      float mraw = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int e = 0; e < BN; ++e) mraw = fmaxf(mraw, x[e]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < BN; ++e) mraw = (e < nv) ? fmaxf(mraw, x[e]) : mraw;
+      }
+      float alpha = 1.f;
+      if (nv > 0) {
+        const float mt = mraw * c;
+        if (mt > m_used + 8.0f) {
+          alpha = ex2_approx(m_used - mt);
+          m_used = mt;
+        }
+      }
+      l *= alpha;
+      const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+      uint32_t pk[BN / 2];
+      float rs = 0.f;
+#pragma unroll
+      for (int e = 0; e < BN; e += 2) {
+        float p0 = ex2_approx(fmaf(x[e], c, -msub));
+        float p1 = ex2_approx(fmaf(x[e + 1], c, -msub));
+        if (!full) {
+          p0 = (e < nv) ? p0 : 0.f;
+          p1 = (e + 1 < nv) ? p1 : 0.f;
+        }
+        rs += p0 + p1;
+        pk[e >> 1] = pack_half2(p0, p1);
+      }
+      l += rs;
+      if (j > 0) {
+        // O holds sum_{t<j} P_t V_t once PV_{j-1} has completed.
+        if (!mbar_wait(bar(B_ODONE), (j - 1) & 1, p.err, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        __syncwarp();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + C::O_COL + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(lane_addr + C::O_COL + cc * 32, o);
+          }
+        }
+      }
+      __syncwarp();
+      {
+        uint32_t w32[32];
+#pragma unroll
+        for (int cc = 0; cc < BN / 64; ++cc) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w32[e] = pk[cc * 32 + e];
+          tmem_st32(lane_addr + static_cast<uint32_t>(j & 1) * BN + cc * 32, w32);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PFULL + (j & 1)));
+    }
+    // ---- epilogue: out = O / l (0 for rows without a visible key)
+    bool have_o = false;
+    if (ok && nJ > 0) {
+      have_o = mbar_wait(bar(B_ODONE), (nJ - 1) & 1, p.err, abort_flag);
+      tc_fence_after();
+    }
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    __syncwarp();
+    __half* orow = p.out + (sq.start + i_row) * p.out_st + static_cast<int64_t>(h) * p.out_sh;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      if (have_o) {
+        tmem_ld32(lane_addr + C::O_COL + cc * 32, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (row_ok) {
+        uint4 pkt[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pkt);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pw[e] = pack_half2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = pkt[e];
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+std::mutex g_attr_mu;
+
+template <int D, int BN>
+tm_status launch(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                 const int32_t* cu, int32_t batch, int32_t max_seqlen, const uint32_t* bitmask,
+                 int64_t mask_hs, int32_t tile_m, int32_t g, int32_t causal, cudaStream_t stream) {
+  using C = Cfg<D, BN>;
+  static bool attr_done = false;
+  {
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    if (!attr_done) {
+      tm_status st = check_cuda(cudaFuncSetAttribute(attn_fwd_kernel<D, BN>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     C::SMEM_BYTES));
+      if (st != TM_OK) return st;
+      attr_done = true;
+    }
+  }
+  CUtensorMap mQ16, mQ8, mK16, mK8, mV16;
+  tm_status st;
+  st = encode_thd_map(&mQ16, q->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q->T, q->H, D, q->stride_t,
+                      q->stride_h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TM_OK) return st;
+  st = encode_thd_map(&mK16, k->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, k->T, k->H, D, k->stride_t,
+                      k->stride_h, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TM_OK) return st;
+  st = encode_thd_map(&mV16, v->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, v->T, v->H, D, v->stride_t,
+                      v->stride_h, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TM_OK) return st;
+  const CUtensorMapSwizzle swz8 = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (bitmask != nullptr) {
+    st = encode_thd_map(&mQ8, q->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q->T, q->H, D, q->H * D, D,
+                        D, 128, swz8);
+    if (st != TM_OK) return st;
+    st = encode_thd_map(&mK8, k->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k->T, k->H, D, k->H * D, D,
+                        D, BN, swz8);
+    if (st != TM_OK) return st;
+  } else {
+    mQ8 = mQ16;
+    mK8 = mK16;
+  }
+  Params p;
+  p.out = static_cast<__half*>(out->data);
+  p.out_st = out->stride_t;
+  p.out_sh = out->stride_h;
+  p.q_scales = static_cast<const float*>(q->scales);
+  p.k_scales = static_cast<const float*>(k->scales);
+  p.bitmask = bitmask;
+  p.mask_hs = mask_hs;
+  p.cu = cu;
+  p.Lq = q->T;
+  p.Lk = k->T;
+  p.Hq = static_cast<int>(q->H);
+  p.Hkv = static_cast<int>(k->H);
+  p.tile_m = tile_m;
+  p.g = g;
+  p.causal = causal ? 1 : 0;
+  p.batch = cu ? batch : 1;
+  const int64_t maxq = cu ? max_seqlen : q->T;
+  const int64_t maxk = cu ? max_seqlen : k->T;
+  p.n_qt_max = static_cast<int>((maxq + tile_m - 1) / tile_m);
+  p.W = tm_mask_words(maxk, BN, g);
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
+  p.err = DevErr{device_error_word()};
+  const int64_t grid = static_cast<int64_t>(p.n_qt_max) * p.batch * p.Hq;
+  if (grid == 0) return TM_OK;
+  if (grid > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
+  attn_fwd_kernel<D, BN><<<static_cast<unsigned>(grid), 192, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16,
+                                                                                      mK8, mV16, p);
+  return check_cuda(cudaGetLastError());
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tm_status check_fp16(const tm_tensor* t, int64_t d) {
+  if (t == nullptr || t->data == nullptr || !aligned16(t->data)) return TM_ERR_INVALID_ARG;
+  if (t->T < 0 || t->H <= 0 || t->d != d) return TM_ERR_INVALID_ARG;
+  if (t->stride_h < d || (t->stride_h % 8) || (t->stride_t % 8)) return TM_ERR_INVALID_ARG;
+  if (t->H > 1 && t->stride_t < t->stride_h * (t->H - 1) + d) return TM_ERR_INVALID_ARG;
+  if (t->H == 1 && t->stride_t < d) return TM_ERR_INVALID_ARG;
+  return TM_OK;
+}
+
+}  // namespace
+}  // namespace tmk
+
+extern "C" tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v,
+                                 tm_tensor* out, const int32_t* cu_seqlens, int32_t batch,
+                                 int32_t max_seqlen, const uint32_t* bitmask,
+                                 int64_t mask_head_stride, int32_t tile_m, int32_t tile_n,
+                                 int32_t g, int32_t causal, void* stream) {
+  using namespace tmk;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return TM_ERR_INVALID_ARG;
+  const int64_t D = q->d;
+  if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
+  if ((tile_m != 64 && tile_m != 128) || (tile_n != 64 && tile_n != 128)) return TM_ERR_UNSUPPORTED;
+  if (g < 1 || mask_head_stride < 0) return TM_ERR_INVALID_ARG;
+  tm_status st = check_fp16(q, D);
+  if (st != TM_OK) return st;
+  st = check_fp16(out, D);
+  if (st != TM_OK) return st;
+  if (out->T != q->T || out->H != q->H) return TM_ERR_INVALID_ARG;
+  const bool cache = (k->scale_kind == TM_SCALE_TOKEN) || (v->scale_kind == TM_SCALE_TOKEN);
+  if (cache) return TM_ERR_UNSUPPORTED;   // INT8 K/V cache: see tm_attn_cache.cu
+  st = check_fp16(k, D);
+  if (st != TM_OK) return st;
+  st = check_fp16(v, D);
+  if (st != TM_OK) return st;
+  if (k->T != v->T || k->H != v->H) return TM_ERR_INVALID_ARG;
+  if (q->H % k->H != 0 || q->H > 65535) return TM_ERR_INVALID_ARG;
+  if (cu_seqlens != nullptr) {
+    if (batch <= 0 || max_seqlen <= 0 || k->T != q->T) return TM_ERR_INVALID_ARG;
+  }
+  if (bitmask != nullptr) {
+    if (reinterpret_cast<uintptr_t>(bitmask) & 3u) return TM_ERR_INVALID_ARG;
+    if (q->codes == nullptr || k->codes == nullptr || !aligned16(q->codes) || !aligned16(k->codes))
+      return TM_ERR_INVALID_ARG;
+    if (q->scale_kind != TM_SCALE_TILE || k->scale_kind != TM_SCALE_TILE || q->scales == nullptr ||
+        k->scales == nullptr)
+      return TM_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = as_stream(stream);
+  if (D == 128) {
+    if (tile_n == 128)
+      return launch<128, 128>(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride,
+                              tile_m, g, causal, s);
+    return launch<128, 64>(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride,
+                           tile_m, g, causal, s);
+  }
+  if (tile_n == 128)
+    return launch<64, 128>(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride,
+                           tile_m, g, causal, s);
+  return launch<64, 64>(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride,
+                        tile_m, g, causal, s);
+}

@@ -1,0 +1,157 @@
+// tm_quant.cu -- per-tile symmetric INT8 quantisation of Q and K
+// (tm_quantize_qk).
+//
+// TileMix (Lattice paper page), abstract: the INT8 route computes score tiles
+// from INT8 operands.  Rule implemented here, per (head, tile of `tile` rows of
+// one sequence):  amax = max|x|;  s = fl32(amax / 127);
+// code = clamp(rne(fl32(x / s)), -127, 127);  s == 0 gives codes 0.
+//
+// One CTA per (tile, sequence, head): the tile's rows x d fp16 values are
+// read once with 16-byte loads and kept in registers between the absmax pass
+// and the quantise pass, so HBM traffic is one read of x plus one write of
+// the codes.  Division is the IEEE round-to-nearest __fdiv_rn and the code
+// conversion is round-to-nearest-even, so the result is bit-identical to the
+// definition.  HBM-bound: bytes per element = 2 (read) + 1 (write).
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "tm_device.cuh"
+#include "tm_host.h"
+
+namespace tmk {
+namespace {
+
+constexpr int kQuantThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kQuantThreads)
+    quantize_tiles_kernel(const __half* __restrict__ x, int64_t stride_t, int64_t stride_h, int H,
+                          int8_t* __restrict__ codes, float* __restrict__ scales,
+                          const int32_t* __restrict__ cu, int64_t L, int tile, DevErr err) {
+  constexpr int VPR = D / 8;                       // 16-byte vectors per row
+  constexpr int MAXV = 128 * VPR / kQuantThreads;  // vectors per thread at tile = 128
+  __shared__ float red[kQuantThreads / 32];
+  __shared__ SeqInfo sinfo;
+  __shared__ float s_scale;
+
+  const int I = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
+  if (threadIdx.x == 0) {
+    sinfo = seq_info(cu, b, L, tile);
+    if (cu != nullptr && I == 0 && sinfo.len > static_cast<int64_t>(gridDim.x) * tile)
+      dev_error(err, TM_DEVERR_SEQLEN);
+  }
+  __syncthreads();
+  const SeqInfo s = sinfo;
+  const int64_t r0 = static_cast<int64_t>(I) * tile;
+  if (r0 >= s.len) return;
+  const int rows = static_cast<int>(min(static_cast<int64_t>(tile), s.len - r0));
+  const int nvec = rows * VPR;
+
+  uint4 v[MAXV];
+  __half2 m2 = __float2half2_rn(0.f);
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int idx = threadIdx.x + k * kQuantThreads;
+    if (idx < nvec) {
+      const int row = idx / VPR, c = idx % VPR;
+      const __half* src = x + (s.start + r0 + row) * stride_t + static_cast<int64_t>(h) * stride_h + c * 8;
+      v[k] = *reinterpret_cast<const uint4*>(src);
+      const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(hv[e]));
+    }
+  }
+  float m = fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = red[0];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[w]);
+    const float sc = __fdiv_rn(a, 127.0f);
+    s_scale = sc;
+    scales[(s.tile_base + I) * H + h] = sc;
+  }
+  __syncthreads();
+  const float sc = s_scale;
+  const int64_t code_row_stride = static_cast<int64_t>(H) * D;
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k) {
+    const int idx = threadIdx.x + k * kQuantThreads;
+    if (idx < nvec) {
+      const int row = idx / VPR, c = idx % VPR;
+      const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
+      uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float f = (e & 1) ? __high2float(hv[e >> 1]) : __low2float(hv[e >> 1]);
+        int qv = 0;
+        if (sc != 0.f) {
+          qv = __float2int_rn(__fdiv_rn(f, sc));
+          qv = max(-127, min(127, qv));
+        }
+        packed[e >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
+      }
+      int8_t* dst = codes + (s.start + r0 + row) * code_row_stride + static_cast<int64_t>(h) * D + c * 8;
+      *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    }
+  }
+}
+
+tm_status check_operand(const tm_tensor* t) {
+  if (t == nullptr || t->data == nullptr) return TM_ERR_INVALID_ARG;
+  if (t->T < 0 || t->H <= 0 || t->d <= 0) return TM_ERR_INVALID_ARG;
+  if (t->d != 64 && t->d != 128) return TM_ERR_UNSUPPORTED;
+  if (t->stride_h < t->d || t->stride_t < t->stride_h * (t->H - 1) + t->d) return TM_ERR_INVALID_ARG;
+  if ((t->stride_h % 8) || (t->stride_t % 8)) return TM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(t->data) % 16) return TM_ERR_INVALID_ARG;
+  return TM_OK;
+}
+
+tm_status launch_quant(const tm_tensor* x, int8_t* codes, float* scales, const int32_t* cu,
+                       int32_t batch, int32_t max_seqlen, int32_t tile, cudaStream_t stream) {
+  if (codes == nullptr || scales == nullptr) return TM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(codes) % 16 || reinterpret_cast<uintptr_t>(scales) % 4)
+    return TM_ERR_INVALID_ARG;
+  const int64_t maxlen = cu ? max_seqlen : x->T;
+  const int nb = cu ? batch : 1;
+  if (maxlen <= 0 || nb <= 0) return TM_OK;   // nothing to quantise
+  const int64_t ntile = (maxlen + tile - 1) / tile;
+  if (ntile > 0x7fffffff || nb > 65535 || x->H > 65535) return TM_ERR_UNSUPPORTED;
+  dim3 grid(static_cast<unsigned>(ntile), static_cast<unsigned>(nb), static_cast<unsigned>(x->H));
+  DevErr err{device_error_word()};
+  const __half* xp = static_cast<const __half*>(x->data);
+  if (x->d == 128)
+    quantize_tiles_kernel<128><<<grid, kQuantThreads, 0, stream>>>(
+        xp, x->stride_t, x->stride_h, static_cast<int>(x->H), codes, scales, cu, x->T, tile, err);
+  else
+    quantize_tiles_kernel<64><<<grid, kQuantThreads, 0, stream>>>(
+        xp, x->stride_t, x->stride_h, static_cast<int>(x->H), codes, scales, cu, x->T, tile, err);
+  return check_cuda(cudaGetLastError());
+}
+
+}  // namespace
+}  // namespace tmk
+
+extern "C" tm_status tm_quantize_qk(const tm_tensor* q, const tm_tensor* k, int8_t* q_codes,
+                                    float* q_scales, int8_t* k_codes, float* k_scales,
+                                    const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen,
+                                    int32_t tile_m, int32_t tile_n, void* stream) {
+  using namespace tmk;
+  if ((tile_m != 64 && tile_m != 128) || (tile_n != 64 && tile_n != 128)) return TM_ERR_UNSUPPORTED;
+  tm_status st = check_operand(q);
+  if (st != TM_OK) return st;
+  if (k != nullptr) {
+    st = check_operand(k);
+    if (st != TM_OK) return st;
+    if (k->d != q->d) return TM_ERR_INVALID_ARG;
+    if (cu_seqlens != nullptr && k->T != q->T) return TM_ERR_INVALID_ARG;
+  }
+  if (cu_seqlens != nullptr && (batch <= 0 || max_seqlen <= 0)) return TM_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  st = launch_quant(q, q_codes, q_scales, cu_seqlens, batch, max_seqlen, tile_m, s);
+  if (st != TM_OK || k == nullptr) return st;
+  return launch_quant(k, k_codes, k_scales, cu_seqlens, batch, max_seqlen, tile_n, s);
+}

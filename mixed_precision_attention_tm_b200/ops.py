@@ -1,0 +1,281 @@
+"""Thin Python binding of libtm (ctypes).
+
+Argument marshalling only: every step of tile-routed attention runs in the
+library's CUDA kernels.  PyTorch supplies device memory and the current
+stream; outputs are allocated here with torch and passed to the library as
+raw pointers.  There is no CPU fallback: if libtm.so is missing the import
+fails, and a CUDA tensor is required wherever the library expects device
+memory.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtm.so")
+HEADER = os.path.join(_HERE, "..", "include", "tm.h")
+
+TM_OK, TM_ERR_INVALID_ARG, TM_ERR_UNSUPPORTED, TM_ERR_CUDA, TM_ERR_TIMEOUT = range(5)
+TM_SCALE_NONE, TM_SCALE_TILE, TM_SCALE_TOKEN = range(3)
+
+
+class TmError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {_lib().tm_status_string(status).decode()} (status {status}"
+                         + (f", cuda {_lib().tm_last_cuda_error()})" if status == TM_ERR_CUDA else ")"))
+
+
+class TmTensor(ctypes.Structure):
+    _fields_ = [
+        ("data", ctypes.c_void_p),
+        ("T", ctypes.c_int64), ("H", ctypes.c_int64), ("d", ctypes.c_int64),
+        ("stride_t", ctypes.c_int64), ("stride_h", ctypes.c_int64),
+        ("codes", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+        ("scale_kind", ctypes.c_int32),
+    ]
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libtm.so not built at {LIB_PATH}; run "
+                              "`python -m mixed_precision_attention_tm_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, U64, D = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_double
+        TP = ctypes.POINTER(TmTensor)
+        sig = {
+            "tm_quantize_qk": (I32, [TP, TP, P, P, P, P, P, I32, I32, I32, I32, P]),
+            "tm_mask_words": (I32, [I64, I32, I32]),
+            "tm_count_tiles": (I64, [P, I32, I64, I32]),
+            "tm_build_mask": (I32, [P, I32, P, I32, I32, I64, I64, I32, I32, I32, I32, D, U64, I32, I32,
+                                    I64, P]),
+            "tm_build_mask_host": (I32, [P, I32, P, I32, I64, I64, I32, I32, I32, I32, D, U64, I32, I32]),
+            "tm_route_stats": (I32, [P, I64, I32, P, I32, I64, I64, I32, I32, I32, I32,
+                                     ctypes.POINTER(D), ctypes.POINTER(D)]),
+            "tm_attn_fwd": (I32, [TP, TP, TP, TP, P, I32, I32, P, I64, I32, I32, I32, I32, P]),
+            "tm_get_device_error": (I32, [P]),
+            "tm_status_string": (ctypes.c_char_p, [I32]),
+            "tm_last_cuda_error": (I32, []),
+            "tm_version": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def header_functions():
+    """Names of the functions declared in include/tm.h."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tm_[a-z0-9_]+)\s*\(", src)))
+
+
+def _check(st, what):
+    if st != TM_OK:
+        raise TmError(st, what)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _cuda(t, name):
+    if t is not None and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _desc(x, codes=None, scales=None, scale_kind=TM_SCALE_NONE, shape_from=None):
+    """tm_tensor for a [T, H, d] tensor (x may be None for an INT8 cache)."""
+    ref = x if x is not None else shape_from
+    T, H, d = ref.shape
+    if x is not None:
+        if x.dtype != torch.float16:
+            raise ValueError("fp16 tensor expected")
+        if x.stride(2) != 1:
+            raise ValueError("innermost dimension must be contiguous")
+        st, sh = x.stride(0), x.stride(1)
+    else:
+        st, sh = H * d, d
+    return TmTensor(None if x is None else x.data_ptr(), T, H, d, st, sh,
+                    None if codes is None else codes.data_ptr(),
+                    None if scales is None else scales.data_ptr(), scale_kind)
+
+
+def _cu_host(cu_seqlens):
+    if cu_seqlens is None:
+        return None
+    return cu_seqlens.detach().to("cpu", torch.int32).contiguous()
+
+
+def count_tiles(L=None, tile=128, cu_seqlens_host=None):
+    lib = _lib()
+    if cu_seqlens_host is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
+        return int(lib.tm_count_tiles(cu.ctypes.data, len(cu) - 1, 0, tile))
+    return int(lib.tm_count_tiles(None, 0, int(L), tile))
+
+
+def mask_words(max_lk, tile_n, g):
+    return int(_lib().tm_mask_words(int(max_lk), int(tile_n), int(g)))
+
+
+# ---------------------------------------------------------------- quantise
+def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqlen=None):
+    """Per-tile INT8 codes and fp32 scales of Q (tile_m rows) and K (tile_n
+    rows): returns (q_codes [Tq,Hq,d] int8, q_scales [n_qt, Hq] fp32,
+    k_codes, k_scales) (the K pair is None when k is None)."""
+    _cuda(q, "q")
+    _cuda(k, "k")
+    lib = _lib()
+    cu_h = _cu_host(cu_seqlens)
+    batch = 0 if cu_h is None else cu_h.numel() - 1
+    if cu_seqlens is not None and max_seqlen is None:
+        max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0
+    nqt = count_tiles(q.shape[0], tile_m, None if cu_h is None else cu_h.numpy())
+    qc = torch.empty(q.shape, dtype=torch.int8, device=q.device)
+    qs = torch.empty((nqt, q.shape[1]), dtype=torch.float32, device=q.device)
+    kc = ks = None
+    if k is not None:
+        nkt = count_tiles(k.shape[0], tile_n, None if cu_h is None else cu_h.numpy())
+        kc = torch.empty(k.shape, dtype=torch.int8, device=k.device)
+        ks = torch.empty((nkt, k.shape[1]), dtype=torch.float32, device=k.device)
+    qd = _desc(q)
+    kd = _desc(k) if k is not None else None
+    st = lib.tm_quantize_qk(ctypes.byref(qd), None if kd is None else ctypes.byref(kd),
+                            _ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks), _ptr(cu_seqlens), batch,
+                            int(max_seqlen or 0), tile_m, tile_n, _stream())
+    _check(st, "tm_quantize_qk")
+    return qc, qs, kc, ks
+
+
+# ---------------------------------------------------------------- mask
+def build_mask(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False, force_sink=False,
+               Lq=None, Lk=None, cu_seqlens=None, max_seqlen=None, device="cuda"):
+    """Seeded routing bitmask on the device, int32 view [Hq, n_qt, W] of the
+    uint32 words (bit 1 = INT8)."""
+    lib = _lib()
+    cu_h = _cu_host(cu_seqlens)
+    batch = 0 if cu_h is None else cu_h.numel() - 1
+    if cu_h is not None:
+        lens = (cu_h[1:] - cu_h[:-1])
+        maxk = int(lens.max()) if batch else 0
+        if max_seqlen is None:
+            max_seqlen = maxk
+        nqt = count_tiles(None, tile_m, cu_h.numpy())
+    else:
+        maxk = Lk
+        nqt = count_tiles(Lq, tile_m)
+    W = mask_words(maxk, tile_n, g)
+    out = torch.zeros((Hq, nqt, W), dtype=torch.int32, device=device)
+    st = lib.tm_build_mask(_ptr(out), Hq, _ptr(cu_seqlens), batch, int(max_seqlen or 0),
+                           int(Lq or 0), int(Lk or 0), tile_m, tile_n, g, int(bool(causal)),
+                           float(p), ctypes.c_uint64(int(seed) & (2 ** 64 - 1)),
+                           int(bool(force_diag)), int(bool(force_sink)), nqt * W, _stream())
+    _check(st, "tm_build_mask")
+    return out
+
+
+def build_mask_host(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False, force_sink=False,
+                    Lq=None, Lk=None, cu_seqlens_host=None):
+    """Host twin of build_mask: numpy uint32 [Hq, n_qt, W]."""
+    lib = _lib()
+    cu = None if cu_seqlens_host is None else np.ascontiguousarray(np.asarray(cu_seqlens_host, np.int32))
+    batch = 0 if cu is None else len(cu) - 1
+    if cu is not None:
+        maxk = int((cu[1:] - cu[:-1]).max()) if batch else 0
+        nqt = count_tiles(None, tile_m, cu)
+    else:
+        maxk = Lk
+        nqt = count_tiles(Lq, tile_m)
+    W = mask_words(maxk, tile_n, g)
+    out = np.zeros((Hq, nqt, W), dtype=np.uint32)
+    st = lib.tm_build_mask_host(out.ctypes.data, Hq, None if cu is None else cu.ctypes.data, batch,
+                                int(Lq or 0), int(Lk or 0), tile_m, tile_n, g, int(bool(causal)),
+                                float(p), ctypes.c_uint64(int(seed) & (2 ** 64 - 1)),
+                                int(bool(force_diag)), int(bool(force_sink)))
+    _check(st, "tm_build_mask_host")
+    return out
+
+
+def route_stats(mask_host, *, Hq, tile_m, tile_n, g, causal, Lq=None, Lk=None, cu_seqlens_host=None):
+    """(n_vis, e8) from a host mask (numpy uint32 [Hm, n_qt, W]) or None."""
+    lib = _lib()
+    cu = None if cu_seqlens_host is None else np.ascontiguousarray(np.asarray(cu_seqlens_host, np.int32))
+    batch = 0 if cu is None else len(cu) - 1
+    nv, e8 = ctypes.c_double(), ctypes.c_double()
+    ptr, hs = None, 0
+    if mask_host is not None:
+        m = np.ascontiguousarray(mask_host.astype(np.uint32, copy=False))
+        ptr = m.ctypes.data
+        hs = 0 if m.shape[0] == 1 else m.shape[1] * m.shape[2]
+    st = lib.tm_route_stats(ptr, hs, Hq, None if cu is None else cu.ctypes.data, batch, int(Lq or 0),
+                            int(Lk or 0), tile_m, tile_n, g, int(bool(causal)), ctypes.byref(nv),
+                            ctypes.byref(e8))
+    _check(st, "tm_route_stats")
+    return nv.value, e8.value
+
+
+# ---------------------------------------------------------------- attention
+def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal=False,
+             bitmask=None, mask_head_stride=None, q_quant=None, k_quant=None, kv_cache=None,
+             cu_seqlens=None, max_seqlen=None):
+    """Fused tile-routed attention.  q: fp16 [Tq,Hq,d]; k, v: fp16 [Tk,Hkv,d]
+    (or kv_cache = (k_codes, k_scale16, v_codes, v_scale16)); bitmask: int32
+    view [Hm, n_qt, W] (Hm = Hq or 1) or None (all FP16); q_quant / k_quant:
+    (codes, scales) from quantize_qk, needed with a bitmask.  Returns out."""
+    _cuda(q, "q")
+    lib = _lib()
+    if out is None:
+        out = torch.empty_like(q)
+    cu_h = _cu_host(cu_seqlens)
+    batch = 0 if cu_h is None else cu_h.numel() - 1
+    if cu_seqlens is not None and max_seqlen is None:
+        max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0
+    qd = _desc(q, *(q_quant if q_quant is not None else (None, None)),
+               scale_kind=TM_SCALE_TILE if q_quant is not None else TM_SCALE_NONE)
+    if kv_cache is not None:
+        kcod, ksc, vcod, vsc = kv_cache
+        kd = _desc(None, kcod, ksc, TM_SCALE_TOKEN, shape_from=kcod)
+        vd = _desc(None, vcod, vsc, TM_SCALE_TOKEN, shape_from=vcod)
+    else:
+        _cuda(k, "k")
+        _cuda(v, "v")
+        kd = _desc(k, *(k_quant if k_quant is not None else (None, None)),
+                   scale_kind=TM_SCALE_TILE if k_quant is not None else TM_SCALE_NONE)
+        vd = _desc(v)
+    od = _desc(out)
+    if bitmask is not None and mask_head_stride is None:
+        mask_head_stride = 0 if bitmask.shape[0] == 1 else bitmask.shape[1] * bitmask.shape[2]
+    st = lib.tm_attn_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
+                         _ptr(cu_seqlens), batch, int(max_seqlen or 0), _ptr(bitmask),
+                         int(mask_head_stride or 0), tile_m, tile_n, g, int(bool(causal)), _stream())
+    _check(st, "tm_attn_fwd")
+    return out
+
+
+def get_device_error():
+    return int(_lib().tm_get_device_error(_stream()))
+
+
+def sm_scale(d):
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,241 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the fp64 oracle on
+identical seeded inputs.
+
+Bars: INT8 codes, tile scales and routing bits bit-exact; attention output
+max-abs error <= 3e-3 (fp16 output, unit-variance inputs).  Sizes span
+several tiles and a ragged tail while the oracle still finishes in seconds.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import TOL, max_err, oracle_mask, run_gpu, run_oracle, seqs_of
+from mixed_precision_attention_tm_b200 import inputs, ops
+
+pytestmark = pytest.mark.gpu
+
+
+def W(Lq, Lk, hq, hkv, d, causal, tm=128, tn=128, g=1, p=None, seed=0, fd=False, fs=False,
+      outliers=False, cu=None):
+    if cu is not None:
+        cu_t = torch.tensor(cu, dtype=torch.int32)
+        lens = cu_t[1:] - cu_t[:-1]
+        Lq = Lk = int(cu[-1])
+    else:
+        cu_t = lens = None
+    if outliers:
+        q, k, _ = inputs.qk_with_outliers(Lq, Lk, hq, hkv, d, seed)
+    else:
+        q, k = inputs.randn_f16((Lq, hq, d), seed), inputs.randn_f16((Lk, hkv, d), seed + 1)
+    v = inputs.randn_f16((Lk, hkv, d), seed + 2)
+    return inputs.Workload(f"w{Lq}x{Lk}", q, k, v, hq, hkv, d, causal, tm, tn, g, p, mask_seed=seed + 4,
+                           force_diag=fd, force_sink=fs, cu_seqlens=cu_t, lens=lens)
+
+
+# ------------------------------------------------------------------ quantiser
+QUANT_CASES = [
+    # (T, H, d, tile, cu, scale)
+    (256, 2, 64, 64, None, 1.0),
+    (1000, 4, 128, 128, None, 1.0),
+    (777, 3, 64, 128, None, 20.0),
+    (1400, 2, 128, 64, [0, 300, 300, 1100, 1400], 1.0),
+    (50, 1, 128, 128, None, 1e-3),
+]
+
+
+@pytest.mark.parametrize("case", QUANT_CASES)
+def test_quantizer_bit_exact(case):
+    T, H, d, tile, cu, scale = case
+    x = inputs.randn_f16((T, H, d), 7, scale)
+    x[3:5] = 0                                    # zeros inside a tile
+    if T >= 256:
+        x[tile:2 * tile, 0] = 0                   # an all-zero (tile, head) block
+    cu_t = None if cu is None else torch.tensor(cu, dtype=torch.int32, device="cuda")
+    maxlen = None if cu is None else max(b - a for a, b in zip(cu[:-1], cu[1:]))
+    qc, qs, _, _ = ops.quantize_qk(x.cuda(), None, tile_m=tile, tile_n=tile, cu_seqlens=cu_t, max_seqlen=maxlen)
+    torch.cuda.synchronize()
+    seqs = oracle.seq_table(T, T, cu)
+    rc, rs = oracle.quantize_tiles(x.numpy(), seqs, tile, "q")
+    assert np.array_equal(qs.cpu().numpy(), rs)
+    assert np.array_equal(qc.cpu().numpy(), rc)
+
+
+def test_quantizer_q_and_k_tiles_differ():
+    q = inputs.randn_f16((500, 4, 128), 1)
+    k = inputs.randn_f16((500, 2, 128), 2)
+    qc, qs, kc, ks = ops.quantize_qk(q.cuda(), k.cuda(), tile_m=64, tile_n=128)
+    torch.cuda.synchronize()
+    seqs = oracle.seq_table(500, 500)
+    rqc, rqs = oracle.quantize_tiles(q.numpy(), seqs, 64, "q")
+    rkc, rks = oracle.quantize_tiles(k.numpy(), seqs, 128, "k")
+    assert np.array_equal(qs.cpu().numpy(), rqs) and np.array_equal(qc.cpu().numpy(), rqc)
+    assert np.array_equal(ks.cpu().numpy(), rks) and np.array_equal(kc.cpu().numpy(), rkc)
+
+
+# ------------------------------------------------------------------ mask
+MASK_CASES = [
+    # (Hq, Lq, Lk, cu, tm, tn, g, causal, p, fd, fs)
+    (2, 256, 256, None, 64, 64, 1, False, 0.5, False, False),
+    (32, 16384, 16384, None, 128, 128, 4, True, 0.75, True, True),
+    (3, 700, 2100, None, 128, 64, 3, True, 0.4, True, False),
+    (4, 1500, 300, None, 64, 128, 1, True, 0.9, False, True),
+    (5, 0, 0, [0, 1000, 1000, 5000, 5001], 128, 128, 4, True, 0.75, True, True),
+    (28, 65536, 65536, None, 128, 128, 8, True, 0.5, True, True),
+]
+
+
+@pytest.mark.parametrize("case", MASK_CASES)
+def test_device_mask_bit_exact(case):
+    Hq, Lq, Lk, cu, tm, tn, g, causal, p, fd, fs = case
+    seed = 1234 + Hq
+    cu_t = None if cu is None else torch.tensor(cu, dtype=torch.int32, device="cuda")
+    m = ops.build_mask(Hq, tile_m=tm, tile_n=tn, g=g, causal=causal, p=p, seed=seed, force_diag=fd,
+                       force_sink=fs, Lq=Lq, Lk=Lk, cu_seqlens=cu_t)
+    torch.cuda.synchronize()
+    got = m.cpu().numpy().view(np.uint32)
+    if cu is not None:
+        Lq = Lk = cu[-1]
+    ref = oracle.build_mask(Hq, oracle.seq_table(Lq, Lk, cu), tm, tn, g, causal, p, seed, fd, fs)
+    assert np.array_equal(got, ref)
+    host = ops.build_mask_host(Hq, tile_m=tm, tile_n=tn, g=g, causal=causal, p=p, seed=seed,
+                               force_diag=fd, force_sink=fs, Lq=Lq, Lk=Lk, cu_seqlens_host=cu)
+    assert np.array_equal(got, host)
+
+
+# ------------------------------------------------------------------ attention vs oracle
+ATTN_CASES = [
+    # id, workload kwargs
+    ("tiny_fp16", dict(Lq=256, Lk=256, hq=2, hkv=1, d=64, causal=False, tm=64, tn=64)),
+    ("tiny_int8_half", dict(Lq=256, Lk=256, hq=2, hkv=1, d=64, causal=False, tm=64, tn=64, p=0.5)),
+    ("d128_causal_ragged", dict(Lq=1000, Lk=1000, hq=4, hkv=2, d=128, causal=True)),
+    ("d128_noncausal_ragged", dict(Lq=1000, Lk=1000, hq=4, hkv=2, d=128, causal=False)),
+    ("d64_causal_ragged", dict(Lq=1000, Lk=1000, hq=4, hkv=1, d=64, causal=True)),
+    ("d128_routed_g2", dict(Lq=1000, Lk=1000, hq=4, hkv=2, d=128, causal=True, g=2, p=0.5, fd=True, fs=True)),
+    ("d128_all_int8", dict(Lq=700, Lk=700, hq=2, hkv=1, d=128, causal=False, p=1.0)),
+    ("d64_routed", dict(Lq=900, Lk=900, hq=4, hkv=2, d=64, causal=True, p=0.6)),
+    ("q_shorter", dict(Lq=300, Lk=1000, hq=2, hkv=2, d=128, causal=True, p=0.5)),
+    ("q_longer_empty_rows", dict(Lq=1000, Lk=300, hq=2, hkv=1, d=128, causal=True, p=0.5)),
+    ("tm64_tn128", dict(Lq=600, Lk=600, hq=2, hkv=1, d=128, causal=True, tm=64, tn=128, p=0.5)),
+    ("tm128_tn64", dict(Lq=600, Lk=600, hq=2, hkv=1, d=128, causal=True, tm=128, tn=64, p=0.5)),
+    ("d64_tn128_tm64", dict(Lq=600, Lk=600, hq=2, hkv=1, d=64, causal=False, tm=64, tn=128, p=0.5)),
+    ("outliers_routed", dict(Lq=1024, Lk=1024, hq=4, hkv=1, d=128, causal=True, g=4, p=0.75, fd=True, fs=True,
+                              outliers=True)),
+    ("varlen_routed", dict(Lq=0, Lk=0, hq=4, hkv=2, d=128, causal=True, g=2, p=0.5, fd=True, fs=True,
+                           cu=[0, 300, 300, 1100, 1400])),
+    ("varlen_fp16_noncausal", dict(Lq=0, Lk=0, hq=2, hkv=1, d=64, causal=False, cu=[0, 129, 200, 457])),
+    ("short_T", dict(Lq=50, Lk=50, hq=1, hkv=1, d=128, causal=True, p=0.5)),
+    ("single_token", dict(Lq=1, Lk=1, hq=2, hkv=1, d=64, causal=True)),
+]
+
+
+@pytest.mark.parametrize("name,kw", ATTN_CASES, ids=[c[0] for c in ATTN_CASES])
+def test_attention_matches_oracle(name, kw):
+    w = W(**kw)
+    out, m, quant = run_gpu(w)
+    mask_u32 = None if m is None else m.numpy().view(np.uint32)
+    if mask_u32 is not None:
+        assert np.array_equal(mask_u32, oracle_mask(w))        # device bits == oracle bits
+        seqs, _ = seqs_of(w)
+        rqc, rqs = oracle.quantize_tiles(w.q.numpy(), seqs, w.tile_m, "q")
+        assert np.array_equal(quant[1].numpy(), rqs) and np.array_equal(quant[0].numpy(), rqc)
+    ref = run_oracle(w, mask_u32)
+    assert torch.isfinite(out).all()
+    err = max_err(out, ref)
+    assert err <= TOL, f"{name}: max abs err {err}"
+
+
+# ------------------------------------------------------------------ GPU invariants
+def test_lossless_inputs_route_invisible_on_gpu():
+    L, hq, hkv, d = 640, 2, 1, 128
+    q, k = inputs.lossless_qk([(0, L)], [(0, L)], L, L, hq, hkv, d, 128, 128, seed=3)
+    v = inputs.randn_f16((L, hkv, d), 5)
+    base = inputs.Workload("ll", q, k, v, hq, hkv, d, True, 128, 128, 1, None)
+    routed = inputs.Workload("ll", q, k, v, hq, hkv, d, True, 128, 128, 1, 0.6, mask_seed=9)
+    o0, _, _ = run_gpu(base)
+    o1, m, _ = run_gpu(routed)
+    assert m.numpy().any()
+    # INT8 and FP16 scores are the same numbers here, so the outputs agree bit for bit
+    assert torch.equal(o0, o1)
+
+
+def test_constant_values_give_ones():
+    w = W(Lq=800, Lk=800, hq=2, hkv=1, d=128, causal=True, p=0.5)
+    w.v = torch.ones_like(w.v)
+    out, _, _ = run_gpu(w)
+    assert (out.float() - 1).abs().max().item() <= 2e-3
+
+
+def test_gqa_equals_repeated_heads_on_gpu():
+    w = W(Lq=640, Lk=640, hq=8, hkv=2, d=128, causal=True, p=0.5)
+    o1, m, _ = run_gpu(w)
+    w2 = W(Lq=640, Lk=640, hq=8, hkv=2, d=128, causal=True, p=0.5)
+    w2.k = w.k.repeat_interleave(4, dim=1)
+    w2.v = w.v.repeat_interleave(4, dim=1)
+    w2.hkv = 8
+    o2, _, _ = run_gpu(w2, mask=m.numpy().view(np.uint32))
+    assert torch.equal(o1, o2)
+
+
+def test_varlen_equals_separate_calls_on_gpu():
+    cu = [0, 300, 300, 1100, 1400]
+    w = W(Lq=0, Lk=0, hq=4, hkv=2, d=128, causal=True, g=2, p=0.5, cu=cu)
+    whole, m, _ = run_gpu(w)
+    mask = m.numpy().view(np.uint32)
+    qt0 = 0
+    for b in range(len(cu) - 1):
+        a, e = cu[b], cu[b + 1]
+        n = oracle.n_tiles(e - a, 128)
+        sub = mask[:, qt0:qt0 + n, :]
+        qt0 += n
+        if e == a:
+            continue
+        wb = inputs.Workload("part", w.q[a:e].clone(), w.k[a:e].clone(), w.v[a:e].clone(), 4, 2, 128, True,
+                             128, 128, 2, 0.5)
+        part, _, _ = run_gpu(wb, mask=np.ascontiguousarray(sub[:, :, :oracle.mask_words(e - a, 128, 2)]))
+        assert torch.equal(whole[a:e], part), b
+
+
+def test_grouping_equals_replicated_bits_on_gpu():
+    w = W(Lq=1024, Lk=1024, hq=2, hkv=1, d=128, causal=True, g=3, p=0.5)
+    o3, m, _ = run_gpu(w)
+    mg = m.numpy().view(np.uint32)
+    nkt = 1024 // 128
+    m1 = np.zeros((2, mg.shape[1], 1), dtype=np.uint32)
+    for h in range(2):
+        for I in range(mg.shape[1]):
+            for J in range(nkt):
+                if oracle.mask_bit(mg, h, I, J // 3):
+                    m1[h, I, 0] |= np.uint32(1 << J)
+    w1 = W(Lq=1024, Lk=1024, hq=2, hkv=1, d=128, causal=True, g=1, p=0.5)
+    o1, _, _ = run_gpu(w1, mask=m1)
+    assert torch.equal(o3, o1)
+
+
+def test_shared_mask_plane_on_gpu():
+    w = W(Lq=512, Lk=512, hq=4, hkv=1, d=128, causal=False, p=0.5)
+    seqs, _ = seqs_of(w)
+    one = oracle.build_mask(1, seqs, 128, 128, 1, False, 0.5, 77)
+    o_shared, _, _ = run_gpu(w, mask=one)
+    o_full, _, _ = run_gpu(w, mask=np.repeat(one, 4, axis=0))
+    assert torch.equal(o_shared, o_full)
+
+
+def test_deterministic():
+    w = W(Lq=1000, Lk=1000, hq=4, hkv=2, d=128, causal=True, p=0.5)
+    a, _, _ = run_gpu(w)
+    b, _, _ = run_gpu(w)
+    assert torch.equal(a, b)
+
+
+def test_noncontiguous_head_strides():
+    # Q / K / V as slices of one packed [T, Hq + 2 Hkv, d] projection output
+    L, hq, hkv, d = 700, 4, 2, 128
+    packed = inputs.randn_f16((L, hq + 2 * hkv, d), 21)
+    q, k, v = packed[:, :hq], packed[:, hq:hq + hkv], packed[:, hq + hkv:]
+    pc = packed.cuda()
+    out = ops.attn_fwd(pc[:, :hq], pc[:, hq:hq + hkv], pc[:, hq + hkv:], causal=True)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q.numpy(), k.numpy(), v.numpy(), causal=True)
+    assert max_err(out.cpu(), ref) <= TOL

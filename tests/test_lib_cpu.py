@@ -1,0 +1,121 @@
+"""CPU checks of the C-ABI library: it loads, exports every function that
+include/tm.h declares, its host-side routing functions agree bit for bit with
+the oracle, and argument validation rejects bad calls before any launch.
+No GPU compute is called here."""
+
+import ctypes
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from mixed_precision_attention_tm_b200 import build as tmbuild
+
+tmbuild.build()
+from mixed_precision_attention_tm_b200 import ops  # noqa: E402
+
+
+def test_library_exports_every_declared_symbol():
+    names = ops.header_functions()
+    assert len(names) >= 10
+    lib = ops._lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", ops.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if l.strip()}
+    assert set(names) <= exported
+
+
+def test_status_strings_and_version():
+    lib = ops._lib()
+    assert lib.tm_status_string(0) == b"ok"
+    assert lib.tm_status_string(4) == b"device wait timed out"
+    assert lib.tm_version().count(b".") == 2
+
+
+@pytest.mark.parametrize("L,tile_n,g", [(16384, 128, 4), (16385, 128, 4), (65536, 128, 8), (256, 64, 1),
+                                        (1, 128, 1), (0, 64, 3)])
+def test_mask_words_matches_oracle(L, tile_n, g):
+    assert ops.mask_words(L, tile_n, g) == oracle.mask_words(L, tile_n, g)
+
+
+def test_count_tiles():
+    assert ops.count_tiles(1000, 128) == 8
+    assert ops.count_tiles(None, 64, [0, 70, 70, 231, 300]) == 2 + 0 + 3 + 2
+
+
+MASK_CASES = [
+    # (Hq, Lq, Lk, cu, tm, tn, g, causal, p, fd, fs)
+    (2, 256, 256, None, 64, 64, 1, False, 0.5, False, False),
+    (32, 16384, 16384, None, 128, 128, 4, True, 0.75, True, True),
+    (3, 700, 2100, None, 128, 64, 3, True, 0.4, True, False),
+    (4, 1500, 300, None, 64, 128, 1, True, 0.9, False, True),
+    (5, 0, 0, [0, 1000, 1000, 5000, 5001], 128, 128, 4, True, 0.75, True, True),
+    (28, 65536, 65536, None, 128, 128, 8, True, 0.5, True, True),
+    (2, 4096, 4096, None, 128, 128, 1, False, 1.0, False, False),
+    (2, 4096, 4096, None, 128, 128, 1, True, 0.0, False, False),
+]
+
+
+@pytest.mark.parametrize("case", MASK_CASES)
+def test_host_mask_builder_bit_exact_vs_oracle(case):
+    Hq, Lq, Lk, cu, tm, tn, g, causal, p, fd, fs = case
+    seed = 0xC0FFEE + Hq
+    got = ops.build_mask_host(Hq, tile_m=tm, tile_n=tn, g=g, causal=causal, p=p, seed=seed,
+                              force_diag=fd, force_sink=fs, Lq=Lq, Lk=Lk, cu_seqlens_host=cu)
+    if cu is not None:
+        Lq = Lk = cu[-1]
+    seqs = oracle.seq_table(Lq, Lk, cu)
+    ref = oracle.build_mask(Hq, seqs, tm, tn, g, causal, p, seed, fd, fs)
+    assert got.shape == ref.shape
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("case", MASK_CASES[:5])
+def test_route_stats_matches_oracle(case):
+    Hq, Lq, Lk, cu, tm, tn, g, causal, p, fd, fs = case
+    m = ops.build_mask_host(Hq, tile_m=tm, tile_n=tn, g=g, causal=causal, p=p, seed=3,
+                            force_diag=fd, force_sink=fs, Lq=Lq, Lk=Lk, cu_seqlens_host=cu)
+    nv, e8 = ops.route_stats(m, Hq=Hq, tile_m=tm, tile_n=tn, g=g, causal=causal, Lq=Lq, Lk=Lk,
+                             cu_seqlens_host=cu)
+    if cu is not None:
+        Lq = Lk = cu[-1]
+    seqs = oracle.seq_table(Lq, Lk, cu)
+    rnv, re8 = oracle.route_stats(m, seqs, Hq, tm, tn, g, causal)
+    assert (nv, e8) == (rnv, re8)
+
+
+def _t(T=256, H=2, d=64, data=1 << 20):
+    return ops.TmTensor(data, T, H, d, H * d, d, None, None, 0)
+
+
+def test_validation_rejects_before_launch():
+    lib = ops._lib()
+    q, k, v, o = _t(), _t(H=1), _t(H=1), _t()
+    by = ctypes.byref
+    # d outside {64, 128}
+    bad = _t(d=96)
+    assert lib.tm_attn_fwd(by(bad), by(k), by(v), by(o), None, 0, 0, None, 0, 64, 64, 1, 0, None) == ops.TM_ERR_UNSUPPORTED
+    # tile sizes
+    assert lib.tm_attn_fwd(by(q), by(k), by(v), by(o), None, 0, 0, None, 0, 32, 64, 1, 0, None) == ops.TM_ERR_UNSUPPORTED
+    # Hq not a multiple of Hkv
+    k3, v3 = _t(H=3), _t(H=3)
+    assert lib.tm_attn_fwd(by(q), by(k3), by(v3), by(o), None, 0, 0, None, 0, 64, 64, 1, 0, None) == ops.TM_ERR_INVALID_ARG
+    # misaligned pointer
+    qm = _t(data=(1 << 20) + 2)
+    assert lib.tm_attn_fwd(by(qm), by(k), by(v), by(o), None, 0, 0, None, 0, 64, 64, 1, 0, None) == ops.TM_ERR_INVALID_ARG
+    # bitmask without codes / scales
+    assert lib.tm_attn_fwd(by(q), by(k), by(v), by(o), None, 0, 0, ctypes.c_void_p(1 << 20), 0, 64, 64, 1, 0,
+                           None) == ops.TM_ERR_INVALID_ARG
+    # g < 1
+    assert lib.tm_attn_fwd(by(q), by(k), by(v), by(o), None, 0, 0, None, 0, 64, 64, 0, 0, None) == ops.TM_ERR_INVALID_ARG
+    # varlen without batch
+    assert lib.tm_attn_fwd(by(q), by(k), by(v), by(o), ctypes.c_void_p(1 << 20), 0, 16, None, 0, 64, 64, 1, 0,
+                           None) == ops.TM_ERR_INVALID_ARG
+    # quantiser: null outputs, bad tile
+    assert lib.tm_quantize_qk(by(q), None, None, None, None, None, None, 0, 0, 64, 64, None) == ops.TM_ERR_INVALID_ARG
+    assert lib.tm_quantize_qk(by(q), None, None, None, None, None, None, 0, 0, 48, 64, None) == ops.TM_ERR_UNSUPPORTED
+    # mask builder: p outside [0, 1]
+    assert lib.tm_build_mask(ctypes.c_void_p(1 << 20), 2, None, 0, 0, 256, 256, 64, 64, 1, 0, 1.5,
+                             ctypes.c_uint64(0), 0, 0, 8, None) == ops.TM_ERR_INVALID_ARG

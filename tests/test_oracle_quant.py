@@ -74,7 +74,7 @@ def test_random_tiles_vs_scalar_bruteforce(seed):
             rows = range(r0, min(T, r0 + tile))
             vals = [float(x[r, h, c]) for r in rows for c in range(d)]
             s, cs = quant_block(vals)
-            assert scales[h, ti] == np.float32(s)
+            assert scales[ti, h] == np.float32(s)
             got = [int(codes[r, h, c]) for r in rows for c in range(d)]
             assert got == cs
 
@@ -88,10 +88,10 @@ def test_varlen_tiles_restart_per_sequence():
     codes, scales = oracle.quantize_tiles(x, seqs, tile, "k")
     # tiles: seq0 rows 0-3, 4-6; seq2 rows 7-10, 11-14, 15-18, 19
     bounds = [(0, 4), (4, 7), (7, 11), (11, 15), (15, 19), (19, 20)]
-    assert scales.shape == (1, len(bounds))
+    assert scales.shape == (len(bounds), 1)
     for t, (a, b) in enumerate(bounds):
         s, cs = quant_block([float(v) for v in x[a:b, 0, :].reshape(-1)])
-        assert scales[0, t] == np.float32(s)
+        assert scales[t, 0] == np.float32(s)
         assert codes[a:b, 0, :].reshape(-1).tolist() == cs
 
 
