@@ -140,21 +140,22 @@ def quantize_tiles(x16, seqs, tile, side):
     and every head h: amax = max |x| over the tile's rows x d (exact: fp16 ->
     fp32 is exact); s = fl32(amax / 127) by IEEE fp32 division; codes =
     clamp(rne(fl32(x / s)), -127, 127), x and s in fp32; amax == 0 gives s = 0
-    and codes 0.  Returns (codes int8 [T, H, d], scales float32 [H, n_tiles]).
+    and codes 0.  Returns (codes int8 [T, H, d], scales float32 [n_tiles, H]),
+    tiles in the global order of ``tile_table``.
     Rows outside every tile keep code 0.
     """
     x16 = np.asarray(x16, dtype=np.float16)
     T, H, d = x16.shape
     tiles = tile_table(seqs, tile, side)
     codes = np.zeros((T, H, d), dtype=np.int8)
-    scales = np.zeros((H, len(tiles)), dtype=np.float32)
+    scales = np.zeros((len(tiles), H), dtype=np.float32)
     x32 = x16.astype(np.float32)
     for (_b, _i, r0, rows, ig) in tiles:
         for h in range(H):
             blk = x32[r0:r0 + rows, h, :]
             amax = np.float32(np.max(np.abs(blk))) if blk.size else np.float32(0)
             s = np.float32(amax / np.float32(127.0))
-            scales[h, ig] = s
+            scales[ig, h] = s
             if s == 0:
                 continue
             q = np.rint(blk / s)                      # fp32 division, then RNE
@@ -289,8 +290,8 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
 
     q: float16 [Tq, Hq, d]; k, v: float16 [Tk, Hkv, d] (or None with an INT8
     cache).  mask: uint32 [Hq or 1, n_qtiles, W] or None (all FP16).
-    q_quant = (codes, scales[Hq, n_qtiles]) and k_quant = (codes,
-    scales[Hkv, n_ktiles]) are the tile-quantised operands of the INT8 route.
+    q_quant = (codes, scales[n_qtiles, Hq]) and k_quant = (codes,
+    scales[n_ktiles, Hkv]) are the tile-quantised operands of the INT8 route.
     kv_cache = (k_codes, k_scale16[Tk, Hkv], v_codes, v_scale16) replaces k, v:
     the FP16 route and P.V use the fp16 view (dequant_cache), the INT8 route
     uses k_codes with the per-token scale of each key.
@@ -299,7 +300,7 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
     For each sequence, query head h (KV head hk = h // (Hq/Hkv)) and visible
     pair (i, j) in query tile I (global I_glob), key tile J, group G = J // g:
       FP16 route: S_ij = sigma * sum_t q_it k_jt   (fp16 values, fp64 sums)
-      INT8 route: S_ij = sigma * s_q[h, I_glob] * s_k * sum_t cq_it ck_jt
+      INT8 route: S_ij = sigma * s_q[I_glob, h] * s_k * sum_t cq_it ck_jt
     with s_k = k tile scale (or the cache scale of key j); the integer sum is
     exact in fp64.  O_i = sum_j softmax_j(S_i.) V_j over visible j; a row with
     no visible key gives 0.
@@ -332,9 +333,8 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
     out = np.full((Tq, Hq, d), np.nan if rows is not None else 0.0, dtype=np.float64)
     kf = k16.astype(np.float64)
     vf = v16.astype(np.float64)
-    qf = q.astype(np.float64)
     if mask is not None:
-        q_codes = np.asarray(q_quant[0]).astype(np.float64)
+        q_codes = np.asarray(q_quant[0])
         q_scales = np.asarray(q_quant[1], dtype=np.float32)
         if kv_cache is not None:
             k_codes = np.asarray(kv_cache[0]).astype(np.float64)
@@ -357,17 +357,17 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
             hk = h // grp
             Kb = kf[ks:ks + lk, hk, :]
             Vb = vf[ks:ks + lk, hk, :]
-            Qr = qf[r0 + sel, h, :]
+            Qr = q[r0 + sel, h, :].astype(np.float64)
             S = sigma * (Qr @ Kb.T)
             if mask is not None:
                 route8 = _group_bits(mask, h, ig, n_groups(n_tiles(lk, tile_n), g))[(jj // tile_n) // g]
                 if route8.any():
-                    acc8 = q_codes[r0 + sel, h, :] @ k_codes[ks:ks + lk, hk, :].T
+                    acc8 = q_codes[r0 + sel, h, :].astype(np.float64) @ k_codes[ks:ks + lk, hk, :].T
                     if kv_cache is not None:
                         col_scale = k_tok_scale[ks:ks + lk, hk]
                     else:
-                        col_scale = k_tile_scale[hk, kt_off[b] + jj // tile_n].astype(np.float64)
-                    S8 = sigma * float(q_scales[h, ig]) * acc8 * col_scale[None, :]
+                        col_scale = k_tile_scale[kt_off[b] + jj // tile_n, hk].astype(np.float64)
+                    S8 = sigma * float(q_scales[ig, h]) * acc8 * col_scale[None, :]
                     S = np.where(route8[None, :], S8, S)
             S = np.where(vis, S, -np.inf)
             has = vis.any(axis=1)
