@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of tile-routed FP16/INT8 fused prefill attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload sweep|long|varlen|mlx|tiny] [--p P]
+
+One step = one pass of the whole hot path over one seeded synthetic batch:
+per-tile INT8 quantisation of Q and K, the seeded routing bitmask, and the
+fused attention kernel (for an all-FP16 workload only the attention kernel).
+Default workload: the TileMix routing sweep shape (L = 16384, Hq = 32,
+Hkv = 8, d = 128, causal, 128x128 tiles, g = 4, outlier channels x20,
+diagonal and sink groups FP16) at INT8 group probability 0.75.
+
+Prints ONE JSON line (rank 0).  `value` is the whole-job algorithmic
+TFLOP/s: 4 * d FLOP per visible query-key pair (QK^T and P.V, causal-aware),
+the same convention as the tflops column of the MLX fused-SDPA tables,
+summed over all ranks and divided by the max-over-ranks device time.
+With N > 1 every rank processes its own independently seeded batch of the
+same shape (weak scaling, no collective on the data path).
+
+`--impl reference` times the CPU oracle (fp64 NumPy) on the host cores
+instead, one sampled (query tile, head) pair of the same workload per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixed_precision_attention_tm_b200 import inputs  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL = {"f16_tflops": 2250.0, "i8_tops": 4500.0}
+
+
+# ---------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            ident = str(device_index)
+        self.cmd = ["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "100"]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 7:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        reasons = set()
+        for s in self.samples:
+            for name, val in zip(self.NAMES, s[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+def make_workload(name, p, seed):
+    if name == "sweep":
+        return inputs.routing_sweep(p, seed=seed)
+    if name == "long":
+        return inputs.long_context(p=p if p is not None else 0.5, seed=seed)
+    if name == "varlen":
+        return inputs.varlen_int8_cache(p=p if p is not None else 0.75, seed=seed)
+    if name == "mlx":
+        return inputs.mlx_shape(4096, 4096, 128, 32, 8, True, seed=seed)
+    if name == "tiny":
+        return inputs.tiny(seed=seed, p=p)
+    raise ValueError(name)
+
+
+def describe(w):
+    cfg = {"workload": w.name, "Lq": w.Lq, "Lk": w.Lk, "Hq": w.hq, "Hkv": w.hkv, "d": w.d, "causal": w.causal,
+           "tile_m": w.tile_m, "tile_n": w.tile_n, "g": w.g, "int8_group_probability": w.p,
+           "force_diag": w.force_diag, "force_sink": w.force_sink,
+           "l2": "inputs larger than L2 (126 MB), no flush" }
+    if w.lens is not None:
+        cfg["seq_lens"] = [int(x) for x in w.lens]
+        cfg["int8_kv_cache"] = w.kv_cache is not None
+    return cfg
+
+
+def route_stats_of(w, mask_host):
+    from mixed_precision_attention_tm_b200 import ops
+    cu = None if w.cu_seqlens is None else w.cu_seqlens.numpy()
+    return ops.route_stats(mask_host, Hq=w.hq, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g, causal=w.causal,
+                           Lq=w.Lq, Lk=w.Lk, cu_seqlens_host=cu)
+
+
+def roofline_time(d, n_vis, e8, p16, p8):
+    """Mix-weighted tensor roofline (seconds): QK^T of FP16 pairs at p16, of
+    INT8 pairs at p8, and P.V of every pair at p16 (FLOP/s)."""
+    e16 = n_vis - e8
+    return 2 * d * e16 / p16 + 2 * d * e8 / p8 + 2 * d * n_vis / p16
+
+
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    from mixed_precision_attention_tm_b200 import ops
+    from mixed_precision_attention_tm_b200.api import TileMixPrefill
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    w = make_workload(args.workload, args.p, seed=args.seed + 1000 * rank)
+    plan = TileMixPrefill(w.Lq, w.Lk, w.hq, w.hkv, w.d, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n,
+                          g=w.g, p=w.p, seed=w.mask_seed, force_diag=w.force_diag, force_sink=w.force_sink,
+                          cu_seqlens=w.cu_seqlens, int8_cache=w.kv_cache is not None, device=dev)
+    plan.load(w.q, w.k, w.v, w.kv_cache)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        plan.run()
+    torch.cuda.synchronize()
+    if ops.get_device_error() != ops.TM_OK:
+        raise RuntimeError("device error after warm-up")
+
+    # routing statistics of the mask the step builds
+    mask_host = None
+    if plan.routed:
+        mask_host = plan.bitmask.cpu().numpy().view(np.uint32)
+    n_vis, e8 = route_stats_of(w, mask_host)
+    flops = 4.0 * w.d * n_vis
+
+    K = args.steps
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    for i in range(K):
+        if plan.routed:
+            plan.quantize()
+            plan.mask()
+        ev_a[i].record(stream)
+        plan.attend()
+        ev_b[i].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t0.elapsed_time(t1)
+    attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev_a, ev_b)) / K
+    if ops.get_device_error() != ops.TM_OK:
+        raise RuntimeError("device error in timed region")
+    t = torch.tensor([total_ms, attn_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms, attn_ms = float(t[0]), float(t[1])
+    ms_step = total_ms / K
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    # roofline of the attention kernel (dominant launch)
+    p16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * 1e12
+    p8 = 2.0 * p16                              # nominal INT8 : FP16 dense ratio (4.5 : 2.25)
+    t_roof = roofline_time(w.d, n_vis, e8, p16, p8)
+    peak_eff = flops / t_roof / 1e12
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    t_roof_nom = roofline_time(w.d, n_vis, e8, NOMINAL["f16_tflops"] * 1e12, NOMINAL["i8_tops"] * 1e12)
+
+    # end-to-end through the public API from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        qh = w.q.pin_memory()
+        kh = None if w.k is None else w.k.pin_memory()
+        vh = None if w.v is None else w.v.pin_memory()
+        kvh = None if w.kv_cache is None else tuple(x.pin_memory() for x in w.kv_cache)
+        out_h = torch.empty(plan.out.shape, dtype=torch.float16, pin_memory=True)
+        for _ in range(2):
+            plan.run_host(qh, kh, vh, kvh, out_h)
+        torch.cuda.synchronize()
+        ke = max(3, min(K, 20))
+        if world > 1:
+            torch.distributed.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(ke):
+            plan.run_host(qh, kh, vh, kvh, out_h)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([s0.elapsed_time(s1) / ke], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": world * flops / (float(te[0]) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": float(te[0]), "h2d_bytes_per_step": plan.input_bytes(),
+               "d2h_bytes_per_step": plan.output_bytes(), "steps": ke}
+
+    # INT8-fraction sweep (outside the timed region; context for the metric)
+    sweep = None
+    if args.workload == "sweep" and not args.no_sweep:
+        sweep = []
+        for ps in (0.0, 0.25, 0.5, 0.75, 1.0):
+            ws = inputs.Workload(w.name, w.q, w.k, w.v, w.hq, w.hkv, w.d, w.causal, w.tile_m, w.tile_n, w.g, ps,
+                                 mask_seed=w.mask_seed, force_diag=True, force_sink=True)
+            pl = TileMixPrefill(ws.Lq, ws.Lk, ws.hq, ws.hkv, ws.d, causal=True, tile_m=128, tile_n=128, g=ws.g,
+                                p=ps, seed=ws.mask_seed, force_diag=True, force_sink=True, device=dev)
+            pl.q, pl.k, pl.v = plan.q, plan.k, plan.v
+            for _ in range(3):
+                pl.run()
+            torch.cuda.synchronize()
+            mh = pl.bitmask.cpu().numpy().view(np.uint32)
+            nv_s, e8_s = route_stats_of(ws, mh)
+            ns = max(5, min(K, 30))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_ms = 0.0
+            for _ in range(ns):
+                pl.quantize()
+                pl.mask()
+                a.record(stream)
+                pl.attend()
+                b.record(stream)
+                b.synchronize()
+                a_ms += a.elapsed_time(b)
+            a_ms /= ns
+            fl = 4.0 * ws.d * nv_s
+            tr = roofline_time(ws.d, nv_s, e8_s, p16, p8)
+            sweep.append({"p": ps, "realised_int8_fraction": e8_s / nv_s, "attn_ms": a_ms,
+                          "tflops": fl / (a_ms * 1e-3) / 1e12, "mixed_roofline_frac": tr / (a_ms * 1e-3),
+                          "tokens_per_s": ws.Lq / (a_ms * 1e-3)})
+            del pl
+
+    launches = plan.launches_per_step * K
+    line = {
+        "metric": "prefill attention TFLOPS (tile-routed FP16/INT8 QK^T, FP16 P.V)",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16+i8 (fp32 accumulate)",
+        "data": "synthetic (seeded N(0,1) fp16, outlier channels x20)",
+        "config": describe(w),
+        "tokens_per_s": world * w.Lq / (ms_step * 1e-3),
+        "realised_int8_fraction": e8 / n_vis,
+        "visible_pairs": n_vis,
+        "attn_ms": attn_ms,
+        "mixed_roofline_frac_of_measured": t_roof / (attn_ms * 1e-3),
+        "mixed_roofline_frac_of_nominal": t_roof_nom / (attn_ms * 1e-3),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff, "unit": "TFLOP/s",
+                     "frac": achieved / peak_eff, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 burst {p16 / 1e12:.1f} TFLOP/s for FP16 pairs, x2 "
+                                    "(nominal INT8:FP16 ratio) for INT8 QK^T, mix-weighted by visible pairs"},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if sweep is not None:
+        line["sweep"] = sweep
+    return line, w
+
+
+def cpu_sample_spec(w, n_pairs):
+    """Evenly spaced (query tile, head) pairs of the workload."""
+    import oracle
+    cu = None if w.cu_seqlens is None else w.cu_seqlens.tolist()
+    seqs = oracle.seq_table(w.Lq, w.Lk, cu)
+    qt = oracle.tile_table(seqs, w.tile_m, "q")
+    out = []
+    n = len(qt) * w.hq
+    for i in range(n_pairs):
+        idx = (i * n) // n_pairs + (n // (2 * n_pairs))
+        out.append((qt[(idx // w.hq) % len(qt)], idx % w.hq))
+    return seqs, out
+
+
+def oracle_pair(w, seqs, tile, h, prep):
+    """Run the oracle on one (query tile, head): all rows of the tile, the
+    head's slice of Q; returns algorithmic FLOPs of the pair."""
+    import oracle
+    b, I, r0, rows, ig = tile
+    q1 = w.q.numpy()[:, h:h + 1]
+    kw = dict(prep)
+    if kw.get("mask") is not None:
+        kw["mask"] = kw["mask"][h:h + 1]
+        qc, qs = kw["q_quant"]
+        kw["q_quant"] = (qc[:, h:h + 1], qs[:, h:h + 1])
+    hk = h // (w.hq // w.hkv)
+    if w.kv_cache is not None:
+        kc, ks, vc, vs = kw["kv_cache"]
+        kw["kv_cache"] = (kc[:, hk:hk + 1], ks[:, hk:hk + 1], vc[:, hk:hk + 1], vs[:, hk:hk + 1])
+        k1 = v1 = None
+    else:
+        k1, v1 = w.k.numpy()[:, hk:hk + 1], w.v.numpy()[:, hk:hk + 1]
+        if kw.get("k_quant") is not None:
+            kc, ks = kw["k_quant"]
+            kw["k_quant"] = (kc[:, hk:hk + 1], ks[:, hk:hk + 1])
+    oracle.attention(q1, k1, v1, rows=range(r0, r0 + rows), **kw)
+    _qs, lq, _ks, lk = seqs[b]
+    ii = I * w.tile_m + np.arange(rows)
+    lim = np.minimum(lk - 1, ii + lk - lq) if w.causal else np.full(rows, lk - 1)
+    return 4.0 * w.d * float(np.maximum(lim + 1, 0).sum())
+
+
+def oracle_prep(w, seqs):
+    import oracle
+    cu = None if w.cu_seqlens is None else w.cu_seqlens.tolist()
+    prep = dict(cu_seqlens=cu, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g)
+    if w.kv_cache is not None:
+        prep["kv_cache"] = tuple(t.numpy() for t in w.kv_cache)
+    if w.p is not None:
+        prep["mask"] = oracle.build_mask(w.hq, seqs, w.tile_m, w.tile_n, w.g, w.causal, w.p, w.mask_seed,
+                                         w.force_diag, w.force_sink)
+        prep["q_quant"] = oracle.quantize_tiles(w.q.numpy(), seqs, w.tile_m, "q")
+        if w.kv_cache is None:
+            prep["k_quant"] = oracle.quantize_tiles(w.k.numpy(), seqs, w.tile_n, "k")
+    return prep
+
+
+def cpu_baseline(w, target_s):
+    """Time the oracle as it stands on evenly spaced (query tile, head) pairs
+    until about target_s seconds of CPU work have run."""
+    cores = len(os.sched_getaffinity(0))
+    seqs, _ = cpu_sample_spec(w, 1)
+    prep = oracle_prep(w, seqs)            # quantisation and mask: not timed
+    n_try = 64
+    _, pairs = cpu_sample_spec(w, n_try)
+    flops = 0.0
+    t0 = time.perf_counter()
+    done = 0
+    for tile, h in pairs:
+        flops += oracle_pair(w, seqs, tile, h, prep)
+        done += 1
+        if time.perf_counter() - t0 > target_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} evenly spaced (query tile, head) pairs of {w.name} (all rows of each tile, "
+                      f"fp64 NumPy/BLAS), {dt:.1f} s; quantisation and mask built beforehand, untimed"}
+
+
+def run_reference(args):
+    """CPU oracle arm: one (query tile, head) pair of the workload per step."""
+    w = make_workload(args.workload, args.p, seed=args.seed)
+    cores = len(os.sched_getaffinity(0))
+    seqs, pairs = cpu_sample_spec(w, max(1, args.steps + args.warmup))
+    prep = oracle_prep(w, seqs)
+    for tile, h in pairs[:args.warmup]:
+        oracle_pair(w, seqs, tile, h, prep)
+    flops = 0.0
+    t0 = time.perf_counter()
+    for tile, h in pairs[args.warmup:args.warmup + args.steps]:
+        flops += oracle_pair(w, seqs, tile, h, prep)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    line = {
+        "impl": "reference",
+        "metric": "prefill attention TFLOPS (tile-routed FP16/INT8 QK^T, FP16 P.V)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / max(1, args.steps), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) fp16, outlier channels x20)",
+        "config": describe(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"one (query tile, head) pair of {w.name} per step, fp64 NumPy/BLAS; "
+                                   "quantisation and mask built beforehand, untimed"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="sweep", choices=["sweep", "long", "varlen", "mlx", "tiny"])
+    ap.add_argument("--p", type=float, default=0.75)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line, w = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,109 @@
+"""User-facing prefill plan: device buffers plus the three library calls.
+
+``TileMixPrefill`` owns the device tensors of one problem shape (Q, K, V or
+the INT8 cache, INT8 codes and tile scales, the routing bitmask, the output)
+and runs one prefill step:
+
+    tm_quantize_qk  ->  tm_build_mask  ->  tm_attn_fwd
+
+on the current CUDA stream.  ``run_host`` is the same step fed from host
+memory: pinned host -> device copies of the inputs, the step, and a device ->
+host copy of the output.  Everything that computes is in libtm; this module
+only allocates and passes pointers.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import ops
+
+
+class TileMixPrefill:
+    def __init__(self, Lq, Lk, hq, hkv, d, *, causal=True, tile_m=128, tile_n=128, g=1, p=None,
+                 seed=0, force_diag=False, force_sink=False, cu_seqlens=None, int8_cache=False,
+                 device="cuda"):
+        self.shape = (Lq, Lk, hq, hkv, d)
+        self.causal, self.tile_m, self.tile_n, self.g = causal, tile_m, tile_n, g
+        self.p, self.seed, self.force_diag, self.force_sink = p, seed, force_diag, force_sink
+        self.int8_cache = int8_cache
+        self.device = torch.device(device)
+        self.cu = None if cu_seqlens is None else cu_seqlens.to(self.device, torch.int32)
+        cu_h = None if cu_seqlens is None else cu_seqlens.to("cpu", torch.int32)
+        self.max_seqlen = None if cu_h is None else int((cu_h[1:] - cu_h[:-1]).max())
+        dev = self.device
+        self.q = torch.empty((Lq, hq, d), dtype=torch.float16, device=dev)
+        if int8_cache:
+            self.k = self.v = None
+            self.kc = torch.empty((Lk, hkv, d), dtype=torch.int8, device=dev)
+            self.vc = torch.empty((Lk, hkv, d), dtype=torch.int8, device=dev)
+            self.ks = torch.empty((Lk, hkv), dtype=torch.float16, device=dev)
+            self.vs = torch.empty((Lk, hkv), dtype=torch.float16, device=dev)
+        else:
+            self.k = torch.empty((Lk, hkv, d), dtype=torch.float16, device=dev)
+            self.v = torch.empty((Lk, hkv, d), dtype=torch.float16, device=dev)
+        self.out = torch.empty((Lq, hq, d), dtype=torch.float16, device=dev)
+        self.routed = p is not None
+        self.launches_per_step = 1 + (3 if self.routed and not int8_cache else 2 if self.routed else 0)
+
+    # -- inputs -----------------------------------------------------------
+    def load(self, q, k=None, v=None, kv_cache=None):
+        """Copy device or host tensors into the plan's resident buffers."""
+        self.q.copy_(q, non_blocking=True)
+        if self.int8_cache:
+            kc, ks, vc, vs = kv_cache
+            self.kc.copy_(kc, non_blocking=True)
+            self.ks.copy_(ks, non_blocking=True)
+            self.vc.copy_(vc, non_blocking=True)
+            self.vs.copy_(vs, non_blocking=True)
+        else:
+            self.k.copy_(k, non_blocking=True)
+            self.v.copy_(v, non_blocking=True)
+
+    def input_bytes(self):
+        t = [self.q] + ([self.kc, self.ks, self.vc, self.vs] if self.int8_cache else [self.k, self.v])
+        return sum(x.numel() * x.element_size() for x in t)
+
+    def output_bytes(self):
+        return self.out.numel() * self.out.element_size()
+
+    # -- the step ---------------------------------------------------------
+    def quantize(self):
+        qc, qs, kc, ks = ops.quantize_qk(self.q, None if self.int8_cache else self.k,
+                                         tile_m=self.tile_m, tile_n=self.tile_n, cu_seqlens=self.cu,
+                                         max_seqlen=self.max_seqlen)
+        self.q_quant = (qc, qs)
+        self.k_quant = None if self.int8_cache else (kc, ks)
+
+    def mask(self):
+        Lq, Lk = self.shape[0], self.shape[1]
+        self.bitmask = ops.build_mask(self.shape[2], tile_m=self.tile_m, tile_n=self.tile_n, g=self.g,
+                                      causal=self.causal, p=self.p, seed=self.seed,
+                                      force_diag=self.force_diag, force_sink=self.force_sink,
+                                      Lq=Lq, Lk=Lk, cu_seqlens=self.cu, max_seqlen=self.max_seqlen,
+                                      device=self.device)
+
+    def attend(self):
+        kv = (self.kc, self.ks, self.vc, self.vs) if self.int8_cache else None
+        return ops.attn_fwd(self.q, self.k, self.v, out=self.out, tile_m=self.tile_m, tile_n=self.tile_n,
+                            g=self.g, causal=self.causal,
+                            bitmask=self.bitmask if self.routed else None,
+                            q_quant=self.q_quant if self.routed else None,
+                            k_quant=self.k_quant if self.routed else None, kv_cache=kv,
+                            cu_seqlens=self.cu, max_seqlen=self.max_seqlen)
+
+    def run(self):
+        """One prefill step on the resident inputs; returns the device output."""
+        if self.routed:
+            self.quantize()
+            self.mask()
+        return self.attend()
+
+    def run_host(self, q, k=None, v=None, kv_cache=None, out_host=None):
+        """Step fed from (pinned) host tensors; the output lands in out_host."""
+        self.load(q, k, v, kv_cache)
+        self.run()
+        if out_host is None:
+            out_host = torch.empty(self.out.shape, dtype=self.out.dtype, pin_memory=True)
+        out_host.copy_(self.out, non_blocking=True)
+        return out_host

@@ -285,86 +285,75 @@ __global__ void __launch_bounds__(192, 1)
     for (int j = 0; j < nJ; ++j) {
       const bool i8 = route_int8(mrow, p.g, j);
       float c = p.scale_log2;
-      if (i8) c = c8_row * __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk);
+      // INT8 tile: S = acc * s_q * s_k * sigma; kept > 0 so that masked -inf
+      // scores stay -inf (an all-zero tile has acc = 0 and gives S = 0).
+      if (i8) c = fmaxf(c8_row * __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk), 1e-30f);
       if (!mbar_wait(bar(B_SFULL + (j & 1)), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
       tc_fence_after();
       __syncwarp();
       float x[BN];
       {
-        uint32_t u[32];
+        uint32_t u[BN];
 #pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          tmem_ld32(lane_addr + static_cast<uint32_t>(j & 1) * BN + cc * 32, u);
-          tmem_wait_ld();
+        for (int cc = 0; cc < BN / 32; ++cc)
+          tmem_ld32p(lane_addr + static_cast<uint32_t>(j & 1) * BN + cc * 32, u + cc * 32);
+        tmem_wait_ld();
+        if (i8) {
+          // exact int32 -> fp32 for |acc| < 2^22: add the bits of 1.5 * 2^23
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (i8) x[cc * 32 + e] = __int_as_float(static_cast<int>(u[e]) + 0x4B400000) - 12582912.0f;
-            else x[cc * 32 + e] = __uint_as_float(u[e]);
-          }
+          for (int e = 0; e < BN; ++e) x[e] = __int_as_float(static_cast<int>(u[e]) + 0x4B400000) - 12582912.0f;
+        } else {
+#pragma unroll
+          for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(u[e]);
         }
       }
       const int64_t nv64 = lim - static_cast<int64_t>(j) * BN + 1;
       const int nv = nv64 <= 0 ? 0 : (nv64 >= BN ? BN : static_cast<int>(nv64));
-      const bool full = __all_sync(0xffffffffu, nv == BN);   // warp-uniform fast path
-      float mraw = -INFINITY;
-      if (full) {
+      if (!__all_sync(0xffffffffu, nv == BN)) {
 #pragma unroll
-        for (int e = 0; e < BN; ++e) mraw = fmaxf(mraw, x[e]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < BN; ++e) mraw = (e < nv) ? fmaxf(mraw, x[e]) : mraw;
+        for (int e = 0; e < BN; ++e) x[e] = (e < nv) ? x[e] : -INFINITY;
       }
       float alpha = 1.f;
       if (nv > 0) {
-        const float mt = mraw * c;
-        if (mt > m_used + 8.0f) {
+        const float mt = row_max<BN>(x) * c;
+        if (mt > m_used + 8.0f) {           // lazy rescale: only when the max grows by > 2^8
           alpha = ex2_approx(m_used - mt);
           m_used = mt;
         }
       }
-      l *= alpha;
       const float msub = (m_used == -INFINITY) ? 0.f : m_used;
       uint32_t pk[BN / 2];
-      float rs = 0.f;
+      float acc[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] = 0.f;
 #pragma unroll
       for (int e = 0; e < BN; e += 2) {
-        float p0 = ex2_approx(fmaf(x[e], c, -msub));
-        float p1 = ex2_approx(fmaf(x[e + 1], c, -msub));
-        if (!full) {
-          p0 = (e < nv) ? p0 : 0.f;
-          p1 = (e + 1 < nv) ? p1 : 0.f;
-        }
-        rs += p0 + p1;
+        const float p0 = ex2_approx(fmaf(x[e], c, -msub));
+        const float p1 = ex2_approx(fmaf(x[e + 1], c, -msub));
+        acc[(e >> 1) & 7] += p0 + p1;
         pk[e >> 1] = pack_half2(p0, p1);
       }
-      l += rs;
+      l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       if (j > 0) {
         // O holds sum_{t<j} P_t V_t once PV_{j-1} has completed.
         if (!mbar_wait(bar(B_ODONE), (j - 1) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
         __syncwarp();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          uint32_t o[D];
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + C::O_COL + cc * 32, o);
-            tmem_wait_ld();
+          for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(lane_addr + C::O_COL + cc * 32, o);
-          }
+          for (int e = 0; e < D; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) tmem_st32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
         }
       }
       __syncwarp();
-      {
-        uint32_t w32[32];
 #pragma unroll
-        for (int cc = 0; cc < BN / 64; ++cc) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) w32[e] = pk[cc * 32 + e];
-          tmem_st32(lane_addr + static_cast<uint32_t>(j & 1) * BN + cc * 32, w32);
-        }
-      }
+      for (int cc = 0; cc < BN / 64; ++cc)
+        tmem_st32p(lane_addr + static_cast<uint32_t>(j & 1) * BN + cc * 32, pk + cc * 32);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PFULL + (j & 1)));
@@ -377,26 +366,25 @@ __global__ void __launch_bounds__(192, 1)
     }
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
     __syncwarp();
-    __half* orow = p.out + (sq.start + i_row) * p.out_st + static_cast<int64_t>(h) * p.out_sh;
+    uint32_t o[D];
+    if (__all_sync(0xffffffffu, have_o)) {
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t o[32];
-      if (have_o) {
-        tmem_ld32(lane_addr + C::O_COL + cc * 32, o);
-        tmem_wait_ld();
-      } else {
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
+      tmem_wait_ld();
+    } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = 0u;
-      }
-      if (row_ok) {
-        uint4 pkt[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(pkt);
+      for (int e = 0; e < D; ++e) o[e] = 0u;
+    }
+    if (row_ok) {
+      __half* orow = p.out + (sq.start + i_row) * p.out_st + static_cast<int64_t>(h) * p.out_sh;
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pw[e] = pack_half2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = pkt[e];
+      for (int cc = 0; cc < D / 8; ++cc) {
+        uint4 pkt;
+        pkt.x = pack_half2(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv);
+        pkt.y = pack_half2(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv);
+        pkt.z = pack_half2(__uint_as_float(o[8 * cc + 4]) * inv, __uint_as_float(o[8 * cc + 5]) * inv);
+        pkt.w = pack_half2(__uint_as_float(o[8 * cc + 6]) * inv, __uint_as_float(o[8 * cc + 7]) * inv);
+        reinterpret_cast<uint4*>(orow)[cc] = pkt;
       }
     }
   }
