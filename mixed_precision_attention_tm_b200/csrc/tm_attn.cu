@@ -28,6 +28,7 @@
 
 #include <mutex>
 
+#include "tm_attn_internal.h"
 #include "tm_device.cuh"
 #include "tm_host.h"
 
@@ -521,6 +522,9 @@ extern "C" tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const t
       return TM_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);
+  if (tile_m == 128 && tile_n == 128)
+    return launch_attn_pair(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride, g,
+                            causal, s);
   if (D == 128) {
     if (tile_n == 128)
       return launch<128, 128>(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride,

@@ -1,0 +1,691 @@
+// tm_attn2.cu -- fused tile-routed attention, two 128-row query tiles per CTA.
+//
+// TileMix (Lattice paper page), abstract: score tiles routed per group of g
+// key tiles to an FP16 or an INT8 QK^T, both feeding one online-softmax state.
+// This is the production layout for 128 x 128 score tiles.  On B200 the
+// softmax (one exp2 per score, plus max / sum / conversion) costs about as
+// much as the FP16 MMAs of a tile, so the kernel is built to keep the tensor
+// pipe and the softmax warps busy at the same time:
+//
+//   * one CTA owns query tiles A = 2P and B = 2P+1 of one head; its two
+//     softmax warpgroups (warps 0-3 on tile A, warps 4-7 on tile B) alternate
+//     on the tensor core: while one warpgroup computes exp2 on its score
+//     tile, the tensor pipe runs the other tile's P.V and next QK^T;
+//   * TMEM holds S_A, S_B (128 columns each; P overwrites S in place as fp16)
+//     and the fp32 accumulators O_A, O_B;
+//   * K / V arrive through a ring of tile-sized shared-memory slots: per key
+//     tile the producer loads the fp16 K tile if either query tile routes it
+//     FP16, the int8 K-code tile if either routes it INT8 (both when they
+//     differ), and the fp16 V tile; slots are released by tcgen05.commit once
+//     the MMAs reading them have completed;
+//   * the softmax arithmetic runs on packed fp32 pairs (f32x2 FMA / ADD),
+//     and 3 of every 8 exp2 pairs run as a degree-3 minimax polynomial on the
+//     FMA pipe (Cody-Waite split 2^y = 2^n * 2^f, f in [-1/2, 1/2];
+//     coefficients fitted by the Remez exchange, max relative error 7.5e-5,
+//     below the fp16 rounding of P), the rest on MUFU.ex2, so that neither
+//     the MUFU pipe nor instruction issue alone bounds the softmax;
+//   * K / V loads carry an evict-last L2 policy and Q an evict-first one,
+//     and the output is written with streaming stores.
+// Every mbarrier wait is bounded (tm_device.cuh).
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "tm_attn_internal.h"
+#include "tm_device.cuh"
+#include "tm_host.h"
+
+#ifdef TM_TRACE
+extern "C" int tm_debug_trace_read(unsigned long long* host, unsigned int block) {
+  if (host == nullptr) {
+    static unsigned long long zero[TM_TRACE_ROLES][TM_TRACE_EVENTS];
+    if (cudaMemcpyToSymbol(g_tm_trace, zero, sizeof(zero)) != cudaSuccess) return -1;
+    return cudaMemcpyToSymbol(g_tm_trace_block, &block, sizeof(block)) == cudaSuccess ? 0 : -1;
+  }
+  return cudaMemcpyFromSymbol(host, g_tm_trace, sizeof(g_tm_trace)) == cudaSuccess ? 0 : -1;
+}
+#endif
+
+namespace tmk {
+namespace {
+
+// trace event ids (roles: 0 = softmax A, 1 = softmax B, 2 = producer, 3 = issuer)
+enum : unsigned {
+  EV_S_READY = 1, EV_EXP_DONE = 2, EV_O_READY = 3, EV_RESCALED = 4, EV_P_RELEASED = 5, EV_EPI_DONE = 6,
+  EV_ACQUIRED = 10, EV_K_READY = 20, EV_PV_A = 21, EV_S_A = 22, EV_PV_B = 23, EV_S_B = 24, EV_V_READY = 25,
+  EV_START = 30, EV_KWAIT_BEGIN = 31, EV_KWAIT_END = 32, EV_VWAIT_BEGIN = 33, EV_SLOADED = 7, EV_MAXED = 8
+};
+
+template <int D>
+struct Cfg2 {
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int SLOT = BN * D * 2;                // one fp16 K or V tile
+  static constexpr int NSLOT = 131072 / SLOT;            // 4 (d=128) or 8 (d=64)
+  static constexpr int Q16_BYTES = BM * D * 2;           // per query tile
+  static constexpr int Q8_BYTES = BM * D;
+  static constexpr int HALF = BM * 128;                  // one 64-column fp16 slab (128 rows)
+  static constexpr int OFF_Q16 = 0;
+  static constexpr int OFF_Q8 = 2 * Q16_BYTES;
+  static constexpr int OFF_SLOT = OFF_Q8 + 2 * Q8_BYTES;
+  static constexpr int OFF_BAR = OFF_SLOT + NSLOT * SLOT;
+  static constexpr int BAR_BYTES = 1024;                 // barriers + routing words
+  static constexpr int MAXW = 64;                        // routing words per query tile kept in smem
+  static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_S16 = idesc_f16(BM, BN, false);
+  static constexpr uint32_t IDESC_S8 = idesc_i8(BM, BN);
+  static constexpr uint32_t IDESC_PV = idesc_f16(BM, D, true);
+  static constexpr uint32_t SW8 = (D == 128) ? kSwizzle128 : kSwizzle64;
+  static constexpr uint32_t SBO8 = (D == 128) ? 1024u : 512u;
+  // 8 softmax warps + (producer, MMA issuer, 2 idle) warps.  Launch: 168
+  // registers per thread (3 warps per SM sub-partition); the softmax
+  // warpgroups then take 216 and the control warpgroup keeps 72:
+  // 2 * 128 * 216 + 128 * 72 = 384 * 168.
+  static constexpr int THREADS = 384;
+  static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, CONTROL_REGS = 72;
+  static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS == THREADS * LAUNCH_REGS,
+                "register split must equal the launch allocation");
+  __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
+  __host__ __device__ static constexpr uint32_t o_col(int t) { return 256u + D * t; }
+};
+
+enum {
+  C_QFULL = 0,
+  C_SFULL = 1,   // +2 (tile A, B)
+  C_PFULL = 3,   // +2
+  C_ODONE = 5,   // +2
+  C_DRAIN = 7,
+  C_FULL = 8,    // +NSLOT (<= 8)
+  C_EMPTY = 16,  // +NSLOT
+  C_COUNT = 24
+};
+
+struct Params2 {
+  __half* out;
+  int64_t out_st, out_sh;
+  const float* q_scales;
+  const float* k_scales;
+  const uint32_t* bitmask;
+  int64_t mask_hs;
+  int W;
+  const int32_t* cu;
+  int64_t Lq, Lk;
+  int Hq, Hkv, g, causal, n_pair_max, n_qt_max, batch;
+  float scale_log2;
+  DevErr err;
+};
+
+// 2^y for y <= 8 on the FMA pipe, two lanes at a time (f32x2).  y = n + f
+// with n = rne(y) obtained by adding 1.5 * 2^23 (whose float ulp is 1), f in
+// [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (relative error <= 7.5e-5
+// on that interval, coefficients from a Remez fit); 2^n enters the exponent
+// field with one integer shift-add per lane.  y is clamped at -125 so masked
+// (-inf) scores give a normal ~2^-125, which rounds to 0 in fp16.
+__device__ __forceinline__ void exp2_poly2(uint64_t y2, float& p0, float& p1) {
+  float y0, y1;
+  f2unpack(y2, y0, y1);
+  y2 = f2pack(fmaxf(y0, -125.0f), fmaxf(y1, -125.0f));
+  const uint64_t magic = f2pack(12582912.0f, 12582912.0f);
+  const uint64_t nmagic = f2pack(-12582912.0f, -12582912.0f);
+  const uint64_t t2 = f2add(y2, magic);
+  const uint64_t n2 = f2add(t2, nmagic);
+  const uint64_t f2 = f2fma(n2, f2pack(-1.0f, -1.0f), y2);
+  uint64_t q = f2fma(f2pack(0.0551716685f, 0.0551716685f), f2, f2pack(0.2426111251f, 0.2426111251f));
+  q = f2fma(q, f2, f2pack(0.6932609677f, 0.6932609677f));
+  q = f2fma(q, f2, f2pack(0.9999280572f, 0.9999280572f));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t2, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// Routing bit of key tile j (group j / g); row is a shared- or global-memory
+// copy of the query tile's bitmask words, or null (all FP16).
+__device__ __forceinline__ bool route8(const uint32_t* row, int g, int j) {
+  if (row == nullptr) return false;
+  const int G = j / g;
+  return (row[G >> 5] >> (G & 31)) & 1u;
+}
+
+struct TileInfo {
+  int64_t row0;      // first global row of the tile
+  int rows;          // valid rows (0: tile absent)
+  int nJ;            // key tiles with a visible pair
+  int64_t ig;        // global query-tile index
+  const uint32_t* mrow;
+};
+
+template <int D, int EMU>
+__global__ void __launch_bounds__(384, 1)
+    attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmQ8,
+                     const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmK8,
+                     const __grid_constant__ CUtensorMap tmV16, const Params2 p) {
+  using C = Cfg2<D>;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_s + pad;
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * C_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * C_COUNT + 4);
+  uint32_t* route_words = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 256);   // [2][MAXW]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit (pair P of sequence b, head h), heaviest pairs first
+  const int h = blockIdx.x % p.Hq;
+  const int t1 = blockIdx.x / p.Hq;
+  const int b = t1 % p.batch;
+  const int P = p.n_pair_max - 1 - t1 / p.batch;
+  const SeqInfo sq = seq_info(p.cu, b, p.Lq, 128);
+  const int64_t Lq = sq.len;
+  const int64_t Lk = p.cu ? sq.len : p.Lk;
+  const int64_t kstart = p.cu ? sq.start : 0;
+  if (p.cu != nullptr && P == 0 && threadIdx.x == 0 &&
+      Lq > static_cast<int64_t>(p.n_qt_max) * 128)
+    dev_error(p.err, TM_DEVERR_SEQLEN);
+  if (static_cast<int64_t>(2 * P) * 128 >= Lq) return;
+
+  TileInfo ti[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int64_t I = 2 * P + t;
+    const int64_t r0 = I * 128;
+    ti[t].row0 = sq.start + r0;
+    ti[t].rows = r0 < Lq ? static_cast<int>(min(static_cast<int64_t>(128), Lq - r0)) : 0;
+    ti[t].ig = sq.tile_base + I;
+    ti[t].nJ = 0;
+    if (ti[t].rows > 0 && Lk > 0) {
+      int64_t jmax = Lk - 1;
+      if (p.causal) jmax = min(jmax, r0 + ti[t].rows - 1 + Lk - Lq);
+      ti[t].nJ = jmax < 0 ? 0 : static_cast<int>(jmax / BN + 1);
+    }
+    ti[t].mrow = (p.bitmask && ti[t].rows > 0)
+                     ? p.bitmask + static_cast<int64_t>(h) * p.mask_hs + ti[t].ig * p.W : nullptr;
+  }
+  const int nJ = max(ti[0].nJ, ti[1].nJ);
+  const int hk = h / (p.Hq / p.Hkv);
+  const int nJA = ti[0].nJ, nJB = ti[1].nJ;
+  // Routing words of both query tiles, staged in shared memory when they fit.
+  const bool words_in_smem = p.W <= C::MAXW;
+  const uint32_t* rrow[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+    rrow[t] = ti[t].mrow == nullptr ? nullptr : (words_in_smem ? route_words + t * C::MAXW : ti[t].mrow);
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C_QFULL), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C_SFULL + t), 1);
+      mbar_init(bar(C_PFULL + t), 128);
+      mbar_init(bar(C_ODONE + t), 1);
+    }
+    mbar_init(bar(C_DRAIN), 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(bar(C_FULL + s), 1);
+      mbar_init(bar(C_EMPTY + s), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 8) {
+    if (lane == 0) {
+      prefetch_tmap(&tmQ16);
+      prefetch_tmap(&tmK16);
+      prefetch_tmap(&tmV16);
+    }
+    if (words_in_smem)
+      for (int t = 0; t < 2; ++t)
+        if (ti[t].mrow != nullptr)
+          for (int w = lane; w < p.W; w += 32) route_words[t * C::MAXW + w] = __ldg(ti[t].mrow + w);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // item needs of key tile j (identical in producer and MMA issuer)
+  auto needs = [&](int j, bool& r0, bool& r1, bool& n16, bool& n8) {
+    const bool a = j < nJA, c = j < nJB;
+    r0 = a && route8(rrow[0], p.g, j);
+    r1 = c && route8(rrow[1], p.g, j);
+    n16 = (a && !r0) || (c && !r1);
+    n8 = r0 || r1;
+  };
+
+  if (warp >= 8) {
+   regs_dec<C::CONTROL_REGS>();
+   if (warp == 8) {
+    // ======================= TMA producer =======================
+    if (lane == 0 && nJ > 0) {
+      TM_TRACE_DECL
+      TM_TRACE_EV(2, EV_START);
+      bool any8[2] = {false, false};
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (ti[t].mrow != nullptr)
+          for (int w = 0; w < p.W; ++w) any8[t] |= (__ldg(ti[t].mrow + w) != 0u);
+      uint32_t qbytes = 0;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) qbytes += (ti[t].rows > 0 ? C::Q16_BYTES : 0) + (any8[t] ? C::Q8_BYTES : 0);
+      // Q is read once (evict first); K / V are re-read by every query tile
+      // of the KV head (evict last).
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
+      mbar_arrive_expect_tx(bar(C_QFULL), qbytes);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (ti[t].rows == 0) continue;
+        const int32_t qr = static_cast<int32_t>(ti[t].row0);
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d_hint(sbase + C::OFF_Q16 + t * C::Q16_BYTES + hh * C::HALF, &tmQ16, bar(C_QFULL), hh * 64, h,
+                           qr, pol_q);
+        if (any8[t]) tma_load_3d_hint(sbase + C::OFF_Q8 + t * C::Q8_BYTES, &tmQ8, bar(C_QFULL), 0, h, qr, pol_q);
+      }
+
+      uint32_t n = 0;   // ring position
+      auto acquire = [&](uint32_t& slot) -> bool {
+        slot = n % C::NSLOT;
+        const uint32_t lap = n / C::NSLOT;
+        if (lap > 0 && !mbar_wait(bar(C_EMPTY + slot), (lap - 1) & 1, p.err, abort_flag)) return false;
+        ++n;
+        TM_TRACE_EV(2, EV_ACQUIRED);
+        return true;
+      };
+      bool ok = true;
+      for (int j = 0; ok && j < nJ; ++j) {
+        bool r0, r1, n16, n8;
+        needs(j, r0, r1, n16, n8);
+        const int32_t krow = static_cast<int32_t>(kstart + static_cast<int64_t>(j) * BN);
+        uint32_t s;
+        if (n16) {
+          if (!(ok = acquire(s))) break;
+          mbar_arrive_expect_tx(bar(C_FULL + s), C::SLOT);
+#pragma unroll
+          for (int hh = 0; hh < D / 64; ++hh)
+            tma_load_3d_hint(sbase + C::OFF_SLOT + s * C::SLOT + hh * C::HALF, &tmK16, bar(C_FULL + s), hh * 64, hk,
+                             krow, pol_kv);
+        }
+        if (n8) {
+          if (!(ok = acquire(s))) break;
+          mbar_arrive_expect_tx(bar(C_FULL + s), BN * D);
+          tma_load_3d_hint(sbase + C::OFF_SLOT + s * C::SLOT, &tmK8, bar(C_FULL + s), 0, hk, krow, pol_kv);
+        }
+        if (!(ok = acquire(s))) break;
+        mbar_arrive_expect_tx(bar(C_FULL + s), C::SLOT);
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d_hint(sbase + C::OFF_SLOT + s * C::SLOT + hh * C::HALF, &tmV16, bar(C_FULL + s), hh * 64, hk,
+                           krow, pol_kv);
+      }
+      // Drain: every issued copy has landed before the CTA may exit.
+      volatile int never = 0;
+      mbar_wait(bar(C_QFULL), 0, p.err, &never);
+      for (uint32_t i = (n > C::NSLOT ? n - C::NSLOT : 0); i < n; ++i)
+        mbar_wait(bar(C_FULL + i % C::NSLOT), (i / C::NSLOT) & 1, p.err, &never);
+    }
+  } else if (warp == 9) {
+    // ======================= tcgen05 issuer =======================
+    if (lane == 0 && nJ > 0) {
+      TM_TRACE_DECL
+      TM_TRACE_EV(3, EV_START);
+      bool ok = mbar_wait(bar(C_QFULL), 0, p.err, abort_flag);
+      uint32_t n = 0;
+      auto take = [&](uint32_t& slot, uint32_t& par) {
+        slot = n % C::NSLOT;
+        par = (n / C::NSLOT) & 1;
+        ++n;
+      };
+      auto issue_s = [&](int t, bool i8, uint32_t kslot) {
+        const uint32_t d_tmem = tmem + C::s_col(t);
+        const uint32_t kb = sbase + C::OFF_SLOT + kslot * C::SLOT;
+        if (i8) {
+          const uint32_t qa = sbase + C::OFF_Q8 + t * C::Q8_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_i8_ss(d_tmem, smem_desc(qa + kk * 32, 16, C::SBO8, C::SW8),
+                      smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8), C::IDESC_S8, kk > 0 ? 1u : 0u);
+        } else {
+          const uint32_t qa = sbase + C::OFF_Q16 + t * C::Q16_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::HALF + (kk & 3) * 32;
+            mma_f16_ss(d_tmem, smem_desc(qa + off, 16, 1024, kSwizzle128),
+                       smem_desc(kb + off, 16, 1024, kSwizzle128), C::IDESC_S16, kk > 0 ? 1u : 0u);
+          }
+        }
+        tc_commit(bar(C_SFULL + t));
+      };
+      auto issue_pv = [&](int t, int jj, uint32_t vslot) -> bool {
+        if (!mbar_wait(bar(C_PFULL + t), jj & 1, p.err, abort_flag)) return false;
+        tc_fence_after();   // orders the softmax warps' TMEM stores of P before the MMA reads it
+        const uint32_t vb = sbase + C::OFF_SLOT + vslot * C::SLOT;
+        const uint32_t a_tmem = tmem + C::s_col(t);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_f16_ts(tmem + C::o_col(t), a_tmem + kk * 8, smem_desc(vb + kk * 2048, C::HALF, 1024, kSwizzle128),
+                     C::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(C_ODONE + t));
+        return true;
+      };
+      uint32_t v_prev = 0;
+      for (int j = 0; ok && j < nJ; ++j) {
+        bool r0, r1, n16, n8;
+        needs(j, r0, r1, n16, n8);
+        uint32_t s16 = 0, s8 = 0, sv = 0, par;
+        TM_TRACE_EV(3, EV_KWAIT_BEGIN);
+        if (n16) {
+          take(s16, par);
+          if (!(ok = mbar_wait(bar(C_FULL + s16), par, p.err, abort_flag))) break;
+        }
+        if (n8) {
+          take(s8, par);
+          if (!(ok = mbar_wait(bar(C_FULL + s8), par, p.err, abort_flag))) break;
+        }
+        take(sv, par);
+        const uint32_t v_par = par;
+        TM_TRACE_EV(3, EV_KWAIT_END);
+        TM_TRACE_EV(3, EV_K_READY);
+        if (j > 0 && j - 1 < nJA && !(ok = issue_pv(0, j - 1, v_prev))) break;
+        TM_TRACE_EV(3, EV_PV_A);
+        if (j < nJA) issue_s(0, r0, r0 ? s8 : s16);
+        TM_TRACE_EV(3, EV_S_A);
+        if (j > 0 && j - 1 < nJB && !(ok = issue_pv(1, j - 1, v_prev))) break;
+        TM_TRACE_EV(3, EV_PV_B);
+        if (j > 0) tc_commit(bar(C_EMPTY + v_prev));
+        if (j < nJB) issue_s(1, r1, r1 ? s8 : s16);
+        TM_TRACE_EV(3, EV_S_B);
+        if (n16) tc_commit(bar(C_EMPTY + s16));
+        if (n8) tc_commit(bar(C_EMPTY + s8));
+        TM_TRACE_EV(3, EV_VWAIT_BEGIN);
+        // V of this tile must have landed before its P.V is issued next round
+        if (!(ok = mbar_wait(bar(C_FULL + sv), v_par, p.err, abort_flag))) break;
+        TM_TRACE_EV(3, EV_V_READY);
+        v_prev = sv;
+      }
+      if (ok) {
+        if (nJ - 1 < nJA) ok = issue_pv(0, nJ - 1, v_prev);
+        if (ok && nJ - 1 < nJB) ok = issue_pv(1, nJ - 1, v_prev);
+        tc_commit(bar(C_EMPTY + v_prev));
+      }
+      tc_commit(bar(C_DRAIN));
+      volatile int never = 0;
+      mbar_wait(bar(C_DRAIN), 0, p.err, &never);
+    }
+   }
+  } else {
+    // ======================= softmax (warpgroup t = tile t) =======================
+    regs_inc<C::SOFTMAX_REGS>();
+    const int t = warp >> 2;
+    const TileInfo& T = ti[t];
+    const int r = threadIdx.x & 127;                 // row in the tile = TMEM lane
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t s_addr = lane_addr + C::s_col(t);
+    const uint32_t o_addr = lane_addr + C::o_col(t);
+    const bool row_ok = r < T.rows;
+    const int64_t i_row = static_cast<int64_t>(2 * P + t) * 128 + r;
+    int64_t lim = -1;
+    if (row_ok) lim = p.causal ? min(Lk - 1, i_row + Lk - Lq) : Lk - 1;
+    float c8_row = 0.f;
+    if (T.mrow != nullptr) c8_row = __ldg(p.q_scales + T.ig * p.Hq + h) * p.scale_log2;
+    const SeqInfo sk = seq_info(p.cu, b, p.Lk, BN);
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    TM_TRACE_DECL
+    const bool tracer = (threadIdx.x & 127) == 0;
+    if (tracer) TM_TRACE_EV(t, EV_START);
+    for (int j = 0; j < T.nJ; ++j) {
+      const bool i8 = route8(rrow[t], p.g, j);
+      float c = p.scale_log2;
+      if (i8) c = fmaxf(c8_row * __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk), 1e-30f);
+      if (!mbar_wait(bar(C_SFULL + t), j & 1, p.err, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      if (tracer) TM_TRACE_EV(t, EV_S_READY);
+      __syncwarp();
+      float x[BN];
+      {
+        uint32_t u[BN];
+#pragma unroll
+        for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32p(s_addr + cc * 32, u + cc * 32);
+        tmem_wait_ld();
+        if (tracer) TM_TRACE_EV(t, EV_SLOADED);
+        if (i8) {
+          // exact int32 -> fp32 for |acc| < 2^22: add the bits of 1.5 * 2^23,
+          // then subtract 1.5 * 2^23 in packed fp32
+          const uint64_t nmagic = f2pack(-12582912.0f, -12582912.0f);
+#pragma unroll
+          for (int e = 0; e < BN; e += 2) {
+            const uint64_t v = f2add(f2pack(__int_as_float(static_cast<int>(u[e]) + 0x4B400000),
+                                            __int_as_float(static_cast<int>(u[e + 1]) + 0x4B400000)),
+                                     nmagic);
+            f2unpack(v, x[e], x[e + 1]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(u[e]);
+        }
+      }
+      const int64_t nv64 = lim - static_cast<int64_t>(j) * BN + 1;
+      const int nv = nv64 <= 0 ? 0 : (nv64 >= BN ? BN : static_cast<int>(nv64));
+      if (!__all_sync(0xffffffffu, nv == BN)) {
+#pragma unroll
+        for (int e = 0; e < BN; ++e) x[e] = (e < nv) ? x[e] : -INFINITY;
+      }
+      float alpha = 1.f;
+      if (nv > 0) {
+        const float mt = row_max<BN>(x) * c;
+        if (mt > m_used + 8.0f) {
+          alpha = ex2_approx(m_used - mt);
+          m_used = mt;
+        }
+      }
+      const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+      if (tracer) TM_TRACE_EV(t, EV_MAXED);
+      const uint64_t c2 = f2pack(c, c);
+      const uint64_t nm2 = f2pack(-msub, -msub);
+      uint32_t pk[BN / 2];
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int e = 0; e < BN; e += 2) {
+        const uint64_t y2 = f2fma(f2pack(x[e], x[e + 1]), c2, nm2);
+        float p0, p1;
+        if (EMU > 0 && ((e >> 1) & 7) < EMU) {
+          exp2_poly2(y2, p0, p1);
+        } else {
+          float y0, y1;
+          f2unpack(y2, y0, y1);
+          p0 = ex2_approx(y0);
+          p1 = ex2_approx(y1);
+        }
+        acc2[(e >> 1) & 3] = f2add(acc2[(e >> 1) & 3], f2pack(p0, p1));
+        pk[e >> 1] = pack_half2(p0, p1);
+      }
+      {
+        const uint64_t s2 = f2add(f2add(acc2[0], acc2[1]), f2add(acc2[2], acc2[3]));
+        float s0, s1;
+        f2unpack(s2, s0, s1);
+        l = l * alpha + (s0 + s1);
+      }
+      if (tracer) TM_TRACE_EV(t, EV_EXP_DONE);
+      // O is rescaled only when a row of this warp raised its running max.
+      // Then PV_{j-1} must have completed: o_done has finished phase j-2 at
+      // least (S_j completed after PV_{j-2}), so waiting for phase j-1 by
+      // parity is unambiguous even though earlier phases were not waited on.
+      if (tracer) TM_TRACE_EV(t, EV_O_READY);
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!mbar_wait(bar(C_ODONE + t), (j - 1) & 1, p.err, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        __syncwarp();
+        {
+          if (tracer) TM_TRACE_EV(t, EV_RESCALED);
+          uint32_t o[D];
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
+          tmem_wait_ld();
+          const uint64_t a2 = f2pack(alpha, alpha);
+#pragma unroll
+          for (int e = 0; e < D; e += 2) {
+            float o0, o1;
+            f2unpack(f2mul(f2pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), o0, o1);
+            o[e] = __float_as_uint(o0);
+            o[e + 1] = __float_as_uint(o1);
+          }
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) tmem_st32p(o_addr + cc * 32, o + cc * 32);
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int cc = 0; cc < BN / 64; ++cc) tmem_st32p(s_addr + cc * 32, pk + cc * 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C_PFULL + t));
+      if (tracer) TM_TRACE_EV(t, EV_P_RELEASED);
+    }
+    // ---- epilogue
+    bool have_o = false;
+    if (ok && T.nJ > 0) {
+      have_o = mbar_wait(bar(C_ODONE + t), (T.nJ - 1) & 1, p.err, abort_flag);
+      tc_fence_after();
+    }
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    __syncwarp();
+    uint32_t o[D];
+    if (__all_sync(0xffffffffu, have_o)) {
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < D; ++e) o[e] = 0u;
+    }
+    if (row_ok) {
+      __half* orow = p.out + (T.row0 + r) * p.out_st + static_cast<int64_t>(h) * p.out_sh;
+#pragma unroll
+      for (int cc = 0; cc < D / 8; ++cc) {
+        uint4 pkt;
+        pkt.x = pack_half2(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv);
+        pkt.y = pack_half2(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv);
+        pkt.z = pack_half2(__uint_as_float(o[8 * cc + 4]) * inv, __uint_as_float(o[8 * cc + 5]) * inv);
+        pkt.w = pack_half2(__uint_as_float(o[8 * cc + 6]) * inv, __uint_as_float(o[8 * cc + 7]) * inv);
+        st_global_stream_v4(reinterpret_cast<uint4*>(orow) + cc, pkt);
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+#ifndef TM_EXP2_EMU_PAIRS
+#define TM_EXP2_EMU_PAIRS 3       // exp2 pairs (of every 8) evaluated on the FMA pipe
+#endif
+
+std::mutex g_mu2;
+
+template <int D>
+tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                      const int32_t* cu, int32_t batch, int32_t max_seqlen, const uint32_t* bitmask,
+                      int64_t mask_hs, int32_t g, int32_t causal, cudaStream_t stream) {
+  using C = Cfg2<D>;
+  auto kern = attn_pair_kernel<D, TM_EXP2_EMU_PAIRS>;
+  static bool attr_done = false;
+  {
+    std::lock_guard<std::mutex> lk(g_mu2);
+    if (!attr_done) {
+      // The warpgroup register split assumes exactly LAUNCH_REGS per thread
+      // at launch; any other allocation could leave setmaxnreg.inc waiting.
+      cudaFuncAttributes fa;
+      tm_status st = check_cuda(cudaFuncGetAttributes(&fa, kern));
+      if (st != TM_OK) return st;
+      if (fa.numRegs != C::LAUNCH_REGS) return TM_ERR_UNSUPPORTED;
+      st = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           C::SMEM_BYTES));
+      if (st != TM_OK) return st;
+      attr_done = true;
+    }
+  }
+  CUtensorMap mQ16, mQ8, mK16, mK8, mV16;
+  tm_status st;
+  st = encode_thd_map(&mQ16, q->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q->T, q->H, D, q->stride_t,
+                      q->stride_h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TM_OK) return st;
+  st = encode_thd_map(&mK16, k->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, k->T, k->H, D, k->stride_t,
+                      k->stride_h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TM_OK) return st;
+  st = encode_thd_map(&mV16, v->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, v->T, v->H, D, v->stride_t,
+                      v->stride_h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TM_OK) return st;
+  const CUtensorMapSwizzle swz8 = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (bitmask != nullptr) {
+    st = encode_thd_map(&mQ8, q->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q->T, q->H, D, q->H * D, D, D,
+                        128, swz8);
+    if (st != TM_OK) return st;
+    st = encode_thd_map(&mK8, k->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k->T, k->H, D, k->H * D, D, D,
+                        128, swz8);
+    if (st != TM_OK) return st;
+  } else {
+    mQ8 = mQ16;
+    mK8 = mK16;
+  }
+  Params2 p;
+  p.out = static_cast<__half*>(out->data);
+  p.out_st = out->stride_t;
+  p.out_sh = out->stride_h;
+  p.q_scales = static_cast<const float*>(q->scales);
+  p.k_scales = static_cast<const float*>(k->scales);
+  p.bitmask = bitmask;
+  p.mask_hs = mask_hs;
+  p.cu = cu;
+  p.Lq = q->T;
+  p.Lk = k->T;
+  p.Hq = static_cast<int>(q->H);
+  p.Hkv = static_cast<int>(k->H);
+  p.g = g;
+  p.causal = causal ? 1 : 0;
+  p.batch = cu ? batch : 1;
+  const int64_t maxq = cu ? max_seqlen : q->T;
+  const int64_t maxk = cu ? max_seqlen : k->T;
+  p.n_qt_max = static_cast<int>((maxq + 127) / 128);
+  p.n_pair_max = (p.n_qt_max + 1) / 2;
+  p.W = tm_mask_words(maxk, 128, g);
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
+  p.err = DevErr{device_error_word()};
+  const int64_t grid = static_cast<int64_t>(p.n_pair_max) * p.batch * p.Hq;
+  if (grid == 0) return TM_OK;
+  if (grid > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
+  return check_cuda(cudaGetLastError());
+}
+
+}  // namespace
+
+tm_status launch_attn_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                           const int32_t* cu, int32_t batch, int32_t max_seqlen,
+                           const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
+                           cudaStream_t stream) {
+  if (q->d == 128)
+    return launch_pair<128>(q, k, v, out, cu, batch, max_seqlen, bitmask, mask_hs, g, causal, stream);
+  return launch_pair<64>(q, k, v, out, cu, batch, max_seqlen, bitmask, mask_hs, g, causal, stream);
+}
+
+}  // namespace tmk

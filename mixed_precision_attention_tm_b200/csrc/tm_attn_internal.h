@@ -1,0 +1,17 @@
+// tm_attn_internal.h -- launchers shared between the attention translation
+// units (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "../../include/tm.h"
+
+namespace tmk {
+
+// Two 128-row query tiles per CTA, 128-key tiles, fp16 K/V (d = 64 or 128).
+tm_status launch_attn_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                           const int32_t* cu, int32_t batch, int32_t max_seqlen,
+                           const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
+                           cudaStream_t stream);
+
+}  // namespace tmk

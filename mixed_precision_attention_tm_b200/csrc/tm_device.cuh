@@ -19,6 +19,31 @@
 #define TM_WAIT_LIMIT_NS 2000000000ull   // 2 s
 #endif
 
+// Optional event tracing (compiled out unless TM_TRACE is defined): one
+// traced CTA records (event id, SM clock) pairs per role into a device buffer
+// that tm_debug_trace_read copies out.  Used to read pipeline timelines.
+#ifdef TM_TRACE
+#define TM_TRACE_ROLES 4
+#define TM_TRACE_EVENTS 4096
+static __device__ unsigned long long g_tm_trace[TM_TRACE_ROLES][TM_TRACE_EVENTS];
+static __device__ unsigned int g_tm_trace_block;
+#define TM_TRACE_DECL unsigned int tm_trace_n = 0;
+#define TM_TRACE_EV(role, ev)                                                                   \
+  do {                                                                                          \
+    if (blockIdx.x == g_tm_trace_block && tm_trace_n < TM_TRACE_EVENTS) {                        \
+      long long tm_c;                                                                           \
+      asm volatile("mov.u64 %0, %%clock64;" : "=l"(tm_c));                                     \
+      g_tm_trace[role][tm_trace_n++] = (static_cast<unsigned long long>(ev) << 56) |             \
+                                       (static_cast<unsigned long long>(tm_c) & 0xFFFFFFFFFFFFFFull); \
+    }                                                                                           \
+  } while (0)
+#else
+#define TM_TRACE_DECL
+#define TM_TRACE_EV(role, ev) \
+  do {                        \
+  } while (0)
+#endif
+
 namespace tmk {
 
 // Defined in tm_api.cu (relocatable device code is not used, so each
@@ -93,6 +118,55 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const D
   }
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Spinning wait for a single latency-critical thread (the MMA issuer): polls
+// with the non-suspending test_wait; same time limit and abort rules as
+// mbar_wait.
+__device__ __forceinline__ bool mbar_spin(uint32_t bar, uint32_t parity, const DevErr& err,
+                                          volatile int* abort) {
+  for (int i = 0; i < 256; ++i)
+    if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    for (int i = 0; i < 256; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > TM_WAIT_LIMIT_NS) {
+      dev_error(err, TM_DEVERR_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Warp-cooperative wait: lane 0 polls, the other lanes wait at __syncwarp and
+// then confirm with one try_wait each (so every lane observes the phase with
+// acquire semantics).  Keeps 31 of 32 threads off the shared-memory barrier
+// while a warp waits.  Must be called by all 32 lanes of a converged warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const DevErr& err,
+                                               volatile int* abort) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, abort);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok && (threadIdx.x & 31) != 0) {
+    while (!mbar_try_wait(bar, parity)) {
+    }
+  }
+  __syncwarp();
+  return ok;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int32_t c0, int32_t c1, int32_t c2) {
@@ -101,6 +175,35 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+// Same load with an L2 cache policy (from createpolicy).
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int32_t c0, int32_t c1, int32_t c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+
+// Brings a tensor tile into L2 ahead of its shared-memory load (no completion).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int32_t c0, int32_t c1, int32_t c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -256,6 +359,47 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Warpgroup register reallocation (all four warps of the warpgroup execute it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: two lanes per instruction).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ void st_global_stream_v4(void* ptr, uint4 v) {
+  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
