@@ -502,8 +502,28 @@ extern "C" tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const t
   st = check_fp16(out, D);
   if (st != TM_OK) return st;
   if (out->T != q->T || out->H != q->H) return TM_ERR_INVALID_ARG;
+  if (q->H % k->H != 0 || q->H > 65535 || k->H <= 0) return TM_ERR_INVALID_ARG;
+  if (cu_seqlens != nullptr && (batch <= 0 || max_seqlen <= 0)) return TM_ERR_INVALID_ARG;
+  if (bitmask != nullptr) {
+    if (reinterpret_cast<uintptr_t>(bitmask) & 3u) return TM_ERR_INVALID_ARG;
+    if (q->codes == nullptr || !aligned16(q->codes) || q->scale_kind != TM_SCALE_TILE || q->scales == nullptr)
+      return TM_ERR_INVALID_ARG;
+  }
   const bool cache = (k->scale_kind == TM_SCALE_TOKEN) || (v->scale_kind == TM_SCALE_TOKEN);
-  if (cache) return TM_ERR_UNSUPPORTED;   // INT8 K/V cache: see tm_attn_cache.cu
+  if (cache) {
+    // INT8 K/V cache: both K and V as codes + per-(token, head) fp16 scales.
+    if (k->scale_kind != TM_SCALE_TOKEN || v->scale_kind != TM_SCALE_TOKEN) return TM_ERR_INVALID_ARG;
+    if (k->codes == nullptr || v->codes == nullptr || k->scales == nullptr || v->scales == nullptr)
+      return TM_ERR_INVALID_ARG;
+    if (!aligned16(k->codes) || !aligned16(v->codes) || (reinterpret_cast<uintptr_t>(k->scales) & 1u) ||
+        (reinterpret_cast<uintptr_t>(v->scales) & 1u))
+      return TM_ERR_INVALID_ARG;
+    if (k->T != v->T || k->H != v->H || k->d != D || v->d != D || k->T < 0) return TM_ERR_INVALID_ARG;
+    if (cu_seqlens != nullptr && k->T != q->T) return TM_ERR_INVALID_ARG;
+    if (D != 128 || tile_n != 128) return TM_ERR_UNSUPPORTED;
+    return launch_attn_cache(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride, tile_m, g,
+                             causal, as_stream(stream));
+  }
   st = check_fp16(k, D);
   if (st != TM_OK) return st;
   st = check_fp16(v, D);
@@ -514,11 +534,7 @@ extern "C" tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const t
     if (batch <= 0 || max_seqlen <= 0 || k->T != q->T) return TM_ERR_INVALID_ARG;
   }
   if (bitmask != nullptr) {
-    if (reinterpret_cast<uintptr_t>(bitmask) & 3u) return TM_ERR_INVALID_ARG;
-    if (q->codes == nullptr || k->codes == nullptr || !aligned16(q->codes) || !aligned16(k->codes))
-      return TM_ERR_INVALID_ARG;
-    if (q->scale_kind != TM_SCALE_TILE || k->scale_kind != TM_SCALE_TILE || q->scales == nullptr ||
-        k->scales == nullptr)
+    if (k->codes == nullptr || !aligned16(k->codes) || k->scale_kind != TM_SCALE_TILE || k->scales == nullptr)
       return TM_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);

@@ -14,4 +14,10 @@ tm_status launch_attn_pair(const tm_tensor* q, const tm_tensor* k, const tm_tens
                            const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
                            cudaStream_t stream);
 
+// INT8 K/V cache (codes + per-token fp16 scales), d = 128, 128-key tiles.
+tm_status launch_attn_cache(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                            const int32_t* cu, int32_t batch, int32_t max_seqlen,
+                            const uint32_t* bitmask, int64_t mask_hs, int32_t tile_m, int32_t g,
+                            int32_t causal, cudaStream_t stream);
+
 }  // namespace tmk

@@ -239,3 +239,56 @@ def test_noncontiguous_head_strides():
     torch.cuda.synchronize()
     ref = oracle.attention(q.numpy(), k.numpy(), v.numpy(), causal=True)
     assert max_err(out.cpu(), ref) <= TOL
+
+
+# ------------------------------------------------------------------ INT8 K/V cache
+def Wc(hq, hkv, causal, p=None, g=1, tm=128, cu=None, Lq=None, Lk=None, seed=0, fd=False, fs=False):
+    if cu is not None:
+        cu_t = torch.tensor(cu, dtype=torch.int32)
+        lens = cu_t[1:] - cu_t[:-1]
+        Lq = Lk = int(cu[-1])
+    else:
+        cu_t = lens = None
+    d = 128
+    q = inputs.randn_f16((Lq, hq, d), seed)
+    k = inputs.randn_f16((Lk, hkv, d), seed + 1)
+    v = inputs.randn_f16((Lk, hkv, d), seed + 2)
+    kc, ks = inputs.int8_kv_cache(k)
+    vc, vs = inputs.int8_kv_cache(v)
+    return inputs.Workload("cache", q, None, None, hq, hkv, d, causal, tm, 128, g, p, mask_seed=seed + 4,
+                           force_diag=fd, force_sink=fs, cu_seqlens=cu_t, lens=lens, kv_cache=(kc, ks, vc, vs))
+
+
+CACHE_CASES = [
+    ("varlen_cache_routed", dict(hq=4, hkv=2, causal=True, p=0.5, g=2, cu=[0, 300, 300, 1100, 1400], fd=True, fs=True)),
+    ("varlen_cache_fp16", dict(hq=4, hkv=1, causal=True, p=None, cu=[0, 257, 900])),
+    ("cache_all_int8", dict(hq=2, hkv=1, causal=False, p=1.0, Lq=700, Lk=700)),
+    ("cache_q_shorter", dict(hq=2, hkv=2, causal=True, p=0.5, Lq=300, Lk=1000)),
+    ("cache_tm64", dict(hq=2, hkv=1, causal=True, p=0.5, tm=64, Lq=600, Lk=600)),
+]
+
+
+@pytest.mark.parametrize("name,kw", CACHE_CASES, ids=[c[0] for c in CACHE_CASES])
+def test_int8_cache_matches_oracle(name, kw):
+    w = Wc(**kw)
+    out, m, _ = run_gpu(w)
+    mask_u32 = None if m is None else m.numpy().view(np.uint32)
+    if mask_u32 is not None:
+        assert np.array_equal(mask_u32, oracle_mask(w))
+    ref = run_oracle(w, mask_u32)
+    assert torch.isfinite(out).all()
+    err = max_err(out, ref)
+    assert err <= TOL, f"{name}: max abs err {err}"
+
+
+def test_int8_cache_fp16_route_equals_dequantised_fp16_inputs():
+    # With every group FP16, the cache path must equal the fp16 path fed with
+    # the cache's fp16 view fp16(code * scale) (the same numbers reach the MMAs).
+    w = Wc(hq=4, hkv=2, causal=True, p=None, Lq=640, Lk=640)
+    out_c, _, _ = run_gpu(w)
+    kc, ks, vc, vs = w.kv_cache
+    k16 = torch.from_numpy(oracle.dequant_cache(kc.numpy(), ks.numpy()))
+    v16 = torch.from_numpy(oracle.dequant_cache(vc.numpy(), vs.numpy()))
+    wf = inputs.Workload("f", w.q, k16, v16, 4, 2, 128, True, 128, 128, 1, None)
+    out_f, _, _ = run_gpu(wf)
+    assert max_err(out_c, out_f.to(torch.float64).numpy()) <= 2e-3
