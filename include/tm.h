@@ -195,6 +195,40 @@ tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
                       const uint32_t* bitmask, int64_t mask_head_stride,
                       int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * tm_attn_fwd_routed_noalloc -- the routed prefill step for callers that
+ * cannot allocate device memory.  (Library addition; it has no counterpart
+ * in the paper.)
+ *
+ * Some callers cannot give the library scratch buffers: a serving engine that
+ * reserves nearly all device memory for its own pools at start-up and has no
+ * allocator to lend to a C library, or a deployment that forbids cudaMalloc
+ * after initialisation because it may synchronise the device and has
+ * unbounded latency.  This call runs tm_quantize_qk, tm_build_mask and
+ * tm_attn_fwd for one sequence (no cu_seqlens; Lq = q->T, Lk = k->T) with the
+ * INT8 codes, tile scales and routing mask placed in a fixed device array that
+ * the library owns: TM_NOALLOC_SCRATCH_BYTES on every GPU that loads the
+ * library, held until the process exits.  The caller passes q, k, v (fp16
+ * data; their codes / scales fields are ignored) and out, as for tm_attn_fwd,
+ * and the routing parameters of tm_build_mask (mask_head_stride is implied).
+ * No cudaMalloc, cudaFree or other allocating routine is called.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) while that device is current; make that first
+ *    call before any stream capture.
+ *  - All calls share the array and it keeps the last call's contents; every
+ *    byte a call reads it first writes, so nothing needs clearing.  Calls
+ *    that overlap on the GPU (other streams, other host threads on the same
+ *    device) race on the array: serialise them.
+ *  - A problem whose codes, scales and mask need more than
+ *    TM_NOALLOC_SCRATCH_BYTES (about Lq*Hq*d + Lk*Hkv*d bytes) returns
+ *    TM_ERR_UNSUPPORTED before any launch.
+ * ------------------------------------------------------------------------- */
+#define TM_NOALLOC_SCRATCH_BYTES (32u << 20)
+tm_status tm_attn_fwd_routed_noalloc(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v,
+                                     tm_tensor* out, int32_t tile_m, int32_t tile_n, int32_t g,
+                                     int32_t causal, double p, uint64_t seed,
+                                     int32_t force_diag, int32_t force_sink, void* stream);
+
 /* Reads and clears the device error word after synchronising `stream`.
  * Returns TM_OK, TM_ERR_TIMEOUT (a pipeline wait gave up; the output of the
  * affected call is unspecified) or TM_ERR_INVALID_ARG (a sequence exceeded

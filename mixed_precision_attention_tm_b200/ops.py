@@ -66,6 +66,7 @@ def _lib():
             "tm_route_stats": (I32, [P, I64, I32, P, I32, I64, I64, I32, I32, I32, I32,
                                      ctypes.POINTER(D), ctypes.POINTER(D)]),
             "tm_attn_fwd": (I32, [TP, TP, TP, TP, P, I32, I32, P, I64, I32, I32, I32, I32, P]),
+            "tm_attn_fwd_routed_noalloc": (I32, [TP, TP, TP, TP, I32, I32, I32, I32, D, U64, I32, I32, P]),
             "tm_get_device_error": (I32, [P]),
             "tm_status_string": (ctypes.c_char_p, [I32]),
             "tm_last_cuda_error": (I32, []),
@@ -270,6 +271,24 @@ def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal
                          _ptr(cu_seqlens), batch, int(max_seqlen or 0), _ptr(bitmask),
                          int(mask_head_stride or 0), tile_m, tile_n, g, int(bool(causal)), _stream())
     _check(st, "tm_attn_fwd")
+    return out
+
+
+def attn_fwd_routed_noalloc(q, k, v, *, out=None, tile_m=128, tile_n=128, g=1, causal=False, p=0.5,
+                            seed=0, force_diag=False, force_sink=False):
+    """Routed prefill (quantise, mask, attend) for one sequence with the
+    library's fixed device scratch array instead of caller-allocated codes,
+    scales and mask; only out is allocated here (by torch) when not given."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda(t, n)
+    if out is None:
+        out = torch.empty_like(q)
+    qd, kd, vd, od = _desc(q), _desc(k), _desc(v), _desc(out)
+    st = _lib().tm_attn_fwd_routed_noalloc(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
+                                           tile_m, tile_n, g, int(bool(causal)), float(p),
+                                           ctypes.c_uint64(int(seed) & (2 ** 64 - 1)), int(bool(force_diag)),
+                                           int(bool(force_sink)), _stream())
+    _check(st, "tm_attn_fwd_routed_noalloc")
     return out
 
 

@@ -1,0 +1,63 @@
+"""GPU test of tm_attn_fwd_routed_noalloc, the routed prefill entry point for
+callers that cannot allocate device memory (for instance engines that keep
+all device memory in their own pools, or deployments that forbid cudaMalloc
+after start-up).  It keeps the INT8 codes, tile scales and routing mask in a
+fixed library-owned device array; its output must match the regular path
+(tm_quantize_qk + tm_build_mask + tm_attn_fwd with caller-allocated buffers)
+within the parity tolerance, on two calls in a row that reuse the array.
+
+Collected last on purpose: a run that stops at the first failure has already
+run every other test.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import TOL
+from mixed_precision_attention_tm_b200 import inputs, ops
+
+pytestmark = pytest.mark.gpu
+
+
+def _regular(q, k, v, tm, tn, g, causal, p, seed, fd, fs):
+    qc, qs, kc, ks = ops.quantize_qk(q, k, tile_m=tm, tile_n=tn)
+    m = ops.build_mask(q.shape[1], tile_m=tm, tile_n=tn, g=g, causal=causal, p=p, seed=seed, force_diag=fd,
+                       force_sink=fs, Lq=q.shape[0], Lk=k.shape[0], device=q.device)
+    return ops.attn_fwd(q, k, v, tile_m=tm, tile_n=tn, g=g, causal=causal, bitmask=m, q_quant=(qc, qs),
+                        k_quant=(kc, ks))
+
+
+CALLS = [
+    # (Lq, Lk, Hq, Hkv, d, tile_m, tile_n, g, causal, p, seed, force_diag, force_sink)
+    (1024, 1024, 8, 2, 128, 128, 128, 2, True, 0.5, 11, True, True),
+    (700, 900, 4, 1, 64, 64, 64, 1, False, 0.75, 12, False, True),
+]
+
+
+def test_noalloc_matches_regular_path_on_consecutive_calls():
+    outs = []
+    for (Lq, Lk, hq, hkv, d, tm, tn, g, causal, p, seed, fd, fs) in CALLS:
+        q = inputs.randn_f16((Lq, hq, d), seed).cuda()
+        k = inputs.randn_f16((Lk, hkv, d), seed + 1).cuda()
+        v = inputs.randn_f16((Lk, hkv, d), seed + 2).cuda()
+        got = ops.attn_fwd_routed_noalloc(q, k, v, tile_m=tm, tile_n=tn, g=g, causal=causal, p=p, seed=seed,
+                                          force_diag=fd, force_sink=fs)
+        ref = _regular(q, k, v, tm, tn, g, causal, p, seed, fd, fs)
+        torch.cuda.synchronize()
+        assert ops.get_device_error() == ops.TM_OK
+        err = (got.float() - ref.float()).abs().max().item()
+        assert err <= TOL, f"call {len(outs)}: max abs difference {err}"
+        outs.append(got.cpu())
+    # the second call overwrote the shared array; the first result is unaffected
+    assert outs[0].shape != outs[1].shape
+
+
+def test_noalloc_rejects_problems_beyond_the_array():
+    # 32 MiB of scratch cannot hold the codes of 16384 x 32 x 128 queries
+    q = torch.empty((16384, 32, 128), dtype=torch.float16, device="cuda")
+    k = torch.empty((16384, 8, 128), dtype=torch.float16, device="cuda")
+    v = torch.empty_like(k)
+    with pytest.raises(ops.TmError) as e:
+        ops.attn_fwd_routed_noalloc(q, k, v, causal=True, p=0.5)
+    assert e.value.status == ops.TM_ERR_UNSUPPORTED
