@@ -113,6 +113,7 @@ struct Params2 {
   const int32_t* cu;
   int64_t Lq, Lk;
   int Hq, Hkv, g, causal, n_pair_max, n_qt_max, batch;
+  int kv_chunk;            // KV heads per scheduling chunk (divides Hkv)
   float scale_log2;
   DevErr err;
 };
@@ -179,11 +180,19 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit (pair P of sequence b, head h), heaviest pairs first
-  const int h = blockIdx.x % p.Hq;
-  const int t1 = blockIdx.x / p.Hq;
-  const int b = t1 % p.batch;
-  const int P = p.n_pair_max - 1 - t1 / p.batch;
+  // ---- work unit (pair P of sequence b, head h).  Grid order: chunk of
+  // kv_chunk KV heads (slowest), pair (heaviest first), sequence, query head
+  // within the chunk (fastest).  The CTAs resident at any time then read the
+  // K / V of one chunk, sized on the host to stay in L2, while the pairs of a
+  // chunk still run longest first.
+  const int heads_per_chunk = p.kv_chunk * (p.Hq / p.Hkv);
+  const int units_per_chunk = heads_per_chunk * p.batch * p.n_pair_max;
+  const int chunk = blockIdx.x / units_per_chunk;
+  int rest = blockIdx.x - chunk * units_per_chunk;
+  const int h = chunk * heads_per_chunk + rest % heads_per_chunk;
+  rest /= heads_per_chunk;
+  const int b = rest % p.batch;
+  const int P = p.n_pair_max - 1 - rest / p.batch;
   const SeqInfo sq = seq_info(p.cu, b, p.Lq, 128);
   const int64_t Lq = sq.len;
   const int64_t Lk = p.cu ? sq.len : p.Lk;
@@ -670,6 +679,17 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
   p.W = tm_mask_words(maxk, 128, g);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   p.err = DevErr{device_error_word()};
+  // KV heads per scheduling chunk: as many as keep their K / V (fp16 K, int8
+  // K, fp16 V) within ~40 MB of L2, widened until a chunk fills two waves of
+  // 148 CTAs; always a divisor of Hkv.
+  {
+    const double kv_bytes = static_cast<double>(maxk) * D * (2 + 1 + 2);
+    int c = static_cast<int>(40.0e6 / (kv_bytes > 1.0 ? kv_bytes : 1.0));
+    c = c < 1 ? 1 : (c > p.Hkv ? p.Hkv : c);
+    while (c < p.Hkv && static_cast<int64_t>(c) * (p.Hq / p.Hkv) * p.batch * p.n_pair_max < 2 * 148) ++c;
+    while (p.Hkv % c) ++c;
+    p.kv_chunk = c;
+  }
   const int64_t grid = static_cast<int64_t>(p.n_pair_max) * p.batch * p.Hq;
   if (grid == 0) return TM_OK;
   if (grid > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
