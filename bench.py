@@ -39,7 +39,38 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from mixed_precision_attention_tm_b200 import inputs  # noqa: E402
+from mixed_precision_attention_tm_b200 import dist, inputs  # noqa: E402
+
+PROFILE = os.path.join(ROOT, "profiles", "attn_pair_routing_sweep.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "mixed_precision_attention_tm_b200", "csrc", f)
+                  for f in ("tm_attn2.cu", "tm_device.cuh")]
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, or
+    None when the kernel sources changed since that capture."""
+    if not os.path.exists(PROFILE):
+        return None, "no committed capture"
+    fields = {}
+    for line in open(PROFILE):
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            fields[k.strip().strip("`")] = v.strip().strip("`")
+    if fields.get("kernel_source_sha256") != kernel_source_hash():
+        return None, "kernel changed since the committed capture"
+    try:
+        return float(fields["dram_bytes_per_launch"]), fields.get("workload", "")
+    except (KeyError, ValueError):
+        return None, "capture summary unreadable"
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL = {"f16_tflops": 2250.0, "i8_tops": 4500.0}
@@ -154,7 +185,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    w = make_workload(args.workload, args.p, seed=args.seed + 1000 * rank)
+    w = make_workload(args.workload, args.p, seed=dist.rank_seed(args.seed, rank))
     plan = TileMixPrefill(w.Lq, w.Lk, w.hq, w.hkv, w.d, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n,
                           g=w.g, p=w.p, seed=w.mask_seed, force_diag=w.force_diag, force_sink=w.force_sink,
                           cu_seqlens=w.cu_seqlens, int8_cache=w.kv_cache is not None, device=dev)
@@ -180,8 +211,7 @@ def run_ours(args, rank, world, local_rank):
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
-    if world > 1:
-        torch.distributed.barrier()
+    dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
@@ -196,18 +226,14 @@ def run_ours(args, rank, world, local_rank):
     t1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
-    if world > 1:
-        torch.distributed.barrier()
+    dist.barrier()
     total_ms = t0.elapsed_time(t1)
     attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev_a, ev_b)) / K
     if ops.get_device_error() != ops.TM_OK:
         raise RuntimeError("device error in timed region")
-    t = torch.tensor([total_ms, attn_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms, attn_ms = float(t[0]), float(t[1])
+    total_ms, attn_ms = dist.max_over_ranks([total_ms, attn_ms], device=dev)
     ms_step = total_ms / K
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = dist.job_throughput(world, flops, ms_step)
 
     # roofline of the attention kernel (dominant launch)
     p16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * 1e12
@@ -229,19 +255,16 @@ def run_ours(args, rank, world, local_rank):
             plan.run_host(qh, kh, vh, kvh, out_h)
         torch.cuda.synchronize()
         ke = max(3, min(K, 20))
-        if world > 1:
-            torch.distributed.barrier()
+        dist.barrier()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(stream)
         for _ in range(ke):
             plan.run_host(qh, kh, vh, kvh, out_h)
         s1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([s0.elapsed_time(s1) / ke], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": world * flops / (float(te[0]) * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "ms_per_step": float(te[0]), "h2d_bytes_per_step": plan.input_bytes(),
+        (te,) = dist.max_over_ranks([s0.elapsed_time(s1) / ke], device=dev)
+        e2e = {"value": dist.job_throughput(world, flops, te), "unit": "TFLOP/s",
+               "ms_per_step": te, "h2d_bytes_per_step": plan.input_bytes(),
                "d2h_bytes_per_step": plan.output_bytes(), "steps": ke}
 
     # INT8-fraction sweep (outside the timed region; context for the metric)
@@ -279,6 +302,9 @@ def run_ours(args, rank, world, local_rank):
             del pl
 
     launches = plan.launches_per_step * K
+    traffic, traffic_note = (None, "traffic captured for the routing-sweep workload only")
+    if args.workload == "sweep" and w.p == 0.75:
+        traffic, traffic_note = profiled_traffic()
     line = {
         "metric": "prefill attention TFLOPS (tile-routed FP16/INT8 QK^T, FP16 P.V)",
         "value": value,
@@ -300,7 +326,7 @@ def run_ours(args, rank, world, local_rank):
         "mixed_roofline_frac_of_measured": t_roof / (attn_ms * 1e-3),
         "mixed_roofline_frac_of_nominal": t_roof_nom / (attn_ms * 1e-3),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff, "unit": "TFLOP/s",
-                     "frac": achieved / peak_eff, "traffic": None,
+                     "frac": achieved / peak_eff, "traffic": traffic, "traffic_note": traffic_note,
                      "peak_source": f"{peak_src} bf16 burst {p16 / 1e12:.1f} TFLOP/s for FP16 pairs, x2 "
                                     "(nominal INT8:FP16 ratio) for INT8 QK^T, mix-weighted by visible pairs"},
         "gpu_launches": launches,
@@ -437,9 +463,7 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, local_rank, world = dist.world_info()
 
     if args.impl == "reference":
         if rank == 0:

@@ -235,6 +235,14 @@ tm_status tm_attn_fwd_routed_noalloc(const tm_tensor* q, const tm_tensor* k, con
  * max_seqlen; its extra tiles were not computed). */
 tm_status tm_get_device_error(void* stream);
 
+/* Failure-detection self-test: launches one thread that waits, with the
+ * library's bounded mbarrier wait, on a barrier nothing arrives on, giving up
+ * after limit_ns (1 ns .. 10 s) of GPU global time.  The wait records a
+ * timeout in the device error word, so a following tm_get_device_error
+ * returns TM_ERR_TIMEOUT (and clears it); the context stays usable.  Nothing
+ * faults, traps or hangs. */
+tm_status tm_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
 /* Static description of a status code. */
 const char* tm_status_string(tm_status s);
 

@@ -5,6 +5,7 @@
 
 #include <mutex>
 
+#include "tm_device.cuh"
 #include "tm_host.h"
 
 namespace {
@@ -23,6 +24,19 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
+
+// One thread waits, with the library's bounded wait, on an mbarrier that
+// nothing arrives on; the wait gives up after limit_ns and records
+// TM_DEVERR_TIMEOUT.  No copy or MMA is in flight, so the kernel just returns.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns, tmk::DevErr err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  tmk::mbar_init(tmk::smem_u32(&bar), 1);
+  abort_flag = 0;
+  tmk::fence_barrier_init();
+  tmk::mbar_wait_limit(tmk::smem_u32(&bar), 0, err, &abort_flag, limit_ns);
+}
 
 }  // namespace
 
@@ -109,6 +123,14 @@ tm_status tm_get_device_error(void* stream) {
   if (host & 1u) return TM_ERR_TIMEOUT;
   if (host & 2u) return TM_ERR_INVALID_ARG;
   return TM_OK;
+}
+
+tm_status tm_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return TM_ERR_INVALID_ARG;
+  tmk::DevErr err{tmk::device_error_word()};
+  if (err.word == nullptr) return tmk::cuda_fail(static_cast<int>(cudaErrorInvalidSymbol));
+  wait_timeout_selftest_kernel<<<1, 32, 0, tmk::as_stream(stream)>>>(limit_ns, err);
+  return tmk::check_cuda(cudaGetLastError());
 }
 
 int32_t tm_mask_words(int64_t max_lk, int32_t tile_n, int32_t g) {

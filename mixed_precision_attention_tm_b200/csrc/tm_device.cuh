@@ -102,20 +102,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity has completed.  Gives up (and
-// reports) after TM_WAIT_LIMIT_NS, or early when *abort becomes non-zero.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const DevErr& err,
-                                          volatile int* abort) {
+// reports) after limit_ns of global time, or early when *abort becomes
+// non-zero.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, const DevErr& err,
+                                                volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_ns() - t0 > TM_WAIT_LIMIT_NS) {
+    if (global_ns() - t0 > limit_ns) {
       dev_error(err, TM_DEVERR_TIMEOUT);
       *abort = 1;
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const DevErr& err,
+                                          volatile int* abort) {
+  return mbar_wait_limit(bar, parity, err, abort, TM_WAIT_LIMIT_NS);
 }
 
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {

@@ -67,6 +67,7 @@ def _lib():
                                      ctypes.POINTER(D), ctypes.POINTER(D)]),
             "tm_attn_fwd": (I32, [TP, TP, TP, TP, P, I32, I32, P, I64, I32, I32, I32, I32, P]),
             "tm_attn_fwd_routed_noalloc": (I32, [TP, TP, TP, TP, I32, I32, I32, I32, D, U64, I32, I32, P]),
+            "tm_selftest_wait_timeout": (I32, [U64, P]),
             "tm_get_device_error": (I32, [P]),
             "tm_status_string": (ctypes.c_char_p, [I32]),
             "tm_last_cuda_error": (I32, []),
@@ -290,6 +291,11 @@ def attn_fwd_routed_noalloc(q, k, v, *, out=None, tile_m=128, tile_n=128, g=1, c
                                            int(bool(force_sink)), _stream())
     _check(st, "tm_attn_fwd_routed_noalloc")
     return out
+
+
+def selftest_wait_timeout(limit_ns=1_000_000):
+    """Launch the bounded-wait self-test (a wait that must time out)."""
+    _check(_lib().tm_selftest_wait_timeout(int(limit_ns), _stream()), "tm_selftest_wait_timeout")
 
 
 def get_device_error():
