@@ -1,0 +1,76 @@
+"""GPU parity at the benchmark configurations' full sizes, through the same
+calls bench.py times: the whole output is computed on the GPU, and sampled
+query rows (tile boundaries plus seeded random rows, every head) are compared
+with the fp64 oracle, which evaluates those rows one by one.  Routing bits,
+INT8 codes and tile scales are compared in full (bit-exact).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import TOL, max_err, oracle_mask, run_gpu, run_oracle, seqs_of
+from mixed_precision_attention_tm_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _sample_rows(seqs, tile, n_random, seed):
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for (qs, lq, _ks, _lk) in seqs:
+        if lq == 0:
+            continue
+        rows.update([qs, qs + lq - 1])
+        for r0 in range(0, lq, tile * 16):       # first and last row of every 16th tile
+            rows.update([qs + r0, qs + min(lq, r0 + tile) - 1])
+        rows.update(int(x) for x in rng.integers(qs, qs + lq, max(1, n_random // len(seqs))))
+    return sorted(rows)
+
+
+def _check(w, n_random=48):
+    out, m, quant = run_gpu(w)
+    assert torch.isfinite(out).all()
+    seqs, _ = seqs_of(w)
+    mask_u32 = None if m is None else m.numpy().view(np.uint32)
+    if mask_u32 is not None:
+        assert np.array_equal(mask_u32, oracle_mask(w))
+        rq = oracle.quantize_tiles(w.q.numpy(), seqs, w.tile_m, "q")
+        assert np.array_equal(quant[1].numpy(), rq[1]) and np.array_equal(quant[0].numpy(), rq[0])
+        if quant[2] is not None:
+            rk = oracle.quantize_tiles(w.k.numpy(), seqs, w.tile_n, "k")
+            assert np.array_equal(quant[3].numpy(), rk[1]) and np.array_equal(quant[2].numpy(), rk[0])
+    rows = _sample_rows(seqs, w.tile_m, n_random, 17)
+    ref = run_oracle(w, mask_u32, rows=rows)
+    err = max_err(out, ref, rows=rows)
+    assert err <= TOL, f"{w.name}: max abs err {err} over {len(rows)} rows"
+
+
+@pytest.mark.parametrize("Lq,Lk,d,hq,hkv,causal", [
+    (4096, 4096, 128, 32, 8, True), (4096, 4096, 64, 16, 2, False), (512, 4096, 128, 32, 8, True),
+    (2048, 2048, 64, 32, 32, True),
+])
+def test_mlx_shapes_full_size(Lq, Lk, d, hq, hkv, causal):
+    _check(inputs.mlx_shape(Lq, Lk, d, hq, hkv, causal))
+
+
+@pytest.mark.parametrize("p", [0.0, 0.75, 1.0])
+def test_routing_sweep_full_size(p):
+    _check(inputs.routing_sweep(p))
+
+
+def test_varlen_int8_cache_full_size():
+    _check(inputs.varlen_int8_cache(), n_random=64)
+
+
+def test_long_context_full_size():
+    _check(inputs.long_context(), n_random=24)
+
+
+def test_tiny_config_both_runs():
+    for p in (None, 0.5):
+        w = inputs.tiny(seed=0, p=p)
+        out, m, _ = run_gpu(w)
+        ref = run_oracle(w, None if m is None else m.numpy().view(np.uint32))
+        assert max_err(out, ref) <= TOL
