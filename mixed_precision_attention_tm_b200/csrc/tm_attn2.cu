@@ -394,6 +394,11 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; ok && j < nJ; ++j) {
         bool r0, r1, n16, n8;
         needs(j, r0, r1, n16, n8);
+        // P.V of tile A for the previous key tile first: its operands (P_A,
+        // V) are ready as soon as softmax A releases P, and the wait for this
+        // key tile's K below then overlaps its execution.
+        if (j > 0 && j - 1 < nJA && !(ok = issue_pv(0, j - 1, v_prev))) break;
+        TM_TRACE_EV(3, EV_PV_A);
         uint32_t s16 = 0, s8 = 0, sv = 0, par;
         TM_TRACE_EV(3, EV_KWAIT_BEGIN);
         if (n16) {
@@ -408,8 +413,6 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t v_par = par;
         TM_TRACE_EV(3, EV_KWAIT_END);
         TM_TRACE_EV(3, EV_K_READY);
-        if (j > 0 && j - 1 < nJA && !(ok = issue_pv(0, j - 1, v_prev))) break;
-        TM_TRACE_EV(3, EV_PV_A);
         if (j < nJA) issue_s(0, r0, r0 ? s8 : s16);
         TM_TRACE_EV(3, EV_S_A);
         if (j > 0 && j - 1 < nJB && !(ok = issue_pv(1, j - 1, v_prev))) break;
