@@ -107,3 +107,60 @@ class TileMixPrefill:
             out_host = torch.empty(self.out.shape, dtype=self.out.dtype, pin_memory=True)
         out_host.copy_(self.out, non_blocking=True)
         return out_host
+
+
+class HostPipeline:
+    """Prefill steps fed from pinned host memory with the copies overlapped.
+
+    Holds `depth` plans (device buffer sets) and three streams: host->device
+    copies of step i+1 and device->host copies of step i-1 run while step i
+    computes.  Events order each buffer set: a step's inputs are uploaded
+    after the buffer's previous output has been downloaded, computed after
+    its upload, and downloaded after its compute.  Every step still moves its
+    own inputs and output across PCIe.
+    """
+
+    def __init__(self, *plan_args, depth=2, device="cuda", **plan_kw):
+        self.device = torch.device(device)
+        self.plans = [TileMixPrefill(*plan_args, device=self.device, **plan_kw) for _ in range(depth)]
+        self.h2d = torch.cuda.Stream(device=self.device)
+        self.comp = torch.cuda.Stream(device=self.device)
+        self.d2h = torch.cuda.Stream(device=self.device)
+        self.depth = depth
+        self.freed = [None] * depth
+
+    def input_bytes(self):
+        return self.plans[0].input_bytes()
+
+    def output_bytes(self):
+        return self.plans[0].output_bytes()
+
+    def run(self, host_inputs, host_outputs):
+        """host_inputs: list of (q, k, v, kv_cache) pinned host tensors per step
+        (k, v or kv_cache may be None); host_outputs: list of pinned host
+        tensors receiving each step's output.  Returns the d2h stream's last
+        event (completion of the final download)."""
+        last = None
+        for i, (inp, out_h) in enumerate(zip(host_inputs, host_outputs)):
+            b = i % self.depth
+            plan = self.plans[b]
+            q, k, v, kv = inp
+            with torch.cuda.stream(self.h2d):
+                if self.freed[b] is not None:
+                    self.h2d.wait_event(self.freed[b])
+                plan.load(q, k, v, kv)
+                loaded = torch.cuda.Event()
+                loaded.record(self.h2d)
+            with torch.cuda.stream(self.comp):
+                self.comp.wait_event(loaded)
+                plan.run()
+                done = torch.cuda.Event()
+                done.record(self.comp)
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(done)
+                out_h.copy_(plan.out, non_blocking=True)
+                freed = torch.cuda.Event()
+                freed.record(self.d2h)
+            self.freed[b] = freed
+            last = freed
+        return last
