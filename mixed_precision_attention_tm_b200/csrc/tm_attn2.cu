@@ -118,31 +118,6 @@ struct Params2 {
   DevErr err;
 };
 
-// 2^y for y <= 8 on the FMA pipe, two lanes at a time (f32x2).  y = n + f
-// with n = rne(y) obtained by adding 1.5 * 2^23 (whose float ulp is 1), f in
-// [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (relative error <= 7.5e-5
-// on that interval, coefficients from a Remez fit); 2^n enters the exponent
-// field with one integer shift-add per lane.  y is clamped at -125 so masked
-// (-inf) scores give a normal ~2^-125, which rounds to 0 in fp16.
-__device__ __forceinline__ void exp2_poly2(uint64_t y2, float& p0, float& p1) {
-  float y0, y1;
-  f2unpack(y2, y0, y1);
-  y2 = f2pack(fmaxf(y0, -125.0f), fmaxf(y1, -125.0f));
-  const uint64_t magic = f2pack(12582912.0f, 12582912.0f);
-  const uint64_t nmagic = f2pack(-12582912.0f, -12582912.0f);
-  const uint64_t t2 = f2add(y2, magic);
-  const uint64_t n2 = f2add(t2, nmagic);
-  const uint64_t f2 = f2fma(n2, f2pack(-1.0f, -1.0f), y2);
-  uint64_t q = f2fma(f2pack(0.0551716685f, 0.0551716685f), f2, f2pack(0.2426111251f, 0.2426111251f));
-  q = f2fma(q, f2, f2pack(0.6932609677f, 0.6932609677f));
-  q = f2fma(q, f2, f2pack(0.9999280572f, 0.9999280572f));
-  float q0, q1, t0, t1;
-  f2unpack(q, q0, q1);
-  f2unpack(t2, t0, t1);
-  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
 // Routing bit of key tile j (group j / g); row is a shared- or global-memory
 // copy of the query tile's bitmask words, or null (all FP16).
 __device__ __forceinline__ bool route8(const uint32_t* row, int g, int j) {

@@ -35,7 +35,7 @@ struct CfgC {
   static constexpr int C8 = BN * D;                  // one int8 code tile, 16 KB
   static constexpr int F16 = BN * D * 2;             // one fp16 tile, 32 KB
   static constexpr int HALF = BN * 128;              // 64-column fp16 slab
-  static constexpr int NKC = 2, NK16 = 2, NVC = 1, NV16 = 2;
+  static constexpr int NKC = 2, NK16 = 1, NVC = 2, NV16 = 2;
   static constexpr int OFF_Q16 = 0;
   static constexpr int OFF_Q8 = OFF_Q16 + Q16_BYTES;
   static constexpr int OFF_KC = OFF_Q8 + Q8_BYTES;
@@ -63,9 +63,9 @@ enum {
   K_KCFULL = 1,    // +NKC
   K_KCEMPTY = 3,   // +NKC (count 129: dequant threads + issuer commit)
   K_K16FULL = 5,   // +NK16 (count 128)
-  K_K16EMPTY = 7,  // +NK16
-  K_VCFULL = 9,
-  K_VCEMPTY = 10,  // count 128
+  K_K16EMPTY = 6,  // +NK16
+  K_VCFULL = 7,    // +NVC
+  K_VCEMPTY = 9,   // +NVC (count 128)
   K_V16FULL = 11,  // +NV16 (count 128)
   K_V16EMPTY = 13, // +NV16
   K_SFULL = 15,    // +2
@@ -91,6 +91,12 @@ struct ParamsC {
   DevErr err;
 };
 
+// exp2 pairs (of every 8) the softmax evaluates on the FMA pipe instead of MUFU
+#ifndef TM_CACHE_EXP2_EMU_PAIRS
+#define TM_CACHE_EXP2_EMU_PAIRS 3
+#endif
+constexpr int kCacheEmuPairs = TM_CACHE_EXP2_EMU_PAIRS;
+
 __device__ __forceinline__ bool route_c(const uint32_t* row, int g, int j) {
   if (row == nullptr) return false;
   const int G = j / g;
@@ -99,22 +105,28 @@ __device__ __forceinline__ bool route_c(const uint32_t* row, int g, int j) {
 
 // Row r of a 128-byte-swizzled int8 code tile (128 codes) -> the same row of a
 // 128-byte-swizzled fp16 tile (two 64-column slabs), each value
-// fp16_rn(code * scale).
-__device__ __forceinline__ void dequant_row(const uint8_t* codes, uint8_t* f16, int r, float scale) {
+// fp16_rn(code * scale).  Codes become fp16 without integer-to-float
+// conversions: XOR 0x80 turns a code x into the byte x + 128, which placed
+// under the fp16 exponent byte 0x64 reads as 1024 + x + 128 exactly (ulp 1);
+// subtracting 1152 gives x exactly, and one fp16 multiply by the (fp16)
+// scale rounds the exact product once, as fp16_rn(x * scale) requires.
+__device__ __forceinline__ void dequant_row(const uint8_t* codes, uint8_t* f16, int r, __half scale) {
   const int sw = r & 7;
+  const __half2 bias = __float2half2_rn(1152.0f);
+  const __half2 s2 = __half2half2(scale);
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const uint4 raw = *reinterpret_cast<const uint4*>(codes + r * 128 + ((c ^ sw) << 4));
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u, raw.z ^ 0x80808080u, raw.w ^ 0x80808080u};
     uint32_t h[8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float f0 = static_cast<float>(static_cast<int8_t>(w[q] & 0xFF)) * scale;
-      const float f1 = static_cast<float>(static_cast<int8_t>((w[q] >> 8) & 0xFF)) * scale;
-      const float f2 = static_cast<float>(static_cast<int8_t>((w[q] >> 16) & 0xFF)) * scale;
-      const float f3 = static_cast<float>(static_cast<int8_t>((w[q] >> 24) & 0xFF)) * scale;
-      h[2 * q] = pack_half2(f0, f1);
-      h[2 * q + 1] = pack_half2(f2, f3);
+      uint32_t lo = __byte_perm(w[q], 0x64646464u, 0x4140u);   // bytes b0, 0x64, b1, 0x64
+      uint32_t hi = __byte_perm(w[q], 0x64646464u, 0x4342u);   // bytes b2, 0x64, b3, 0x64
+      __half2 vlo = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&lo), bias), s2);
+      __half2 vhi = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&hi), bias), s2);
+      h[2 * q] = *reinterpret_cast<uint32_t*>(&vlo);
+      h[2 * q + 1] = *reinterpret_cast<uint32_t*>(&vhi);
     }
     // codes 16c..16c+15 = fp16 columns 16c..16c+15: slab c/4, chunks 2(c%4), 2(c%4)+1
     uint8_t* slab = f16 + (c >> 2) * CfgC::HALF + r * 128;
@@ -169,8 +181,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar(K_QFULL), 1);
     for (int s = 0; s < C::NKC; ++s) { mbar_init(bar(K_KCFULL + s), 1); mbar_init(bar(K_KCEMPTY + s), 129); }
     for (int s = 0; s < C::NK16; ++s) { mbar_init(bar(K_K16FULL + s), 128); mbar_init(bar(K_K16EMPTY + s), 1); }
-    mbar_init(bar(K_VCFULL), 1);
-    mbar_init(bar(K_VCEMPTY), 128);
+    for (int s = 0; s < C::NVC; ++s) { mbar_init(bar(K_VCFULL + s), 1); mbar_init(bar(K_VCEMPTY + s), 128); }
     for (int s = 0; s < C::NV16; ++s) { mbar_init(bar(K_V16FULL + s), 128); mbar_init(bar(K_V16EMPTY + s), 1); }
     for (int s = 0; s < 2; ++s) { mbar_init(bar(K_SFULL + s), 1); mbar_init(bar(K_PFULL + s), 128); }
     mbar_init(bar(K_ODONE), 1);
@@ -206,9 +217,10 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(bar(K_KCFULL + s), C::C8);
         tma_load_3d(sbase + C::OFF_KC + s * C::C8, &tmKc, bar(K_KCFULL + s), 0, hk, krow);
         ++nkc;
-        if (j > 0 && !mbar_wait(bar(K_VCEMPTY), (j - 1) & 1, p.err, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(K_VCFULL), C::C8);
-        tma_load_3d(sbase + C::OFF_VC, &tmVc, bar(K_VCFULL), 0, hk, krow);
+        const int vs = j % C::NVC, vlap = j / C::NVC;
+        if (vlap > 0 && !mbar_wait(bar(K_VCEMPTY + vs), (vlap - 1) & 1, p.err, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(K_VCFULL + vs), C::C8);
+        tma_load_3d(sbase + C::OFF_VC + vs * C::C8, &tmVc, bar(K_VCFULL + vs), 0, hk, krow);
         ++nvc;
       }
       volatile int never = 0;
@@ -217,7 +229,10 @@ __global__ void __launch_bounds__(384, 1)
         const int cnt = nkc > s ? (nkc - 1 - s) / C::NKC + 1 : 0;
         if (cnt > 0) mbar_wait(bar(K_KCFULL + s), (cnt - 1) & 1, p.err, &never);
       }
-      if (nvc > 0) mbar_wait(bar(K_VCFULL), (nvc - 1) & 1, p.err, &never);
+      for (int s = 0; s < C::NVC; ++s) {
+        const int cnt = nvc > s ? (nvc - 1 - s) / C::NVC + 1 : 0;
+        if (cnt > 0) mbar_wait(bar(K_VCFULL + s), (cnt - 1) & 1, p.err, &never);
+      }
     } else if (warp == 9 && lane == 0 && nJ > 0) {
       // ======================= tcgen05 issuer =======================
       bool ok = mbar_wait(bar(K_QFULL), 0, p.err, abort_flag);
@@ -280,8 +295,8 @@ __global__ void __launch_bounds__(384, 1)
       const bool i8 = route_c(mrow, p.g, j);
       const int64_t tok = kstart + static_cast<int64_t>(j) * BN + r;
       const bool in = tok < kstart + Lk;
-      const float ks = in ? __half2float(p.k_tok_scale[tok * p.Hkv + hk]) : 0.f;
-      const float vs = in ? __half2float(p.v_tok_scale[tok * p.Hkv + hk]) : 0.f;
+      const __half ks = in ? p.k_tok_scale[tok * p.Hkv + hk] : __float2half(0.f);
+      const __half vs = in ? p.v_tok_scale[tok * p.Hkv + hk] : __float2half(0.f);
       const int s = j % C::NKC;
       if (!mbar_wait(bar(K_KCFULL + s), (j / C::NKC) & 1, p.err, abort_flag)) break;
       if (!i8) {
@@ -293,13 +308,14 @@ __global__ void __launch_bounds__(384, 1)
         ++n16;
       }
       mbar_arrive(bar(K_KCEMPTY + s));
-      if (!mbar_wait(bar(K_VCFULL), j & 1, p.err, abort_flag)) break;
+      const int vcs = j % C::NVC;
+      if (!mbar_wait(bar(K_VCFULL + vcs), (j / C::NVC) & 1, p.err, abort_flag)) break;
       const int v16 = j % C::NV16;
       if (j >= C::NV16 && !mbar_wait(bar(K_V16EMPTY + v16), ((j / C::NV16) - 1) & 1, p.err, abort_flag)) break;
-      dequant_row(smem + C::OFF_VC, smem + C::OFF_V16 + v16 * C::F16, r, vs);
+      dequant_row(smem + C::OFF_VC + vcs * C::C8, smem + C::OFF_V16 + v16 * C::F16, r, vs);
       fence_async_shared();
       mbar_arrive(bar(K_V16FULL + v16));
-      mbar_arrive(bar(K_VCEMPTY));
+      mbar_arrive(bar(K_VCEMPTY + vcs));
     }
   } else {
     // ======================= softmax (warps 0-3) =======================
@@ -335,15 +351,26 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld32p(lane_addr + static_cast<uint32_t>(j & 1) * BN + cc * 32, u + cc * 32);
         tmem_wait_ld();
         if (i8) {
-          // exact int32 -> fp32 (|acc| < 2^22), times the column's s_q s_k sigma log2(e)
+          // exact int32 -> fp32 (|acc| < 2^22: add the bits of 1.5 * 2^23, then
+          // subtract it), times the column's s_q s_k sigma log2(e), in f32x2
+          const uint64_t nmagic = f2pack(-12582912.0f, -12582912.0f);
+          const float2* ks2 = reinterpret_cast<const float2*>(kscale_s);
 #pragma unroll
-          for (int e = 0; e < BN; ++e)
-            x[e] = (__int_as_float(static_cast<int>(u[e]) + 0x4B400000) - 12582912.0f) * kscale_s[e];
+          for (int e = 0; e < BN; e += 2) {
+            const float2 kk = ks2[e >> 1];
+            const uint64_t v = f2mul(f2add(f2pack(__int_as_float(static_cast<int>(u[e]) + 0x4B400000),
+                                                  __int_as_float(static_cast<int>(u[e + 1]) + 0x4B400000)),
+                                           nmagic),
+                                     f2pack(kk.x, kk.y));
+            f2unpack(v, x[e], x[e + 1]);
+          }
         } else {
 #pragma unroll
-          for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(u[e]) * p.scale_log2;
+          for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(u[e]);
         }
       }
+      // scores in log2 units are x * c (INT8 tiles are already scaled)
+      const float c = i8 ? 1.0f : p.scale_log2;
       const int64_t nv64 = lim - static_cast<int64_t>(j) * BN + 1;
       const int nv = nv64 <= 0 ? 0 : (nv64 >= BN ? BN : static_cast<int>(nv64));
       if (!__all_sync(0xffffffffu, nv == BN)) {
@@ -352,39 +379,60 @@ __global__ void __launch_bounds__(384, 1)
       }
       float alpha = 1.f;
       if (nv > 0) {
-        const float mt = row_max<BN>(x);
+        const float mt = row_max<BN>(x) * c;
         if (mt > m_used + 8.0f) {
           alpha = ex2_approx(m_used - mt);
           m_used = mt;
         }
       }
       const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+      const uint64_t c2 = f2pack(c, c);
+      const uint64_t nm2 = f2pack(-msub, -msub);
       uint32_t pk[BN / 2];
-      float acc[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int e = 0; e < BN; e += 2) {
-        const float p0 = ex2_approx(x[e] - msub);
-        const float p1 = ex2_approx(x[e + 1] - msub);
-        acc[(e >> 1) & 7] += p0 + p1;
+        const uint64_t y2 = f2fma(f2pack(x[e], x[e + 1]), c2, nm2);
+        float p0, p1;
+        if (kCacheEmuPairs > 0 && ((e >> 1) & 7) < kCacheEmuPairs) {
+          exp2_poly2(y2, p0, p1);
+        } else {
+          float y0, y1;
+          f2unpack(y2, y0, y1);
+          p0 = ex2_approx(y0);
+          p1 = ex2_approx(y1);
+        }
+        acc2[(e >> 1) & 3] = f2add(acc2[(e >> 1) & 3], f2pack(p0, p1));
         pk[e >> 1] = pack_half2(p0, p1);
       }
-      l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-      if (j > 0) {
+      {
+        const uint64_t s2 = f2add(f2add(acc2[0], acc2[1]), f2add(acc2[2], acc2[3]));
+        float s0, s1;
+        f2unpack(s2, s0, s1);
+        l = l * alpha + (s0 + s1);
+      }
+      // O is rescaled only when a row of this warp raised its running max;
+      // then PV_{j-1} must have completed.  S_j was committed after PV_{j-2}
+      // was issued, so o_done has finished phase j-2 and waiting for phase
+      // j-1 by parity is unambiguous although earlier phases were skipped.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         if (!mbar_wait(bar(K_ODONE), (j - 1) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
         __syncwarp();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          uint32_t o[D];
+        uint32_t o[D];
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
-          tmem_wait_ld();
+        for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
+        tmem_wait_ld();
+        const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
-          for (int e = 0; e < D; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) tmem_st32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
+        for (int e = 0; e < D; e += 2) {
+          float o0, o1;
+          f2unpack(f2mul(f2pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), o0, o1);
+          o[e] = __float_as_uint(o0);
+          o[e + 1] = __float_as_uint(o1);
         }
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) tmem_st32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
       }
       __syncwarp();
 #pragma unroll
