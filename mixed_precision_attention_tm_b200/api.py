@@ -29,7 +29,8 @@ class TileMixPrefill:
         self.int8_cache = int8_cache
         self.device = torch.device(device)
         self.cu = None if cu_seqlens is None else cu_seqlens.to(self.device, torch.int32)
-        cu_h = None if cu_seqlens is None else cu_seqlens.to("cpu", torch.int32)
+        cu_h = None if cu_seqlens is None else cu_seqlens.to("cpu", torch.int32).contiguous()
+        self.cu_h = cu_h
         self.max_seqlen = None if cu_h is None else int((cu_h[1:] - cu_h[:-1]).max())
         dev = self.device
         self.q = torch.empty((Lq, hq, d), dtype=torch.float16, device=dev)
@@ -44,6 +45,20 @@ class TileMixPrefill:
             self.v = torch.empty((Lk, hkv, d), dtype=torch.float16, device=dev)
         self.out = torch.empty((Lq, hq, d), dtype=torch.float16, device=dev)
         self.routed = p is not None
+        self.q_quant = self.k_quant = self.bitmask = None
+        if self.routed:
+            # codes, tile scales and the routing mask: allocated once, rewritten every step
+            cu_np = None if cu_h is None else cu_h.numpy()
+            nqt = ops.count_tiles(Lq, tile_m, cu_np)
+            self.q_quant = (torch.empty((Lq, hq, d), dtype=torch.int8, device=dev),
+                            torch.empty((nqt, hq), dtype=torch.float32, device=dev))
+            if not int8_cache:
+                nkt = ops.count_tiles(Lk, tile_n, cu_np)
+                self.k_quant = (torch.empty((Lk, hkv, d), dtype=torch.int8, device=dev),
+                                torch.empty((nkt, hkv), dtype=torch.float32, device=dev))
+            maxk = Lk if cu_h is None else self.max_seqlen
+            self.bitmask = torch.empty((hq, nqt, ops.mask_words(maxk, tile_n, g)), dtype=torch.int32,
+                                       device=dev)
         self.launches_per_step = 1 + (3 if self.routed and not int8_cache else 2 if self.routed else 0)
 
     # -- inputs -----------------------------------------------------------
@@ -69,19 +84,18 @@ class TileMixPrefill:
 
     # -- the step ---------------------------------------------------------
     def quantize(self):
-        qc, qs, kc, ks = ops.quantize_qk(self.q, None if self.int8_cache else self.k,
-                                         tile_m=self.tile_m, tile_n=self.tile_n, cu_seqlens=self.cu,
-                                         max_seqlen=self.max_seqlen)
-        self.q_quant = (qc, qs)
-        self.k_quant = None if self.int8_cache else (kc, ks)
+        kq = (None, None) if self.k_quant is None else self.k_quant
+        ops.quantize_qk(self.q, None if self.int8_cache else self.k, tile_m=self.tile_m, tile_n=self.tile_n,
+                        cu_seqlens=self.cu, max_seqlen=self.max_seqlen, cu_seqlens_host=self.cu_h,
+                        out=(*self.q_quant, *kq))
 
     def mask(self):
         Lq, Lk = self.shape[0], self.shape[1]
-        self.bitmask = ops.build_mask(self.shape[2], tile_m=self.tile_m, tile_n=self.tile_n, g=self.g,
-                                      causal=self.causal, p=self.p, seed=self.seed,
-                                      force_diag=self.force_diag, force_sink=self.force_sink,
-                                      Lq=Lq, Lk=Lk, cu_seqlens=self.cu, max_seqlen=self.max_seqlen,
-                                      device=self.device)
+        ops.build_mask(self.shape[2], tile_m=self.tile_m, tile_n=self.tile_n, g=self.g,
+                       causal=self.causal, p=self.p, seed=self.seed, force_diag=self.force_diag,
+                       force_sink=self.force_sink, Lq=Lq, Lk=Lk, cu_seqlens=self.cu,
+                       max_seqlen=self.max_seqlen, device=self.device, cu_seqlens_host=self.cu_h,
+                       out=self.bitmask)
 
     def attend(self):
         kv = (self.kc, self.ks, self.vc, self.vs) if self.int8_cache else None
@@ -90,7 +104,7 @@ class TileMixPrefill:
                             bitmask=self.bitmask if self.routed else None,
                             q_quant=self.q_quant if self.routed else None,
                             k_quant=self.k_quant if self.routed else None, kv_cache=kv,
-                            cu_seqlens=self.cu, max_seqlen=self.max_seqlen)
+                            cu_seqlens=self.cu, max_seqlen=self.max_seqlen, cu_seqlens_host=self.cu_h)
 
     def run(self):
         """One prefill step on the resident inputs; returns the device output."""

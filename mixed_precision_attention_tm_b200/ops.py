@@ -123,10 +123,20 @@ def _desc(x, codes=None, scales=None, scale_kind=TM_SCALE_NONE, shape_from=None)
                     None if scales is None else scales.data_ptr(), scale_kind)
 
 
-def _cu_host(cu_seqlens):
+def _cu_host(cu_seqlens, cu_seqlens_host=None):
+    """Host int32 copy of cu_seqlens.  Callers that run many steps pass the
+    host copy they keep (cu_seqlens_host) so no step reads the device array
+    back (a blocking copy)."""
     if cu_seqlens is None:
         return None
+    if cu_seqlens_host is not None:
+        return torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
     return cu_seqlens.detach().to("cpu", torch.int32).contiguous()
+
+
+def _check_buf(t, shape, dtype, name):
+    if t is None or tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise TmError(f"{name}: expected a contiguous {dtype} tensor of shape {tuple(shape)}")
 
 
 def count_tiles(L=None, tile=128, cu_seqlens_host=None):
@@ -142,22 +152,35 @@ def mask_words(max_lk, tile_n, g):
 
 
 # ---------------------------------------------------------------- quantise
-def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqlen=None):
+def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqlen=None,
+                cu_seqlens_host=None, out=None):
     """Per-tile INT8 codes and fp32 scales of Q (tile_m rows) and K (tile_n
     rows): returns (q_codes [Tq,Hq,d] int8, q_scales [n_qt, Hq] fp32,
-    k_codes, k_scales) (the K pair is None when k is None)."""
+    k_codes, k_scales) (the K pair is None when k is None).  out: the same
+    4-tuple of preallocated tensors to write into (reused across steps)."""
     _cuda(q, "q")
     _cuda(k, "k")
     lib = _lib()
-    cu_h = _cu_host(cu_seqlens)
+    cu_h = _cu_host(cu_seqlens, cu_seqlens_host)
     batch = 0 if cu_h is None else cu_h.numel() - 1
     if cu_seqlens is not None and max_seqlen is None:
         max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0
     nqt = count_tiles(q.shape[0], tile_m, None if cu_h is None else cu_h.numpy())
-    qc = torch.empty(q.shape, dtype=torch.int8, device=q.device)
-    qs = torch.empty((nqt, q.shape[1]), dtype=torch.float32, device=q.device)
-    kc = ks = None
-    if k is not None:
+    if out is not None:
+        qc, qs, kc, ks = out
+        _check_buf(qc, q.shape, torch.int8, "q_codes")
+        _check_buf(qs, (nqt, q.shape[1]), torch.float32, "q_scales")
+        if k is None:
+            kc = ks = None
+    else:
+        qc = torch.empty(q.shape, dtype=torch.int8, device=q.device)
+        qs = torch.empty((nqt, q.shape[1]), dtype=torch.float32, device=q.device)
+        kc = ks = None
+    if k is not None and out is not None:
+        nkt = count_tiles(k.shape[0], tile_n, None if cu_h is None else cu_h.numpy())
+        _check_buf(kc, k.shape, torch.int8, "k_codes")
+        _check_buf(ks, (nkt, k.shape[1]), torch.float32, "k_scales")
+    elif k is not None:
         nkt = count_tiles(k.shape[0], tile_n, None if cu_h is None else cu_h.numpy())
         kc = torch.empty(k.shape, dtype=torch.int8, device=k.device)
         ks = torch.empty((nkt, k.shape[1]), dtype=torch.float32, device=k.device)
@@ -172,11 +195,13 @@ def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqle
 
 # ---------------------------------------------------------------- mask
 def build_mask(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False, force_sink=False,
-               Lq=None, Lk=None, cu_seqlens=None, max_seqlen=None, device="cuda"):
+               Lq=None, Lk=None, cu_seqlens=None, max_seqlen=None, device="cuda",
+               cu_seqlens_host=None, out=None):
     """Seeded routing bitmask on the device, int32 view [Hq, n_qt, W] of the
-    uint32 words (bit 1 = INT8)."""
+    uint32 words (bit 1 = INT8).  The library writes every word, so the
+    buffer (out, or a new one) needs no initialisation."""
     lib = _lib()
-    cu_h = _cu_host(cu_seqlens)
+    cu_h = _cu_host(cu_seqlens, cu_seqlens_host)
     batch = 0 if cu_h is None else cu_h.numel() - 1
     if cu_h is not None:
         lens = (cu_h[1:] - cu_h[:-1])
@@ -188,7 +213,10 @@ def build_mask(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False, forc
         maxk = Lk
         nqt = count_tiles(Lq, tile_m)
     W = mask_words(maxk, tile_n, g)
-    out = torch.zeros((Hq, nqt, W), dtype=torch.int32, device=device)
+    if out is None:
+        out = torch.empty((Hq, nqt, W), dtype=torch.int32, device=device)
+    else:
+        _check_buf(out, (Hq, nqt, W), torch.int32, "bitmask")
     st = lib.tm_build_mask(_ptr(out), Hq, _ptr(cu_seqlens), batch, int(max_seqlen or 0),
                            int(Lq or 0), int(Lk or 0), tile_m, tile_n, g, int(bool(causal)),
                            float(p), ctypes.c_uint64(int(seed) & (2 ** 64 - 1)),
@@ -240,7 +268,7 @@ def route_stats(mask_host, *, Hq, tile_m, tile_n, g, causal, Lq=None, Lk=None, c
 # ---------------------------------------------------------------- attention
 def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal=False,
              bitmask=None, mask_head_stride=None, q_quant=None, k_quant=None, kv_cache=None,
-             cu_seqlens=None, max_seqlen=None):
+             cu_seqlens=None, max_seqlen=None, cu_seqlens_host=None):
     """Fused tile-routed attention.  q: fp16 [Tq,Hq,d]; k, v: fp16 [Tk,Hkv,d]
     (or kv_cache = (k_codes, k_scale16, v_codes, v_scale16)); bitmask: int32
     view [Hm, n_qt, W] (Hm = Hq or 1) or None (all FP16); q_quant / k_quant:
@@ -249,7 +277,7 @@ def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal
     lib = _lib()
     if out is None:
         out = torch.empty_like(q)
-    cu_h = _cu_host(cu_seqlens)
+    cu_h = _cu_host(cu_seqlens, cu_seqlens_host)
     batch = 0 if cu_h is None else cu_h.numel() - 1
     if cu_seqlens is not None and max_seqlen is None:
         max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0

@@ -119,3 +119,25 @@ def test_validation_rejects_before_launch():
     # mask builder: p outside [0, 1]
     assert lib.tm_build_mask(ctypes.c_void_p(1 << 20), 2, None, 0, 0, 256, 256, 64, 64, 1, 0, 1.5,
                              ctypes.c_uint64(0), 0, 0, 8, None) == ops.TM_ERR_INVALID_ARG
+
+
+def test_prefill_plan_buffers_match_library_sizes():
+    """The plan preallocates codes, tile scales and the routing mask once; their
+    shapes must be the ones the library writes (tile counts per sequence, mask
+    words from the longest sequence)."""
+    import torch
+    from mixed_precision_attention_tm_b200.api import TileMixPrefill
+    lens = [300, 129, 1000]
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    T = int(cu[-1])
+    pl = TileMixPrefill(T, T, 8, 2, 128, causal=True, tile_m=64, tile_n=128, g=2, p=0.5,
+                        cu_seqlens=cu, device="cpu")
+    nqt = sum(-(-n // 64) for n in lens)
+    nkt = sum(-(-n // 128) for n in lens)
+    assert pl.q_quant[0].shape == (T, 8, 128) and pl.q_quant[1].shape == (nqt, 8)
+    assert pl.k_quant[0].shape == (T, 2, 128) and pl.k_quant[1].shape == (nkt, 2)
+    assert pl.bitmask.shape == (8, nqt, oracle.mask_words(max(lens), 128, 2))
+    cache = TileMixPrefill(T, T, 8, 2, 128, p=0.5, cu_seqlens=cu, int8_cache=True, device="cpu")
+    assert cache.k_quant is None and cache.launches_per_step == 3
+    plain = TileMixPrefill(256, 256, 8, 2, 128, device="cpu")
+    assert plain.bitmask is None and plain.launches_per_step == 1
