@@ -233,23 +233,34 @@ __global__ void __launch_bounds__(384, 1)
         const int cnt = nvc > s ? (nvc - 1 - s) / C::NVC + 1 : 0;
         if (cnt > 0) mbar_wait(bar(K_VCFULL + s), (cnt - 1) & 1, p.err, &never);
       }
-    } else if (warp == 9 && lane == 0 && nJ > 0) {
+    } else if (warp == 9 && nJ > 0) {
       // ======================= tcgen05 issuer =======================
-      bool ok = mbar_wait(bar(K_QFULL), 0, p.err, abort_flag);
+      // Whole warp: descriptors are warp-uniform values built ahead of each
+      // group; one elected lane issues the group and its commits.
+      bool ok = mbar_wait_warp(bar(K_QFULL), 0, p.err, abort_flag);
       int n16 = 0;
+      auto commit1 = [&](uint32_t b) {
+        if (elect_one()) tc_commit(b);
+        __syncwarp();
+      };
       auto issue_pv = [&](int t) -> bool {
-        if (!mbar_wait(bar(K_PFULL + (t & 1)), (t >> 1) & 1, p.err, abort_flag)) return false;
         const int vs = t % C::NV16;
-        if (!mbar_wait(bar(K_V16FULL + vs), (t / C::NV16) & 1, p.err, abort_flag)) return false;
-        tc_fence_after();
         const uint32_t vb = sbase + C::OFF_V16 + vs * C::F16;
-        const uint32_t a_tmem = tmem + static_cast<uint32_t>(t & 1) * BN;
+        uint64_t bd[BN / 16];
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_f16_ts(tmem + C::O_COL, a_tmem + kk * 8, smem_desc(vb + kk * 2048, C::HALF, 1024, kSwizzle128),
-                     C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(K_ODONE));
-        tc_commit(bar(K_V16EMPTY + vs));
+        for (int kk = 0; kk < BN / 16; ++kk) bd[kk] = smem_desc(vb + kk * 2048, C::HALF, 1024, kSwizzle128);
+        if (!mbar_wait_warp(bar(K_PFULL + (t & 1)), (t >> 1) & 1, p.err, abort_flag)) return false;
+        if (!mbar_wait_warp(bar(K_V16FULL + vs), (t / C::NV16) & 1, p.err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t a_tmem = tmem + static_cast<uint32_t>(t & 1) * BN;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_f16_ts(tmem + C::O_COL, a_tmem + kk * 8, bd[kk], C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(K_ODONE));
+          tc_commit(bar(K_V16EMPTY + vs));
+        }
+        __syncwarp();
         return true;
       };
       for (int j = 0; ok && j < nJ; ++j) {
@@ -257,35 +268,48 @@ __global__ void __launch_bounds__(384, 1)
         const int s = j % C::NKC;
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
         if (i8) {
-          if (!(ok = mbar_wait(bar(K_KCFULL + s), (j / C::NKC) & 1, p.err, abort_flag))) break;
           const uint32_t kb = sbase + C::OFF_KC + s * C::C8;
+          uint64_t ad[D / 32], bd[D / 32];
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk)
-            mma_i8_ss(d_tmem, smem_desc(sbase + C::OFF_Q8 + kk * 32, 16, 1024, kSwizzle128),
-                      smem_desc(kb + kk * 32, 16, 1024, kSwizzle128), C::IDESC_S8, kk > 0 ? 1u : 0u);
-          tc_commit(bar(K_SFULL + (j & 1)));
+          for (int kk = 0; kk < D / 32; ++kk) {
+            ad[kk] = smem_desc(sbase + C::OFF_Q8 + kk * 32, 16, 1024, kSwizzle128);
+            bd[kk] = smem_desc(kb + kk * 32, 16, 1024, kSwizzle128);
+          }
+          if (!(ok = mbar_wait_warp(bar(K_KCFULL + s), (j / C::NKC) & 1, p.err, abort_flag))) break;
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < D / 32; ++kk) mma_i8_ss(d_tmem, ad[kk], bd[kk], C::IDESC_S8, kk > 0 ? 1u : 0u);
+            tc_commit(bar(K_SFULL + (j & 1)));
+          }
+          __syncwarp();
         } else {
           const int s16 = n16 % C::NK16;
-          if (!(ok = mbar_wait(bar(K_K16FULL + s16), (n16 / C::NK16) & 1, p.err, abort_flag))) break;
-          tc_fence_after();   // dequantised tile written by the generic proxy, fenced by its writers
           const uint32_t kb = sbase + C::OFF_K16 + s16 * C::F16;
+          uint64_t ad[D / 16], bd[D / 16];
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::HALF + (kk & 3) * 32;
-            mma_f16_ss(d_tmem, smem_desc(sbase + C::OFF_Q16 + off, 16, 1024, kSwizzle128),
-                       smem_desc(kb + off, 16, 1024, kSwizzle128), C::IDESC_S16, kk > 0 ? 1u : 0u);
+            ad[kk] = smem_desc(sbase + C::OFF_Q16 + off, 16, 1024, kSwizzle128);
+            bd[kk] = smem_desc(kb + off, 16, 1024, kSwizzle128);
           }
-          tc_commit(bar(K_SFULL + (j & 1)));
-          tc_commit(bar(K_K16EMPTY + s16));
+          if (!(ok = mbar_wait_warp(bar(K_K16FULL + s16), (n16 / C::NK16) & 1, p.err, abort_flag))) break;
+          tc_fence_after();   // dequantised tile written by the generic proxy, fenced by its writers
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) mma_f16_ss(d_tmem, ad[kk], bd[kk], C::IDESC_S16, kk > 0 ? 1u : 0u);
+            tc_commit(bar(K_SFULL + (j & 1)));
+            tc_commit(bar(K_K16EMPTY + s16));
+          }
+          __syncwarp();
           ++n16;
         }
-        tc_commit(bar(K_KCEMPTY + s));
+        commit1(bar(K_KCEMPTY + s));
         if (j >= 1 && !(ok = issue_pv(j - 1))) break;
       }
       if (ok) issue_pv(nJ - 1);
-      tc_commit(bar(K_DRAIN));
+      commit1(bar(K_DRAIN));
       volatile int never = 0;
-      mbar_wait(bar(K_DRAIN), 0, p.err, &never);
+      mbar_wait_warp(bar(K_DRAIN), 0, p.err, &never);
     }
   } else if (warp >= 4) {
     // ======================= dequantisation (one key row per thread) ==========
@@ -413,12 +437,18 @@ __global__ void __launch_bounds__(384, 1)
       }
       // O is rescaled only when a row of this warp raised its running max;
       // then PV_{j-1} must have completed.  S_j was committed after PV_{j-2}
-      // was issued, so o_done has finished phase j-2 and waiting for phase
-      // j-1 by parity is unambiguous although earlier phases were skipped.
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      // was issued, so o_done has finished phase j-2, and PV_j cannot start
+      // before this warp releases P_j: waiting for phase j-1 by parity is
+      // unambiguous although earlier phases were skipped.  The last tile
+      // always waits, so that the epilogue's wait for phase nJ-1 can only
+      // see phase nJ-1 or nJ (parity alone cannot tell nJ-2 from nJ).
+      const bool rescale = j > 0 && __any_sync(0xffffffffu, alpha != 1.f);
+      if (j > 0 && (rescale || j == nJ - 1)) {
         if (!mbar_wait(bar(K_ODONE), (j - 1) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
         __syncwarp();
+      }
+      if (rescale) {
         uint32_t o[D];
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
