@@ -55,7 +55,8 @@ namespace {
 enum : unsigned {
   EV_S_READY = 1, EV_EXP_DONE = 2, EV_O_READY = 3, EV_RESCALED = 4, EV_P_RELEASED = 5, EV_EPI_DONE = 6,
   EV_ACQUIRED = 10, EV_K_READY = 20, EV_PV_A = 21, EV_S_A = 22, EV_PV_B = 23, EV_S_B = 24, EV_V_READY = 25,
-  EV_START = 30, EV_KWAIT_BEGIN = 31, EV_KWAIT_END = 32, EV_VWAIT_BEGIN = 33, EV_SLOADED = 7, EV_MAXED = 8
+  EV_START = 30, EV_KWAIT_BEGIN = 31, EV_KWAIT_END = 32, EV_VWAIT_BEGIN = 33, EV_SLOADED = 7, EV_MAXED = 8,
+  EV_P_SEEN = 26, EV_MMA_ISSUED = 27
 };
 
 template <int D>
@@ -323,94 +324,172 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 9) {
     // ======================= tcgen05 issuer =======================
-    if (lane == 0 && nJ > 0) {
+    // The issuing warp never touches shared memory inside its loop: on this
+    // SM a barrier poll (or any shared-memory access) by the thread that
+    // issues tcgen05.mma holds back its next MMA for ~200 cycles while the
+    // MMAs saturate the shared-memory port, and the MMA queue is too short to
+    // cover that.  Every mbarrier wait is made by the wait helper (warp 10),
+    // which then meets this warp at named barrier 1; the two walk the same
+    // sequence of handoffs.  Routing words are kept in registers.  One
+    // elected lane issues each group of MMAs and its commits.
+    if (nJ > 0) {
       TM_TRACE_DECL
-      TM_TRACE_EV(3, EV_START);
-      bool ok = mbar_wait(bar(C_QFULL), 0, p.err, abort_flag);
+      const bool tracer = lane == 0;
+      if (tracer) TM_TRACE_EV(3, EV_START);
+      auto handoff = [&]() { named_bar_sync(1, 64); };
+      handoff();   // Q tiles landed
       uint32_t n = 0;
-      auto take = [&](uint32_t& slot, uint32_t& par) {
+      auto take = [&](uint32_t& slot) {
         slot = n % C::NSLOT;
-        par = (n / C::NSLOT) & 1;
         ++n;
+      };
+      int wwin = -1;
+      uint32_t rw0 = 0, rw1 = 0;
+      auto route_reg = [&](int j, bool& r0, bool& r1, bool& n16, bool& n8) {
+        const bool a = j < nJA, c = j < nJB;
+        const int G = j / p.g;
+        if ((G >> 5) != wwin) {   // one shared-memory read per 32 routing groups
+          wwin = G >> 5;
+          rw0 = rrow[0] != nullptr ? rrow[0][wwin] : 0u;
+          rw1 = rrow[1] != nullptr ? rrow[1][wwin] : 0u;
+        }
+        r0 = a && ((rw0 >> (G & 31)) & 1u);
+        r1 = c && ((rw1 >> (G & 31)) & 1u);
+        n16 = (a && !r0) || (c && !r1);
+        n8 = r0 || r1;
       };
       auto issue_s = [&](int t, bool i8, uint32_t kslot) {
         const uint32_t d_tmem = tmem + C::s_col(t);
         const uint32_t kb = sbase + C::OFF_SLOT + kslot * C::SLOT;
         if (i8) {
           const uint32_t qa = sbase + C::OFF_Q8 + t * C::Q8_BYTES;
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk)
-            mma_i8_ss(d_tmem, smem_desc(qa + kk * 32, 16, C::SBO8, C::SW8),
-                      smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8), C::IDESC_S8, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 32; ++kk)
+              mma_i8_ss(d_tmem, smem_desc(qa + kk * 32, 16, C::SBO8, C::SW8),
+                        smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8), C::IDESC_S8, kk > 0 ? 1u : 0u);
+            tc_commit(bar(C_SFULL + t));
+          }
         } else {
           const uint32_t qa = sbase + C::OFF_Q16 + t * C::Q16_BYTES;
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::HALF + (kk & 3) * 32;
-            mma_f16_ss(d_tmem, smem_desc(qa + off, 16, 1024, kSwizzle128),
-                       smem_desc(kb + off, 16, 1024, kSwizzle128), C::IDESC_S16, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::HALF + (kk & 3) * 32;
+              mma_f16_ss(d_tmem, smem_desc(qa + off, 16, 1024, kSwizzle128),
+                         smem_desc(kb + off, 16, 1024, kSwizzle128), C::IDESC_S16, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(C_SFULL + t));
           }
         }
-        tc_commit(bar(C_SFULL + t));
+        __syncwarp();
       };
-      auto issue_pv = [&](int t, int jj, uint32_t vslot) -> bool {
-        if (!mbar_wait(bar(C_PFULL + t), jj & 1, p.err, abort_flag)) return false;
+      auto issue_pv = [&](int t, int jj, uint32_t vslot) {
+        handoff();          // softmax t released P_t(jj)
+        if (tracer) TM_TRACE_EV(3, EV_P_SEEN);
         tc_fence_after();   // orders the softmax warps' TMEM stores of P before the MMA reads it
         const uint32_t vb = sbase + C::OFF_SLOT + vslot * C::SLOT;
         const uint32_t a_tmem = tmem + C::s_col(t);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_f16_ts(tmem + C::o_col(t), a_tmem + kk * 8, smem_desc(vb + kk * 2048, C::HALF, 1024, kSwizzle128),
-                     C::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(C_ODONE + t));
-        return true;
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            mma_f16_ts(tmem + C::o_col(t), a_tmem + kk * 8, smem_desc(vb + kk * 2048, C::HALF, 1024, kSwizzle128),
+                       C::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+#ifdef TM_TRACE_MMA
+            TM_TRACE_EV(3, EV_MMA_ISSUED);
+#endif
+          }
+          tc_commit(bar(C_ODONE + t));
+        }
+        __syncwarp();
+      };
+      auto commit1 = [&](uint32_t b) {
+        if (elect_one()) tc_commit(b);
+        __syncwarp();
       };
       uint32_t v_prev = 0;
-      for (int j = 0; ok && j < nJ; ++j) {
+      for (int j = 0; j < nJ; ++j) {
         bool r0, r1, n16, n8;
-        needs(j, r0, r1, n16, n8);
+        route_reg(j, r0, r1, n16, n8);
         // P.V of tile A for the previous key tile first: its operands (P_A,
         // V) are ready as soon as softmax A releases P, and the wait for this
-        // key tile's K below then overlaps its execution.
-        if (j > 0 && j - 1 < nJA && !(ok = issue_pv(0, j - 1, v_prev))) break;
-        TM_TRACE_EV(3, EV_PV_A);
-        uint32_t s16 = 0, s8 = 0, sv = 0, par;
-        TM_TRACE_EV(3, EV_KWAIT_BEGIN);
-        if (n16) {
-          take(s16, par);
-          if (!(ok = mbar_wait(bar(C_FULL + s16), par, p.err, abort_flag))) break;
-        }
-        if (n8) {
-          take(s8, par);
-          if (!(ok = mbar_wait(bar(C_FULL + s8), par, p.err, abort_flag))) break;
-        }
-        take(sv, par);
-        const uint32_t v_par = par;
-        TM_TRACE_EV(3, EV_KWAIT_END);
-        TM_TRACE_EV(3, EV_K_READY);
+        // key tile's K then overlaps its execution.
+        if (j > 0 && j - 1 < nJA) issue_pv(0, j - 1, v_prev);
+        if (tracer) TM_TRACE_EV(3, EV_PV_A);
+        uint32_t s16 = 0, s8 = 0, sv = 0;
+        if (n16) take(s16);
+        if (n8) take(s8);
+        take(sv);
+        handoff();   // K tiles of j landed
+        if (tracer) TM_TRACE_EV(3, EV_K_READY);
         if (j < nJA) issue_s(0, r0, r0 ? s8 : s16);
-        TM_TRACE_EV(3, EV_S_A);
-        if (j > 0 && j - 1 < nJB && !(ok = issue_pv(1, j - 1, v_prev))) break;
-        TM_TRACE_EV(3, EV_PV_B);
-        if (j > 0) tc_commit(bar(C_EMPTY + v_prev));
+        if (tracer) TM_TRACE_EV(3, EV_S_A);
+        if (j > 0 && j - 1 < nJB) issue_pv(1, j - 1, v_prev);
+        if (tracer) TM_TRACE_EV(3, EV_PV_B);
+        if (j > 0) commit1(bar(C_EMPTY + v_prev));
         if (j < nJB) issue_s(1, r1, r1 ? s8 : s16);
-        TM_TRACE_EV(3, EV_S_B);
-        if (n16) tc_commit(bar(C_EMPTY + s16));
-        if (n8) tc_commit(bar(C_EMPTY + s8));
-        TM_TRACE_EV(3, EV_VWAIT_BEGIN);
-        // V of this tile must have landed before its P.V is issued next round
-        if (!(ok = mbar_wait(bar(C_FULL + sv), v_par, p.err, abort_flag))) break;
-        TM_TRACE_EV(3, EV_V_READY);
+        if (tracer) TM_TRACE_EV(3, EV_S_B);
+        if (n16) commit1(bar(C_EMPTY + s16));
+        if (n8) commit1(bar(C_EMPTY + s8));
+        handoff();   // V of j landed (its P.V is issued next round)
+        if (tracer) TM_TRACE_EV(3, EV_V_READY);
         v_prev = sv;
       }
-      if (ok) {
-        if (nJ - 1 < nJA) ok = issue_pv(0, nJ - 1, v_prev);
-        if (ok && nJ - 1 < nJB) ok = issue_pv(1, nJ - 1, v_prev);
-        tc_commit(bar(C_EMPTY + v_prev));
+      if (nJ - 1 < nJA) issue_pv(0, nJ - 1, v_prev);
+      if (nJ - 1 < nJB) issue_pv(1, nJ - 1, v_prev);
+      commit1(bar(C_EMPTY + v_prev));
+      commit1(bar(C_DRAIN));
+      if (lane == 0) {
+        volatile int never = 0;
+        mbar_wait(bar(C_DRAIN), 0, p.err, &never);
       }
-      tc_commit(bar(C_DRAIN));
-      volatile int never = 0;
-      mbar_wait(bar(C_DRAIN), 0, p.err, &never);
+      __syncwarp();
+    }
+  } else if (warp == 10) {
+    // ======================= wait helper =======================
+    // Makes the issuer's mbarrier waits (operands landed, P released) in the
+    // issuer's order and meets it at named barrier 1 after each.  A wait that
+    // times out or sees the abort flag only records the failure: the helper
+    // still takes every handoff, so neither warp is left at the barrier, and
+    // the issuer's remaining MMAs run on stale operands whose results the
+    // failed launch discards.
+    if (nJ > 0) {
+      auto wait1 = [&](uint32_t b, uint32_t par) {
+        if (lane == 0) mbar_wait(b, par, p.err, abort_flag);
+      };
+      auto handoff = [&]() {
+        __syncwarp();
+        named_bar_sync(1, 64);
+      };
+      auto wait_p = [&](int t, int jj) {   // P_t(jj) released
+        wait1(bar(C_PFULL + t), jj & 1);
+        handoff();
+      };
+      wait1(bar(C_QFULL), 0);
+      handoff();
+      uint32_t n = 0;
+      auto take = [&](uint32_t& slot, uint32_t& par) {
+        slot = n % C::NSLOT;
+        par = (n / C::NSLOT) & 1;
+        ++n;
+      };
+      for (int j = 0; j < nJ; ++j) {
+        bool r0, r1, n16, n8;
+        needs(j, r0, r1, n16, n8);
+        if (j > 0 && j - 1 < nJA) wait_p(0, j - 1);
+        uint32_t s16 = 0, s8 = 0, sv = 0, par16 = 0, par8 = 0, parv = 0;
+        if (n16) take(s16, par16);
+        if (n8) take(s8, par8);
+        take(sv, parv);
+        if (n16) wait1(bar(C_FULL + s16), par16);
+        if (n8) wait1(bar(C_FULL + s8), par8);
+        handoff();
+        if (j > 0 && j - 1 < nJB) wait_p(1, j - 1);
+        wait1(bar(C_FULL + sv), parv);
+        handoff();
+      }
+      if (nJ - 1 < nJA) wait_p(0, nJ - 1);
+      if (nJ - 1 < nJB) wait_p(1, nJ - 1);
     }
    }
   } else {
@@ -432,7 +511,10 @@ __global__ void __launch_bounds__(384, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     TM_TRACE_DECL
-    const bool tracer = (threadIdx.x & 127) == 0;
+#ifndef TM_TRACE_WARP
+#define TM_TRACE_WARP 0
+#endif
+    const bool tracer = (threadIdx.x & 127) == 32 * TM_TRACE_WARP;
     if (tracer) TM_TRACE_EV(t, EV_START);
     for (int j = 0; j < T.nJ; ++j) {
       const bool i8 = route8(rrow[t], p.g, j);

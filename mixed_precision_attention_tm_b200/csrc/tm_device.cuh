@@ -156,6 +156,19 @@ __device__ __forceinline__ bool mbar_spin(uint32_t bar, uint32_t parity, const D
   }
 }
 
+// True in exactly one lane of a converged warp (elect.sync: the same lane
+// every time for a full mask, so the tcgen05 operations it issues and their
+// commits come from one thread).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Warp-cooperative wait: lane 0 polls, the other lanes wait at __syncwarp and
 // then confirm with one try_wait each (so every lane observes the phase with
 // acquire semantics).  Keeps 31 of 32 threads off the shared-memory barrier
