@@ -19,7 +19,7 @@
 //               from TMEM, int32 -> fp32 and dequantisation by
 //               s_q * s_k * sigma for INT8 tiles, causal / ragged masking,
 //               online max / sum with a lazy rescale of O (only when the row
-//               max grows by more than 2^8), P rounded to fp16 and written back
+//               max grows by more than 2^15), P rounded to fp16 and written back
 //               over S in TMEM, and the final O / l epilogue.
 // Every mbarrier wait is bounded (tm_device.cuh).
 #include <cuda.h>
@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(192, 1)
       float alpha = 1.f;
       if (nv > 0) {
         const float mt = row_max<BN>(x) * c;
-        if (mt > m_used + 8.0f) {           // lazy rescale: only when the max grows by > 2^8
+        if (mt > m_used + kLazyRescaleLog2) {   // lazy rescale
           alpha = ex2_approx(m_used - mt);
           m_used = mt;
         }

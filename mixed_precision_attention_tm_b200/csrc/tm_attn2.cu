@@ -48,6 +48,20 @@ extern "C" int tm_debug_trace_read(unsigned long long* host, unsigned int block)
 }
 #endif
 
+
+// Softmax phase profile (compiled only with TM_PHASES, together with
+// TM_TRACE): the tracing thread sums SM-clock deltas per phase in registers
+// and stores the sums once, so the profile costs a few cycles per phase.
+#ifdef TM_PHASES
+#define TM_SM_EV(ev) do { } while (0)
+#define TM_PH_DECL long long tm_ph[8] = {0, 0, 0, 0, 0, 0, 0, 0}; long long tm_ph_t = clock64();
+#define TM_PH(i) do { const long long tm_now = clock64(); tm_ph[i] += tm_now - tm_ph_t; tm_ph_t = tm_now; } while (0)
+#else
+#define TM_SM_EV(ev) do { if (tracer) TM_TRACE_EV(t, ev); } while (0)
+#define TM_PH_DECL
+#define TM_PH(i) do { } while (0)
+#endif
+
 namespace tmk {
 namespace {
 
@@ -56,7 +70,8 @@ enum : unsigned {
   EV_S_READY = 1, EV_EXP_DONE = 2, EV_O_READY = 3, EV_RESCALED = 4, EV_P_RELEASED = 5, EV_EPI_DONE = 6,
   EV_ACQUIRED = 10, EV_K_READY = 20, EV_PV_A = 21, EV_S_A = 22, EV_PV_B = 23, EV_S_B = 24, EV_V_READY = 25,
   EV_START = 30, EV_KWAIT_BEGIN = 31, EV_KWAIT_END = 32, EV_VWAIT_BEGIN = 33, EV_SLOADED = 7, EV_MAXED = 8,
-  EV_P_SEEN = 26, EV_MMA_ISSUED = 27
+  EV_P_SEEN = 26, EV_MMA_ISSUED = 27, EV_HW_KV_BEGIN = 40, EV_HW_KV_END = 41, EV_HW_P_BEGIN = 42,
+  EV_HW_P_END = 43
 };
 
 template <int D>
@@ -95,13 +110,18 @@ struct Cfg2 {
 enum {
   C_QFULL = 0,
   C_SFULL = 1,   // +2 (tile A, B)
-  C_PFULL = 3,   // +2
-  C_ODONE = 5,   // +2
-  C_DRAIN = 7,
-  C_FULL = 8,    // +NSLOT (<= 8)
-  C_EMPTY = 16,  // +NSLOT
-  C_COUNT = 24
+  C_ODONE = 3,   // +2
+  C_DRAIN = 5,   // +2 (one per issuer)
+  C_PFULL = 7,   // +2: P_t stored (single-issuer mode; count 128)
+  C_FULL = 9,    // +NSLOT (<= 8)
+  C_EMPTY = 17,  // +NSLOT; one release per issuer that reads the slot's tiles
+  C_COUNT = 25
 };
+// Named barriers (0 is __syncthreads):
+//   NB_P + t:  softmax warpgroup t (128, arrive) -> issuer t (32, sync): P_t stored
+//   NB_KV + t: wait helper (32) <-> issuer t (32): operands landed
+//   NB_START: softmax A (128, arrive) -> issuer B (32, sync), once: P_A(0) stored
+enum : int { NB_P = 1, NB_KV = 3, NB_START = 5 };
 
 struct Params2 {
   __half* out;
@@ -135,7 +155,7 @@ struct TileInfo {
   const uint32_t* mrow;
 };
 
-template <int D, int EMU>
+template <int D, int EMU, bool DUAL>
 __global__ void __launch_bounds__(384, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmQ8,
                      const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmK8,
@@ -210,13 +230,13 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar(C_QFULL), 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(C_SFULL + t), 1);
-      mbar_init(bar(C_PFULL + t), 128);
       mbar_init(bar(C_ODONE + t), 1);
+      mbar_init(bar(C_DRAIN + t), 1);
+      mbar_init(bar(C_PFULL + t), 128);
     }
-    mbar_init(bar(C_DRAIN), 1);
     for (int s = 0; s < C::NSLOT; ++s) {
       mbar_init(bar(C_FULL + s), 1);
-      mbar_init(bar(C_EMPTY + s), 1);
+      mbar_init(bar(C_EMPTY + s), DUAL ? 2 : 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -255,8 +275,10 @@ __global__ void __launch_bounds__(384, 1)
    if (warp == 8) {
     // ======================= TMA producer =======================
     if (lane == 0 && nJ > 0) {
+#ifndef TM_TRACE_HELPER
       TM_TRACE_DECL
       TM_TRACE_EV(2, EV_START);
+#endif
       bool any8[2] = {false, false};
 #pragma unroll
       for (int t = 0; t < 2; ++t)
@@ -287,7 +309,9 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t lap = n / C::NSLOT;
         if (lap > 0 && !mbar_wait(bar(C_EMPTY + slot), (lap - 1) & 1, p.err, abort_flag)) return false;
         ++n;
+#ifndef TM_TRACE_HELPER
         TM_TRACE_EV(2, EV_ACQUIRED);
+#endif
         return true;
       };
       bool ok = true;
@@ -322,7 +346,193 @@ __global__ void __launch_bounds__(384, 1)
       for (uint32_t i = (n > C::NSLOT ? n - C::NSLOT : 0); i < n; ++i)
         mbar_wait(bar(C_FULL + i % C::NSLOT), (i / C::NSLOT) & 1, p.err, &never);
     }
-  } else if (warp == 9) {
+   } else if (DUAL) {
+   if (warp == 9 || warp == 10) {
+    // ======================= tcgen05 issuers (warp 9: tile A, warp 10: tile B) ====
+    // One issuing warp per query tile, so that neither tile's P.V and next
+    // S wait behind the other tile's MMAs.  An issuing warp never touches
+    // shared memory inside its loop: on this SM a barrier poll (or any
+    // shared-memory access) by the thread that issues tcgen05.mma holds back
+    // its next MMA by ~200 cycles while the MMAs saturate the shared-memory
+    // port, and the MMA queue is too short to cover that.  It learns that P
+    // is stored from its softmax warpgroup at named barrier NB_P + t, and
+    // that K / V landed from the wait helper at NB_KV + t.  One elected lane
+    // issues each group of MMAs and its commits.  Each ring slot is released
+    // by two commits (one per query tile); a tile past its last key tile
+    // leaves its share to the other tile's issuer.
+    const int t = warp - 9;
+    const int nJt = t == 0 ? nJA : nJB;
+    const int nJo = t == 0 ? nJB : nJA;
+    if (nJt > 0) {
+      TM_TRACE_DECL
+      const bool tracer = lane == 0 && t == 0;
+      if (tracer) TM_TRACE_EV(3, EV_START);
+      auto kv_handoff = [&]() { named_bar_sync(NB_KV + t, 64); };
+      auto p_handoff = [&]() { named_bar_sync(NB_P + t, 160); };
+      kv_handoff();   // Q tiles landed
+      uint32_t n = 0;
+      auto take = [&](uint32_t& slot) {
+        slot = n % C::NSLOT;
+        ++n;
+      };
+      int wwin = -1;
+      uint32_t rw0 = 0, rw1 = 0;
+      auto route_reg = [&](int j, bool& r0, bool& r1, bool& n16, bool& n8) {
+        const bool a = j < nJA, c = j < nJB;
+        const int G = j / p.g;
+        if ((G >> 5) != wwin) {   // one shared-memory read per 32 routing groups
+          wwin = G >> 5;
+          rw0 = rrow[0] != nullptr ? rrow[0][wwin] : 0u;
+          rw1 = rrow[1] != nullptr ? rrow[1][wwin] : 0u;
+        }
+        r0 = a && ((rw0 >> (G & 31)) & 1u);
+        r1 = c && ((rw1 >> (G & 31)) & 1u);
+        n16 = (a && !r0) || (c && !r1);
+        n8 = r0 || r1;
+      };
+      // release a ring slot: this tile's share, plus the other tile's when
+      // that tile has no key tile jj
+      auto release = [&](uint32_t slot, int jj) {
+        if (elect_one()) {
+          tc_commit(bar(C_EMPTY + slot));
+          if (jj >= nJo) tc_commit(bar(C_EMPTY + slot));
+        }
+        __syncwarp();
+      };
+      const uint32_t d_s = tmem + C::s_col(t), d_o = tmem + C::o_col(t);
+      auto issue_s = [&](bool i8, uint32_t kslot) {
+        const uint32_t kb = sbase + C::OFF_SLOT + kslot * C::SLOT;
+        if (i8) {
+          const uint32_t qa = sbase + C::OFF_Q8 + t * C::Q8_BYTES;
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < D / 32; ++kk)
+              mma_i8_ss(d_s, smem_desc(qa + kk * 32, 16, C::SBO8, C::SW8),
+                        smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8), C::IDESC_S8, kk > 0 ? 1u : 0u);
+            tc_commit(bar(C_SFULL + t));
+          }
+        } else {
+          const uint32_t qa = sbase + C::OFF_Q16 + t * C::Q16_BYTES;
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::HALF + (kk & 3) * 32;
+              mma_f16_ss(d_s, smem_desc(qa + off, 16, 1024, kSwizzle128),
+                         smem_desc(kb + off, 16, 1024, kSwizzle128), C::IDESC_S16, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(C_SFULL + t));
+          }
+        }
+        __syncwarp();
+      };
+      auto issue_pv = [&](int jj, uint32_t vslot) {
+        p_handoff();        // softmax t stored P_t(jj)
+        if (tracer) TM_TRACE_EV(3, EV_P_SEEN);
+        tc_fence_after();   // orders the softmax warps' TMEM stores of P before the MMA reads it
+        const uint32_t vb = sbase + C::OFF_SLOT + vslot * C::SLOT;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_f16_ts(d_o, d_s + kk * 8, smem_desc(vb + kk * 2048, C::HALF, 1024, kSwizzle128), C::IDESC_PV,
+                       (jj > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(C_ODONE + t));
+        }
+        __syncwarp();
+        release(vslot, jj);
+      };
+      uint32_t v_prev = 0;
+      for (int j = 0; j < nJt; ++j) {
+        bool r0, r1, n16, n8;
+        route_reg(j, r0, r1, n16, n8);
+        uint32_t s16 = 0, s8 = 0, sv = 0;
+        if (n16) take(s16);
+        if (n8) take(s8);
+        take(sv);
+        kv_handoff();   // K tiles of j (and V of j-1) landed
+        // P.V of the previous key tile first (S_t(j) overwrites P_t(j-1))
+        if (j > 0) issue_pv(j - 1, v_prev);
+        if (tracer) TM_TRACE_EV(3, EV_K_READY);
+        const bool r = t == 0 ? r0 : r1;
+        // Tile B starts half a period behind tile A: its first S waits until
+        // softmax A has stored P_A(0), so that the two tiles' softmax and
+        // MMA phases alternate instead of running in lockstep.  (This waits
+        // only on S_A(0); nothing it waits for depends on tile B.)
+        if (t == 1 && j == 0 && nJA > 0) named_bar_sync(NB_START, 160);
+        issue_s(r, r ? s8 : s16);
+        if (tracer) TM_TRACE_EV(3, EV_S_A);
+        if (n16) release(s16, j);
+        if (n8) release(s8, j);
+        v_prev = sv;
+      }
+      kv_handoff();   // V of the last key tile landed
+      issue_pv(nJt - 1, v_prev);
+      if (elect_one()) tc_commit(bar(C_DRAIN + t));
+      __syncwarp();
+      if (lane == 0) {
+        volatile int never = 0;
+        mbar_wait(bar(C_DRAIN + t), 0, p.err, &never);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 11) {
+    // ======================= wait helper =======================
+    // Makes both issuers' operand waits (Q, then per key tile j: K of j and
+    // V of j-1, then the last V) and meets issuer t at named barrier
+    // NB_KV + t after each, tile A's handoff of a round before tile B's.  A
+    // wait that times out or sees the abort flag only records the failure:
+    // the helper still takes every handoff, so no warp is left at a barrier,
+    // and the remaining MMAs run on stale operands of a launch that reports
+    // the error.
+    if (nJ > 0) {
+#ifdef TM_TRACE_HELPER
+      TM_TRACE_DECL
+#endif
+      auto wait1 = [&](uint32_t b, uint32_t par) {
+#ifdef TM_TRACE_HELPER
+        if (lane == 0) TM_TRACE_EV(2, EV_HW_KV_BEGIN);
+#endif
+        if (lane == 0) mbar_wait(b, par, p.err, abort_flag);
+#ifdef TM_TRACE_HELPER
+        if (lane == 0) TM_TRACE_EV(2, EV_HW_KV_END);
+#endif
+      };
+      auto handoff = [&](int t) {
+        __syncwarp();
+        named_bar_sync(NB_KV + t, 64);
+      };
+      wait1(bar(C_QFULL), 0);
+      if (nJA > 0) handoff(0);
+      if (nJB > 0) handoff(1);
+      uint32_t n = 0;
+      auto take = [&](uint32_t& slot, uint32_t& par) {
+        slot = n % C::NSLOT;
+        par = (n / C::NSLOT) & 1;
+        ++n;
+      };
+      uint32_t sv_prev = 0, pv_prev = 0;
+      for (int j = 0; j < nJ; ++j) {
+        bool r0, r1, n16, n8;
+        needs(j, r0, r1, n16, n8);
+        uint32_t s16 = 0, s8 = 0, sv = 0, par16 = 0, par8 = 0, parv = 0;
+        if (n16) take(s16, par16);
+        if (n8) take(s8, par8);
+        take(sv, parv);
+        if (j > 0) wait1(bar(C_FULL + sv_prev), pv_prev);
+        if (n16) wait1(bar(C_FULL + s16), par16);
+        if (n8) wait1(bar(C_FULL + s8), par8);
+        if (j < nJA) handoff(0);
+        if (j < nJB) handoff(1);
+        // after a tile's last key tile: the V of that key tile
+        if (j == nJA - 1 || j == nJB - 1) wait1(bar(C_FULL + sv), parv);
+        if (j == nJA - 1) handoff(0);
+        if (j == nJB - 1) handoff(1);
+        sv_prev = sv;
+        pv_prev = parv;
+      }
+    }
+   }
+   } else {
+   if (warp == 9) {
     // ======================= tcgen05 issuer =======================
     // The issuing warp never touches shared memory inside its loop: on this
     // SM a barrier poll (or any shared-memory access) by the thread that
@@ -492,6 +702,7 @@ __global__ void __launch_bounds__(384, 1)
       if (nJ - 1 < nJB) wait_p(1, nJ - 1);
     }
    }
+   }
   } else {
     // ======================= softmax (warpgroup t = tile t) =======================
     regs_inc<C::SOFTMAX_REGS>();
@@ -515,14 +726,18 @@ __global__ void __launch_bounds__(384, 1)
 #define TM_TRACE_WARP 0
 #endif
     const bool tracer = (threadIdx.x & 127) == 32 * TM_TRACE_WARP;
-    if (tracer) TM_TRACE_EV(t, EV_START);
+    TM_SM_EV(EV_START);
+    TM_PH_DECL
     for (int j = 0; j < T.nJ; ++j) {
       const bool i8 = route8(rrow[t], p.g, j);
       float c = p.scale_log2;
       if (i8) c = fmaxf(c8_row * __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk), 1e-30f);
-      if (!mbar_wait(bar(C_SFULL + t), j & 1, p.err, abort_flag)) { ok = false; break; }
+      // No early exit: the issuer expects one P handoff per key tile, so a
+      // failed wait only marks the launch failed and the loop runs on.
+      if (!mbar_wait(bar(C_SFULL + t), j & 1, p.err, abort_flag)) ok = false;
       tc_fence_after();
-      if (tracer) TM_TRACE_EV(t, EV_S_READY);
+      TM_PH(0);
+      TM_SM_EV(EV_S_READY);
       __syncwarp();
       float x[BN];
       {
@@ -530,7 +745,8 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32p(s_addr + cc * 32, u + cc * 32);
         tmem_wait_ld();
-        if (tracer) TM_TRACE_EV(t, EV_SLOADED);
+        TM_PH(1);
+        TM_SM_EV(EV_SLOADED);
         if (i8) {
           // exact int32 -> fp32 for |acc| < 2^22: add the bits of 1.5 * 2^23,
           // then subtract 1.5 * 2^23 in packed fp32
@@ -556,13 +772,14 @@ __global__ void __launch_bounds__(384, 1)
       float alpha = 1.f;
       if (nv > 0) {
         const float mt = row_max<BN>(x) * c;
-        if (mt > m_used + 8.0f) {
+        if (mt > m_used + kLazyRescaleLog2) {
           alpha = ex2_approx(m_used - mt);
           m_used = mt;
         }
       }
       const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-      if (tracer) TM_TRACE_EV(t, EV_MAXED);
+      TM_PH(2);
+      TM_SM_EV(EV_MAXED);
       const uint64_t c2 = f2pack(c, c);
       const uint64_t nm2 = f2pack(-msub, -msub);
       uint32_t pk[BN / 2];
@@ -588,18 +805,19 @@ __global__ void __launch_bounds__(384, 1)
         f2unpack(s2, s0, s1);
         l = l * alpha + (s0 + s1);
       }
-      if (tracer) TM_TRACE_EV(t, EV_EXP_DONE);
+      TM_PH(3);
+      TM_SM_EV(EV_EXP_DONE);
       // O is rescaled only when a row of this warp raised its running max.
       // Then PV_{j-1} must have completed: o_done has finished phase j-2 at
       // least (S_j completed after PV_{j-2}), so waiting for phase j-1 by
       // parity is unambiguous even though earlier phases were not waited on.
-      if (tracer) TM_TRACE_EV(t, EV_O_READY);
+      TM_SM_EV(EV_O_READY);
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if (!mbar_wait(bar(C_ODONE + t), (j - 1) & 1, p.err, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(C_ODONE + t), (j - 1) & 1, p.err, abort_flag)) ok = false;
         tc_fence_after();
         __syncwarp();
         {
-          if (tracer) TM_TRACE_EV(t, EV_RESCALED);
+          TM_SM_EV(EV_RESCALED);
           uint32_t o[D];
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
@@ -616,14 +834,25 @@ __global__ void __launch_bounds__(384, 1)
           for (int cc = 0; cc < D / 32; ++cc) tmem_st32p(o_addr + cc * 32, o + cc * 32);
         }
       }
+      TM_PH(4);
       __syncwarp();
 #pragma unroll
       for (int cc = 0; cc < BN / 64; ++cc) tmem_st32p(s_addr + cc * 32, pk + cc * 32);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C_PFULL + t));
-      if (tracer) TM_TRACE_EV(t, EV_P_RELEASED);
+      if (DUAL) {
+        named_bar_arrive(NB_P + t, 160);   // P_t(j) stored: hand it to issuer t
+        if (t == 0 && j == 0 && ti[1].nJ > 0) named_bar_arrive(NB_START, 160);
+      } else {
+        mbar_arrive(bar(C_PFULL + t));     // the wait helper hands it to the issuer
+      }
+      TM_PH(5);
+      TM_SM_EV(EV_P_RELEASED);
     }
+#ifdef TM_PHASES
+    if (tracer && blockIdx.x == g_tm_trace_block)
+      for (int i = 0; i < 8; ++i) g_tm_trace[t][TM_TRACE_EVENTS - 8 + i] = static_cast<unsigned long long>(tm_ph[i]);
+#endif
     // ---- epilogue
     bool have_o = false;
     if (ok && T.nJ > 0) {
@@ -671,30 +900,43 @@ __global__ void __launch_bounds__(384, 1)
 
 std::mutex g_mu2;
 
+// One-time kernel attributes; the warpgroup register split assumes exactly
+// LAUNCH_REGS per thread at launch (any other allocation could leave
+// setmaxnreg.inc waiting), so a build that differs is refused.
+template <int D, bool DUAL>
+tm_status prepare_pair_kernel() {
+  using C = Cfg2<D>;
+  static bool attr_done = false;
+  std::lock_guard<std::mutex> lk(g_mu2);
+  if (attr_done) return TM_OK;
+  auto kern = attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, DUAL>;
+  cudaFuncAttributes fa;
+  tm_status st = check_cuda(cudaFuncGetAttributes(&fa, kern));
+  if (st != TM_OK) return st;
+  if (fa.numRegs != C::LAUNCH_REGS) return TM_ERR_UNSUPPORTED;
+  st = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  if (st != TM_OK) return st;
+  attr_done = true;
+  return TM_OK;
+}
+
+// Key tiles from which the two query tiles of a CTA get one tcgen05 issuer
+// each.  With short rows of key tiles the single shared issuer measured
+// faster (its fixed issue order keeps the tiles' softmax phases
+// alternating); with long rows one issuer per tile removes the wait of each
+// tile's P.V and next S behind the other tile's MMAs.
+constexpr int64_t kDualIssuerKeyTiles = 64;
+
 template <int D>
 tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                       const int32_t* cu, int32_t batch, int32_t max_seqlen, const uint32_t* bitmask,
                       int64_t mask_hs, int32_t g, int32_t causal, cudaStream_t stream) {
   using C = Cfg2<D>;
-  auto kern = attn_pair_kernel<D, TM_EXP2_EMU_PAIRS>;
-  static bool attr_done = false;
-  {
-    std::lock_guard<std::mutex> lk(g_mu2);
-    if (!attr_done) {
-      // The warpgroup register split assumes exactly LAUNCH_REGS per thread
-      // at launch; any other allocation could leave setmaxnreg.inc waiting.
-      cudaFuncAttributes fa;
-      tm_status st = check_cuda(cudaFuncGetAttributes(&fa, kern));
-      if (st != TM_OK) return st;
-      if (fa.numRegs != C::LAUNCH_REGS) return TM_ERR_UNSUPPORTED;
-      st = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           C::SMEM_BYTES));
-      if (st != TM_OK) return st;
-      attr_done = true;
-    }
-  }
+  const int64_t maxk_tiles = ((cu ? max_seqlen : k->T) + 127) / 128;
+  const bool dual = maxk_tiles >= kDualIssuerKeyTiles;
+  tm_status st = dual ? prepare_pair_kernel<D, true>() : prepare_pair_kernel<D, false>();
+  if (st != TM_OK) return st;
   CUtensorMap mQ16, mQ8, mK16, mK8, mV16;
-  tm_status st;
   st = encode_thd_map(&mQ16, q->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q->T, q->H, D, q->stride_t,
                       q->stride_h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != TM_OK) return st;
@@ -753,7 +995,12 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
   const int64_t grid = static_cast<int64_t>(p.n_pair_max) * p.batch * p.Hq;
   if (grid == 0) return TM_OK;
   if (grid > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
-  kern<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
+  if (dual)
+    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true>
+        <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
+  else
+    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, false>
+        <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   return check_cuda(cudaGetLastError());
 }
 

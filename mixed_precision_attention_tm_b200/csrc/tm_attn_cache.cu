@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(384, 1)
       float alpha = 1.f;
       if (nv > 0) {
         const float mt = row_max<BN>(x) * c;
-        if (mt > m_used + 8.0f) {
+        if (mt > m_used + kLazyRescaleLog2) {
           alpha = ex2_approx(m_used - mt);
           m_used = mt;
         }

@@ -385,6 +385,13 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
 }
 
 // ---------------------------------------------------------------- misc
+// Lazy online-softmax rescaling: a row's running max m is raised (and O and
+// the row sum rescaled) only when a score exceeds it by more than this many
+// powers of two.  P = 2^(s - m) then stays below 2^15, inside fp16's range
+// (max 65504) at full relative precision, and the fp32 row sum and O
+// accumulator are unaffected; a larger margin means fewer rescales.
+constexpr float kLazyRescaleLog2 = 15.0f;
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -426,7 +433,7 @@ __device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^y for y <= 8 on the FMA pipe, two lanes at a time (f32x2).  y = n + f
+// 2^y for y <= kLazyRescaleLog2 on the FMA pipe, two lanes at a time (f32x2).  y = n + f
 // with n = rne(y) obtained by adding 1.5 * 2^23 (whose float ulp is 1), f in
 // [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (relative error <= 7.5e-5
 // on that interval, coefficients from a Remez fit); 2^n enters the exponent
@@ -481,6 +488,11 @@ __device__ __forceinline__ float row_max(const float* x) {
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Arrives on named barrier `id` (expected count nthreads) without waiting;
+// executed by whole warps.
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {

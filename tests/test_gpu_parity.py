@@ -292,3 +292,46 @@ def test_int8_cache_fp16_route_equals_dequantised_fp16_inputs():
     wf = inputs.Workload("f", w.q, k16, v16, 4, 2, 128, True, 128, 128, 1, None)
     out_f, _, _ = run_gpu(wf)
     assert max_err(out_c, out_f.to(torch.float64).numpy()) <= 2e-3
+
+
+# ------------------------------------------------------------------ two-issuer mode
+# Rows of 64 or more key tiles run the 128x128 kernel with one tcgen05 issuer
+# per query tile (shorter rows share one issuer); these cases reach that mode
+# with an absent second query tile, ragged key tails, causal rows of different
+# lengths, varlen batches mixing long and short sequences, and d = 64.
+DUAL_CASES = [
+    ("dual_noncausal_tileB_absent", dict(Lq=384, Lk=8269, hq=2, hkv=1, d=128, causal=False, g=2, p=0.5)),
+    ("dual_causal_ragged_outliers", dict(Lq=8269, Lk=8269, hq=2, hkv=1, d=128, causal=True, g=1, p=0.5,
+                                         fd=True, fs=True, outliers=True)),
+    ("dual_causal_fp16", dict(Lq=8205, Lk=8205, hq=2, hkv=2, d=128, causal=True)),
+    ("dual_varlen_mixed", dict(Lq=0, Lk=0, hq=4, hkv=2, d=128, causal=True, g=4, p=0.75,
+                               cu=[0, 300, 8500, 8629, 8800])),
+    ("dual_d64", dict(Lq=320, Lk=8192, hq=2, hkv=1, d=64, causal=False, g=1, p=1.0)),
+]
+
+
+def _rows_for(w, seed=5, n_random=40):
+    seqs, _ = seqs_of(w)
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for (qs, lq, _ks, _lk) in seqs:
+        if lq == 0:
+            continue
+        for r0 in range(0, lq, 128):      # first and last row of every query tile
+            rows.update([qs + r0, qs + min(lq, r0 + 128) - 1])
+        rows.update(int(x) for x in rng.integers(qs, qs + lq, max(1, n_random // len(seqs))))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name,kw", DUAL_CASES, ids=[c[0] for c in DUAL_CASES])
+def test_two_issuer_mode_matches_oracle(name, kw):
+    w = W(**kw)
+    out, m, _ = run_gpu(w)
+    assert torch.isfinite(out).all()
+    mask_u32 = None if m is None else m.numpy().view(np.uint32)
+    if mask_u32 is not None:
+        assert np.array_equal(mask_u32, oracle_mask(w))
+    rows = _rows_for(w)
+    ref = run_oracle(w, mask_u32, rows=rows)
+    err = max_err(out, ref, rows=rows)
+    assert err <= TOL, f"{name}: max abs err {err} over {len(rows)} rows"
