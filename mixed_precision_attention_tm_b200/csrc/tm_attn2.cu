@@ -744,7 +744,7 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t u[BN];
 #pragma unroll
         for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32p(s_addr + cc * 32, u + cc * 32);
-        tmem_wait_ld();
+        tmem_wait_ld_regs<BN>(u);
         TM_PH(1);
         TM_SM_EV(EV_SLOADED);
         if (i8) {
@@ -821,7 +821,7 @@ __global__ void __launch_bounds__(384, 1)
           uint32_t o[D];
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
-          tmem_wait_ld();
+          tmem_wait_ld_regs<D>(o);
           const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
           for (int e = 0; e < D; e += 2) {
@@ -865,7 +865,7 @@ __global__ void __launch_bounds__(384, 1)
     if (__all_sync(0xffffffffu, have_o)) {
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
-      tmem_wait_ld();
+      tmem_wait_ld_regs<D>(o);
     } else {
 #pragma unroll
       for (int e = 0; e < D; ++e) o[e] = 0u;

@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int cc = 0; cc < BN / 32; ++cc)
           tmem_ld32p(lane_addr + static_cast<uint32_t>(j & 1) * BN + cc * 32, u + cc * 32);
-        tmem_wait_ld();
+        tmem_wait_ld_regs<BN>(u);
         if (i8) {
           // exact int32 -> fp32 (|acc| < 2^22: add the bits of 1.5 * 2^23, then
           // subtract it), times the column's s_q s_k sigma log2(e), in f32x2
@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t o[D];
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
-        tmem_wait_ld();
+        tmem_wait_ld_regs<D>(o);
         const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
         for (int e = 0; e < D; e += 2) {
@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(384, 1)
     if (__all_sync(0xffffffffu, have_o)) {
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) tmem_ld32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
-      tmem_wait_ld();
+      tmem_wait_ld_regs<D>(o);
     } else {
 #pragma unroll
       for (int e = 0; e < D; ++e) o[e] = 0u;

@@ -348,6 +348,15 @@ __device__ __forceinline__ void reg_fence32(uint32_t* r) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// Waits for this thread's TMEM loads into r[0, N) and then pins those
+// registers: the empty asm statement "modifies" them after the wait, so the
+// compiler cannot schedule a use of a loaded value ahead of the wait.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t* r) {
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < N / 32; ++c) reg_fence32(r + c * 32);
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
