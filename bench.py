@@ -312,6 +312,33 @@ def run_ours(args, rank, world, local_rank):
                           "tokens_per_s": ws.Lq / (a_ms * 1e-3)})
             del pl
 
+    # secondary bounds: instruction rates probed on this GPU, turned into
+    # floors for this workload at the clock sampled during the timed region
+    secondary = None
+    try:
+        rates = ops.probe_rates()
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        f_hz = float(clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0) * 1e6
+        per_sm_clk = lambda cyc: 4 * 32 / cyc            # values per clock per SM (4 sub-partitions)
+        ex2 = per_sm_clk(rates["ex2_cycles_per_warp_instr"])
+        cvt = per_sm_clk(rates["cvt_s32_f32_cycles_per_warp_instr"])
+        mag = per_sm_clk(rates["magic_conversion_cycles_per_warp_value"])
+        secondary = {
+            "probe": rates,
+            "sm_clock_mhz": f_hz / 1e6,
+            "exp2_per_clk_per_sm": ex2,
+            "exp_floor_ms_all_mufu": n_vis / (ex2 * sms * f_hz) * 1e3,
+            "exp_floor_ms_mufu_share": 5.0 / 8.0 * n_vis / (ex2 * sms * f_hz) * 1e3,
+            "int8_pair_conversion_floor_ms_cvt": e8 / (cvt * sms * f_hz) * 1e3,
+            "int8_pair_conversion_floor_ms_kernel": e8 / (mag * sms * f_hz) * 1e3,
+            "mma_f16_tflops_back_to_back": 2.0 * 128 * 128 * 16 / rates["mma_f16_m128n128k16_cycles"]
+                                           * sms * f_hz / 1e12,
+            "note": "exp: one exp2 per visible pair; the kernels evaluate 3 of every 8 on the FMA pipe "
+                    "(mufu_share); conversion: one int32->fp32 per INT8-routed pair",
+        }
+    except Exception as exc:                                   # a probe failure must not hide the run
+        secondary = {"unavailable": str(exc)}
+
     launches = plan.launches_per_step * K
     traffic, traffic_note = (None, "traffic captured for the routing-sweep workload only")
     if args.workload == "sweep" and w.p == 0.75:
@@ -342,6 +369,7 @@ def run_ours(args, rank, world, local_rank):
                                     "(nominal INT8:FP16 ratio) for INT8 QK^T, mix-weighted by visible pairs"},
         "gpu_launches": launches,
         "clocks": clk,
+        "secondary_bounds": secondary,
     }
     if e2e is not None:
         line["e2e"] = e2e
@@ -458,13 +486,64 @@ def run_reference(args):
     return line
 
 
+def run_mlx_table(args):
+    """All 48 runs of the MLX-shaped all-FP16 configuration (24 shapes x
+    causal / non-causal), timed as the MLX table times them: 10 warm-up and
+    64 timed calls, median and mean of per-call CUDA-event times.  A 256 MiB
+    buffer is written between timed calls so that no call finds its inputs
+    in L2 (the flush is outside the timed region)."""
+    from mixed_precision_attention_tm_b200 import metrics, ops
+    from mixed_precision_attention_tm_b200.api import TileMixPrefill
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    p16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rows = []
+    for (Lq, Lk, d, hq, hkv) in inputs.MLX_SHAPES:
+        for causal in (False, True):
+            w = inputs.mlx_shape(Lq, Lk, d, hq, hkv, causal, seed=args.seed)
+            plan = TileMixPrefill(w.Lq, w.Lk, w.hq, w.hkv, w.d, causal=w.causal, device=dev)
+            plan.load(w.q, w.k, w.v)
+            for _ in range(10):
+                plan.run()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(64):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                plan.run()
+                b.record()
+                b.synchronize()
+                ts.append(a.elapsed_time(b))
+            if ops.get_device_error() != ops.TM_OK:
+                raise RuntimeError(f"device error on {w.name}")
+            med, mean = float(np.median(ts)), float(np.mean(ts))
+            nvis = metrics.visible_pairs(Lq, Lk, causal) * hq
+            alg = metrics.algorithmic_flops(d, nvis) / (med * 1e-3) / 1e12
+            mlx = metrics.mlx_flops(1, hq, Lq, Lk, d, causal) / (med * 1e-3) / 1e12
+            rows.append({"qsl": Lq, "ksl": Lk, "hdim": d, "n_qh": hq, "n_kvh": hkv, "causal": int(causal),
+                         "ms_median": round(med, 4), "ms_mean": round(mean, 4),
+                         "tflops_alg": round(alg, 1), "tflops_mlx": round(mlx, 1),
+                         "tokens_per_s": round(Lq / (med * 1e-3), 0),
+                         "frac_of_fp16_roofline": round(alg / p16, 3)})
+            del plan
+    return {"metric": "prefill attention TFLOPS, MLX-shaped all-FP16 table", "unit": "TFLOP/s",
+            "n_gpus": 1, "dtype": "f16 (fp32 accumulate)", "data": "synthetic (seeded N(0,1) fp16)",
+            "timing": "10 warm-up + 64 calls, per-call CUDA events, 256 MiB L2 flush between calls",
+            "peak": {"bf16_tflops": p16, "source": peak_src}, "table": rows}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="sweep", choices=["sweep", "long", "varlen", "mlx", "tiny"])
+    ap.add_argument("--workload", default="sweep",
+                    choices=["sweep", "long", "varlen", "mlx", "tiny", "mlx_table"])
     ap.add_argument("--p", type=float, default=0.75)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-sweep", action="store_true")
@@ -475,6 +554,11 @@ def main():
     args.warmup = max(args.warmup, 3)
 
     rank, local_rank, world = dist.world_info()
+
+    if args.workload == "mlx_table":      # a report of config 2's 48 runs, not a bench line
+        if rank == 0:
+            print(json.dumps(run_mlx_table(args)), flush=True)
+        return
 
     if args.impl == "reference":
         if rank == 0:

@@ -243,6 +243,27 @@ tm_status tm_get_device_error(void* stream);
  * faults, traps or hangs. */
 tm_status tm_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
+/* Instruction-rate probes behind the kernels' secondary bounds (a
+ * measurement utility; the pages have no counterpart).  On the current
+ * device, writes out[0..4]:
+ *   out[0]  MUFU ex2.approx.f32, SM-clock cycles per warp instruction per SM
+ *           sub-partition (4 warps per sub-partition);
+ *   out[1]  cvt.rn.f32.s32 (int32 -> fp32), same unit, one integer shift
+ *           per value included;
+ *   out[2]  the kernels' exact int32 -> fp32 conversion (integer add of the
+ *           bits of 1.5 * 2^23, one fp32 subtract), cycles per value per
+ *           sub-partition, one integer shift per value included;
+ *   out[3]  tcgen05.mma kind::f16 M128 N128 K16, cycles per MMA on one SM,
+ *           issued back to back;
+ *   out[4]  tcgen05.mma kind::i8 M128 N128 K32, same.
+ * A tensor probe whose bounded wait expired reports -1.
+ * scratch: caller-owned device memory of at least tm_probe_scratch_bytes()
+ * bytes, 16-byte aligned (the probe allocates nothing).  Synchronises
+ * `stream` (a cudaStream_t) before returning.  TM_ERR_INVALID_ARG for a
+ * null or short buffer or n_out < 5. */
+int64_t tm_probe_scratch_bytes(void);
+tm_status tm_probe_rates(double* out, int32_t n_out, void* scratch, int64_t scratch_bytes, void* stream);
+
 /* Static description of a status code. */
 const char* tm_status_string(tm_status s);
 

@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(C_SFULL + t), 1);
       mbar_init(bar(C_ODONE + t), 1);
       mbar_init(bar(C_DRAIN + t), 1);
-      mbar_init(bar(C_PFULL + t), 128);
+      mbar_init(bar(C_PFULL + t), 4);   // one arrival per softmax warp
     }
     for (int s = 0; s < C::NSLOT; ++s) {
       mbar_init(bar(C_FULL + s), 1);
@@ -844,7 +844,8 @@ __global__ void __launch_bounds__(384, 1)
         named_bar_arrive(NB_P + t, 160);   // P_t(j) stored: hand it to issuer t
         if (t == 0 && j == 0 && ti[1].nJ > 0) named_bar_arrive(NB_START, 160);
       } else {
-        mbar_arrive(bar(C_PFULL + t));     // the wait helper hands it to the issuer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C_PFULL + t));   // the wait helper hands it to the issuer
       }
       TM_PH(5);
       TM_SM_EV(EV_P_RELEASED);

@@ -72,6 +72,8 @@ def _lib():
             "tm_status_string": (ctypes.c_char_p, [I32]),
             "tm_last_cuda_error": (I32, []),
             "tm_version": (ctypes.c_char_p, []),
+            "tm_probe_scratch_bytes": (I64, []),
+            "tm_probe_rates": (I32, [ctypes.POINTER(D), I32, P, I64, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -319,6 +321,22 @@ def attn_fwd_routed_noalloc(q, k, v, *, out=None, tile_m=128, tile_n=128, g=1, c
                                            int(bool(force_sink)), _stream())
     _check(st, "tm_attn_fwd_routed_noalloc")
     return out
+
+
+def probe_rates():
+    """Instruction rates behind the kernels' secondary bounds, measured on the
+    current GPU (see tm_probe_rates in include/tm.h): cycles per warp
+    instruction per SM sub-partition for MUFU ex2, cvt int32->fp32 and the
+    kernels' exact conversion; cycles per tcgen05 MMA (f16 M128N128K16, i8
+    M128N128K32) on one SM."""
+    lib = _lib()
+    n = int(lib.tm_probe_scratch_bytes())
+    scratch = torch.empty(n, dtype=torch.uint8, device="cuda")
+    out = (ctypes.c_double * 5)()
+    _check(lib.tm_probe_rates(out, 5, _ptr(scratch), n, _stream()), "tm_probe_rates")
+    keys = ("ex2_cycles_per_warp_instr", "cvt_s32_f32_cycles_per_warp_instr", "magic_conversion_cycles_per_warp_value",
+            "mma_f16_m128n128k16_cycles", "mma_i8_m128n128k32_cycles")
+    return dict(zip(keys, list(out)))
 
 
 def selftest_wait_timeout(limit_ns=1_000_000):
