@@ -25,6 +25,34 @@
 #include "tm_device.cuh"
 #include "tm_host.h"
 
+
+// Phase profile (compiled only with TM_PHASES and TM_TRACE): thread 0 (softmax)
+// and thread 128 (dequantisation) of the traced CTA sum SM-clock deltas per
+// phase in registers and store the sums once.
+#if defined(TM_PHASES) && defined(TM_TRACE)
+#define TMC_PH_DECL long long tm_ph[8] = {0, 0, 0, 0, 0, 0, 0, 0}; long long tm_ph_t = clock64();
+#define TMC_PH(i) do { const long long tm_now = clock64(); tm_ph[i] += tm_now - tm_ph_t; tm_ph_t = tm_now; } while (0)
+#define TMC_PH_STORE(role) do { if ((threadIdx.x & 127) == 0 && blockIdx.x == g_tm_trace_block) \
+  for (int i = 0; i < 8; ++i) g_tm_trace[role][TM_TRACE_EVENTS - 8 + i] = static_cast<unsigned long long>(tm_ph[i]); } while (0)
+#else
+#define TMC_PH_DECL
+#define TMC_PH(i) do { } while (0)
+#define TMC_PH_STORE(role) do { } while (0)
+#endif
+
+#ifdef TM_TRACE
+// Trace-build reader of this translation unit's trace buffer (same contract
+// as tm_debug_trace_read for the pair kernel).
+extern "C" int tm_debug_trace_read_cache(unsigned long long* host, unsigned int block) {
+  if (host == nullptr) {
+    static unsigned long long zero[TM_TRACE_ROLES][TM_TRACE_EVENTS];
+    if (cudaMemcpyToSymbol(g_tm_trace, zero, sizeof(zero)) != cudaSuccess) return -1;
+    return cudaMemcpyToSymbol(g_tm_trace_block, &block, sizeof(block)) == cudaSuccess ? 0 : -1;
+  }
+  return cudaMemcpyFromSymbol(host, g_tm_trace, sizeof(g_tm_trace)) == cudaSuccess ? 0 : -1;
+}
+#endif
+
 namespace tmk {
 namespace {
 
@@ -315,6 +343,7 @@ __global__ void __launch_bounds__(384, 1)
     // ======================= dequantisation (one key row per thread) ==========
     const int r = threadIdx.x - 128;
     int n16 = 0;
+    TMC_PH_DECL
     for (int j = 0; j < nJ; ++j) {
       const bool i8 = route_c(mrow, p.g, j);
       const int64_t tok = kstart + static_cast<int64_t>(j) * BN + r;
@@ -323,24 +352,31 @@ __global__ void __launch_bounds__(384, 1)
       const __half vs = in ? p.v_tok_scale[tok * p.Hkv + hk] : __float2half(0.f);
       const int s = j % C::NKC;
       if (!mbar_wait(bar(K_KCFULL + s), (j / C::NKC) & 1, p.err, abort_flag)) break;
+      TMC_PH(0);
       if (!i8) {
         const int s16 = n16 % C::NK16;
         if (n16 >= C::NK16 && !mbar_wait(bar(K_K16EMPTY + s16), ((n16 / C::NK16) - 1) & 1, p.err, abort_flag)) break;
+        TMC_PH(1);
         dequant_row(smem + C::OFF_KC + s * C::C8, smem + C::OFF_K16 + s16 * C::F16, r, ks);
         fence_async_shared();
         mbar_arrive(bar(K_K16FULL + s16));
         ++n16;
       }
       mbar_arrive(bar(K_KCEMPTY + s));
+      TMC_PH(2);
       const int vcs = j % C::NVC;
       if (!mbar_wait(bar(K_VCFULL + vcs), (j / C::NVC) & 1, p.err, abort_flag)) break;
+      TMC_PH(3);
       const int v16 = j % C::NV16;
       if (j >= C::NV16 && !mbar_wait(bar(K_V16EMPTY + v16), ((j / C::NV16) - 1) & 1, p.err, abort_flag)) break;
+      TMC_PH(4);
       dequant_row(smem + C::OFF_VC + vcs * C::C8, smem + C::OFF_V16 + v16 * C::F16, r, vs);
       fence_async_shared();
       mbar_arrive(bar(K_V16FULL + v16));
       mbar_arrive(bar(K_VCEMPTY + vcs));
+      TMC_PH(5);
     }
+    TMC_PH_STORE(1);
   } else {
     // ======================= softmax (warps 0-3) =======================
     regs_inc<C::SOFTMAX_REGS>();
@@ -354,6 +390,7 @@ __global__ void __launch_bounds__(384, 1)
     if (mrow != nullptr) c8_row = __ldg(p.q_scales + ig * p.Hq + h) * p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    TMC_PH_DECL
     for (int j = 0; j < nJ; ++j) {
       const bool i8 = route_c(mrow, p.g, j);
       if (i8) {
@@ -367,6 +404,7 @@ __global__ void __launch_bounds__(384, 1)
       if (!mbar_wait(bar(K_SFULL + (j & 1)), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
       tc_fence_after();
       __syncwarp();
+      TMC_PH(0);
       float x[BN];
       {
         uint32_t u[BN];
@@ -374,6 +412,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int cc = 0; cc < BN / 32; ++cc)
           tmem_ld32p(lane_addr + static_cast<uint32_t>(j & 1) * BN + cc * 32, u + cc * 32);
         tmem_wait_ld_regs<BN>(u);
+        TMC_PH(1);
         if (i8) {
           // exact int32 -> fp32 (|acc| < 2^22: add the bits of 1.5 * 2^23, then
           // subtract it), times the column's s_q s_k sigma log2(e), in f32x2
@@ -410,6 +449,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+      TMC_PH(2);
       const uint64_t c2 = f2pack(c, c);
       const uint64_t nm2 = f2pack(-msub, -msub);
       uint32_t pk[BN / 2];
@@ -435,6 +475,7 @@ __global__ void __launch_bounds__(384, 1)
         f2unpack(s2, s0, s1);
         l = l * alpha + (s0 + s1);
       }
+      TMC_PH(3);
       // O is rescaled only when a row of this warp raised its running max;
       // then PV_{j-1} must have completed.  S_j was committed after PV_{j-2}
       // was issued, so o_done has finished phase j-2, and PV_j cannot start
@@ -464,6 +505,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) tmem_st32p(lane_addr + C::O_COL + cc * 32, o + cc * 32);
       }
+      TMC_PH(4);
       __syncwarp();
 #pragma unroll
       for (int cc = 0; cc < BN / 64; ++cc)
@@ -471,7 +513,9 @@ __global__ void __launch_bounds__(384, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(K_PFULL + (j & 1)));
+      TMC_PH(5);
     }
+    TMC_PH_STORE(0);
     bool have_o = false;
     if (ok && nJ > 0) {
       have_o = mbar_wait(bar(K_ODONE), (nJ - 1) & 1, p.err, abort_flag);
