@@ -28,6 +28,7 @@ from .tilemix_oracle import (  # noqa: F401
     attention,
     attention_rows,
     build_mask,
+    build_mask_scale_policy,
     dequant_cache,
     last_visible_key,
     mask_bit,

@@ -241,6 +241,60 @@ def build_mask(Hq, seqs, tile_m, tile_n, g, causal, p, seed,
     return out
 
 
+def build_mask_scale_policy(Hq, Hkv, seqs, tile_m, tile_n, g, causal, q_scales, k_scales, tau,
+                            force_diag=False, force_sink=False, words=None):
+    """Content-driven routing bitmask from the tile quantisation scales,
+    uint32 [Hq, n_qtiles, W] in the layout of ``build_mask``.
+
+    TileMix (Lattice paper page, abstract) adjusts precision during inference
+    and claims a controllable accuracy-efficiency frontier, but gives no
+    policy.  Plainest content signal: with symmetric absmax/127 codes every
+    element's rounding error is at most half a step, so the INT8 score of a
+    tile pair differs from the fp16 one by at most
+        d * s_q[I] * s_k[J] * (127 + 1/4)
+    (|q| <= 127 s_q, |k| <= 127 s_k).  A group is routed INT8 when this bound,
+    taken over the group's key tiles that query tile I sees, is at most a
+    threshold: with mk = max of s_k over key tiles J in
+    [G*g, min((G+1)*g, nj)) (nj = key tiles visible to I; kv head
+    h // (Hq/Hkv)), bit = fl32(s_q[I, h] * mk) <= tau (fp32).  Legality and
+    forcing are those of ``build_mask``.  tau = +inf routes every eligible
+    group INT8; tau < 0 none.
+    q_scales: fp32 [n_qtiles, Hq]; k_scales: fp32 [n_ktiles, Hkv], global
+    tile order of ``tile_table``.
+    """
+    qt = tile_table(seqs, tile_m, "q")
+    kt = tile_table(seqs, tile_n, "k")
+    kbase = {}
+    for (b, i, _r0, _rows, ig) in kt:
+        if i == 0:
+            kbase[b] = ig
+    if words is None:
+        words = mask_words(max([s[3] for s in seqs] + [1]), tile_n, g)
+    q_scales = np.asarray(q_scales, dtype=np.float32)
+    k_scales = np.asarray(k_scales, dtype=np.float32)
+    tau = np.float32(tau)
+    grp = Hq // Hkv
+    out = np.zeros((Hq, len(qt), words), dtype=np.uint32)
+    for t in qt:
+        b, _i, _r0, _rows, ig = t
+        ng, gdiag = _legal_groups(t, seqs, tile_m, tile_n, g, causal)
+        if ng == 0:
+            continue
+        jmax = last_visible_key(t[1] * tile_m + t[3] - 1, seqs[b][1], seqs[b][3], causal)
+        nj = jmax // tile_n + 1
+        for h in range(Hq):
+            hk = h // grp
+            sq = q_scales[ig, h]
+            for G in range(ng):
+                if (force_sink and G == 0) or (force_diag and G == gdiag):
+                    continue
+                js = range(G * g, min((G + 1) * g, nj))
+                mk = max(k_scales[kbase[b] + j, hk] for j in js)
+                if np.float32(sq * mk) <= tau:
+                    out[h, ig, G // 32] |= np.uint32(1 << (G % 32))
+    return out
+
+
 def mask_bit(mask, h, ig, G):
     """Routing bit of group G of query tile ig for head h (head stride 0 when
     the mask has a single head plane)."""

@@ -146,3 +146,79 @@ def test_route_stats_counts_pairs():
     seqs = oracle.seq_table(12, 5)
     n_vis, _ = oracle.route_stats(None, seqs, 1, 4, 4, 1, True)
     assert n_vis == sum(max(0, min(5, i + 5 - 12 + 1)) for i in range(12))
+
+
+# ------------------------------------------------------------------ scale policy
+# Content-driven routing (the frontier item): a group is INT8 when
+# s_q * max s_k over its key tiles is at most tau.  Pins: the extremes reduce
+# to the Bernoulli builder's p = 1 / p = 0 masks, the mask is monotone in tau,
+# a key tile made an outlier by construction is exactly the one kept FP16, and
+# the error bound the policy thresholds holds for INT8 scores.
+
+def _policy_case(lens, causal, tile, g, hq=4, hkv=2, d=16, seed=3, outlier=None):
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    seqs = oracle.seq_table(cu[-1], cu[-1], cu)
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((cu[-1], hq, d)).astype(np.float16)
+    k = rng.standard_normal((cu[-1], hkv, d)).astype(np.float16)
+    if outlier is not None:
+        rows, val = outlier
+        k[rows, :, 0] = np.float16(val)
+    _, qs = oracle.quantize_tiles(q, seqs, tile, "q")
+    _, ks = oracle.quantize_tiles(k, seqs, tile, "k")
+    return seqs, qs, ks
+
+
+@pytest.mark.parametrize("lens,causal,g,fd,fs", [
+    ([300], True, 1, False, False), ([300], False, 2, True, True), ([70, 200, 129], True, 3, True, False),
+])
+def test_scale_policy_extremes_equal_bernoulli_p1_and_p0(lens, causal, g, fd, fs):
+    seqs, qs, ks = _policy_case(lens, causal, 32, g)
+    kw = dict(force_diag=fd, force_sink=fs)
+    all_on = oracle.build_mask_scale_policy(4, 2, seqs, 32, 32, g, causal, qs, ks, np.inf, **kw)
+    assert np.array_equal(all_on, oracle.build_mask(4, seqs, 32, 32, g, causal, 1.0, 7, **kw))
+    none = oracle.build_mask_scale_policy(4, 2, seqs, 32, 32, g, causal, qs, ks, -1.0, **kw)
+    assert not none.any()
+
+
+def test_scale_policy_monotone_in_tau():
+    seqs, qs, ks = _policy_case([257, 96], True, 32, 2)
+    prods = np.sort(np.outer(qs.ravel(), ks.ravel()).ravel())
+    prev = None
+    for tau in np.quantile(prods, [0.0, 0.1, 0.3, 0.5, 0.7, 0.9, 1.0]):
+        m = oracle.build_mask_scale_policy(4, 2, seqs, 32, 32, 2, True, qs, ks, tau)
+        if prev is not None:
+            assert np.array_equal(prev & m, prev)       # bits only ever turn on
+        prev = m
+
+
+def test_scale_policy_keeps_the_outlier_key_tile_fp16():
+    # one sequence of 8 key tiles of 32 rows; key tile 5 carries a value 100x
+    # the others in channel 0 of every kv head, so its scale is ~25x larger
+    tile, g = 32, 2
+    seqs, qs, ks = _policy_case([256], False, tile, g, outlier=(slice(5 * tile, 6 * tile), 400.0))
+    normal = np.float32(qs.max()) * np.float32(np.delete(ks, 5, axis=0).max())
+    tau = np.float32(normal * 1.01)
+    m = oracle.build_mask_scale_policy(4, 2, seqs, tile, tile, g, False, qs, ks, tau)
+    outlier_group = 5 // g
+    for h in range(4):
+        for ig in range(8):
+            bits = [oracle.mask_bit(m, h, ig, G) for G in range(4)]
+            assert bits == [0 if G == outlier_group else 1 for G in range(4)], (h, ig, bits)
+
+
+def test_int8_score_error_within_the_policy_bound():
+    # |s_q s_k (c_q . c_k) - q . k| <= d * s_q * s_k * (127 + 1/4), per score
+    rng = np.random.default_rng(11)
+    d = 64
+    for scale_q, scale_k in ((1.0, 1.0), (20.0, 0.05), (1e-3, 300.0)):
+        q = (rng.standard_normal((32, 1, d)) * scale_q).astype(np.float16)
+        k = (rng.standard_normal((32, 1, d)) * scale_k).astype(np.float16)
+        q[3, 0, :4] *= np.float16(20)                                # outlier channels
+        seqs = oracle.seq_table(32, 32)
+        qc, qs = oracle.quantize_tiles(q, seqs, 32, "q")
+        kc, ks = oracle.quantize_tiles(k, seqs, 32, "k")
+        s8 = float(qs[0, 0]) * float(ks[0, 0]) * (qc[:, 0].astype(np.float64) @ kc[:, 0].astype(np.float64).T)
+        s16 = q[:, 0].astype(np.float64) @ k[:, 0].astype(np.float64).T
+        bound = d * float(qs[0, 0]) * float(ks[0, 0]) * (127 + 0.25)
+        assert np.abs(s8 - s16).max() <= bound
