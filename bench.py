@@ -536,6 +536,78 @@ def run_mlx_table(args):
             "peak": {"bf16_tflops": p16, "source": peak_src}, "table": rows}
 
 
+def run_frontier(args):
+    """Accuracy-efficiency curve on the routing-sweep inputs: for random
+    routing (Bernoulli p) and for the scale policy (INT8 iff s_q * s_k <=
+    tau, tau at quantiles of the tile-scale products), the realised INT8
+    fraction, the attention time (median of 20 calls) and the output error
+    against the all-FP16 output of the same kernel (max, mean and rms of the
+    absolute difference over every output element)."""
+    from mixed_precision_attention_tm_b200 import ops
+    from mixed_precision_attention_tm_b200.api import TileMixPrefill
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    p16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * 1e12
+    w = (inputs.routing_sweep_token_outliers(0.0, seed=args.seed) if args.frontier_input == "tokens"
+         else inputs.routing_sweep(0.0, seed=args.seed))
+    common = dict(causal=True, tile_m=128, tile_n=128, g=w.g, force_diag=True, force_sink=True, device=dev)
+
+    def run(**kw):
+        pl = TileMixPrefill(w.Lq, w.Lk, w.hq, w.hkv, w.d, **common, **kw)
+        pl.load(w.q, w.k, w.v)
+        for _ in range(3):
+            pl.run()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(20):
+            if pl.routed:
+                pl.quantize()
+                pl.mask()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            pl.attend()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        if ops.get_device_error() != ops.TM_OK:
+            raise RuntimeError("device error in the frontier run")
+        mh = pl.bitmask.cpu().numpy().view(np.uint32) if pl.routed else None
+        nv, e8 = route_stats_of(w, mh)
+        return pl, float(np.median(ts)), nv, e8
+
+    ref_plan, ref_ms, nv, _ = run(p=None)
+    ref = ref_plan.out.float()
+
+    def point(kind, knob, pl, ms, nv_, e8_):
+        diff = (pl.out.float() - ref).abs()
+        t_roof = roofline_time(w.d, nv_, e8_, p16, 2.0 * p16)
+        return {"policy": kind, "knob": knob, "realised_int8_fraction": e8_ / nv_, "attn_ms": ms,
+                "tflops": 4.0 * w.d * nv_ / (ms * 1e-3) / 1e12, "mixed_roofline_frac": t_roof / (ms * 1e-3),
+                "err_max_abs": float(diff.max()), "err_mean_abs": float(diff.mean()),
+                "err_rms": float(diff.pow(2).mean().sqrt())}
+
+    rows = [point("fp16", None, ref_plan, ref_ms, nv, 0.0)]
+    for p in (0.25, 0.5, 0.75, 1.0):
+        pl, ms, nv_, e8_ = run(p=p, seed=w.mask_seed)
+        rows.append(point("random", p, pl, ms, nv_, e8_))
+        del pl
+    # tau at quantiles of s_q * s_k over (query tile, head) x (key tile, kv head)
+    qc, qs, kc, ks = ops.quantize_qk(ref_plan.q, ref_plan.k, tile_m=128, tile_n=128)
+    prods = (qs.reshape(-1, 1) * ks.reshape(1, -1)).flatten()
+    qv = torch.tensor([0.2, 0.4, 0.6, 0.8, 0.9, 0.97], device=dev)
+    taus = torch.quantile(prods[torch.randperm(prods.numel(), device=dev)[:1 << 20]], qv).tolist()
+    for tau in taus + [float("inf")]:
+        pl, ms, nv_, e8_ = run(tau=tau)
+        rows.append(point("scale", tau, pl, ms, nv_, e8_))
+        del pl
+    return {"metric": "accuracy-efficiency frontier: output error vs realised INT8 fraction", "unit": "mixed",
+            "n_gpus": 1, "workload": w.name, "config": describe(w), "inputs": args.frontier_input,
+            "reference": "all-FP16 output of the same kernel on the same inputs",
+            "peak": {"bf16_tflops": p16 / 1e12, "source": peak_src}, "points": rows}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -543,21 +615,25 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="sweep",
-                    choices=["sweep", "long", "varlen", "mlx", "tiny", "mlx_table"])
+                    choices=["sweep", "long", "varlen", "mlx", "tiny", "mlx_table", "frontier"])
     ap.add_argument("--p", type=float, default=0.75)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--frontier-input", default="channels", choices=["channels", "tokens"],
+                    help="frontier report: outlier channels in every token (the routing sweep's inputs) "
+                         "or outliers in 0.2%% of the key tokens")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     rank, local_rank, world = dist.world_info()
 
-    if args.workload == "mlx_table":      # a report of config 2's 48 runs, not a bench line
+    if args.workload in ("mlx_table", "frontier"):   # reports, not the contract's bench line
         if rank == 0:
-            print(json.dumps(run_mlx_table(args)), flush=True)
+            fn = run_mlx_table if args.workload == "mlx_table" else run_frontier
+            print(json.dumps(fn(args)), flush=True)
         return
 
     if args.impl == "reference":

@@ -148,6 +148,24 @@ tm_status tm_build_mask(uint32_t* bitmask, int32_t Hq,
                         int32_t force_diag, int32_t force_sink, int64_t mask_head_stride,
                         void* stream);
 
+/* Content-driven routing bitmask (the frontier policy; the pages adjust
+ * precision during inference but give no policy).  Same layout, legality and
+ * forcing as tm_build_mask.  With symmetric absmax/127 codes the INT8 score
+ * of a tile pair differs from the fp16 score by at most
+ * d * s_q * s_k * (127 + 1/4); group G of query tile I (head h, kv head
+ * h / (Hq / Hkv)) is routed INT8 iff fl32(s_q[I, h] * mk) <= tau, where mk is
+ * the largest s_k over the group's key tiles that I sees.  tau = +inf routes
+ * every eligible group INT8, tau < 0 none.
+ *   q_scales: device fp32 [n_qtiles, Hq], k_scales: device fp32 [n_ktiles, Hkv]
+ *             (the tile scales written by tm_quantize_qk).
+ *   Other arguments as for tm_build_mask.  TM_ERR_INVALID_ARG for Hq % Hkv
+ *   != 0, a NaN tau, null scales or the conditions of tm_build_mask. */
+tm_status tm_build_mask_scale_policy(uint32_t* bitmask, int32_t Hq, int32_t Hkv, const int32_t* cu_seqlens,
+                                     int32_t batch, int32_t max_seqlen, int64_t Lq, int64_t Lk, int32_t tile_m,
+                                     int32_t tile_n, int32_t g, int32_t causal, const float* q_scales,
+                                     const float* k_scales, float tau, int32_t force_diag, int32_t force_sink,
+                                     int64_t mask_head_stride, void* stream);
+
 /* Same bits computed on the host (bitmask_host and cu_seqlens_host are host
  * pointers), written with mask_head_stride = n_qtiles * W; bit-identical to
  * tm_build_mask. */

@@ -22,10 +22,19 @@ from . import ops
 class TileMixPrefill:
     def __init__(self, Lq, Lk, hq, hkv, d, *, causal=True, tile_m=128, tile_n=128, g=1, p=None,
                  seed=0, force_diag=False, force_sink=False, cu_seqlens=None, int8_cache=False,
-                 device="cuda"):
+                 tau=None, device="cuda"):
+        """p: Bernoulli INT8 probability per eligible group (seeded mask);
+        tau: instead of p, the content-driven policy (INT8 iff the tile
+        scales' score-error bound s_q * s_k is at most tau).  Neither: all
+        FP16."""
         self.shape = (Lq, Lk, hq, hkv, d)
         self.causal, self.tile_m, self.tile_n, self.g = causal, tile_m, tile_n, g
+        if p is not None and tau is not None:
+            raise ValueError("give either p (random routing) or tau (scale policy), not both")
+        if tau is not None and int8_cache:
+            raise ValueError("the scale policy needs tile scales of K; the INT8 cache has per-token scales")
         self.p, self.seed, self.force_diag, self.force_sink = p, seed, force_diag, force_sink
+        self.tau = tau
         self.int8_cache = int8_cache
         self.device = torch.device(device)
         self.cu = None if cu_seqlens is None else cu_seqlens.to(self.device, torch.int32)
@@ -44,7 +53,7 @@ class TileMixPrefill:
             self.k = torch.empty((Lk, hkv, d), dtype=torch.float16, device=dev)
             self.v = torch.empty((Lk, hkv, d), dtype=torch.float16, device=dev)
         self.out = torch.empty((Lq, hq, d), dtype=torch.float16, device=dev)
-        self.routed = p is not None
+        self.routed = p is not None or tau is not None
         self.q_quant = self.k_quant = self.bitmask = None
         if self.routed:
             # codes, tile scales and the routing mask: allocated once, rewritten every step
@@ -91,6 +100,13 @@ class TileMixPrefill:
 
     def mask(self):
         Lq, Lk = self.shape[0], self.shape[1]
+        if self.tau is not None:
+            ops.build_mask_scale_policy(self.q_quant[1], self.k_quant[1], self.shape[2], self.shape[3],
+                                        tile_m=self.tile_m, tile_n=self.tile_n, g=self.g, causal=self.causal,
+                                        tau=self.tau, force_diag=self.force_diag, force_sink=self.force_sink,
+                                        Lq=Lq, Lk=Lk, cu_seqlens=self.cu, max_seqlen=self.max_seqlen,
+                                        cu_seqlens_host=self.cu_h, out=self.bitmask)
+            return
         ops.build_mask(self.shape[2], tile_m=self.tile_m, tile_n=self.tile_n, g=self.g,
                        causal=self.causal, p=self.p, seed=self.seed, force_diag=self.force_diag,
                        force_sink=self.force_sink, Lq=Lq, Lk=Lk, cu_seqlens=self.cu,

@@ -86,6 +86,66 @@ __global__ void build_mask_kernel(uint32_t* __restrict__ bm, int64_t head_stride
   for (int w = threadIdx.x; w < a.W; w += blockDim.x) row[w] = mask_word(a, h, ig, I, lq, lk, w);
 }
 
+// Content-driven routing from the tile quantisation scales.  With symmetric
+// absmax/127 codes the INT8 score of a tile pair is within
+// d * s_q * s_k * (127 + 1/4) of the fp16 score (half a step of rounding per
+// element), so a group is routed INT8 when s_q[I] times the largest s_k of
+// the group's key tiles that query tile I sees is at most tau.  The product
+// is one round-to-nearest fp32 multiply (no contraction) so that the decision
+// is reproducible bit for bit.  Legality and forcing as in mask_word.
+struct PolicyArgs {
+  int Hq, Hkv;
+  int tile_m, tile_n, g;
+  int causal;
+  float tau;
+  int force_diag, force_sink;
+  int W;
+};
+
+__device__ inline uint32_t policy_word(const PolicyArgs& a, int h, int64_t ig, int64_t I, int64_t lq,
+                                       int64_t lk, int64_t kbase, const float* qs, const float* ks,
+                                       int w) {
+  const int64_t r0 = I * a.tile_m;
+  const int64_t rows = (lq - r0) < a.tile_m ? (lq - r0) : a.tile_m;
+  const int64_t jmax = last_key(r0 + rows - 1, lq, lk, a.causal);
+  if (jmax < 0) return 0u;
+  const int64_t nj = jmax / a.tile_n + 1;
+  const int64_t ng = (nj - 1) / a.g + 1;
+  const int64_t gdiag = (nj - 1) / a.g;
+  const int hk = h / (a.Hq / a.Hkv);
+  const float sq = qs[ig * a.Hq + h];
+  uint32_t word = 0u;
+  for (int bit = 0; bit < 32; ++bit) {
+    const int64_t G = static_cast<int64_t>(w) * 32 + bit;
+    if (G >= ng) break;
+    if (a.force_diag && G == gdiag) continue;
+    if (a.force_sink && G == 0) continue;
+    const int64_t j1 = (G + 1) * a.g < nj ? (G + 1) * a.g : nj;
+    float mk = 0.f;
+    for (int64_t j = G * a.g; j < j1; ++j) mk = fmaxf(mk, ks[(kbase + j) * a.Hkv + hk]);
+    if (__fmul_rn(sq, mk) <= a.tau) word |= 1u << bit;
+  }
+  return word;
+}
+
+__global__ void build_mask_policy_kernel(uint32_t* __restrict__ bm, int64_t head_stride,
+                                         const int32_t* __restrict__ cu, int64_t Lq, int64_t Lk,
+                                         PolicyArgs a, const float* __restrict__ qs,
+                                         const float* __restrict__ ks, DevErr err) {
+  const int I = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
+  SeqInfo s = seq_info(cu, b, Lq, a.tile_m);
+  const int64_t lq = s.len;
+  const int64_t lk = cu ? s.len : Lk;
+  if (cu != nullptr && I == 0 && threadIdx.x == 0 &&
+      lq > static_cast<int64_t>(gridDim.x) * a.tile_m)
+    dev_error(err, TM_DEVERR_SEQLEN);
+  if (static_cast<int64_t>(I) * a.tile_m >= lq) return;
+  const int64_t kbase = seq_info(cu, b, Lk, a.tile_n).tile_base;
+  const int64_t ig = s.tile_base + I;
+  uint32_t* row = bm + static_cast<int64_t>(h) * head_stride + ig * a.W;
+  for (int w = threadIdx.x; w < a.W; w += blockDim.x) row[w] = policy_word(a, h, ig, I, lq, lk, kbase, qs, ks, w);
+}
+
 tm_status check_mask_args(int32_t Hq, int32_t tile_m, int32_t tile_n, int32_t g, double p) {
   if (Hq <= 0 || Hq >= (1 << 24)) return TM_ERR_INVALID_ARG;
   if (tile_m <= 0 || tile_n <= 0 || g <= 0) return TM_ERR_INVALID_ARG;
@@ -122,6 +182,37 @@ tm_status tm_build_mask(uint32_t* bitmask, int32_t Hq, const int32_t* cu_seqlens
   DevErr err{device_error_word()};
   build_mask_kernel<<<grid, 32, 0, as_stream(stream)>>>(bitmask, mask_head_stride, cu_seqlens, Lq,
                                                         Lk, a, err);
+  return check_cuda(cudaGetLastError());
+}
+
+tm_status tm_build_mask_scale_policy(uint32_t* bitmask, int32_t Hq, int32_t Hkv, const int32_t* cu_seqlens,
+                                     int32_t batch, int32_t max_seqlen, int64_t Lq, int64_t Lk, int32_t tile_m,
+                                     int32_t tile_n, int32_t g, int32_t causal, const float* q_scales,
+                                     const float* k_scales, float tau, int32_t force_diag, int32_t force_sink,
+                                     int64_t mask_head_stride, void* stream) {
+  using namespace tmk;
+  tm_status st = check_mask_args(Hq, tile_m, tile_n, g, 0.5);
+  if (st != TM_OK) return st;
+  if (Hkv <= 0 || Hq % Hkv != 0) return TM_ERR_INVALID_ARG;
+  if (tau != tau) return TM_ERR_INVALID_ARG;   // NaN
+  if (bitmask == nullptr || reinterpret_cast<uintptr_t>(bitmask) % 4) return TM_ERR_INVALID_ARG;
+  if (q_scales == nullptr || k_scales == nullptr) return TM_ERR_INVALID_ARG;
+  const int64_t maxq = cu_seqlens ? max_seqlen : Lq;
+  const int64_t maxk = cu_seqlens ? max_seqlen : Lk;
+  if (cu_seqlens != nullptr && (batch <= 0 || max_seqlen <= 0)) return TM_ERR_INVALID_ARG;
+  if (maxq < 0 || maxk < 0) return TM_ERR_INVALID_ARG;
+  PolicyArgs a{Hq, Hkv, tile_m, tile_n, g, causal ? 1 : 0, tau, force_diag ? 1 : 0, force_sink ? 1 : 0,
+               tm_mask_words(maxk, tile_n, g)};
+  const int64_t nqt_max = (maxq + tile_m - 1) / tile_m;
+  if (nqt_max == 0) return TM_OK;
+  if (mask_head_stride < 0) return TM_ERR_INVALID_ARG;
+  if (cu_seqlens == nullptr && Hq > 1 && mask_head_stride < nqt_max * a.W) return TM_ERR_INVALID_ARG;
+  const int nb = cu_seqlens ? batch : 1;
+  if (nqt_max > 0x7fffffff || nb > 65535 || Hq > 65535) return TM_ERR_UNSUPPORTED;
+  dim3 grid(static_cast<unsigned>(nqt_max), static_cast<unsigned>(nb), static_cast<unsigned>(Hq));
+  DevErr err{device_error_word()};
+  build_mask_policy_kernel<<<grid, 32, 0, as_stream(stream)>>>(bitmask, mask_head_stride, cu_seqlens, Lq, Lk, a,
+                                                               q_scales, k_scales, err);
   return check_cuda(cudaGetLastError());
 }
 

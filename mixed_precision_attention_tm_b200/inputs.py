@@ -59,6 +59,20 @@ def qk_with_outliers(Tq, Tk, hq, hkv, d, seed, factor=20.0, n=4):
     return q.to(torch.float16), k.to(torch.float16), ch
 
 
+def qk_with_token_outliers(Tq, Tk, hq, hkv, d, seed, factor=20.0, frac=0.002):
+    """Q [Tq, hq, d] and K [Tk, hkv, d] ~ N(0, 1), with a seeded fraction of
+    key tokens (the same tokens for every KV head) multiplied by ``factor`` in
+    all channels, in fp32 before the single rounding to fp16: outliers that
+    sit in a few key tiles rather than in every tile.  Returns (q, k, the
+    outlier token indices)."""
+    q = torch.randn(Tq, hq, d, generator=_gen(seed), dtype=torch.float32)
+    k = torch.randn(Tk, hkv, d, generator=_gen(seed + 1), dtype=torch.float32)
+    n = max(1, int(round(frac * Tk)))
+    tok = torch.randperm(Tk, generator=_gen(seed + 3))[:n].sort().values
+    k[tok] *= factor
+    return q.to(torch.float16), k.to(torch.float16), tok
+
+
 def varlen_lengths(batch, lo, hi, seed):
     """batch integer lengths ~ U[lo, hi] (inclusive) and cu_seqlens int32."""
     lens = torch.randint(lo, hi + 1, (batch,), generator=_gen(seed), dtype=torch.int64)
@@ -171,6 +185,16 @@ def routing_sweep(p, L=16384, hq=32, hkv=8, d=128, seed=0):
     return Workload(f"sweep_L{L}_p{p}", q, k, v, hq, hkv, d, True, 128, 128, 4, p,
                     mask_seed=seed + 4, force_diag=True, force_sink=True,
                     extra={"outlier_channels": ch})
+
+
+def routing_sweep_token_outliers(p, L=16384, hq=32, hkv=8, d=128, seed=0, frac=0.002):
+    """The routing-sweep shape with token-localised key outliers
+    (qk_with_token_outliers) instead of outlier channels."""
+    q, k, tok = qk_with_token_outliers(L, L, hq, hkv, d, seed, frac=frac)
+    v = randn_f16((L, hkv, d), seed + 2)
+    return Workload(f"sweep_tokout_L{L}_p{p}", q, k, v, hq, hkv, d, True, 128, 128, 4, p,
+                    mask_seed=seed + 4, force_diag=True, force_sink=True,
+                    extra={"outlier_tokens": int(tok.numel())})
 
 
 def varlen_int8_cache(batch=8, lo=1024, hi=8192, hq=32, hkv=4, d=128, p=0.75, seed=0):

@@ -63,6 +63,8 @@ def _lib():
             "tm_build_mask": (I32, [P, I32, P, I32, I32, I64, I64, I32, I32, I32, I32, D, U64, I32, I32,
                                     I64, P]),
             "tm_build_mask_host": (I32, [P, I32, P, I32, I64, I64, I32, I32, I32, I32, D, U64, I32, I32]),
+            "tm_build_mask_scale_policy": (I32, [P, I32, I32, P, I32, I32, I64, I64, I32, I32, I32, I32, P, P,
+                                                 ctypes.c_float, I32, I32, I64, P]),
             "tm_route_stats": (I32, [P, I64, I32, P, I32, I64, I64, I32, I32, I32, I32,
                                      ctypes.POINTER(D), ctypes.POINTER(D)]),
             "tm_attn_fwd": (I32, [TP, TP, TP, TP, P, I32, I32, P, I64, I32, I32, I32, I32, P]),
@@ -224,6 +226,39 @@ def build_mask(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False, forc
                            float(p), ctypes.c_uint64(int(seed) & (2 ** 64 - 1)),
                            int(bool(force_diag)), int(bool(force_sink)), nqt * W, _stream())
     _check(st, "tm_build_mask")
+    return out
+
+
+def build_mask_scale_policy(q_scales, k_scales, Hq, Hkv, *, tile_m, tile_n, g, causal, tau, force_diag=False,
+                            force_sink=False, Lq=None, Lk=None, cu_seqlens=None, max_seqlen=None,
+                            cu_seqlens_host=None, out=None):
+    """Content-driven routing bitmask (int32 view [Hq, n_qt, W]): group G of
+    query tile I goes INT8 iff s_q[I] * max s_k over its visible key tiles
+    <= tau (see tm_build_mask_scale_policy).  q_scales / k_scales: the device
+    tile scales from quantize_qk."""
+    _cuda(q_scales, "q_scales")
+    _cuda(k_scales, "k_scales")
+    lib = _lib()
+    cu_h = _cu_host(cu_seqlens, cu_seqlens_host)
+    batch = 0 if cu_h is None else cu_h.numel() - 1
+    if cu_h is not None:
+        maxk = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0
+        if max_seqlen is None:
+            max_seqlen = maxk
+        nqt = count_tiles(None, tile_m, cu_h.numpy())
+    else:
+        maxk = Lk
+        nqt = count_tiles(Lq, tile_m)
+    W = mask_words(maxk, tile_n, g)
+    if out is None:
+        out = torch.empty((Hq, nqt, W), dtype=torch.int32, device=q_scales.device)
+    else:
+        _check_buf(out, (Hq, nqt, W), torch.int32, "bitmask")
+    st = lib.tm_build_mask_scale_policy(_ptr(out), Hq, Hkv, _ptr(cu_seqlens), batch, int(max_seqlen or 0),
+                                        int(Lq or 0), int(Lk or 0), tile_m, tile_n, g, int(bool(causal)),
+                                        _ptr(q_scales), _ptr(k_scales), float(tau), int(bool(force_diag)),
+                                        int(bool(force_sink)), nqt * W, _stream())
+    _check(st, "tm_build_mask_scale_policy")
     return out
 
 

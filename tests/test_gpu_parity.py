@@ -335,3 +335,56 @@ def test_two_issuer_mode_matches_oracle(name, kw):
     ref = run_oracle(w, mask_u32, rows=rows)
     err = max_err(out, ref, rows=rows)
     assert err <= TOL, f"{name}: max abs err {err} over {len(rows)} rows"
+
+
+# ------------------------------------------------------------------ scale policy
+POLICY_CASES = [
+    dict(Lq=700, Lk=700, hq=4, hkv=2, d=128, causal=True, g=2, tm=128, tn=128, fd=True, fs=True, outliers=True),
+    dict(Lq=300, Lk=900, hq=2, hkv=1, d=64, causal=False, g=1, tm=64, tn=64, outliers=True),
+    dict(Lq=0, Lk=0, hq=4, hkv=1, d=128, causal=True, g=3, cu=[0, 130, 600, 1000], outliers=True),
+]
+
+
+@pytest.mark.parametrize("kw", POLICY_CASES, ids=["causal_gqa", "noncausal_64", "varlen"])
+def test_scale_policy_mask_bit_exact_and_attention(kw):
+    w = W(**kw)
+    seqs, cu = seqs_of(w)
+    q, k = w.q.cuda(), w.k.cuda()
+    cu_d = None if w.cu_seqlens is None else w.cu_seqlens.cuda()
+    ms = w.max_seqlen if cu is not None else None
+    qc, qs, kc, ks = ops.quantize_qk(q, k, tile_m=w.tile_m, tile_n=w.tile_n, cu_seqlens=cu_d, max_seqlen=ms)
+    rq = oracle.quantize_tiles(w.q.numpy(), seqs, w.tile_m, "q")[1]
+    rk = oracle.quantize_tiles(w.k.numpy(), seqs, w.tile_n, "k")[1]
+    prods = np.sort(np.outer(rq.ravel(), rk.ravel()).ravel())
+    for tau in (float(np.quantile(prods, 0.3)), float(np.quantile(prods, 0.8)), float("inf"), -1.0):
+        m = ops.build_mask_scale_policy(qs, ks, w.hq, w.hkv, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g,
+                                        causal=w.causal, tau=tau, force_diag=w.force_diag, force_sink=w.force_sink,
+                                        Lq=w.Lq, Lk=w.Lk, cu_seqlens=cu_d, max_seqlen=ms)
+        torch.cuda.synchronize()
+        ref = oracle.build_mask_scale_policy(w.hq, w.hkv, seqs, w.tile_m, w.tile_n, w.g, w.causal, rq, rk,
+                                             np.float32(tau), force_diag=w.force_diag, force_sink=w.force_sink)
+        got = m.cpu().numpy().view(np.uint32)
+        assert np.array_equal(got, ref), f"tau={tau}"
+    # the attention with the last non-trivial policy mask matches the oracle
+    tau = float(np.quantile(prods, 0.5))
+    m = ops.build_mask_scale_policy(qs, ks, w.hq, w.hkv, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g,
+                                    causal=w.causal, tau=tau, force_diag=w.force_diag, force_sink=w.force_sink,
+                                    Lq=w.Lq, Lk=w.Lk, cu_seqlens=cu_d, max_seqlen=ms)
+    out, _, _ = run_gpu(w, mask=m.cpu().numpy().view(np.uint32))
+    ref = run_oracle(w, m.cpu().numpy().view(np.uint32))
+    assert max_err(out, ref) <= TOL
+
+
+def test_scale_policy_plan_matches_direct_calls():
+    from mixed_precision_attention_tm_b200.api import TileMixPrefill
+    w = W(Lq=1000, Lk=1000, hq=4, hkv=2, d=128, causal=True, g=2, outliers=True)
+    pl = TileMixPrefill(w.Lq, w.Lk, w.hq, w.hkv, w.d, causal=True, g=2, tau=1e-3)
+    pl.load(w.q, w.k, w.v)
+    out = pl.run().clone()
+    torch.cuda.synchronize()
+    qc, qs, kc, ks = ops.quantize_qk(w.q.cuda(), w.k.cuda())
+    m = ops.build_mask_scale_policy(qs, ks, 4, 2, tile_m=128, tile_n=128, g=2, causal=True, tau=1e-3,
+                                    Lq=w.Lq, Lk=w.Lk)
+    direct = ops.attn_fwd(w.q.cuda(), w.k.cuda(), w.v.cuda(), g=2, causal=True, bitmask=m,
+                          q_quant=(qc, qs), k_quant=(kc, ks))
+    assert torch.equal(out, direct)
