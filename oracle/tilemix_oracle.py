@@ -37,6 +37,11 @@ also listed with its reason in the design notes of this repository):
   (h) GQA: query head h reads KV head h // (Hq / Hkv).
   (j) variable-length batches share one cu_seqlens for Q and K
       (self-attention prefill); query and key tiles restart per sequence.
+      With a separate cu_seqlens_k (prefix-cached prefill, the NEXT-2 item:
+      each sequence's lq new queries attend to lk >= lq keys, prefix first),
+      key rows of sequence b are cu_k[b] .. cu_k[b+1]-1 and causal masking
+      stays bottom-right per sequence (reading (f) with that sequence's Lq,
+      Lk).
   (k) a query row with no visible key outputs 0.
   (m) the mask builder draws an independent Bernoulli(p) per eligible group
       from a counter-based hash (splitmix64); the group holding the query
@@ -63,17 +68,20 @@ _M64 = (1 << 64) - 1
 # geometry: sequences, tiles, visibility
 # --------------------------------------------------------------------------
 
-def seq_table(Tq, Tk=None, cu_seqlens=None):
+def seq_table(Tq, Tk=None, cu_seqlens=None, cu_seqlens_k=None):
     """Sequences as (q_start, Lq, k_start, Lk).
 
     Without ``cu_seqlens`` there is one sequence with Lq = Tq, Lk = Tk (Tq and
     Tk may differ).  With ``cu_seqlens`` (reading (j)) sequence b spans rows
-    cu[b] .. cu[b+1]-1 of both Q and K, so Lq = Lk = cu[b+1] - cu[b].
+    cu[b] .. cu[b+1]-1 of both Q and K, so Lq = Lk = cu[b+1] - cu[b]; with
+    ``cu_seqlens_k`` as well its keys are rows cu_k[b] .. cu_k[b+1]-1 of K.
     """
     if cu_seqlens is None:
         return [(0, int(Tq), 0, int(Tq if Tk is None else Tk))]
     cu = [int(c) for c in cu_seqlens]
-    return [(cu[b], cu[b + 1] - cu[b], cu[b], cu[b + 1] - cu[b]) for b in range(len(cu) - 1)]
+    ck = cu if cu_seqlens_k is None else [int(c) for c in cu_seqlens_k]
+    assert len(ck) == len(cu)
+    return [(cu[b], cu[b + 1] - cu[b], ck[b], ck[b + 1] - ck[b]) for b in range(len(cu) - 1)]
 
 
 def n_tiles(L, tile):
@@ -339,7 +347,7 @@ def route_stats(mask, seqs, Hq, tile_m, tile_n, g, causal):
 
 def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
               tile_m=128, tile_n=128, g=1, mask=None,
-              q_quant=None, k_quant=None, kv_cache=None, rows=None):
+              q_quant=None, k_quant=None, kv_cache=None, rows=None, cu_seqlens_k=None):
     """Tile-routed softmax attention in fp64.  Returns float64 [Tq, Hq, d].
 
     q: float16 [Tq, Hq, d]; k, v: float16 [Tk, Hkv, d] (or None with an INT8
@@ -350,6 +358,8 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
     the FP16 route and P.V use the fp16 view (dequant_cache), the INT8 route
     uses k_codes with the per-token scale of each key.
     rows: optional iterable of global query rows to evaluate (others are NaN).
+    cu_seqlens_k: key offsets per sequence when they differ from cu_seqlens
+    (prefix-cached prefill); reading (j).
 
     For each sequence, query head h (KV head hk = h // (Hq/Hkv)) and visible
     pair (i, j) in query tile I (global I_glob), key tile J, group G = J // g:
@@ -372,7 +382,7 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
     assert Hq % Hkv == 0
     grp = Hq // Hkv
     sigma = 1.0 / math.sqrt(d)
-    seqs = seq_table(Tq, Tk, cu_seqlens)
+    seqs = seq_table(Tq, Tk, cu_seqlens, cu_seqlens_k)
     qtiles = tile_table(seqs, tile_m, "q")
     kt_off = []
     acc = 0

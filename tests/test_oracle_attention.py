@@ -289,3 +289,57 @@ def test_sampled_rows_match_full():
                                  q_quant=qq, k_quant=kq)
     np.testing.assert_allclose(part[rows], full[rows], rtol=1e-12, atol=1e-14)
     assert np.isnan(part[1]).all()
+
+
+# ------------------------------------------------------------------ separate key offsets
+# Prefix-cached prefill (cu_seqlens_k != cu_seqlens): sequence b's lq new query
+# tokens attend to its lk >= lq keys, prefix first, bottom-right causal.
+
+def test_prefix_prefill_equals_last_rows_of_full_self_attention():
+    rng = np.random.default_rng(21)
+    lk_list, lq_list = [300, 129, 520], [77, 129, 5]
+    Hq, Hkv, d = 4, 2, 32
+    # full sequences: K, V of lk tokens; the new queries are the last lq rows of Q_full
+    qf = [rng.standard_normal((lk, Hq, d)).astype(np.float16) for lk in lk_list]
+    kf = [rng.standard_normal((lk, Hkv, d)).astype(np.float16) for lk in lk_list]
+    vf = [rng.standard_normal((lk, Hkv, d)).astype(np.float16) for lk in lk_list]
+    q = np.concatenate([x[-lq:] for x, lq in zip(qf, lq_list)])
+    k, v = np.concatenate(kf), np.concatenate(vf)
+    cu_q = np.concatenate([[0], np.cumsum(lq_list)])
+    cu_k = np.concatenate([[0], np.cumsum(lk_list)])
+    for causal in (True, False):
+        got = oracle.attention(q, k, v, cu_seqlens=cu_q, cu_seqlens_k=cu_k, causal=causal, tile_m=32, tile_n=32)
+        for b, (lq, lk) in enumerate(zip(lq_list, lk_list)):
+            full = oracle.attention(qf[b], kf[b], vf[b], causal=causal, tile_m=32, tile_n=32)
+            np.testing.assert_allclose(got[cu_q[b]:cu_q[b + 1]], full[lk - lq:], rtol=0, atol=1e-12)
+
+
+def test_prefix_prefill_routed_equals_per_sequence_calls():
+    rng = np.random.default_rng(22)
+    lq_list, lk_list = [40, 100], [200, 100]
+    Hq, Hkv, d = 2, 1, 16
+    q = rng.standard_normal((sum(lq_list), Hq, d)).astype(np.float16)
+    k = rng.standard_normal((sum(lk_list), Hkv, d)).astype(np.float16)
+    v = rng.standard_normal((sum(lk_list), Hkv, d)).astype(np.float16)
+    cu_q = np.concatenate([[0], np.cumsum(lq_list)])
+    cu_k = np.concatenate([[0], np.cumsum(lk_list)])
+    seqs = oracle.seq_table(len(q), len(k), cu_q, cu_k)
+    assert seqs == [(0, 40, 0, 200), (40, 100, 200, 100)]
+    mask = oracle.build_mask(Hq, seqs, 32, 32, 2, True, 0.6, 5, force_diag=True)
+    qq = oracle.quantize_tiles(q, seqs, 32, "q")
+    kq = oracle.quantize_tiles(k, seqs, 32, "k")
+    got = oracle.attention(q, k, v, cu_seqlens=cu_q, cu_seqlens_k=cu_k, causal=True, tile_m=32, tile_n=32, g=2,
+                           mask=mask, q_quant=qq, k_quant=kq)
+    qt0 = 0
+    for b, (lq, lk) in enumerate(zip(lq_list, lk_list)):
+        qb, kb, vb = q[cu_q[b]:cu_q[b + 1]], k[cu_k[b]:cu_k[b + 1]], v[cu_k[b]:cu_k[b + 1]]
+        sb = oracle.seq_table(lq, lk)
+        nqt = oracle.n_tiles(lq, 32)
+        mb = oracle.build_mask(Hq, sb, 32, 32, 2, True, 0.6, 5, force_diag=True)
+        # the batched mask rows of this sequence carry the batched hash keys (I_glob); reuse them
+        mb[:, :, :] = mask[:, qt0:qt0 + nqt, :mb.shape[2]]
+        ref = oracle.attention(qb, kb, vb, causal=True, tile_m=32, tile_n=32, g=2, mask=mb,
+                               q_quant=oracle.quantize_tiles(qb, sb, 32, "q"),
+                               k_quant=oracle.quantize_tiles(kb, sb, 32, "k"))
+        np.testing.assert_allclose(got[cu_q[b]:cu_q[b + 1]], ref, rtol=0, atol=1e-12)
+        qt0 += nqt
