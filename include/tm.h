@@ -104,6 +104,18 @@ tm_status tm_quantize_qk(const tm_tensor* q, const tm_tensor* k,
                          const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen,
                          int32_t tile_m, int32_t tile_n, void* stream);
 
+/* tm_quantize_qk with separate key offsets (prefix-cached prefill): Q tiles
+ * restart at every cu_seqlens_q[b], K tiles at every cu_seqlens_k[b]; the
+ * sequence's lq new queries attend to its lk keys.  max_seqlen_q / _k bound
+ * the per-sequence lengths.  Scales are written per side in tile order over
+ * all sequences ([n_qtiles, Hq] and [n_ktiles, Hkv]; tm_count_tiles with the
+ * side's offsets).  TM_ERR_INVALID_ARG when an offset array is null or a
+ * maximum is not positive; otherwise as tm_quantize_qk. */
+tm_status tm_quantize_qk_varlen(const tm_tensor* q, const tm_tensor* k, int8_t* q_codes, float* q_scales,
+                                int8_t* k_codes, float* k_scales, const int32_t* cu_seqlens_q,
+                                const int32_t* cu_seqlens_k, int32_t batch, int32_t max_seqlen_q,
+                                int32_t max_seqlen_k, int32_t tile_m, int32_t tile_n, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Routing bitmask layout (TileMix abstract: "compact bitmasks", one bit per
  * query tile x key-tile group, "each routing bit govern[s] multiple adjacent
@@ -148,6 +160,17 @@ tm_status tm_build_mask(uint32_t* bitmask, int32_t Hq,
                         int32_t force_diag, int32_t force_sink, int64_t mask_head_stride,
                         void* stream);
 
+/* tm_build_mask with separate key offsets: sequence b has lq = cu_q[b+1] -
+ * cu_q[b] queries and lk = cu_k[b+1] - cu_k[b] keys, bottom-right causal;
+ * W = tm_mask_words(max_seqlen_k, tile_n, g).  A key sequence longer than
+ * max_seqlen_k is reported by tm_get_device_error (TM_ERR_INVALID_ARG) and
+ * its rows are not written. */
+tm_status tm_build_mask_varlen(uint32_t* bitmask, int32_t Hq, const int32_t* cu_seqlens_q,
+                               const int32_t* cu_seqlens_k, int32_t batch, int32_t max_seqlen_q,
+                               int32_t max_seqlen_k, int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal,
+                               double p, uint64_t seed, int32_t force_diag, int32_t force_sink,
+                               int64_t mask_head_stride, void* stream);
+
 /* Content-driven routing bitmask (the frontier policy; the pages adjust
  * precision during inference but give no policy).  Same layout, legality and
  * forcing as tm_build_mask.  With symmetric absmax/127 codes the INT8 score
@@ -183,6 +206,12 @@ tm_status tm_route_stats(const uint32_t* bitmask_host, int64_t mask_head_stride,
                          int64_t Lq, int64_t Lk, int32_t tile_m, int32_t tile_n, int32_t g,
                          int32_t causal, double* n_vis, double* e8);
 
+/* tm_route_stats with separate (host) key offsets per sequence. */
+tm_status tm_route_stats_varlen(const uint32_t* mask_host, int64_t mask_head_stride, int32_t Hq,
+                                const int32_t* cu_seqlens_q_host, const int32_t* cu_seqlens_k_host, int32_t batch,
+                                int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal, double* n_vis,
+                                double* e8);
+
 /* ---------------------------------------------------------------------------
  * tm_attn_fwd -- fused tile-routed attention forward (prefill).
  *
@@ -212,6 +241,20 @@ tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
                       const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen,
                       const uint32_t* bitmask, int64_t mask_head_stride,
                       int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal, void* stream);
+
+/* tm_attn_fwd with separate key offsets (prefix-cached prefill, also over an
+ * INT8 K/V cache): sequence b's queries are rows cu_seqlens_q[b] .. of q and
+ * out, its keys rows cu_seqlens_k[b] .. of k and v (or of the cache), and
+ * query i of a sequence sees key j iff j < lk and (not causal or
+ * j <= i + lk - lq).  The bitmask is laid out as by tm_build_mask_varlen and
+ * the tile scales as by tm_quantize_qk_varlen.  A key sequence longer than
+ * max_seqlen_k is reported by tm_get_device_error (TM_ERR_INVALID_ARG); its
+ * query rows are not written.  Otherwise as tm_attn_fwd. */
+tm_status tm_attn_fwd_varlen(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch,
+                             int32_t max_seqlen_q, int32_t max_seqlen_k, const uint32_t* bitmask,
+                             int64_t mask_head_stride, int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal,
+                             void* stream);
 
 /* ---------------------------------------------------------------------------
  * tm_attn_fwd_routed_noalloc -- the routed prefill step for callers that

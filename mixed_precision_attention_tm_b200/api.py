@@ -22,11 +22,13 @@ from . import ops
 class TileMixPrefill:
     def __init__(self, Lq, Lk, hq, hkv, d, *, causal=True, tile_m=128, tile_n=128, g=1, p=None,
                  seed=0, force_diag=False, force_sink=False, cu_seqlens=None, int8_cache=False,
-                 tau=None, device="cuda"):
+                 tau=None, cu_seqlens_k=None, device="cuda"):
         """p: Bernoulli INT8 probability per eligible group (seeded mask);
         tau: instead of p, the content-driven policy (INT8 iff the tile
         scales' score-error bound s_q * s_k is at most tau).  Neither: all
-        FP16."""
+        FP16.  cu_seqlens_k: key offsets per sequence when they differ from
+        cu_seqlens (prefix-cached prefill: Lq = total new queries, Lk = total
+        keys)."""
         self.shape = (Lq, Lk, hq, hkv, d)
         self.causal, self.tile_m, self.tile_n, self.g = causal, tile_m, tile_n, g
         if p is not None and tau is not None:
@@ -41,6 +43,13 @@ class TileMixPrefill:
         cu_h = None if cu_seqlens is None else cu_seqlens.to("cpu", torch.int32).contiguous()
         self.cu_h = cu_h
         self.max_seqlen = None if cu_h is None else int((cu_h[1:] - cu_h[:-1]).max())
+        if cu_seqlens_k is not None and cu_seqlens is None:
+            raise ValueError("cu_seqlens_k needs cu_seqlens")
+        if cu_seqlens_k is not None and tau is not None:
+            raise ValueError("the scale policy takes shared query / key offsets")
+        self.cu_k = None if cu_seqlens_k is None else cu_seqlens_k.to(self.device, torch.int32)
+        self.ck_h = None if cu_seqlens_k is None else cu_seqlens_k.to("cpu", torch.int32).contiguous()
+        self.max_seqlen_k = None if self.ck_h is None else int((self.ck_h[1:] - self.ck_h[:-1]).max())
         dev = self.device
         self.q = torch.empty((Lq, hq, d), dtype=torch.float16, device=dev)
         if int8_cache:
@@ -62,10 +71,11 @@ class TileMixPrefill:
             self.q_quant = (torch.empty((Lq, hq, d), dtype=torch.int8, device=dev),
                             torch.empty((nqt, hq), dtype=torch.float32, device=dev))
             if not int8_cache:
-                nkt = ops.count_tiles(Lk, tile_n, cu_np)
+                ck_np = cu_np if self.ck_h is None else self.ck_h.numpy()
+                nkt = ops.count_tiles(Lk, tile_n, ck_np)
                 self.k_quant = (torch.empty((Lk, hkv, d), dtype=torch.int8, device=dev),
                                 torch.empty((nkt, hkv), dtype=torch.float32, device=dev))
-            maxk = Lk if cu_h is None else self.max_seqlen
+            maxk = Lk if cu_h is None else (self.max_seqlen if self.ck_h is None else self.max_seqlen_k)
             self.bitmask = torch.empty((hq, nqt, ops.mask_words(maxk, tile_n, g)), dtype=torch.int32,
                                        device=dev)
         self.launches_per_step = 1 + (3 if self.routed and not int8_cache else 2 if self.routed else 0)
@@ -96,7 +106,8 @@ class TileMixPrefill:
         kq = (None, None) if self.k_quant is None else self.k_quant
         ops.quantize_qk(self.q, None if self.int8_cache else self.k, tile_m=self.tile_m, tile_n=self.tile_n,
                         cu_seqlens=self.cu, max_seqlen=self.max_seqlen, cu_seqlens_host=self.cu_h,
-                        out=(*self.q_quant, *kq))
+                        out=(*self.q_quant, *kq), cu_seqlens_k=self.cu_k, max_seqlen_k=self.max_seqlen_k,
+                        cu_seqlens_k_host=self.ck_h)
 
     def mask(self):
         Lq, Lk = self.shape[0], self.shape[1]
@@ -111,7 +122,8 @@ class TileMixPrefill:
                        causal=self.causal, p=self.p, seed=self.seed, force_diag=self.force_diag,
                        force_sink=self.force_sink, Lq=Lq, Lk=Lk, cu_seqlens=self.cu,
                        max_seqlen=self.max_seqlen, device=self.device, cu_seqlens_host=self.cu_h,
-                       out=self.bitmask)
+                       out=self.bitmask, cu_seqlens_k=self.cu_k, max_seqlen_k=self.max_seqlen_k,
+                       cu_seqlens_k_host=self.ck_h)
 
     def attend(self):
         kv = (self.kc, self.ks, self.vc, self.vs) if self.int8_cache else None
@@ -120,7 +132,8 @@ class TileMixPrefill:
                             bitmask=self.bitmask if self.routed else None,
                             q_quant=self.q_quant if self.routed else None,
                             k_quant=self.k_quant if self.routed else None, kv_cache=kv,
-                            cu_seqlens=self.cu, max_seqlen=self.max_seqlen, cu_seqlens_host=self.cu_h)
+                            cu_seqlens=self.cu, max_seqlen=self.max_seqlen, cu_seqlens_host=self.cu_h,
+                            cu_seqlens_k=self.cu_k, max_seqlen_k=self.max_seqlen_k)
 
     def run(self):
         """One prefill step on the resident inputs; returns the device output."""

@@ -84,6 +84,8 @@ struct Params {
   int64_t mask_hs;
   int W;
   const int32_t* cu;
+  const int32_t* cu_k;     // key offsets (= cu unless separate)
+  int64_t max_lk;          // longest key row the launch was sized for
   int64_t Lq, Lk;          // lengths without cu_seqlens
   int Hq, Hkv, tile_m, g, causal, n_qt_max, batch;
   float scale_log2;        // sigma * log2(e)
@@ -126,8 +128,16 @@ __global__ void __launch_bounds__(192, 1)
   const int I = p.n_qt_max - 1 - t1 / p.batch;
   const SeqInfo sq = seq_info(p.cu, b, p.Lq, p.tile_m);
   const int64_t Lq = sq.len;
-  const int64_t Lk = p.cu ? sq.len : p.Lk;
-  const int64_t kstart = p.cu ? sq.start : 0;
+  // keys of sequence b: rows cu_k[b] .. (cu_k = cu unless the key offsets
+  // differ, as in prefix-cached prefill); a longer key row than the launch
+  // was sized for (mask words, key scales) is an argument error
+  const SeqInfo skq = seq_info(p.cu_k, b, p.Lk, BN);
+  const int64_t Lk = p.cu_k ? skq.len : p.Lk;
+  const int64_t kstart = p.cu_k ? skq.start : 0;
+  if (p.cu_k != nullptr && Lk > p.max_lk) {
+    if (threadIdx.x == 0) dev_error(p.err, TM_DEVERR_SEQLEN);
+    return;
+  }
   if (p.cu != nullptr && I == 0 && threadIdx.x == 0 &&
       Lq > static_cast<int64_t>(p.n_qt_max) * p.tile_m)
     dev_error(p.err, TM_DEVERR_SEQLEN);
@@ -280,7 +290,7 @@ __global__ void __launch_bounds__(192, 1)
     if (row_ok) lim = p.causal ? min(Lk - 1, i_row + Lk - Lq) : Lk - 1;
     float c8_row = 0.f;
     if (mrow != nullptr) c8_row = __ldg(p.q_scales + ig * p.Hq + h) * p.scale_log2;
-    const SeqInfo sk = seq_info(p.cu, b, p.Lk, BN);  // key-tile numbering of this sequence
+    const SeqInfo sk = seq_info(p.cu_k, b, p.Lk, BN);  // key-tile numbering of this sequence
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nJ; ++j) {
@@ -404,7 +414,8 @@ std::mutex g_attr_mu;
 
 template <int D, int BN>
 tm_status launch(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
-                 const int32_t* cu, int32_t batch, int32_t max_seqlen, const uint32_t* bitmask,
+                 const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
+                 const uint32_t* bitmask,
                  int64_t mask_hs, int32_t tile_m, int32_t g, int32_t causal, cudaStream_t stream) {
   using C = Cfg<D, BN>;
   static bool attr_done = false;
@@ -450,6 +461,7 @@ tm_status launch(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_
   p.bitmask = bitmask;
   p.mask_hs = mask_hs;
   p.cu = cu;
+  p.cu_k = cu ? (cu_k ? cu_k : cu) : nullptr;
   p.Lq = q->T;
   p.Lk = k->T;
   p.Hq = static_cast<int>(q->H);
@@ -458,8 +470,9 @@ tm_status launch(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_
   p.g = g;
   p.causal = causal ? 1 : 0;
   p.batch = cu ? batch : 1;
-  const int64_t maxq = cu ? max_seqlen : q->T;
-  const int64_t maxk = cu ? max_seqlen : k->T;
+  const int64_t maxq = cu ? max_q : q->T;
+  const int64_t maxk = cu ? max_k : k->T;
+  p.max_lk = maxk;
   p.n_qt_max = static_cast<int>((maxq + tile_m - 1) / tile_m);
   p.W = tm_mask_words(maxk, BN, g);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
@@ -486,12 +499,15 @@ tm_status check_fp16(const tm_tensor* t, int64_t d) {
 }  // namespace
 }  // namespace tmk
 
-extern "C" tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v,
-                                 tm_tensor* out, const int32_t* cu_seqlens, int32_t batch,
-                                 int32_t max_seqlen, const uint32_t* bitmask,
-                                 int64_t mask_head_stride, int32_t tile_m, int32_t tile_n,
-                                 int32_t g, int32_t causal, void* stream) {
-  using namespace tmk;
+namespace tmk {
+namespace {
+
+// Shared body of tm_attn_fwd (cu_k null: keys use the query offsets) and
+// tm_attn_fwd_varlen (separate key offsets).
+tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                        const int32_t* cu_seqlens, const int32_t* cu_k, int32_t batch, int32_t max_seqlen,
+                        int32_t max_k, const uint32_t* bitmask, int64_t mask_head_stride, int32_t tile_m,
+                        int32_t tile_n, int32_t g, int32_t causal, void* stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return TM_ERR_INVALID_ARG;
   const int64_t D = q->d;
   if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
@@ -504,6 +520,10 @@ extern "C" tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const t
   if (out->T != q->T || out->H != q->H) return TM_ERR_INVALID_ARG;
   if (q->H % k->H != 0 || q->H > 65535 || k->H <= 0) return TM_ERR_INVALID_ARG;
   if (cu_seqlens != nullptr && (batch <= 0 || max_seqlen <= 0)) return TM_ERR_INVALID_ARG;
+  if (cu_k != nullptr && (cu_seqlens == nullptr || max_k <= 0)) return TM_ERR_INVALID_ARG;
+  // with shared offsets the key rows are the query rows
+  const bool shared = cu_seqlens != nullptr && cu_k == nullptr;
+  if (shared) max_k = max_seqlen;
   if (bitmask != nullptr) {
     if (reinterpret_cast<uintptr_t>(bitmask) & 3u) return TM_ERR_INVALID_ARG;
     if (q->codes == nullptr || !aligned16(q->codes) || q->scale_kind != TM_SCALE_TILE || q->scales == nullptr)
@@ -519,10 +539,10 @@ extern "C" tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const t
         (reinterpret_cast<uintptr_t>(v->scales) & 1u))
       return TM_ERR_INVALID_ARG;
     if (k->T != v->T || k->H != v->H || k->d != D || v->d != D || k->T < 0) return TM_ERR_INVALID_ARG;
-    if (cu_seqlens != nullptr && k->T != q->T) return TM_ERR_INVALID_ARG;
+    if (shared && k->T != q->T) return TM_ERR_INVALID_ARG;
     if (D != 128 || tile_n != 128) return TM_ERR_UNSUPPORTED;
-    return launch_attn_cache(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride, tile_m, g,
-                             causal, as_stream(stream));
+    return launch_attn_cache(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
+                             tile_m, g, causal, as_stream(stream));
   }
   st = check_fp16(k, D);
   if (st != TM_OK) return st;
@@ -530,27 +550,48 @@ extern "C" tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const t
   if (st != TM_OK) return st;
   if (k->T != v->T || k->H != v->H) return TM_ERR_INVALID_ARG;
   if (q->H % k->H != 0 || q->H > 65535) return TM_ERR_INVALID_ARG;
-  if (cu_seqlens != nullptr) {
-    if (batch <= 0 || max_seqlen <= 0 || k->T != q->T) return TM_ERR_INVALID_ARG;
-  }
+  if (shared && k->T != q->T) return TM_ERR_INVALID_ARG;
   if (bitmask != nullptr) {
     if (k->codes == nullptr || !aligned16(k->codes) || k->scale_kind != TM_SCALE_TILE || k->scales == nullptr)
       return TM_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);
   if (tile_m == 128 && tile_n == 128)
-    return launch_attn_pair(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride, g,
-                            causal, s);
+    return launch_attn_pair(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
+                            g, causal, s);
   if (D == 128) {
     if (tile_n == 128)
-      return launch<128, 128>(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride,
+      return launch<128, 128>(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
                               tile_m, g, causal, s);
-    return launch<128, 64>(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride,
+    return launch<128, 64>(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
                            tile_m, g, causal, s);
   }
   if (tile_n == 128)
-    return launch<64, 128>(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride,
+    return launch<64, 128>(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
                            tile_m, g, causal, s);
-  return launch<64, 64>(q, k, v, out, cu_seqlens, batch, max_seqlen, bitmask, mask_head_stride,
+  return launch<64, 64>(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
                         tile_m, g, causal, s);
+}
+
+}  // namespace
+}  // namespace tmk
+
+extern "C" tm_status tm_attn_fwd(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v,
+                                 tm_tensor* out, const int32_t* cu_seqlens, int32_t batch,
+                                 int32_t max_seqlen, const uint32_t* bitmask,
+                                 int64_t mask_head_stride, int32_t tile_m, int32_t tile_n,
+                                 int32_t g, int32_t causal, void* stream) {
+  return tmk::attn_fwd_impl(q, k, v, out, cu_seqlens, nullptr, batch, max_seqlen, 0, bitmask, mask_head_stride,
+                            tile_m, tile_n, g, causal, stream);
+}
+
+extern "C" tm_status tm_attn_fwd_varlen(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v,
+                                        tm_tensor* out, const int32_t* cu_seqlens_q,
+                                        const int32_t* cu_seqlens_k, int32_t batch, int32_t max_seqlen_q,
+                                        int32_t max_seqlen_k, const uint32_t* bitmask,
+                                        int64_t mask_head_stride, int32_t tile_m, int32_t tile_n, int32_t g,
+                                        int32_t causal, void* stream) {
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return TM_ERR_INVALID_ARG;
+  return tmk::attn_fwd_impl(q, k, v, out, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q, max_seqlen_k, bitmask,
+                            mask_head_stride, tile_m, tile_n, g, causal, stream);
 }

@@ -132,6 +132,8 @@ struct Params2 {
   int64_t mask_hs;
   int W;
   const int32_t* cu;
+  const int32_t* cu_k;   // key offsets (= cu unless separate)
+  int64_t max_lk;        // longest key row the launch was sized for
   int64_t Lq, Lk;
   int Hq, Hkv, g, causal, n_pair_max, n_qt_max, batch;
   int kv_chunk;            // KV heads per scheduling chunk (divides Hkv)
@@ -191,8 +193,16 @@ __global__ void __launch_bounds__(384, 1)
   const int P = p.n_pair_max - 1 - rest / p.batch;
   const SeqInfo sq = seq_info(p.cu, b, p.Lq, 128);
   const int64_t Lq = sq.len;
-  const int64_t Lk = p.cu ? sq.len : p.Lk;
-  const int64_t kstart = p.cu ? sq.start : 0;
+  // keys of sequence b: rows cu_k[b] .. (cu_k = cu unless the key offsets
+  // differ, as in prefix-cached prefill); a longer key row than the launch
+  // was sized for (mask words, key scales) is an argument error
+  const SeqInfo skq = seq_info(p.cu_k, b, p.Lk, BN);
+  const int64_t Lk = p.cu_k ? skq.len : p.Lk;
+  const int64_t kstart = p.cu_k ? skq.start : 0;
+  if (p.cu_k != nullptr && Lk > p.max_lk) {
+    if (threadIdx.x == 0) dev_error(p.err, TM_DEVERR_SEQLEN);
+    return;
+  }
   if (p.cu != nullptr && P == 0 && threadIdx.x == 0 &&
       Lq > static_cast<int64_t>(p.n_qt_max) * 128)
     dev_error(p.err, TM_DEVERR_SEQLEN);
@@ -718,7 +728,7 @@ __global__ void __launch_bounds__(384, 1)
     if (row_ok) lim = p.causal ? min(Lk - 1, i_row + Lk - Lq) : Lk - 1;
     float c8_row = 0.f;
     if (T.mrow != nullptr) c8_row = __ldg(p.q_scales + T.ig * p.Hq + h) * p.scale_log2;
-    const SeqInfo sk = seq_info(p.cu, b, p.Lk, BN);
+    const SeqInfo sk = seq_info(p.cu_k, b, p.Lk, BN);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     TM_TRACE_DECL
@@ -930,10 +940,11 @@ constexpr int64_t kDualIssuerKeyTiles = 64;
 
 template <int D>
 tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
-                      const int32_t* cu, int32_t batch, int32_t max_seqlen, const uint32_t* bitmask,
+                      const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
+                      const uint32_t* bitmask,
                       int64_t mask_hs, int32_t g, int32_t causal, cudaStream_t stream) {
   using C = Cfg2<D>;
-  const int64_t maxk_tiles = ((cu ? max_seqlen : k->T) + 127) / 128;
+  const int64_t maxk_tiles = ((cu ? max_k : k->T) + 127) / 128;
   const bool dual = maxk_tiles >= kDualIssuerKeyTiles;
   tm_status st = dual ? prepare_pair_kernel<D, true>() : prepare_pair_kernel<D, false>();
   if (st != TM_OK) return st;
@@ -968,6 +979,7 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
   p.bitmask = bitmask;
   p.mask_hs = mask_hs;
   p.cu = cu;
+  p.cu_k = cu ? (cu_k ? cu_k : cu) : nullptr;
   p.Lq = q->T;
   p.Lk = k->T;
   p.Hq = static_cast<int>(q->H);
@@ -975,8 +987,9 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
   p.g = g;
   p.causal = causal ? 1 : 0;
   p.batch = cu ? batch : 1;
-  const int64_t maxq = cu ? max_seqlen : q->T;
-  const int64_t maxk = cu ? max_seqlen : k->T;
+  const int64_t maxq = cu ? max_q : q->T;
+  const int64_t maxk = cu ? max_k : k->T;
+  p.max_lk = maxk;
   p.n_qt_max = static_cast<int>((maxq + 127) / 128);
   p.n_pair_max = (p.n_qt_max + 1) / 2;
   p.W = tm_mask_words(maxk, 128, g);
@@ -1008,12 +1021,12 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
 }  // namespace
 
 tm_status launch_attn_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
-                           const int32_t* cu, int32_t batch, int32_t max_seqlen,
+                           const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
                            const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
                            cudaStream_t stream) {
   if (q->d == 128)
-    return launch_pair<128>(q, k, v, out, cu, batch, max_seqlen, bitmask, mask_hs, g, causal, stream);
-  return launch_pair<64>(q, k, v, out, cu, batch, max_seqlen, bitmask, mask_hs, g, causal, stream);
+    return launch_pair<128>(q, k, v, out, cu, cu_k, batch, max_q, max_k, bitmask, mask_hs, g, causal, stream);
+  return launch_pair<64>(q, k, v, out, cu, cu_k, batch, max_q, max_k, bitmask, mask_hs, g, causal, stream);
 }
 
 }  // namespace tmk

@@ -113,6 +113,8 @@ struct ParamsC {
   int64_t mask_hs;
   int W;
   const int32_t* cu;
+  const int32_t* cu_k;   // key offsets (= cu unless separate)
+  int64_t max_lk;        // longest key row the launch was sized for
   int64_t Lq, Lk;
   int Hq, Hkv, tile_m, g, causal, n_qt_max, batch;
   float scale_log2;
@@ -190,8 +192,16 @@ __global__ void __launch_bounds__(384, 1)
   const int I = p.n_qt_max - 1 - t1 / p.batch;
   const SeqInfo sq = seq_info(p.cu, b, p.Lq, p.tile_m);
   const int64_t Lq = sq.len;
-  const int64_t Lk = p.cu ? sq.len : p.Lk;
-  const int64_t kstart = p.cu ? sq.start : 0;
+  // keys of sequence b: rows cu_k[b] .. (cu_k = cu unless the key offsets
+  // differ, as in prefix-cached prefill); a longer key row than the launch
+  // was sized for (mask words, key scales) is an argument error
+  const SeqInfo skq = seq_info(p.cu_k, b, p.Lk, BN);
+  const int64_t Lk = p.cu_k ? skq.len : p.Lk;
+  const int64_t kstart = p.cu_k ? skq.start : 0;
+  if (p.cu_k != nullptr && Lk > p.max_lk) {
+    if (threadIdx.x == 0) dev_error(p.err, TM_DEVERR_SEQLEN);
+    return;
+  }
   if (p.cu != nullptr && I == 0 && threadIdx.x == 0 && Lq > static_cast<int64_t>(p.n_qt_max) * p.tile_m)
     dev_error(p.err, TM_DEVERR_SEQLEN);
   if (static_cast<int64_t>(I) * p.tile_m >= Lq) return;
@@ -560,7 +570,7 @@ std::mutex g_mu_c;
 }  // namespace
 
 tm_status launch_attn_cache(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
-                            const int32_t* cu, int32_t batch, int32_t max_seqlen,
+                            const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
                             const uint32_t* bitmask, int64_t mask_hs, int32_t tile_m, int32_t g,
                             int32_t causal, cudaStream_t stream) {
   using C = CfgC;
@@ -606,6 +616,7 @@ tm_status launch_attn_cache(const tm_tensor* q, const tm_tensor* k, const tm_ten
   p.bitmask = bitmask;
   p.mask_hs = mask_hs;
   p.cu = cu;
+  p.cu_k = cu ? (cu_k ? cu_k : cu) : nullptr;
   p.Lq = q->T;
   p.Lk = k->T;
   p.Hq = static_cast<int>(q->H);
@@ -614,8 +625,9 @@ tm_status launch_attn_cache(const tm_tensor* q, const tm_tensor* k, const tm_ten
   p.g = g;
   p.causal = causal ? 1 : 0;
   p.batch = cu ? batch : 1;
-  const int64_t maxq = cu ? max_seqlen : q->T;
-  const int64_t maxk = cu ? max_seqlen : k->T;
+  const int64_t maxq = cu ? max_q : q->T;
+  const int64_t maxk = cu ? max_k : k->T;
+  p.max_lk = maxk;
   p.n_qt_max = static_cast<int>((maxq + tile_m - 1) / tile_m);
   p.W = tm_mask_words(maxk, 128, g);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(C::D)));

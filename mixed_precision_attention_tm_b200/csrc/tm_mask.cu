@@ -71,12 +71,17 @@ __host__ __device__ inline uint32_t mask_word(const MaskArgs& a, int h, int64_t 
 
 // One warp per (query tile, sequence, head); lanes stride over the W words.
 __global__ void build_mask_kernel(uint32_t* __restrict__ bm, int64_t head_stride,
-                                  const int32_t* __restrict__ cu, int64_t Lq, int64_t Lk,
-                                  MaskArgs a, DevErr err) {
+                                  const int32_t* __restrict__ cu, const int32_t* __restrict__ cu_k,
+                                  int64_t Lq, int64_t Lk, int64_t max_lk, MaskArgs a, DevErr err) {
   const int I = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
   SeqInfo s = seq_info(cu, b, Lq, a.tile_m);
   const int64_t lq = s.len;
-  const int64_t lk = cu ? s.len : Lk;
+  // key length: from cu_k when the key offsets differ from the query offsets
+  const int64_t lk = cu_k ? seq_info(cu_k, b, Lk, a.tile_n).len : (cu ? s.len : Lk);
+  if (cu_k != nullptr && lk > max_lk) {   // the row of W words was sized for max_lk
+    if (I == 0 && threadIdx.x == 0) dev_error(err, TM_DEVERR_SEQLEN);
+    return;
+  }
   if (cu != nullptr && I == 0 && threadIdx.x == 0 &&
       lq > static_cast<int64_t>(gridDim.x) * a.tile_m)
     dev_error(err, TM_DEVERR_SEQLEN);
@@ -158,8 +163,9 @@ tm_status check_mask_args(int32_t Hq, int32_t tile_m, int32_t tile_n, int32_t g,
 
 extern "C" {
 
-tm_status tm_build_mask(uint32_t* bitmask, int32_t Hq, const int32_t* cu_seqlens, int32_t batch,
-                        int32_t max_seqlen, int64_t Lq, int64_t Lk, int32_t tile_m, int32_t tile_n,
+static tm_status build_mask_impl(uint32_t* bitmask, int32_t Hq, const int32_t* cu_seqlens,
+                                 const int32_t* cu_k, int32_t batch, int32_t max_seqlen, int32_t max_k,
+                                 int64_t Lq, int64_t Lk, int32_t tile_m, int32_t tile_n,
                         int32_t g, int32_t causal, double p, uint64_t seed, int32_t force_diag,
                         int32_t force_sink, int64_t mask_head_stride, void* stream) {
   using namespace tmk;
@@ -167,7 +173,8 @@ tm_status tm_build_mask(uint32_t* bitmask, int32_t Hq, const int32_t* cu_seqlens
   if (st != TM_OK) return st;
   if (bitmask == nullptr || reinterpret_cast<uintptr_t>(bitmask) % 4) return TM_ERR_INVALID_ARG;
   const int64_t maxq = cu_seqlens ? max_seqlen : Lq;
-  const int64_t maxk = cu_seqlens ? max_seqlen : Lk;
+  const int64_t maxk = cu_seqlens ? (cu_k ? max_k : max_seqlen) : Lk;
+  if (cu_k != nullptr && (cu_seqlens == nullptr || max_k <= 0)) return TM_ERR_INVALID_ARG;
   if (cu_seqlens != nullptr && (batch <= 0 || max_seqlen <= 0)) return TM_ERR_INVALID_ARG;
   if (maxq < 0 || maxk < 0) return TM_ERR_INVALID_ARG;
   MaskArgs a{Hq, tile_m, tile_n, g, causal ? 1 : 0, p, seed, force_diag ? 1 : 0,
@@ -180,9 +187,27 @@ tm_status tm_build_mask(uint32_t* bitmask, int32_t Hq, const int32_t* cu_seqlens
   if (nqt_max > 0x7fffffff || nb > 65535 || Hq > 65535) return TM_ERR_UNSUPPORTED;
   dim3 grid(static_cast<unsigned>(nqt_max), static_cast<unsigned>(nb), static_cast<unsigned>(Hq));
   DevErr err{device_error_word()};
-  build_mask_kernel<<<grid, 32, 0, as_stream(stream)>>>(bitmask, mask_head_stride, cu_seqlens, Lq,
-                                                        Lk, a, err);
+  build_mask_kernel<<<grid, 32, 0, as_stream(stream)>>>(bitmask, mask_head_stride, cu_seqlens, cu_k, Lq,
+                                                        Lk, maxk, a, err);
   return check_cuda(cudaGetLastError());
+}
+
+tm_status tm_build_mask(uint32_t* bitmask, int32_t Hq, const int32_t* cu_seqlens, int32_t batch,
+                        int32_t max_seqlen, int64_t Lq, int64_t Lk, int32_t tile_m, int32_t tile_n,
+                        int32_t g, int32_t causal, double p, uint64_t seed, int32_t force_diag,
+                        int32_t force_sink, int64_t mask_head_stride, void* stream) {
+  return build_mask_impl(bitmask, Hq, cu_seqlens, nullptr, batch, max_seqlen, 0, Lq, Lk, tile_m, tile_n, g,
+                         causal, p, seed, force_diag, force_sink, mask_head_stride, stream);
+}
+
+tm_status tm_build_mask_varlen(uint32_t* bitmask, int32_t Hq, const int32_t* cu_seqlens_q,
+                               const int32_t* cu_seqlens_k, int32_t batch, int32_t max_seqlen_q,
+                               int32_t max_seqlen_k, int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal,
+                               double p, uint64_t seed, int32_t force_diag, int32_t force_sink,
+                               int64_t mask_head_stride, void* stream) {
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return TM_ERR_INVALID_ARG;
+  return build_mask_impl(bitmask, Hq, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q, max_seqlen_k, 0, 0, tile_m,
+                         tile_n, g, causal, p, seed, force_diag, force_sink, mask_head_stride, stream);
 }
 
 tm_status tm_build_mask_scale_policy(uint32_t* bitmask, int32_t Hq, int32_t Hkv, const int32_t* cu_seqlens,
@@ -254,11 +279,13 @@ tm_status tm_build_mask_host(uint32_t* bitmask_host, int32_t Hq, const int32_t* 
   return TM_OK;
 }
 
-tm_status tm_route_stats(const uint32_t* bitmask_host, int64_t mask_head_stride, int32_t Hq,
-                         const int32_t* cu_seqlens_host, int32_t batch, int64_t Lq, int64_t Lk,
-                         int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal, double* n_vis,
-                         double* e8) {
+static tm_status route_stats_impl(const uint32_t* bitmask_host, int64_t mask_head_stride, int32_t Hq,
+                                  const int32_t* cu_seqlens_host, const int32_t* cu_k_host, int32_t batch,
+                                  int64_t Lq, int64_t Lk, int32_t tile_m, int32_t tile_n, int32_t g,
+                                  int32_t causal, double* n_vis, double* e8) {
   using namespace tmk;
+  if (cu_k_host != nullptr && cu_seqlens_host == nullptr) return TM_ERR_INVALID_ARG;
+  const int32_t* ck = cu_k_host ? cu_k_host : cu_seqlens_host;   // key offsets
   if (n_vis == nullptr || e8 == nullptr || Hq <= 0 || tile_m <= 0 || tile_n <= 0 || g <= 0)
     return TM_ERR_INVALID_ARG;
   const int nb = cu_seqlens_host ? batch : 1;
@@ -266,8 +293,7 @@ tm_status tm_route_stats(const uint32_t* bitmask_host, int64_t mask_head_stride,
   int64_t maxk = Lk;
   if (cu_seqlens_host) {
     maxk = 0;
-    for (int b = 0; b < nb; ++b)
-      maxk = std::max<int64_t>(maxk, cu_seqlens_host[b + 1] - cu_seqlens_host[b]);
+    for (int b = 0; b < nb; ++b) maxk = std::max<int64_t>(maxk, ck[b + 1] - ck[b]);
   }
   const int W = tm_mask_words(maxk, tile_n, g);
   long double nv = 0, ne8 = 0;
@@ -275,7 +301,7 @@ tm_status tm_route_stats(const uint32_t* bitmask_host, int64_t mask_head_stride,
   std::vector<int64_t> per_tile;
   for (int b = 0; b < nb; ++b) {
     const int64_t lq = cu_seqlens_host ? cu_seqlens_host[b + 1] - cu_seqlens_host[b] : Lq;
-    const int64_t lk = cu_seqlens_host ? lq : Lk;
+    const int64_t lk = cu_seqlens_host ? ck[b + 1] - ck[b] : Lk;
     const int64_t n = (lq + tile_m - 1) / tile_m;
     for (int64_t I = 0; I < n; ++I, ++ig) {
       const int64_t r0 = I * tile_m;
@@ -306,6 +332,23 @@ tm_status tm_route_stats(const uint32_t* bitmask_host, int64_t mask_head_stride,
   *n_vis = static_cast<double>(nv);
   *e8 = static_cast<double>(ne8);
   return TM_OK;
+}
+
+tm_status tm_route_stats(const uint32_t* bitmask_host, int64_t mask_head_stride, int32_t Hq,
+                         const int32_t* cu_seqlens_host, int32_t batch, int64_t Lq, int64_t Lk,
+                         int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal, double* n_vis,
+                         double* e8) {
+  return route_stats_impl(bitmask_host, mask_head_stride, Hq, cu_seqlens_host, nullptr, batch, Lq, Lk, tile_m,
+                          tile_n, g, causal, n_vis, e8);
+}
+
+tm_status tm_route_stats_varlen(const uint32_t* bitmask_host, int64_t mask_head_stride, int32_t Hq,
+                                const int32_t* cu_seqlens_q_host, const int32_t* cu_seqlens_k_host,
+                                int32_t batch, int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal,
+                                double* n_vis, double* e8) {
+  if (cu_seqlens_q_host == nullptr || cu_seqlens_k_host == nullptr) return TM_ERR_INVALID_ARG;
+  return route_stats_impl(bitmask_host, mask_head_stride, Hq, cu_seqlens_q_host, cu_seqlens_k_host, batch, 0, 0,
+                          tile_m, tile_n, g, causal, n_vis, e8);
 }
 
 }  // extern "C"

@@ -135,6 +135,27 @@ tm_status launch_quant(const tm_tensor* x, int8_t* codes, float* scales, const i
 }  // namespace
 }  // namespace tmk
 
+extern "C" tm_status tm_quantize_qk_varlen(const tm_tensor* q, const tm_tensor* k, int8_t* q_codes,
+                                           float* q_scales, int8_t* k_codes, float* k_scales,
+                                           const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                           int32_t batch, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                           int32_t tile_m, int32_t tile_n, void* stream) {
+  using namespace tmk;
+  if ((tile_m != 64 && tile_m != 128) || (tile_n != 64 && tile_n != 128)) return TM_ERR_UNSUPPORTED;
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr || batch <= 0 || max_seqlen_q <= 0) return TM_ERR_INVALID_ARG;
+  tm_status st = check_operand(q);
+  if (st != TM_OK) return st;
+  if (k != nullptr) {
+    st = check_operand(k);
+    if (st != TM_OK) return st;
+    if (k->d != q->d || max_seqlen_k <= 0) return TM_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = as_stream(stream);
+  st = launch_quant(q, q_codes, q_scales, cu_seqlens_q, batch, max_seqlen_q, tile_m, s);
+  if (st != TM_OK || k == nullptr) return st;
+  return launch_quant(k, k_codes, k_scales, cu_seqlens_k, batch, max_seqlen_k, tile_n, s);
+}
+
 extern "C" tm_status tm_quantize_qk(const tm_tensor* q, const tm_tensor* k, int8_t* q_codes,
                                     float* q_scales, int8_t* k_codes, float* k_scales,
                                     const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen,

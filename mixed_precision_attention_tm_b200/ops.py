@@ -68,6 +68,12 @@ def _lib():
             "tm_route_stats": (I32, [P, I64, I32, P, I32, I64, I64, I32, I32, I32, I32,
                                      ctypes.POINTER(D), ctypes.POINTER(D)]),
             "tm_attn_fwd": (I32, [TP, TP, TP, TP, P, I32, I32, P, I64, I32, I32, I32, I32, P]),
+            "tm_attn_fwd_varlen": (I32, [TP, TP, TP, TP, P, P, I32, I32, I32, P, I64, I32, I32, I32, I32, P]),
+            "tm_quantize_qk_varlen": (I32, [TP, TP, P, P, P, P, P, P, I32, I32, I32, I32, I32, P]),
+            "tm_build_mask_varlen": (I32, [P, I32, P, P, I32, I32, I32, I32, I32, I32, I32, D, U64, I32, I32,
+                                           I64, P]),
+            "tm_route_stats_varlen": (I32, [P, I64, I32, P, P, I32, I32, I32, I32, I32,
+                                            ctypes.POINTER(D), ctypes.POINTER(D)]),
             "tm_attn_fwd_routed_noalloc": (I32, [TP, TP, TP, TP, I32, I32, I32, I32, D, U64, I32, I32, P]),
             "tm_selftest_wait_timeout": (I32, [U64, P]),
             "tm_get_device_error": (I32, [P]),
@@ -157,7 +163,7 @@ def mask_words(max_lk, tile_n, g):
 
 # ---------------------------------------------------------------- quantise
 def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqlen=None,
-                cu_seqlens_host=None, out=None):
+                cu_seqlens_host=None, out=None, cu_seqlens_k=None, max_seqlen_k=None, cu_seqlens_k_host=None):
     """Per-tile INT8 codes and fp32 scales of Q (tile_m rows) and K (tile_n
     rows): returns (q_codes [Tq,Hq,d] int8, q_scales [n_qt, Hq] fp32,
     k_codes, k_scales) (the K pair is None when k is None).  out: the same
@@ -170,6 +176,9 @@ def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqle
     if cu_seqlens is not None and max_seqlen is None:
         max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0
     nqt = count_tiles(q.shape[0], tile_m, None if cu_h is None else cu_h.numpy())
+    ck_h = cu_h if cu_seqlens_k is None else _cu_host(cu_seqlens_k, cu_seqlens_k_host)
+    if cu_seqlens_k is not None and max_seqlen_k is None:
+        max_seqlen_k = int((ck_h[1:] - ck_h[:-1]).max()) if batch else 0
     if out is not None:
         qc, qs, kc, ks = out
         _check_buf(qc, q.shape, torch.int8, "q_codes")
@@ -181,15 +190,22 @@ def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqle
         qs = torch.empty((nqt, q.shape[1]), dtype=torch.float32, device=q.device)
         kc = ks = None
     if k is not None and out is not None:
-        nkt = count_tiles(k.shape[0], tile_n, None if cu_h is None else cu_h.numpy())
+        nkt = count_tiles(k.shape[0], tile_n, None if ck_h is None else ck_h.numpy())
         _check_buf(kc, k.shape, torch.int8, "k_codes")
         _check_buf(ks, (nkt, k.shape[1]), torch.float32, "k_scales")
     elif k is not None:
-        nkt = count_tiles(k.shape[0], tile_n, None if cu_h is None else cu_h.numpy())
+        nkt = count_tiles(k.shape[0], tile_n, None if ck_h is None else ck_h.numpy())
         kc = torch.empty(k.shape, dtype=torch.int8, device=k.device)
         ks = torch.empty((nkt, k.shape[1]), dtype=torch.float32, device=k.device)
     qd = _desc(q)
     kd = _desc(k) if k is not None else None
+    if cu_seqlens_k is not None:       # separate key offsets (prefix-cached prefill)
+        st = lib.tm_quantize_qk_varlen(ctypes.byref(qd), None if kd is None else ctypes.byref(kd),
+                                       _ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks), _ptr(cu_seqlens), _ptr(cu_seqlens_k),
+                                       batch, int(max_seqlen or 0), int(max_seqlen_k or 0), tile_m, tile_n,
+                                       _stream())
+        _check(st, "tm_quantize_qk_varlen")
+        return qc, qs, kc, ks
     st = lib.tm_quantize_qk(ctypes.byref(qd), None if kd is None else ctypes.byref(kd),
                             _ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks), _ptr(cu_seqlens), batch,
                             int(max_seqlen or 0), tile_m, tile_n, _stream())
@@ -200,7 +216,7 @@ def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqle
 # ---------------------------------------------------------------- mask
 def build_mask(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False, force_sink=False,
                Lq=None, Lk=None, cu_seqlens=None, max_seqlen=None, device="cuda",
-               cu_seqlens_host=None, out=None):
+               cu_seqlens_host=None, out=None, cu_seqlens_k=None, max_seqlen_k=None, cu_seqlens_k_host=None):
     """Seeded routing bitmask on the device, int32 view [Hq, n_qt, W] of the
     uint32 words (bit 1 = INT8).  The library writes every word, so the
     buffer (out, or a new one) needs no initialisation."""
@@ -213,6 +229,12 @@ def build_mask(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False, forc
         if max_seqlen is None:
             max_seqlen = maxk
         nqt = count_tiles(None, tile_m, cu_h.numpy())
+        if cu_seqlens_k is not None:       # key lengths from the key offsets
+            ck_h = _cu_host(cu_seqlens_k, cu_seqlens_k_host)
+            maxk = int((ck_h[1:] - ck_h[:-1]).max()) if batch else 0
+            if max_seqlen_k is None:
+                max_seqlen_k = maxk
+            maxk = max_seqlen_k
     else:
         maxk = Lk
         nqt = count_tiles(Lq, tile_m)
@@ -221,6 +243,13 @@ def build_mask(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False, forc
         out = torch.empty((Hq, nqt, W), dtype=torch.int32, device=device)
     else:
         _check_buf(out, (Hq, nqt, W), torch.int32, "bitmask")
+    if cu_seqlens_k is not None:
+        st = lib.tm_build_mask_varlen(_ptr(out), Hq, _ptr(cu_seqlens), _ptr(cu_seqlens_k), batch,
+                                      int(max_seqlen or 0), int(max_seqlen_k or 0), tile_m, tile_n, g,
+                                      int(bool(causal)), float(p), ctypes.c_uint64(int(seed) & (2 ** 64 - 1)),
+                                      int(bool(force_diag)), int(bool(force_sink)), nqt * W, _stream())
+        _check(st, "tm_build_mask_varlen")
+        return out
     st = lib.tm_build_mask(_ptr(out), Hq, _ptr(cu_seqlens), batch, int(max_seqlen or 0),
                            int(Lq or 0), int(Lk or 0), tile_m, tile_n, g, int(bool(causal)),
                            float(p), ctypes.c_uint64(int(seed) & (2 ** 64 - 1)),
@@ -284,10 +313,22 @@ def build_mask_host(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False,
     return out
 
 
-def route_stats(mask_host, *, Hq, tile_m, tile_n, g, causal, Lq=None, Lk=None, cu_seqlens_host=None):
+def route_stats(mask_host, *, Hq, tile_m, tile_n, g, causal, Lq=None, Lk=None, cu_seqlens_host=None,
+                cu_seqlens_k_host=None):
     """(n_vis, e8) from a host mask (numpy uint32 [Hm, n_qt, W]) or None."""
     lib = _lib()
     cu = None if cu_seqlens_host is None else np.ascontiguousarray(np.asarray(cu_seqlens_host, np.int32))
+    if cu_seqlens_k_host is not None:
+        ck = np.ascontiguousarray(np.asarray(cu_seqlens_k_host, np.int32))
+        nv, e8 = ctypes.c_double(), ctypes.c_double()
+        ptr, hs = None, 0
+        if mask_host is not None:
+            m = np.ascontiguousarray(mask_host.astype(np.uint32, copy=False))
+            ptr, hs = m.ctypes.data, (0 if m.shape[0] == 1 else m.shape[1] * m.shape[2])
+        st = lib.tm_route_stats_varlen(ptr, hs, Hq, cu.ctypes.data, ck.ctypes.data, len(cu) - 1, tile_m, tile_n,
+                                       g, int(bool(causal)), ctypes.byref(nv), ctypes.byref(e8))
+        _check(st, "tm_route_stats_varlen")
+        return nv.value, e8.value
     batch = 0 if cu is None else len(cu) - 1
     nv, e8 = ctypes.c_double(), ctypes.c_double()
     ptr, hs = None, 0
@@ -305,7 +346,7 @@ def route_stats(mask_host, *, Hq, tile_m, tile_n, g, causal, Lq=None, Lk=None, c
 # ---------------------------------------------------------------- attention
 def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal=False,
              bitmask=None, mask_head_stride=None, q_quant=None, k_quant=None, kv_cache=None,
-             cu_seqlens=None, max_seqlen=None, cu_seqlens_host=None):
+             cu_seqlens=None, max_seqlen=None, cu_seqlens_host=None, cu_seqlens_k=None, max_seqlen_k=None):
     """Fused tile-routed attention.  q: fp16 [Tq,Hq,d]; k, v: fp16 [Tk,Hkv,d]
     (or kv_cache = (k_codes, k_scale16, v_codes, v_scale16)); bitmask: int32
     view [Hm, n_qt, W] (Hm = Hq or 1) or None (all FP16); q_quant / k_quant:
@@ -333,6 +374,16 @@ def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal
     od = _desc(out)
     if bitmask is not None and mask_head_stride is None:
         mask_head_stride = 0 if bitmask.shape[0] == 1 else bitmask.shape[1] * bitmask.shape[2]
+    if cu_seqlens_k is not None:
+        if max_seqlen_k is None:
+            ck_h = _cu_host(cu_seqlens_k, None)
+            max_seqlen_k = int((ck_h[1:] - ck_h[:-1]).max()) if batch else 0
+        st = lib.tm_attn_fwd_varlen(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
+                                    _ptr(cu_seqlens), _ptr(cu_seqlens_k), batch, int(max_seqlen or 0),
+                                    int(max_seqlen_k or 0), _ptr(bitmask), int(mask_head_stride or 0), tile_m,
+                                    tile_n, g, int(bool(causal)), _stream())
+        _check(st, "tm_attn_fwd_varlen")
+        return out
     st = lib.tm_attn_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
                          _ptr(cu_seqlens), batch, int(max_seqlen or 0), _ptr(bitmask),
                          int(mask_head_stride or 0), tile_m, tile_n, g, int(bool(causal)), _stream())

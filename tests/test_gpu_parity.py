@@ -388,3 +388,80 @@ def test_scale_policy_plan_matches_direct_calls():
     direct = ops.attn_fwd(w.q.cuda(), w.k.cuda(), w.v.cuda(), g=2, causal=True, bitmask=m,
                           q_quant=(qc, qs), k_quant=(kc, ks))
     assert torch.equal(out, direct)
+
+
+# ------------------------------------------------------------------ separate key offsets
+# Prefix-cached prefill: sequence b has lq new queries and lk >= lq keys
+# (cu_seqlens_k), bottom-right causal per sequence; fp16 K/V through the
+# 128x128 pair kernel and the 64-row single-tile kernel, and an INT8 cache.
+PREFIX_CASES = [
+    ("pair_causal", dict(lq=[77, 129, 0, 300], lk=[300, 129, 520, 300], hq=4, hkv=2, d=128, causal=True,
+                         tm=128, tn=128, g=2, p=0.6)),
+    ("pair_noncausal_fp16", dict(lq=[200, 33], lk=[1000, 700], hq=2, hkv=1, d=64, causal=False,
+                                 tm=128, tn=128, g=1, p=None)),
+    ("single_tile_64", dict(lq=[90, 64], lk=[250, 64], hq=2, hkv=2, d=128, causal=True, tm=64, tn=64, g=1, p=0.5)),
+    ("int8_cache", dict(lq=[100, 256, 17], lk=[900, 256, 400], hq=4, hkv=1, d=128, causal=True, tm=128, tn=128,
+                        g=2, p=0.7, cache=True)),
+]
+
+
+@pytest.mark.parametrize("name,kw", PREFIX_CASES, ids=[c[0] for c in PREFIX_CASES])
+def test_prefix_prefill_matches_oracle(name, kw):
+    lq, lk = kw["lq"], kw["lk"]
+    hq, hkv, d, causal, tm, tn, g, p = kw["hq"], kw["hkv"], kw["d"], kw["causal"], kw["tm"], kw["tn"], kw["g"], kw["p"]
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    q = inputs.randn_f16((int(cu_q[-1]), hq, d), 40)
+    k = inputs.randn_f16((int(cu_k[-1]), hkv, d), 41)
+    v = inputs.randn_f16((int(cu_k[-1]), hkv, d), 42)
+    seqs = oracle.seq_table(len(q), len(k), cu_q, cu_k)
+    cq, ck = torch.tensor(cu_q).cuda(), torch.tensor(cu_k).cuda()
+    kv = None
+    if kw.get("cache"):
+        kc, ks16 = inputs.int8_kv_cache(k)
+        vc, vs16 = inputs.int8_kv_cache(v)
+        kv = (kc, ks16, vc, vs16)
+    qd = q.cuda()
+    kd = None if kv is not None else k.cuda()
+    qc, qs, kcd, ksd = ops.quantize_qk(qd, kd, tile_m=tm, tile_n=tn, cu_seqlens=cq, cu_seqlens_k=ck)
+    m = mask_u32 = None
+    if p is not None:
+        m = ops.build_mask(hq, tile_m=tm, tile_n=tn, g=g, causal=causal, p=p, seed=9, force_diag=True,
+                           cu_seqlens=cq, cu_seqlens_k=ck)
+        torch.cuda.synchronize()
+        mask_u32 = m.cpu().numpy().view(np.uint32)
+        assert np.array_equal(mask_u32, oracle.build_mask(hq, seqs, tm, tn, g, causal, p, 9, force_diag=True))
+        rq = oracle.quantize_tiles(q.numpy(), seqs, tm, "q")
+        assert np.array_equal(qs.cpu().numpy(), rq[1]) and np.array_equal(qc.cpu().numpy(), rq[0])
+        if kv is None:
+            rk = oracle.quantize_tiles(k.numpy(), seqs, tn, "k")
+            assert np.array_equal(ksd.cpu().numpy(), rk[1]) and np.array_equal(kcd.cpu().numpy(), rk[0])
+    out = ops.attn_fwd(qd, kd, None if kv is not None else v.cuda(), tile_m=tm, tile_n=tn, g=g, causal=causal,
+                       bitmask=m, q_quant=(qc, qs) if m is not None else None,
+                       k_quant=(kcd, ksd) if (m is not None and kv is None) else None,
+                       kv_cache=None if kv is None else tuple(t.cuda() for t in kv),
+                       cu_seqlens=cq, cu_seqlens_k=ck)
+    torch.cuda.synchronize()
+    assert ops.get_device_error() == ops.TM_OK
+    okw = dict(cu_seqlens=cu_q, cu_seqlens_k=cu_k, causal=causal, tile_m=tm, tile_n=tn, g=g)
+    if mask_u32 is not None:
+        okw.update(mask=mask_u32, q_quant=oracle.quantize_tiles(q.numpy(), seqs, tm, "q"))
+        if kv is None:
+            okw["k_quant"] = oracle.quantize_tiles(k.numpy(), seqs, tn, "k")
+    if kv is not None:
+        ref = oracle.attention(q.numpy(), kv_cache=tuple(t.numpy() for t in kv), **okw)
+    else:
+        ref = oracle.attention(q.numpy(), k.numpy(), v.numpy(), **okw)
+    assert max_err(out.cpu(), ref) <= TOL
+
+
+def test_prefix_prefill_longer_keys_than_declared_is_reported():
+    cu_q = torch.tensor([0, 64], dtype=torch.int32).cuda()
+    cu_k = torch.tensor([0, 512], dtype=torch.int32).cuda()
+    q = inputs.randn_f16((64, 2, 128), 1).cuda()
+    k = inputs.randn_f16((512, 2, 128), 2).cuda()
+    v = inputs.randn_f16((512, 2, 128), 3).cuda()
+    ops.attn_fwd(q, k, v, causal=True, cu_seqlens=cu_q, cu_seqlens_k=cu_k, max_seqlen=64, max_seqlen_k=256)
+    torch.cuda.synchronize()
+    assert ops.get_device_error() == ops.TM_ERR_INVALID_ARG
+    assert ops.get_device_error() == ops.TM_OK          # reading clears the word
