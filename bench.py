@@ -145,6 +145,8 @@ def make_workload(name, p, seed):
         return inputs.long_context(p=p if p is not None else 0.5, seed=seed)
     if name == "varlen":
         return inputs.varlen_int8_cache(p=p if p is not None else 0.75, seed=seed)
+    if name == "prefix":
+        return inputs.prefix_int8_cache(p=p if p is not None else 0.75, seed=seed)
     if name == "mlx":
         return inputs.mlx_shape(4096, 4096, 128, 32, 8, True, seed=seed)
     if name == "tiny":
@@ -152,22 +154,52 @@ def make_workload(name, p, seed):
     raise ValueError(name)
 
 
+L2_BYTES = 126 * 1000 * 1000
+FLUSH_BYTES = 256 << 20
+
+
+def step_input_bytes(w):
+    """Bytes a step reads from its resident inputs (Q, K, V or the cache)."""
+    t = [w.q] + ([w.k, w.v] if w.kv_cache is None else list(w.kv_cache))
+    return sum(x.numel() * x.element_size() for x in t if x is not None)
+
+
+def needs_flush(w):
+    return step_input_bytes(w) < 2 * L2_BYTES
+
+
+def data_note(w):
+    """How the workload's synthetic inputs were drawn."""
+    parts = ["seeded N(0,1) fp16"]
+    if "outlier_channels" in w.extra:
+        parts.append("4 outlier channels per KV head x20")
+    if "outlier_tokens" in w.extra:
+        parts.append(f"{w.extra['outlier_tokens']} outlier key tokens x20")
+    if w.kv_cache is not None:
+        parts.append("K/V as a per-token INT8 cache")
+    return "synthetic (" + ", ".join(parts) + ")"
+
+
 def describe(w):
     cfg = {"workload": w.name, "Lq": w.Lq, "Lk": w.Lk, "Hq": w.hq, "Hkv": w.hkv, "d": w.d, "causal": w.causal,
            "tile_m": w.tile_m, "tile_n": w.tile_n, "g": w.g, "int8_group_probability": w.p,
            "force_diag": w.force_diag, "force_sink": w.force_sink,
-           "l2": "inputs larger than L2 (126 MB), no flush" }
+           "l2": ("inputs smaller than twice L2: a 256 MiB buffer is written before every timed step, outside "
+                  "the per-step events" if needs_flush(w) else "inputs larger than L2 (126 MB), no flush")}
     if w.lens is not None:
         cfg["seq_lens"] = [int(x) for x in w.lens]
         cfg["int8_kv_cache"] = w.kv_cache is not None
+    if w.lens_k is not None:
+        cfg["key_lens"] = [int(x) for x in w.lens_k]
     return cfg
 
 
 def route_stats_of(w, mask_host):
     from mixed_precision_attention_tm_b200 import ops
     cu = None if w.cu_seqlens is None else w.cu_seqlens.numpy()
+    ck = None if w.cu_seqlens_k is None else w.cu_seqlens_k.numpy()
     return ops.route_stats(mask_host, Hq=w.hq, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g, causal=w.causal,
-                           Lq=w.Lq, Lk=w.Lk, cu_seqlens_host=cu)
+                           Lq=w.Lq, Lk=w.Lk, cu_seqlens_host=cu, cu_seqlens_k_host=ck)
 
 
 def roofline_time(d, n_vis, e8, p16, p8):
@@ -188,7 +220,8 @@ def run_ours(args, rank, world, local_rank):
     w = make_workload(args.workload, args.p, seed=dist.rank_seed(args.seed, rank))
     plan = TileMixPrefill(w.Lq, w.Lk, w.hq, w.hkv, w.d, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n,
                           g=w.g, p=w.p, seed=w.mask_seed, force_diag=w.force_diag, force_sink=w.force_sink,
-                          cu_seqlens=w.cu_seqlens, int8_cache=w.kv_cache is not None, device=dev)
+                          cu_seqlens=w.cu_seqlens, int8_cache=w.kv_cache is not None, device=dev,
+                          cu_seqlens_k=w.cu_seqlens_k)
     plan.load(w.q, w.k, w.v, w.kv_cache)
     torch.cuda.synchronize()
 
@@ -213,21 +246,31 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     dist.barrier()
     torch.cuda.synchronize()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if needs_flush(w) else None
+    st_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if flush is not None else None
+    st_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if flush is not None else None
     clocks.start()
     time.sleep(0.3)
     t0.record(stream)
     for i in range(K):
+        if flush is not None:
+            flush.zero_()                      # evict the inputs from L2 (outside the step's events)
+            st_a[i].record(stream)
         if plan.routed:
             plan.quantize()
             plan.mask()
         ev_a[i].record(stream)
         plan.attend()
         ev_b[i].record(stream)
+        if flush is not None:
+            st_b[i].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     dist.barrier()
     total_ms = t0.elapsed_time(t1)
+    if flush is not None:
+        total_ms = sum(a.elapsed_time(b) for a, b in zip(st_a, st_b))
     attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev_a, ev_b)) / K
     if ops.get_device_error() != ops.TM_OK:
         raise RuntimeError("device error in timed region")
@@ -255,7 +298,8 @@ def run_ours(args, rank, world, local_rank):
         kvh = None if w.kv_cache is None else tuple(x.pin_memory() for x in w.kv_cache)
         pipe = HostPipeline(w.Lq, w.Lk, w.hq, w.hkv, w.d, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n,
                             g=w.g, p=w.p, seed=w.mask_seed, force_diag=w.force_diag, force_sink=w.force_sink,
-                            cu_seqlens=w.cu_seqlens, int8_cache=w.kv_cache is not None, device=dev)
+                            cu_seqlens=w.cu_seqlens, int8_cache=w.kv_cache is not None, device=dev,
+                          cu_seqlens_k=w.cu_seqlens_k)
         outs = [torch.empty(plan.out.shape, dtype=torch.float16, pin_memory=True) for _ in range(2)]
         ke = max(4, min(K, 20))
         step_in = [(qh, kh, vh, kvh)]
@@ -355,7 +399,7 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f16+i8 (fp32 accumulate)",
-        "data": "synthetic (seeded N(0,1) fp16, outlier channels x20)",
+        "data": data_note(w),
         "config": describe(w),
         "tokens_per_s": world * w.Lq / (ms_step * 1e-3),
         "realised_int8_fraction": e8 / n_vis,
@@ -382,7 +426,8 @@ def cpu_sample_spec(w, n_pairs):
     """Evenly spaced (query tile, head) pairs of the workload."""
     import oracle
     cu = None if w.cu_seqlens is None else w.cu_seqlens.tolist()
-    seqs = oracle.seq_table(w.Lq, w.Lk, cu)
+    ck = None if w.cu_seqlens_k is None else w.cu_seqlens_k.tolist()
+    seqs = oracle.seq_table(w.Lq, w.Lk, cu, ck)
     qt = oracle.tile_table(seqs, w.tile_m, "q")
     out = []
     n = len(qt) * w.hq
@@ -423,7 +468,8 @@ def oracle_pair(w, seqs, tile, h, prep):
 def oracle_prep(w, seqs):
     import oracle
     cu = None if w.cu_seqlens is None else w.cu_seqlens.tolist()
-    prep = dict(cu_seqlens=cu, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g)
+    ck = None if w.cu_seqlens_k is None else w.cu_seqlens_k.tolist()
+    prep = dict(cu_seqlens=cu, cu_seqlens_k=ck, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g)
     if w.kv_cache is not None:
         prep["kv_cache"] = tuple(t.numpy() for t in w.kv_cache)
     if w.p is not None:
@@ -476,7 +522,7 @@ def run_reference(args):
         "metric": "prefill attention TFLOPS (tile-routed FP16/INT8 QK^T, FP16 P.V)",
         "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3 / max(1, args.steps), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) fp16, outlier channels x20)",
+        "vs_baseline": None, "dtype": "f64", "data": data_note(w),
         "config": describe(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"one (query tile, head) pair of {w.name} per step, fp64 NumPy/BLAS; "
@@ -615,7 +661,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="sweep",
-                    choices=["sweep", "long", "varlen", "mlx", "tiny", "mlx_table", "frontier"])
+                    choices=["sweep", "long", "varlen", "prefix", "mlx", "tiny", "mlx_table", "frontier"])
     ap.add_argument("--p", type=float, default=0.75)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-sweep", action="store_true")

@@ -141,6 +141,8 @@ class Workload:
     lens: torch.Tensor | None = None
     kv_cache: tuple | None = None        # (k_codes, k_scale16, v_codes, v_scale16)
     extra: dict = field(default_factory=dict)
+    cu_seqlens_k: torch.Tensor | None = None   # key offsets when they differ (prefix-cached prefill)
+    lens_k: torch.Tensor | None = None
 
     @property
     def Lq(self):
@@ -155,6 +157,10 @@ class Workload:
         if self.lens is not None:
             return int(self.lens.max())
         return max(self.Lq, self.Lk)
+
+    @property
+    def max_seqlen_k(self):
+        return None if self.lens_k is None else int(self.lens_k.max())
 
 
 def tiny(seed=0, p=None):
@@ -211,6 +217,26 @@ def varlen_int8_cache(batch=8, lo=1024, hi=8192, hq=32, hkv=4, d=128, p=0.75, se
     return Workload(f"varlen_cache_b{batch}", q, None, None, hq, hkv, d, True, 128, 128, 4, p,
                     mask_seed=seed + 4, force_diag=True, force_sink=True,
                     cu_seqlens=cu, lens=lens, kv_cache=(kc, ks, vc, vs))
+
+
+def prefix_int8_cache(batch=8, lo=256, hi=2048, prefix_hi=8192, hq=32, hkv=4, d=128, p=0.75, seed=0):
+    """Prefix-cached prefill over an INT8 K/V cache: sequence b has lq ~
+    U[lo, hi] new query tokens and a cached prefix of U[0, prefix_hi] tokens,
+    so lk = prefix + lq keys (cu_seqlens_k); causal (bottom-right), g=4,
+    Bernoulli(p) mask, diagonal and sink groups forced FP16."""
+    lq, cu = varlen_lengths(batch, lo, hi, seed + 5)
+    pre, _ = varlen_lengths(batch, 0, prefix_hi, seed + 6)
+    lk = lq + pre
+    cu_k = torch.zeros(batch + 1, dtype=torch.int32)
+    cu_k[1:] = torch.cumsum(lk, 0).to(torch.int32)
+    q = randn_f16((int(cu[-1]), hq, d), seed)
+    k = randn_f16((int(cu_k[-1]), hkv, d), seed + 1)
+    v = randn_f16((int(cu_k[-1]), hkv, d), seed + 2)
+    kc, ks = int8_kv_cache(k)
+    vc, vs = int8_kv_cache(v)
+    return Workload(f"prefix_cache_b{batch}", q, None, None, hq, hkv, d, True, 128, 128, 4, p,
+                    mask_seed=seed + 4, force_diag=True, force_sink=True,
+                    cu_seqlens=cu, lens=lq, kv_cache=(kc, ks, vc, vs), cu_seqlens_k=cu_k, lens_k=lk)
 
 
 def long_context(L=65536, hq=28, hkv=4, d=128, p=0.5, seed=0):
