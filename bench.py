@@ -422,6 +422,155 @@ def run_ours(args, rank, world, local_rank):
     return line, w
 
 
+def run_sharded(args, rank, world, local_rank):
+    """One problem split by query heads over the ranks (strong scaling):
+    every rank holds the same seeded workload, computes its block of query
+    heads (api.HeadShardedPrefill) and ends each step with the whole output,
+    through one all-gather and the library's interleaving copy, both inside
+    the timed step."""
+    from mixed_precision_attention_tm_b200 import ops
+    from mixed_precision_attention_tm_b200.api import HeadShardedPrefill
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    w = make_workload(args.workload, args.p, seed=args.seed)     # one problem, the same on every rank
+    plan = HeadShardedPrefill(w.Lq, w.Lk, w.hq, w.hkv, w.d, rank=rank, world=world, causal=w.causal,
+                              tile_m=w.tile_m, tile_n=w.tile_n, g=w.g, p=w.p, seed=w.mask_seed,
+                              force_diag=w.force_diag, force_sink=w.force_sink, cu_seqlens=w.cu_seqlens,
+                              int8_cache=w.kv_cache is not None, cu_seqlens_k=w.cu_seqlens_k, device=dev)
+    plan.load(w.q, w.k, w.v, w.kv_cache)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        plan.run()
+    torch.cuda.synchronize()
+    if ops.get_device_error() != ops.TM_OK:
+        raise RuntimeError("device error after warm-up")
+
+    # work of the whole problem and of this rank's heads
+    cu = None if w.cu_seqlens is None else w.cu_seqlens.numpy()
+    ck = None if w.cu_seqlens_k is None else w.cu_seqlens_k.numpy()
+    full_host = None if plan.full_mask is None else plan.full_mask.cpu().numpy().view(np.uint32)
+
+    def stats(h0, h1):
+        if h1 <= h0:
+            return 0.0, 0.0
+        m = None if full_host is None else np.ascontiguousarray(full_host[h0:h1])
+        return ops.route_stats(m, Hq=h1 - h0, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g, causal=w.causal,
+                               Lq=w.Lq, Lk=w.Lk, cu_seqlens_host=cu, cu_seqlens_k_host=ck)
+    n_vis_r, e8_r = stats(plan.h0, plan.h1)
+    n_vis, e8 = n_vis_r, e8_r
+    if world > 1:
+        t = torch.tensor([n_vis_r, e8_r], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t)
+        n_vis, e8 = float(t[0]), float(t[1])
+    flops = 4.0 * w.d * n_vis
+
+    K = args.steps
+    st_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    st_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    at_a = [[torch.cuda.Event(enable_timing=True) for _ in plan.subs] for _ in range(K)]
+    at_b = [[torch.cuda.Event(enable_timing=True) for _ in plan.subs] for _ in range(K)]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if needs_flush(w) else None
+    clocks = ClockSampler(local_rank)
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(K):
+        if flush is not None:
+            flush.zero_()
+        st_a[i].record(stream)
+        if plan.full_mask is not None:
+            ops.build_mask(w.hq, out=plan.full_mask, **plan._mask_kw)
+        for j, sub in enumerate(plan.subs):
+            if sub.routed:
+                sub.quantize()
+            at_a[i][j].record(stream)
+            sub.attend()
+            at_b[i][j].record(stream)
+        if world > 1:
+            plan.gather()
+            plan.merge()
+        st_b[i].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dist.barrier()
+    if ops.get_device_error() != ops.TM_OK:
+        raise RuntimeError("device error in timed region")
+    step_ms = sum(a.elapsed_time(b) for a, b in zip(st_a, st_b)) / K
+    attn_ms = sum(a.elapsed_time(b) for i in range(K) for a, b in zip(at_a[i], at_b[i])) / K
+    step_max, attn_max = dist.max_over_ranks([step_ms, attn_ms], device=dev)
+    value = flops / (step_max * 1e-3) / 1e12
+
+    p16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * 1e12
+    p8 = 2.0 * p16
+    flops_r = 4.0 * w.d * n_vis_r
+    t_roof_r = roofline_time(w.d, n_vis_r, e8_r, p16, p8) if n_vis_r else 0.0
+    peak_eff = flops_r / t_roof_r / 1e12 if t_roof_r else None
+    achieved = flops_r / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else 0.0
+
+    e2e = None
+    if not args.no_e2e:
+        slices = plan.slice_inputs(w.q, w.k, w.v, w.kv_cache, pin=True)
+        out_h = torch.empty(plan.out.shape, dtype=torch.float16, pin_memory=True)
+        ke = max(4, min(K, 20))
+        for _ in range(2):
+            plan.load_slices(slices)
+            plan.run()
+            out_h.copy_(plan.out, non_blocking=True)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(ke):
+            plan.load_slices(slices)
+            plan.run()
+            out_h.copy_(plan.out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        (te,) = dist.max_over_ranks([e0.elapsed_time(e1) / ke], device=dev)
+        e2e = {"value": flops / (te * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": te,
+               "h2d_bytes_per_step": plan.input_bytes(), "d2h_bytes_per_step": plan.output_bytes(),
+               "steps": ke, "path": "api.HeadShardedPrefill (this rank's heads from pinned host memory, "
+                                    "its step, the all-gather and interleave, the whole output to the host; "
+                                    "no overlap between steps)"}
+
+    cfg = describe(w)
+    cfg["parallelism"] = f"query heads over {world} rank(s)"
+    cfg["head_shards"] = [plan.head_start[r + 1] - plan.head_start[r] for r in range(world)]
+    line = {
+        "metric": "prefill attention TFLOPS (tile-routed FP16/INT8 QK^T, FP16 P.V)",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": step_max,
+        "higher_is_better": True,
+        "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "f16+i8 (fp32 accumulate)",
+        "data": data_note(w),
+        "config": cfg,
+        "tokens_per_s": w.Lq / (step_max * 1e-3),
+        "realised_int8_fraction": e8 / n_vis,
+        "visible_pairs": n_vis,
+        "attn_ms_rank_max": attn_max,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff, "unit": "TFLOP/s",
+                     "frac": None if not peak_eff else achieved / peak_eff, "traffic": None,
+                     "traffic_note": "rank 0's attention launches over its own heads; no capture of this mode",
+                     "peak_source": f"{peak_src} bf16 burst {p16 / 1e12:.1f} TFLOP/s for FP16 pairs, x2 "
+                                    "(nominal INT8:FP16 ratio) for INT8 QK^T, mix-weighted by visible pairs"},
+        "gpu_launches": plan.launches_per_step * K,
+        "clocks": clk,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    return line, w
+
+
 def cpu_sample_spec(w, n_pairs):
     """Evenly spaced (query tile, head) pairs of the workload."""
     import oracle
@@ -668,6 +817,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                    help="batch: every rank runs its own seeded problem (weak scaling); heads: one problem "
+                         "split by query heads over the ranks, output all-gathered (strong scaling)")
     ap.add_argument("--frontier-input", default="channels", choices=["channels", "tokens"],
                     help="frontier report: outlier channels in every token (the routing sweep's inputs) "
                          "or outliers in 0.2%% of the key tokens")
@@ -693,7 +845,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        line, w = run_ours(args, rank, world, local_rank)
+        line, w = (run_sharded if args.shard == "heads" else run_ours)(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
         if rank == 0:

@@ -325,6 +325,27 @@ tm_status tm_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 int64_t tm_probe_scratch_bytes(void);
 tm_status tm_probe_rates(double* out, int32_t n_out, void* scratch, int64_t scratch_bytes, void* stream);
 
+/* Head-sharded prefill: reassembly of the output after the all-gather.
+ * The pages do not speak of more than one GPU.  Every step of the method
+ * (TileMix abstract: per-tile quantisation, routing bits, scores, shared
+ * online softmax) is computed per query head, and grouped-query heads (the
+ * GQA shapes of the MLX PR "Nax Refactor" attention tables) share only their
+ * K / V, so one problem shards over ranks by blocks of consecutive query
+ * heads with no exchange on the data path: rank r computes heads head_start[r] ..
+ * head_start[r+1]-1 of every token into the first head slots of its
+ * [T, h_cap, d] slice, and an all-gather of those equal-size slices gives
+ * `gathered`, fp16 [world, T, h_cap, d] contiguous.  This writes out[t, h, :]
+ * = gathered[r, t, h - head_start[r], :] for the rank r owning h.
+ *   out          device fp16 [T, Hq, d], heads contiguous (stride d), row
+ *                stride out_stride_t elements (>= Hq*d, multiple of 8);
+ *   head_start   HOST int32 [world+1]: head_start[0] = 0, non-decreasing,
+ *                head_start[world] = Hq, every count <= h_cap;
+ *   d            multiple of 8; world in 1..64; both pointers 16-byte aligned.
+ * The two buffers must not overlap.  Asynchronous on `stream`; TM_ERR_INVALID_ARG
+ * on any violated condition (nothing is launched); T = 0 is a no-op. */
+tm_status tm_merge_head_shards(void* out, int64_t out_stride_t, const void* gathered, int64_t T, int32_t Hq,
+                               int32_t d, int32_t world, int32_t h_cap, const int32_t* head_start, void* stream);
+
 /* Static description of a status code. */
 const char* tm_status_string(tm_status s);
 

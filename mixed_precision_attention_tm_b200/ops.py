@@ -82,6 +82,7 @@ def _lib():
             "tm_version": (ctypes.c_char_p, []),
             "tm_probe_scratch_bytes": (I64, []),
             "tm_probe_rates": (I32, [ctypes.POINTER(D), I32, P, I64, P]),
+            "tm_merge_head_shards": (I32, [P, I64, P, I64, I32, I32, I32, I32, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -146,7 +147,7 @@ def _cu_host(cu_seqlens, cu_seqlens_host=None):
 
 def _check_buf(t, shape, dtype, name):
     if t is None or tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
-        raise TmError(f"{name}: expected a contiguous {dtype} tensor of shape {tuple(shape)}")
+        raise ValueError(f"{name}: expected a contiguous {dtype} tensor of shape {tuple(shape)}")
 
 
 def count_tiles(L=None, tile=128, cu_seqlens_host=None):
@@ -406,6 +407,30 @@ def attn_fwd_routed_noalloc(q, k, v, *, out=None, tile_m=128, tile_n=128, g=1, c
                                            ctypes.c_uint64(int(seed) & (2 ** 64 - 1)), int(bool(force_diag)),
                                            int(bool(force_sink)), _stream())
     _check(st, "tm_attn_fwd_routed_noalloc")
+    return out
+
+
+def merge_head_shards(out, gathered, head_start):
+    """Interleave the all-gathered output slices of a head-sharded prefill
+    back into token-major order (tm_merge_head_shards): gathered fp16
+    [world, T, h_cap, d] contiguous, rank r's heads head_start[r] ..
+    head_start[r+1]-1 in its first slots; out fp16 [T, Hq, d] (heads
+    contiguous, rows may be strided).  Returns out."""
+    _cuda(out, "out")
+    _cuda(gathered, "gathered")
+    if out.dtype != torch.float16 or gathered.dtype != torch.float16:
+        raise ValueError("fp16 tensors expected")
+    if gathered.dim() != 4 or not gathered.is_contiguous():
+        raise ValueError("gathered: contiguous [world, T, h_cap, d] expected")
+    world, T, h_cap, d = gathered.shape
+    if out.dim() != 3 or out.shape[0] != T or out.shape[2] != d or out.stride(2) != 1 or out.stride(1) != d:
+        raise ValueError("out: [T, Hq, d] with contiguous heads expected")
+    hs = np.ascontiguousarray(np.asarray(head_start, dtype=np.int32))
+    if hs.shape != (world + 1,):
+        raise ValueError("head_start must hold world + 1 entries")
+    st = _lib().tm_merge_head_shards(_ptr(out), int(out.stride(0)), _ptr(gathered), int(T), int(out.shape[1]),
+                                     int(d), int(world), int(h_cap), hs.ctypes.data, _stream())
+    _check(st, "tm_merge_head_shards")
     return out
 
 
