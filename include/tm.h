@@ -325,6 +325,18 @@ tm_status tm_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 int64_t tm_probe_scratch_bytes(void);
 tm_status tm_probe_rates(double* out, int32_t n_out, void* scratch, int64_t scratch_bytes, void* stream);
 
+/* Kernel choice for d = 128 attention with 128 x 128 tiles (tm_attn_fwd,
+ * tm_attn_fwd_varlen; fp16 K / V).  Two kernels compute the same result: one
+ * holding two 128-row query tiles per CTA (faster per tile once INT8 tiles
+ * are routed) and one holding a single query tile per CTA with three score
+ * buffers in tensor memory (twice as many CTAs).  choice: 0 automatic (the
+ * default: the one-tile kernel when the two-tile kernel would launch fewer
+ * CTAs than the GPU has SMs, or for an all-FP16 launch without a causal
+ * mask whose last wave it fills clearly better), 1 always the two-tile
+ * kernel, 2 always the one-tile kernel.  Process-wide; TM_ERR_INVALID_ARG for
+ * any other value. */
+tm_status tm_set_attn_kernel(int32_t choice);
+
 /* Head-sharded prefill: reassembly of the output after the all-gather.
  * The pages do not speak of more than one GPU.  Every step of the method
  * (TileMix abstract: per-tile quantisation, routing bits, scores, shared

@@ -28,7 +28,60 @@
 
 #include <mutex>
 
+// Which d = 128, 128 x 128-tile launches take the kernel with one query tile
+// per CTA and three score buffers (tm_attn3.cu) instead of the two-tile
+// kernel (tm_attn2.cu): 0 none, 1 by use_one_tile_kernel below, 2 all.
+#ifndef TM_SPLIT_KERNEL
+#define TM_SPLIT_KERNEL 1
+#endif
+#include <atomic>
+
 #include "tm_attn_internal.h"
+
+namespace tmk {
+namespace {
+
+int device_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) ==
+                                                   cudaSuccess && v > 0)
+      sms = v;
+    else
+      return 148;
+  }
+  return sms;
+}
+
+// Measured on B200 (a table of all-FP16 MLX-shaped launches and the routing
+// sweep): per tile the two-tile kernel is as fast as the one-tile kernel on
+// FP16 tiles and faster once INT8 tiles are routed, but it has half as many
+// CTAs.  The one-tile kernel is taken when the two-tile kernel would leave
+// SMs idle (fewer CTAs than SMs), and for all-FP16 launches without a causal
+// mask when its CTAs fill their last wave clearly better (causal launches
+// already balance their waves by running the longest query tiles first).
+std::atomic<int> g_attn_kernel{0};   // tm_set_attn_kernel
+
+bool use_one_tile_kernel(int64_t n_qt, int64_t batch, int64_t hq, bool routed, bool causal) {
+  const int choice = g_attn_kernel.load(std::memory_order_relaxed);
+  if (choice != 0) return choice == 2;
+  const int64_t sms = device_sms();
+  const int64_t pair_ctas = (n_qt + 1) / 2 * batch * hq, one_ctas = n_qt * batch * hq;
+  if (pair_ctas < sms) return true;
+  if (routed || causal) return false;
+  auto fill = [&](int64_t ctas) { return static_cast<double>(ctas) / (((ctas + sms - 1) / sms) * sms); };
+  return fill(one_ctas) > 1.1 * fill(pair_ctas);
+}
+
+}  // namespace
+}  // namespace tmk
+
+extern "C" tm_status tm_set_attn_kernel(int32_t choice) {
+  if (choice < 0 || choice > 2) return TM_ERR_INVALID_ARG;
+  tmk::g_attn_kernel.store(choice, std::memory_order_relaxed);
+  return TM_OK;
+}
 #include "tm_device.cuh"
 #include "tm_host.h"
 
@@ -556,9 +609,16 @@ tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor*
       return TM_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);
-  if (tile_m == 128 && tile_n == 128)
+  if (tile_m == 128 && tile_n == 128) {
+    const int64_t n_qt = ((cu_seqlens ? max_seqlen : q->T) + 127) / 128;
+    if (D == 128 && (TM_SPLIT_KERNEL == 2 ||
+                     (TM_SPLIT_KERNEL == 1 && use_one_tile_kernel(n_qt, cu_seqlens ? batch : 1, q->H,
+                                                                  bitmask != nullptr, causal != 0))))
+      return launch_attn_split(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
+                               g, causal, s);
     return launch_attn_pair(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
                             g, causal, s);
+  }
   if (D == 128) {
     if (tile_n == 128)
       return launch<128, 128>(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,

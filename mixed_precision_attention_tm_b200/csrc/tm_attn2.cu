@@ -86,7 +86,8 @@ struct Cfg2 {
   static constexpr int OFF_Q8 = 2 * Q16_BYTES;
   static constexpr int OFF_SLOT = OFF_Q8 + 2 * Q8_BYTES;
   static constexpr int OFF_BAR = OFF_SLOT + NSLOT * SLOT;
-  static constexpr int BAR_BYTES = 1024;                 // barriers + routing words
+  static constexpr int BAR_BYTES = 2048;                 // barriers, routing words, key-tile scales
+  static constexpr int KSC_MAX = 256;                    // key tiles whose INT8 scales are staged
   static constexpr int MAXW = 64;                        // routing words per query tile kept in smem
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -101,6 +102,7 @@ struct Cfg2 {
   // 2 * 128 * 216 + 128 * 72 = 384 * 168.
   static constexpr int THREADS = 384;
   static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, CONTROL_REGS = 72;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS == THREADS * LAUNCH_REGS,
                 "register split must equal the launch allocation");
   __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
@@ -174,6 +176,7 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * C_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * C_COUNT + 4);
   uint32_t* route_words = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 256);   // [2][MAXW]
+  float* ksc = reinterpret_cast<float*>(smem + C::OFF_BAR + 1024);                 // [KSC_MAX]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -266,6 +269,12 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = 0; t < 2; ++t)
         if (ti[t].mrow != nullptr)
           for (int w = lane; w < p.W; w += 32) route_words[t * C::MAXW + w] = __ldg(ti[t].mrow + w);
+    // the INT8 route's key-tile scales (shared by both query tiles), so that
+    // no softmax step waits on a global load for them
+    if (ti[0].mrow != nullptr || ti[1].mrow != nullptr) {
+      const int nst = nJ < C::KSC_MAX ? nJ : C::KSC_MAX;
+      for (int j = lane; j < nst; j += 32) ksc[j] = __ldg(p.k_scales + (skq.tile_base + j) * p.Hkv + hk);
+    }
   }
   __syncthreads();
   tc_fence_after();
@@ -741,7 +750,10 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; j < T.nJ; ++j) {
       const bool i8 = route8(rrow[t], p.g, j);
       float c = p.scale_log2;
-      if (i8) c = fmaxf(c8_row * __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk), 1e-30f);
+      if (i8) {
+        const float ks = j < C::KSC_MAX ? ksc[j] : __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk);
+        c = fmaxf(c8_row * ks, 1e-30f);
+      }
       // No early exit: the issuer expects one P handoff per key tile, so a
       // failed wait only marks the launch failed and the loop runs on.
       if (!mbar_wait(bar(C_SFULL + t), j & 1, p.err, abort_flag)) ok = false;

@@ -282,6 +282,109 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
+// Groups of tcgen05.mma issued from one asm statement, with every
+// descriptor formed before the first MMA.  Measured on B200: an MMA issued
+// back to back after another from the same thread starts as that one
+// finishes (M128 N128 K16 f16 or K32 i8: 64 SM cycles each), but each
+// instruction the issuing thread executes between two MMAs delays the second
+// one (descriptor arithmetic and a branch between MMAs raised the time per
+// MMA to 70-107 cycles).  acc_first is the accumulate flag of the group's
+// first MMA; the others accumulate.
+template <int N>
+__device__ __forceinline__ void mma_f16_ss_n(uint32_t d, const uint64_t* a, const uint64_t* b, uint32_t idesc,
+                                             uint32_t acc_first);
+template <int N>
+__device__ __forceinline__ void mma_i8_ss_n(uint32_t d, const uint64_t* a, const uint64_t* b, uint32_t idesc,
+                                            uint32_t acc_first);
+// A from TMEM (a[i]: TMEM addresses), B from shared memory, kind::f16
+template <int N>
+__device__ __forceinline__ void mma_f16_ts_n(uint32_t d, const uint32_t* a, const uint64_t* b, uint32_t idesc,
+                                             uint32_t acc_first);
+template <>
+__device__ __forceinline__ void mma_f16_ss_n<4>(uint32_t d, const uint64_t* a, const uint64_t* b, uint32_t idesc,
+                                          uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "setp.ne.b32 q, %11, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %9, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, q;\n\t}"
+      ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(acc_first), "r"(1u));
+}
+template <>
+__device__ __forceinline__ void mma_f16_ss_n<8>(uint32_t d, const uint64_t* a, const uint64_t* b, uint32_t idesc,
+                                          uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %18, 0;\n\t"
+      "setp.ne.b32 q, %19, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %9, %17, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %17, q;\n\t}"
+      ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]), "l"(a[6]), "l"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc), "r"(acc_first), "r"(1u));
+}
+template <>
+__device__ __forceinline__ void mma_i8_ss_n<2>(uint32_t d, const uint64_t* a, const uint64_t* b, uint32_t idesc,
+                                          uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "setp.ne.b32 q, %7, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %3, %5, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %2, %4, %5, q;\n\t}"
+      ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(b[0]), "l"(b[1]), "r"(idesc), "r"(acc_first), "r"(1u));
+}
+template <>
+__device__ __forceinline__ void mma_i8_ss_n<4>(uint32_t d, const uint64_t* a, const uint64_t* b, uint32_t idesc,
+                                          uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "setp.ne.b32 q, %11, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %5, %9, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %2, %6, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %3, %7, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %4, %8, %9, q;\n\t}"
+      ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(acc_first), "r"(1u));
+}
+template <>
+__device__ __forceinline__ void mma_f16_ts_n<4>(uint32_t d, const uint32_t* a, const uint64_t* b, uint32_t idesc,
+                                          uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "setp.ne.b32 q, %11, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, q;\n\t}"
+      ::"r"(d), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(acc_first), "r"(1u));
+}
+template <>
+__device__ __forceinline__ void mma_f16_ts_n<8>(uint32_t d, const uint32_t* a, const uint64_t* b, uint32_t idesc,
+                                          uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %18, 0;\n\t"
+      "setp.ne.b32 q, %19, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %9, %17, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %10, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %11, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %12, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %13, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%6], %14, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %15, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %16, %17, q;\n\t}"
+      ::"r"(d), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc), "r"(acc_first), "r"(1u));
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp receives
 // columns [col, col+32) of TMEM lane (lane base of taddr) + t.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {

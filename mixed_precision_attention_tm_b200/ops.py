@@ -83,6 +83,7 @@ def _lib():
             "tm_probe_scratch_bytes": (I64, []),
             "tm_probe_rates": (I32, [ctypes.POINTER(D), I32, P, I64, P]),
             "tm_merge_head_shards": (I32, [P, I64, P, I64, I32, I32, I32, I32, P, P]),
+            "tm_set_attn_kernel": (I32, [I32]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -408,6 +409,16 @@ def attn_fwd_routed_noalloc(q, k, v, *, out=None, tile_m=128, tile_n=128, g=1, c
                                            int(bool(force_sink)), _stream())
     _check(st, "tm_attn_fwd_routed_noalloc")
     return out
+
+
+ATTN_KERNEL_AUTO, ATTN_KERNEL_TWO_TILE, ATTN_KERNEL_ONE_TILE = 0, 1, 2
+
+
+def set_attn_kernel(choice):
+    """Kernel for d = 128, 128 x 128-tile attention (tm_set_attn_kernel):
+    ATTN_KERNEL_AUTO (default), ATTN_KERNEL_TWO_TILE or ATTN_KERNEL_ONE_TILE.
+    Process-wide."""
+    _check(_lib().tm_set_attn_kernel(int(choice)), "tm_set_attn_kernel")
 
 
 def merge_head_shards(out, gathered, head_start):

@@ -17,6 +17,16 @@ from mixed_precision_attention_tm_b200 import inputs, ops
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True, params=[ops.ATTN_KERNEL_TWO_TILE, ops.ATTN_KERNEL_ONE_TILE],
+                ids=["two_tile", "one_tile"])
+def attn_kernel(request):
+    """Every case runs through both d = 128 attention kernels (the two-tile
+    and the one-tile kernel); other launches are unaffected by the choice."""
+    ops.set_attn_kernel(request.param)
+    yield request.param
+    ops.set_attn_kernel(ops.ATTN_KERNEL_AUTO)
+
+
 def W(Lq, Lk, hq, hkv, d, causal, tm=128, tn=128, g=1, p=None, seed=0, fd=False, fs=False,
       outliers=False, cu=None):
     if cu is not None:

@@ -141,3 +141,11 @@ def test_prefill_plan_buffers_match_library_sizes():
     assert cache.k_quant is None and cache.launches_per_step == 3
     plain = TileMixPrefill(256, 256, 8, 2, 128, device="cpu")
     assert plain.bitmask is None and plain.launches_per_step == 1
+
+
+def test_attn_kernel_choice_rejects_unknown_values():
+    lib = ops._lib()
+    assert lib.tm_set_attn_kernel(3) == ops.TM_ERR_INVALID_ARG
+    assert lib.tm_set_attn_kernel(-1) == ops.TM_ERR_INVALID_ARG
+    for c in (ops.ATTN_KERNEL_TWO_TILE, ops.ATTN_KERNEL_ONE_TILE, ops.ATTN_KERNEL_AUTO):
+        assert lib.tm_set_attn_kernel(c) == ops.TM_OK
