@@ -314,6 +314,10 @@ DUAL_CASES = [
     ("dual_causal_ragged_outliers", dict(Lq=8269, Lk=8269, hq=2, hkv=1, d=128, causal=True, g=1, p=0.5,
                                          fd=True, fs=True, outliers=True)),
     ("dual_causal_fp16", dict(Lq=8205, Lk=8205, hq=2, hkv=2, d=128, causal=True)),
+    # all-FP16 launches with rows of 64 key tiles or more take the chunked
+    # two-tile mode (64-key chunks in two score slots per query tile)
+    ("dual_noncausal_fp16_gqa_ragged", dict(Lq=300, Lk=8269, hq=4, hkv=2, d=128, causal=False)),
+    ("dual_varlen_fp16", dict(Lq=0, Lk=0, hq=2, hkv=1, d=128, causal=True, cu=[0, 8300, 8500])),
     ("dual_varlen_mixed", dict(Lq=0, Lk=0, hq=4, hkv=2, d=128, causal=True, g=4, p=0.75,
                                cu=[0, 300, 8500, 8629, 8800])),
     ("dual_d64", dict(Lq=320, Lk=8192, hq=2, hkv=1, d=64, causal=False, g=1, p=1.0)),
