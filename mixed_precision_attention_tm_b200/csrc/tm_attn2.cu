@@ -25,7 +25,12 @@
 //     below the fp16 rounding of P), the rest on MUFU.ex2, so that neither
 //     the MUFU pipe nor instruction issue alone bounds the softmax;
 //   * K / V loads carry an evict-last L2 policy and Q an evict-first one,
-//     and the output is written with streaming stores.
+//     and the output is written with streaming stores;
+//   * chunked mode (template argument CH; all-FP16 rows of 64 key tiles or
+//     more): each tile's 128 score columns hold two 64-key chunks, and the
+//     QK^T of chunk c+2 follows the P.V of chunk c into the same half, so
+//     the tensor pipe computes the next chunk's scores while the softmax
+//     works on the current one.
 // Every mbarrier wait is bounded (tm_device.cuh).
 #include <cuda.h>
 #include <cuda_fp16.h>
