@@ -139,8 +139,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------
 def make_workload(name, p, seed):
+    """p: INT8 group probability; None takes the workload's configured one
+    (routing sweep 0.75, long context 0.5, varlen and prefix 0.75)."""
     if name == "sweep":
-        return inputs.routing_sweep(p, seed=seed)
+        return inputs.routing_sweep(p if p is not None else 0.75, seed=seed)
     if name == "long":
         return inputs.long_context(p=p if p is not None else 0.5, seed=seed)
     if name == "varlen":
@@ -811,7 +813,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="sweep",
                     choices=["sweep", "long", "varlen", "prefix", "mlx", "tiny", "mlx_table", "frontier"])
-    ap.add_argument("--p", type=float, default=0.75)
+    ap.add_argument("--p", type=float, default=None,
+                    help="INT8 group probability (default: the workload's configuration: 0.75, long context 0.5)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
