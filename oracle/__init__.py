@@ -29,13 +29,17 @@ from .tilemix_oracle import (  # noqa: F401
     attention_rows,
     build_mask,
     build_mask_scale_policy,
+    E4M3_MAX,
     dequant_cache,
+    e4m3_decode,
+    e4m3_encode,
     last_visible_key,
     mask_bit,
     mask_words,
     n_groups,
     n_tiles,
     quantize_tiles,
+    quantize_tiles_fp8,
     route_stats,
     seq_table,
     splitmix64,

@@ -47,6 +47,15 @@ also listed with its reason in the design notes of this repository):
       from a counter-based hash (splitmix64); the group holding the query
       tile's last visible key tile ("diagonal") and group 0 ("sink") can be
       forced to FP16.
+  (n) a third precision (the NEXT-3 item; the pages name FP16 and INT8
+      only, and the fp8 scaling page, pytorch-labs float8_experimental #305,
+      gives per-tensor and per-axis fp8 scales): FP8 E4M3 codes with a
+      symmetric per-tile scale s = fl32(amax / 448) (448 is E4M3's largest
+      finite value), code = E4M3 round-to-nearest-even of fl32(x / s),
+      saturating at +-448; amax == 0 gives s = 0 and codes 0.  A second bit
+      plane in the routing mask's layout selects FP8 for a group whose INT8
+      bit is clear (two bits per group: INT8 wins when both are set).  FP8
+      score = sigma * s_q * s_k * (exact dot product of the decoded codes).
 
 Because online softmax is an exact rewrite of ordinary softmax, the oracle
 computes ordinary softmax attention over the per-tile-routed scores in fp64
@@ -168,6 +177,73 @@ def quantize_tiles(x16, seqs, tile, side):
                 continue
             q = np.rint(blk / s)                      # fp32 division, then RNE
             codes[r0:r0 + rows, h, :] = np.clip(q, -127, 127).astype(np.int8)
+    return codes, scales
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 (reading (n))
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes):
+    """Values of FP8 E4M3 codes (uint8): bit 7 sign, bits 6..3 exponent
+    (bias 7), bits 2..0 mantissa; exponent 0 is subnormal, m/8 * 2^-6;
+    exponent 15 with mantissa 7 is NaN (the format has no infinities, so
+    exponent 15 with mantissa 0..6 are finite values up to 448)."""
+    c = np.asarray(codes).astype(np.int64) & 0xFF
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    mag = np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+    return np.where(c & 0x80, -mag, mag)
+
+
+_E4M3_MAGS = None
+
+
+def e4m3_encode(x):
+    """E4M3 codes (uint8) of fp32 values: the nearest finite E4M3 value, ties
+    to the code with an even mantissa, magnitudes beyond 448 saturating to 448
+    ("satfinite"); the sign bit is the sign of x (so a negative value that
+    rounds to zero gives the code of -0)."""
+    global _E4M3_MAGS
+    if _E4M3_MAGS is None:
+        _E4M3_MAGS = e4m3_decode(np.arange(0, 0x7F))       # codes 0x00..0x7E, ascending magnitudes
+    mags = _E4M3_MAGS
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(mags, a, side="left"), 0, len(mags) - 1)
+    lo = np.maximum(hi - 1, 0)
+    dlo, dhi = a - mags[lo], mags[hi] - a
+    take_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(take_hi, hi, lo).astype(np.int64)
+    code = np.where(np.signbit(x), code | 0x80, code)
+    return code.astype(np.uint8)
+
+
+def quantize_tiles_fp8(x16, seqs, tile, side):
+    """Per-(head, tile) FP8 E4M3 quantisation, reading (n): amax = max |x|
+    over the tile's rows x d; s = fl32(amax / 448); codes = e4m3_encode(
+    fl32(x / s)); amax == 0 gives s = 0 and codes 0.  Returns (codes uint8
+    [T, H, d], scales float32 [n_tiles, H]) in the tile order of
+    ``tile_table``; rows outside every tile keep code 0."""
+    x16 = np.asarray(x16, dtype=np.float16)
+    T, H, d = x16.shape
+    tiles = tile_table(seqs, tile, side)
+    codes = np.zeros((T, H, d), dtype=np.uint8)
+    scales = np.zeros((len(tiles), H), dtype=np.float32)
+    x32 = x16.astype(np.float32)
+    for (_b, _i, r0, rows, ig) in tiles:
+        for h in range(H):
+            blk = x32[r0:r0 + rows, h, :]
+            amax = np.float32(np.max(np.abs(blk))) if blk.size else np.float32(0)
+            s = np.float32(amax / np.float32(E4M3_MAX))
+            scales[ig, h] = s
+            if s == 0:
+                continue
+            codes[r0:r0 + rows, h, :] = e4m3_encode(blk / s)   # fp32 division
     return codes, scales
 
 
@@ -347,7 +423,8 @@ def route_stats(mask, seqs, Hq, tile_m, tile_n, g, causal):
 
 def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
               tile_m=128, tile_n=128, g=1, mask=None,
-              q_quant=None, k_quant=None, kv_cache=None, rows=None, cu_seqlens_k=None):
+              q_quant=None, k_quant=None, kv_cache=None, rows=None, cu_seqlens_k=None,
+              mask_fp8=None, qf8_quant=None, kf8_quant=None):
     """Tile-routed softmax attention in fp64.  Returns float64 [Tq, Hq, d].
 
     q: float16 [Tq, Hq, d]; k, v: float16 [Tk, Hkv, d] (or None with an INT8
@@ -360,6 +437,11 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
     rows: optional iterable of global query rows to evaluate (others are NaN).
     cu_seqlens_k: key offsets per sequence when they differ from cu_seqlens
     (prefix-cached prefill); reading (j).
+    mask_fp8 (reading (n)): a second bit plane in the layout of ``mask``; a
+    legal group whose INT8 bit is clear and FP8 bit is set takes
+    S_ij = sigma * s_q * s_k * (dot product of the E4M3-decoded codes), with
+    qf8_quant = (codes, scales[n_qtiles, Hq]) and kf8_quant = (codes,
+    scales[n_ktiles, Hkv]) from quantize_tiles_fp8 (fp16 K only).
 
     For each sequence, query head h (KV head hk = h // (Hq/Hkv)) and visible
     pair (i, j) in query tile I (global I_glob), key tile J, group G = J // g:
@@ -397,6 +479,13 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
     out = np.full((Tq, Hq, d), np.nan if rows is not None else 0.0, dtype=np.float64)
     kf = k16.astype(np.float64)
     vf = v16.astype(np.float64)
+    if mask_fp8 is not None:
+        if kv_cache is not None:
+            raise ValueError("the FP8 route takes tile-quantised fp16 K, not an INT8 cache")
+        qf8_val = e4m3_decode(qf8_quant[0])
+        kf8_val = e4m3_decode(kf8_quant[0])
+        qf8_scales = np.asarray(qf8_quant[1], dtype=np.float32)
+        kf8_scales = np.asarray(kf8_quant[1], dtype=np.float32)
     if mask is not None:
         q_codes = np.asarray(q_quant[0])
         q_scales = np.asarray(q_quant[1], dtype=np.float32)
@@ -423,6 +512,7 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
             Vb = vf[ks:ks + lk, hk, :]
             Qr = q[r0 + sel, h, :].astype(np.float64)
             S = sigma * (Qr @ Kb.T)
+            route8 = np.zeros(lk, dtype=bool)
             if mask is not None:
                 route8 = _group_bits(mask, h, ig, n_groups(n_tiles(lk, tile_n), g))[(jj // tile_n) // g]
                 if route8.any():
@@ -433,6 +523,13 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
                         col_scale = k_tile_scale[kt_off[b] + jj // tile_n, hk].astype(np.float64)
                     S8 = sigma * float(q_scales[ig, h]) * acc8 * col_scale[None, :]
                     S = np.where(route8[None, :], S8, S)
+            if mask_fp8 is not None:
+                routef8 = ~route8 & _group_bits(mask_fp8, h, ig, n_groups(n_tiles(lk, tile_n), g))[(jj // tile_n) // g]
+                if routef8.any():
+                    accf8 = qf8_val[r0 + sel, h, :] @ kf8_val[ks:ks + lk, hk, :].T    # exact in fp64
+                    colf8 = kf8_scales[kt_off[b] + jj // tile_n, hk].astype(np.float64)
+                    Sf8 = sigma * float(qf8_scales[ig, h]) * accf8 * colf8[None, :]
+                    S = np.where(routef8[None, :], Sf8, S)
             S = np.where(vis, S, -np.inf)
             has = vis.any(axis=1)
             m = np.where(has, S.max(axis=1, initial=-np.inf), 0.0)
