@@ -116,6 +116,19 @@ tm_status tm_quantize_qk_varlen(const tm_tensor* q, const tm_tensor* k, int8_t* 
                                 const int32_t* cu_seqlens_k, int32_t batch, int32_t max_seqlen_q,
                                 int32_t max_seqlen_k, int32_t tile_m, int32_t tile_n, void* stream);
 
+/* FP8 E4M3 codes of the third precision (the pages name FP16 and INT8; the
+ * fp8 scaling page, pytorch-labs float8_experimental #305, describes fp8
+ * operands with per-tensor or per-axis scales).  Per (head, tile) as in
+ * tm_quantize_qk, with s = fl32(amax / 448) (448: the largest finite E4M3
+ * value) and code = E4M3 round-to-nearest-even of fl32(x / s), saturating at
+ * +-448 (bit 7 sign, bits 6..3 exponent with bias 7, bits 2..0 mantissa;
+ * a negative value that rounds to zero gives the code of -0); amax == 0
+ * gives s = 0 and codes 0.  Layouts, arguments and errors as
+ * tm_quantize_qk, codes as uint8.  Bit-identical to the definition. */
+tm_status tm_quantize_qk_fp8(const tm_tensor* q, const tm_tensor* k, uint8_t* q_codes, float* q_scales,
+                             uint8_t* k_codes, float* k_scales, const int32_t* cu_seqlens, int32_t batch,
+                             int32_t max_seqlen, int32_t tile_m, int32_t tile_n, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Routing bitmask layout (TileMix abstract: "compact bitmasks", one bit per
  * query tile x key-tile group, "each routing bit govern[s] multiple adjacent
@@ -324,6 +337,27 @@ tm_status tm_selftest_wait_timeout(uint64_t limit_ns, void* stream);
  * null or short buffer or n_out < 5. */
 int64_t tm_probe_scratch_bytes(void);
 tm_status tm_probe_rates(double* out, int32_t n_out, void* scratch, int64_t scratch_bytes, void* stream);
+
+/* Attention with the FP8 third precision (the pages route between FP16 and
+ * INT8; fp8 scaling page, pytorch-labs float8_experimental #305, for fp8
+ * operands with per-axis scales).  As tm_attn_fwd with 128 x 128 tiles and
+ * d = 128, plus a second routing bit plane `bitmask_fp8` in the layout of
+ * `bitmask` (same mask_head_stride): a legal group whose INT8 bit is clear
+ * and whose FP8 bit is set computes its scores from the E4M3 codes of
+ * tm_quantize_qk_fp8, S_ij = sigma * s_q * s_k * (dot product of the decoded
+ * codes), accumulated in fp32 by the tensor core (kind::f8f6f4); INT8 wins
+ * when both bits are set.  bitmask may be NULL (no INT8 groups; then Q / K
+ * need no INT8 codes).  q_fp8_codes [Tq, Hq, 128] / q_fp8_scales
+ * [n_qtiles, Hq], k_fp8_codes [Tk, Hkv, 128] / k_fp8_scales [n_ktiles, Hkv]
+ * as written by tm_quantize_qk_fp8 with the same tiles and cu_seqlens.
+ * fp16 K / V only (no INT8 cache).  Codes 16-byte aligned, masks and scales
+ * 4-byte aligned, else TM_ERR_INVALID_ARG; other d, tiles or a cache:
+ * TM_ERR_UNSUPPORTED. */
+tm_status tm_attn_fwd_fp8(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                          const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen, const uint32_t* bitmask,
+                          const uint32_t* bitmask_fp8, int64_t mask_head_stride, const uint8_t* q_fp8_codes,
+                          const float* q_fp8_scales, const uint8_t* k_fp8_codes, const float* k_fp8_scales,
+                          int32_t g, int32_t causal, void* stream);
 
 /* Kernel choice for d = 128 attention with 128 x 128 tiles (tm_attn_fwd,
  * tm_attn_fwd_varlen; fp16 K / V).  Two kernels compute the same result: one

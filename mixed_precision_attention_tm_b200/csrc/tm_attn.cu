@@ -560,7 +560,7 @@ namespace {
 tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                         const int32_t* cu_seqlens, const int32_t* cu_k, int32_t batch, int32_t max_seqlen,
                         int32_t max_k, const uint32_t* bitmask, int64_t mask_head_stride, int32_t tile_m,
-                        int32_t tile_n, int32_t g, int32_t causal, void* stream) {
+                        int32_t tile_n, int32_t g, int32_t causal, void* stream, const Fp8Route* f8 = nullptr) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return TM_ERR_INVALID_ARG;
   const int64_t D = q->d;
   if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
@@ -583,6 +583,16 @@ tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor*
       return TM_ERR_INVALID_ARG;
   }
   const bool cache = (k->scale_kind == TM_SCALE_TOKEN) || (v->scale_kind == TM_SCALE_TOKEN);
+  if (f8 != nullptr) {
+    // the FP8 route: d = 128, 128 x 128 tiles, fp16 K / V, one-tile kernel
+    if (cache || D != 128 || tile_m != 128 || tile_n != 128) return TM_ERR_UNSUPPORTED;
+    if (f8->bitmask == nullptr || (reinterpret_cast<uintptr_t>(f8->bitmask) & 3u)) return TM_ERR_INVALID_ARG;
+    if (f8->q_codes == nullptr || f8->k_codes == nullptr || !aligned16(f8->q_codes) || !aligned16(f8->k_codes))
+      return TM_ERR_INVALID_ARG;
+    if (f8->q_scales == nullptr || f8->k_scales == nullptr || (reinterpret_cast<uintptr_t>(f8->q_scales) & 3u) ||
+        (reinterpret_cast<uintptr_t>(f8->k_scales) & 3u))
+      return TM_ERR_INVALID_ARG;
+  }
   if (cache) {
     // INT8 K/V cache: both K and V as codes + per-(token, head) fp16 scales.
     if (k->scale_kind != TM_SCALE_TOKEN || v->scale_kind != TM_SCALE_TOKEN) return TM_ERR_INVALID_ARG;
@@ -609,6 +619,9 @@ tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor*
       return TM_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);
+  if (f8 != nullptr)
+    return launch_attn_split(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride, g,
+                             causal, s, f8);
   if (tile_m == 128 && tile_n == 128) {
     const int64_t n_qt = ((cu_seqlens ? max_seqlen : q->T) + 127) / 128;
     if (D == 128 && (TM_SPLIT_KERNEL == 2 ||
@@ -654,4 +667,15 @@ extern "C" tm_status tm_attn_fwd_varlen(const tm_tensor* q, const tm_tensor* k, 
   if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return TM_ERR_INVALID_ARG;
   return tmk::attn_fwd_impl(q, k, v, out, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q, max_seqlen_k, bitmask,
                             mask_head_stride, tile_m, tile_n, g, causal, stream);
+}
+
+extern "C" tm_status tm_attn_fwd_fp8(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                                     const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen,
+                                     const uint32_t* bitmask, const uint32_t* bitmask_fp8, int64_t mask_head_stride,
+                                     const uint8_t* q_fp8_codes, const float* q_fp8_scales,
+                                     const uint8_t* k_fp8_codes, const float* k_fp8_scales, int32_t g,
+                                     int32_t causal, void* stream) {
+  const tmk::Fp8Route f8{bitmask_fp8, q_fp8_codes, q_fp8_scales, k_fp8_codes, k_fp8_scales};
+  return tmk::attn_fwd_impl(q, k, v, out, cu_seqlens, nullptr, batch, max_seqlen, 0, bitmask, mask_head_stride, 128,
+                            128, g, causal, stream, &f8);
 }

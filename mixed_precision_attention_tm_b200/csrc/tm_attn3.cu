@@ -65,25 +65,28 @@ extern "C" int tm_debug_trace_read_split(unsigned long long* host, unsigned int 
 namespace tmk {
 namespace {
 
+template <bool F8>
 struct Cfg3 {
   static constexpr int D = 128, BM = 128, BN = 128, HN = 64;   // HN: keys per softmax warpgroup
   static constexpr int SLOT = BN * D * 2;                       // one fp16 K or V tile (32 KB)
-  static constexpr int NK = 3, NV = 2;                          // K and V ring slots
+  static constexpr int NK = F8 ? 2 : 3, NV = 2;                 // K and V ring slots
   static constexpr int NSB = 3;                                 // score buffers in TMEM
   static constexpr int Q16_BYTES = BM * D * 2;
   static constexpr int Q8_BYTES = BM * D;
   static constexpr int HALF = BM * 128;                         // one 64-column fp16 slab (128 rows)
   static constexpr int OFF_Q16 = 0;
   static constexpr int OFF_Q8 = OFF_Q16 + Q16_BYTES;
-  static constexpr int OFF_K = OFF_Q8 + Q8_BYTES;
+  static constexpr int OFF_QF8 = OFF_Q8 + Q8_BYTES;             // FP8 route only
+  static constexpr int OFF_K = OFF_QF8 + (F8 ? Q8_BYTES : 0);
   static constexpr int OFF_V = OFF_K + NK * SLOT;
   static constexpr int OFF_BAR = OFF_V + NV * SLOT;
-  static constexpr int OFF_WORDS = OFF_BAR + 256;               // routing words (barriers and TMEM slot below)
+  static constexpr int OFF_WORDS = OFF_BAR + 256;               // routing words [2 planes][MAXW]
   static constexpr int OFF_XMAX = OFF_BAR + 1024;               // row maxima [2 iterations][2 warpgroups][128],
                                                                 // then row sums [2 warpgroups][128]
   static constexpr int OFF_KSC = OFF_XMAX + 3 * 256 * 4;        // key-tile scales of the INT8 route
   static constexpr int MAXJ = 512;                              // key tiles whose scales are staged
-  static constexpr int BAR_BYTES = 1024 + 3 * 256 * 4 + MAXJ * 4;
+  static constexpr int OFF_KSCF8 = OFF_KSC + MAXJ * 4;          // ... of the FP8 route
+  static constexpr int BAR_BYTES = 1024 + 3 * 256 * 4 + MAXJ * 4 * (F8 ? 2 : 1);
   static constexpr int MAXW = 64;                               // routing words kept in shared memory
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -91,6 +94,7 @@ struct Cfg3 {
   static constexpr uint32_t S_COL = 128;                        // + 128 buffer
   static constexpr uint32_t IDESC_S16 = idesc_f16(BM, BN, false);
   static constexpr uint32_t IDESC_S8 = idesc_i8(BM, BN);
+  static constexpr uint32_t IDESC_F8 = idesc_f8_e4m3(BM, BN);
   static constexpr uint32_t IDESC_PV = idesc_f16(BM, D, true);
   // 8 softmax warps + K producer, issuer, wait helper, V producer.  The
   // register split is the two-tile kernel's: 2 * 128 * 216 + 128 * 72 = 384 * 168.
@@ -99,7 +103,7 @@ struct Cfg3 {
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS == THREADS * LAUNCH_REGS,
                 "register split must equal the launch allocation");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static_assert(OFF_WORDS + 4 * MAXW <= OFF_XMAX, "routing words fit");
+  static_assert(OFF_WORDS + 2 * 4 * MAXW <= OFF_XMAX, "routing words fit");
 };
 
 enum {
@@ -132,6 +136,9 @@ struct Params3 {
   const float* q_scales;
   const float* k_scales;
   const uint32_t* bitmask;
+  const float* qf8_scales;     // FP8 route: E4M3 tile scales of Q [n_qtiles, Hq] and K [n_ktiles, Hkv]
+  const float* kf8_scales;
+  const uint32_t* bitmask_f8;  // FP8 route: second bit plane, layout of bitmask
   int64_t mask_hs;
   int W;
   const int32_t* cu;
@@ -150,12 +157,22 @@ __device__ __forceinline__ bool route_bit(const uint32_t* row, int g, int j) {
   return (row[G >> 5] >> (G & 31)) & 1u;
 }
 
-template <int EMU>
+// route of key tile j: 0 FP16, 1 INT8 (first bit plane), 2 FP8 (second
+// plane, when the first bit is clear)
+template <bool F8>
+__device__ __forceinline__ int route_of(const uint32_t* row8, const uint32_t* rowf8, int g, int j) {
+  if (route_bit(row8, g, j)) return 1;
+  if (F8 && route_bit(rowf8, g, j)) return 2;
+  return 0;
+}
+
+template <int EMU, bool F8>
 __global__ void __launch_bounds__(384, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmQ8,
                       const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmK8,
-                      const __grid_constant__ CUtensorMap tmV16, const Params3 p) {
-  using C = Cfg3;
+                      const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmQF8,
+                      const __grid_constant__ CUtensorMap tmKF8, const Params3 p) {
+  using C = Cfg3<F8>;
   constexpr int D = C::D, BN = C::BN, HN = C::HN;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -169,6 +186,7 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* route_words = reinterpret_cast<uint32_t*>(smem + C::OFF_WORDS);
   float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
   float* ksc = reinterpret_cast<float*>(smem + C::OFF_KSC);
+  float* kscf8 = reinterpret_cast<float*>(smem + C::OFF_KSCF8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -211,6 +229,9 @@ __global__ void __launch_bounds__(384, 1)
   const int hk = h / (p.Hq / p.Hkv);
   const bool words_in_smem = p.W <= C::MAXW;
   const uint32_t* rrow = mrow == nullptr ? nullptr : (words_in_smem ? route_words : mrow);
+  const uint32_t* mrowf8 =
+      (F8 && p.bitmask_f8) ? p.bitmask_f8 + static_cast<int64_t>(h) * p.mask_hs + ig * p.W : nullptr;
+  const uint32_t* rrowf8 = mrowf8 == nullptr ? nullptr : (words_in_smem ? route_words + C::MAXW : mrowf8);
 
   // ---- setup
   if (threadIdx.x == 0) {
@@ -244,6 +265,12 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (words_in_smem && mrow != nullptr)
       for (int w = lane; w < p.W; w += 32) route_words[w] = __ldg(mrow + w);
+    if (words_in_smem && mrowf8 != nullptr)
+      for (int w = lane; w < p.W; w += 32) route_words[C::MAXW + w] = __ldg(mrowf8 + w);
+    if (mrowf8 != nullptr) {
+      const int nst = nJ < C::MAXJ ? nJ : C::MAXJ;
+      for (int j = lane; j < nst; j += 32) kscf8[j] = __ldg(p.kf8_scales + (skq.tile_base + j) * p.Hkv + hk);
+    }
     // the INT8 route's key-tile scales, so that no softmax step waits on a
     // global load for them
     if (mrow != nullptr) {
@@ -266,25 +293,30 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t pol_kv = l2_policy_evict_last();
         volatile int never = 0;
         {
-          bool any8 = false;
+          bool any8 = false, anyf8 = false;
           if (mrow != nullptr)
             for (int w = 0; w < p.W; ++w) any8 |= (__ldg(mrow + w) != 0u);
+          if (mrowf8 != nullptr)
+            for (int w = 0; w < p.W; ++w) anyf8 |= (__ldg(mrowf8 + w) != 0u);
           const uint64_t pol_q = l2_policy_evict_first();
           const int32_t qr = static_cast<int32_t>(row0);
-          mbar_arrive_expect_tx(bar(B_QFULL), C::Q16_BYTES + (any8 ? C::Q8_BYTES : 0));
+          mbar_arrive_expect_tx(bar(B_QFULL),
+                                C::Q16_BYTES + (any8 ? C::Q8_BYTES : 0) + (anyf8 ? C::Q8_BYTES : 0));
 #pragma unroll
           for (int hh = 0; hh < D / 64; ++hh)
             tma_load_3d_hint(sbase + C::OFF_Q16 + hh * C::HALF, &tmQ16, bar(B_QFULL), hh * 64, h, qr, pol_q);
           if (any8) tma_load_3d_hint(sbase + C::OFF_Q8, &tmQ8, bar(B_QFULL), 0, h, qr, pol_q);
+          if (anyf8) tma_load_3d_hint(sbase + C::OFF_QF8, &tmQF8, bar(B_QFULL), 0, h, qr, pol_q);
           int nk = 0;
           for (int j = 0; j < nJ; ++j) {
             const int32_t krow = static_cast<int32_t>(kstart + static_cast<int64_t>(j) * BN);
             const int ks = j % C::NK;
             if (j >= C::NK && !mbar_wait(bar(B_KEMPTY + ks), (j / C::NK - 1) & 1, p.err, abort_flag)) break;
             const uint32_t kdst = sbase + C::OFF_K + ks * C::SLOT;
-            if (route_bit(rrow, p.g, j)) {
+            const int rt = route_of<F8>(rrow, rrowf8, p.g, j);
+            if (rt != 0) {   // int8 or E4M3 codes: one 128-byte row per key
               mbar_arrive_expect_tx(bar(B_KFULL + ks), BN * D);
-              tma_load_3d_hint(kdst, &tmK8, bar(B_KFULL + ks), 0, hk, krow, pol_kv);
+              tma_load_3d_hint(kdst, rt == 1 ? &tmK8 : &tmKF8, bar(B_KFULL + ks), 0, hk, krow, pol_kv);
             } else {
               mbar_arrive_expect_tx(bar(B_KFULL + ks), C::SLOT);
 #pragma unroll
@@ -332,30 +364,35 @@ __global__ void __launch_bounds__(384, 1)
       if (nJ > 0) {
         auto kv_handoff = [&]() { named_bar_sync(NB_KV, 64); };
         int wwin = -1;
-        uint32_t rw = 0;
-        auto route_reg = [&](int j) -> bool {
-          if (rrow == nullptr) return false;
+        uint32_t rw = 0, rwf8 = 0;
+        auto route_reg = [&](int j) -> int {
+          if (rrow == nullptr && rrowf8 == nullptr) return 0;
           const int G = j / p.g;
           if ((G >> 5) != wwin) {
             wwin = G >> 5;
-            rw = rrow[wwin];
+            rw = rrow != nullptr ? rrow[wwin] : 0u;
+            rwf8 = rrowf8 != nullptr ? rrowf8[wwin] : 0u;
           }
-          return (rw >> (G & 31)) & 1u;
+          if ((rw >> (G & 31)) & 1u) return 1;
+          return (F8 && ((rwf8 >> (G & 31)) & 1u)) ? 2 : 0;
         };
         auto issue_s = [&](int j) {
-          const bool i8 = route_reg(j);
+          const int rt = route_reg(j);
+          const bool i8 = rt != 0;   // 8-bit codes: int8 or E4M3
           const int ks = j % C::NK, sb = j % C::NSB;
           const uint32_t kb = sbase + C::OFF_K + ks * C::SLOT;
           const uint32_t d_s = tmem + C::S_COL + 128u * static_cast<uint32_t>(sb);
           if (i8) {
             uint64_t ad[D / 32], bd[D / 32];
+            const uint32_t qa = sbase + (rt == 1 ? C::OFF_Q8 : C::OFF_QF8);
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk) {
-              ad[kk] = smem_desc(sbase + C::OFF_Q8 + kk * 32, 16, 1024, kSwizzle128);
+              ad[kk] = smem_desc(qa + kk * 32, 16, 1024, kSwizzle128);
               bd[kk] = smem_desc(kb + kk * 32, 16, 1024, kSwizzle128);
             }
             if (elect_one()) {
-              mma_i8_ss_n<D / 32>(d_s, ad, bd, C::IDESC_S8, 0u);
+              if (F8 && rt == 2) mma_f8_ss_n<D / 32>(d_s, ad, bd, C::IDESC_F8, 0u);
+              else mma_i8_ss_n<D / 32>(d_s, ad, bd, C::IDESC_S8, 0u);
               tc_commit(bar(B_SFULL + sb));
               tc_commit(bar(B_KEMPTY + ks));
             }
@@ -469,8 +506,9 @@ __global__ void __launch_bounds__(384, 1)
     const int64_t i_row = r0 + r;
     int64_t lim = -1;
     if (row_ok) lim = p.causal ? min(Lk - 1, i_row + Lk - Lq) : Lk - 1;
-    float c8_row = 0.f;
+    float c8_row = 0.f, cf8_row = 0.f;
     if (mrow != nullptr) c8_row = __ldg(p.q_scales + ig * p.Hq + h) * p.scale_log2;
+    if (mrowf8 != nullptr) cf8_row = __ldg(p.qf8_scales + ig * p.Hq + h) * p.scale_log2;
     const SeqInfo sk = seq_info(p.cu_k, b, p.Lk, BN);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -478,11 +516,15 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; j < nJ; ++j) {
       const int sb = j % C::NSB;
       const uint32_t s_addr = lane_addr + C::S_COL + 128u * sb + HN * hw;
-      const bool i8 = route_bit(rrow, p.g, j);
+      const int rt = route_of<F8>(rrow, rrowf8, p.g, j);
+      const bool i8 = rt == 1;   // int32 scores to convert; FP8 scores arrive in fp32
       float c = p.scale_log2;
       if (i8) {
         const float ks = j < C::MAXJ ? ksc[j] : __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk);
         c = fmaxf(c8_row * ks, 1e-30f);
+      } else if (F8 && rt == 2) {
+        const float ks = j < C::MAXJ ? kscf8[j] : __ldg(p.kf8_scales + (sk.tile_base + j) * p.Hkv + hk);
+        c = fmaxf(cf8_row * ks, 1e-30f);
       }
       // No early exit: the issuer expects one P handoff per key tile.
       if (!mbar_wait(bar(B_SFULL + sb), (j / C::NSB) & 1, p.err, abort_flag)) ok = false;
@@ -654,16 +696,17 @@ std::mutex g_mu3;
 
 // One-time kernel attributes; the warpgroup register split assumes exactly
 // LAUNCH_REGS per thread at launch, so a build that differs is refused.
+template <bool F8>
 tm_status prepare_split_kernel() {
   static bool attr_done = false;
   std::lock_guard<std::mutex> lk(g_mu3);
   if (attr_done) return TM_OK;
-  auto kern = attn_split_kernel<TM_EXP2_EMU_PAIRS>;
+  auto kern = attn_split_kernel<TM_EXP2_EMU_PAIRS, F8>;
   cudaFuncAttributes fa;
   tm_status st = check_cuda(cudaFuncGetAttributes(&fa, kern));
   if (st != TM_OK) return st;
-  if (fa.numRegs != Cfg3::LAUNCH_REGS) return TM_ERR_UNSUPPORTED;
-  st = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg3::SMEM_BYTES));
+  if (fa.numRegs != Cfg3<F8>::LAUNCH_REGS) return TM_ERR_UNSUPPORTED;
+  st = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg3<F8>::SMEM_BYTES));
   if (st != TM_OK) return st;
   attr_done = true;
   return TM_OK;
@@ -674,13 +717,13 @@ tm_status prepare_split_kernel() {
 tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                             const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
                             const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
-                            cudaStream_t stream) {
-  using C = Cfg3;
-  constexpr int D = C::D;
+                            cudaStream_t stream, const Fp8Route* f8) {
+  constexpr int D = 128;
   if (q->d != D) return TM_ERR_UNSUPPORTED;
-  tm_status st = prepare_split_kernel();
+  const bool use_f8 = f8 != nullptr && f8->bitmask != nullptr;
+  tm_status st = use_f8 ? prepare_split_kernel<true>() : prepare_split_kernel<false>();
   if (st != TM_OK) return st;
-  CUtensorMap mQ16, mQ8, mK16, mK8, mV16;
+  CUtensorMap mQ16, mQ8, mK16, mK8, mV16, mQF8, mKF8;
   st = encode_thd_map(&mQ16, q->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q->T, q->H, D, q->stride_t,
                       q->stride_h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != TM_OK) return st;
@@ -701,6 +744,17 @@ tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_ten
     mQ8 = mQ16;
     mK8 = mK16;
   }
+  if (use_f8) {
+    st = encode_thd_map(&mQF8, f8->q_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q->T, q->H, D, q->H * D, D, D, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TM_OK) return st;
+    st = encode_thd_map(&mKF8, f8->k_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k->T, k->H, D, k->H * D, D, D, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TM_OK) return st;
+  } else {
+    mQF8 = mQ8;
+    mKF8 = mK8;
+  }
   Params3 p;
   p.out = static_cast<__half*>(out->data);
   p.out_st = out->stride_t;
@@ -708,6 +762,9 @@ tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_ten
   p.q_scales = static_cast<const float*>(q->scales);
   p.k_scales = static_cast<const float*>(k->scales);
   p.bitmask = bitmask;
+  p.qf8_scales = use_f8 ? f8->q_scales : nullptr;
+  p.kf8_scales = use_f8 ? f8->k_scales : nullptr;
+  p.bitmask_f8 = use_f8 ? f8->bitmask : nullptr;
   p.mask_hs = mask_hs;
   p.cu = cu;
   p.cu_k = cu ? (cu_k ? cu_k : cu) : nullptr;
@@ -739,8 +796,14 @@ tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_ten
   const int64_t grid = static_cast<int64_t>(p.n_qt_max) * p.batch * p.Hq;
   if (grid == 0) return TM_OK;
   if (grid > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
-  attn_split_kernel<TM_EXP2_EMU_PAIRS>
-      <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
+  if (use_f8)
+    attn_split_kernel<TM_EXP2_EMU_PAIRS, true><<<static_cast<unsigned>(grid), Cfg3<true>::THREADS,
+                                                 Cfg3<true>::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16,
+                                                                                   mQF8, mKF8, p);
+  else
+    attn_split_kernel<TM_EXP2_EMU_PAIRS, false><<<static_cast<unsigned>(grid), Cfg3<false>::THREADS,
+                                                  Cfg3<false>::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16,
+                                                                                     mQF8, mKF8, p);
   return check_cuda(cudaGetLastError());
 }
 

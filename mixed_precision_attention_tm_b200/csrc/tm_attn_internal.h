@@ -16,12 +16,23 @@ tm_status launch_attn_pair(const tm_tensor* q, const tm_tensor* k, const tm_tens
                            const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
                            cudaStream_t stream);
 
-// One 128-row query tile per CTA with two score buffers in TMEM and the keys
-// of each score tile split between two softmax warpgroups (d = 128).
+// The FP8 third precision: a second routing bit plane (layout of the INT8
+// bitmask) and the E4M3 codes and tile scales of Q and K.
+struct Fp8Route {
+  const uint32_t* bitmask;
+  const uint8_t* q_codes;
+  const float* q_scales;
+  const uint8_t* k_codes;
+  const float* k_scales;
+};
+
+// One 128-row query tile per CTA with three score buffers in TMEM and the
+// keys of each score tile split between two softmax warpgroups (d = 128).
+// f8: the FP8 route (null or a null bitmask: FP16 / INT8 only).
 tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                             const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
                             const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
-                            cudaStream_t stream);
+                            cudaStream_t stream, const Fp8Route* f8 = nullptr);
 
 // INT8 K/V cache (codes + per-token fp16 scales), d = 128, 128-key tiles.
 tm_status launch_attn_cache(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,

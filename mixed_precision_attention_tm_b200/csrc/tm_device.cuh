@@ -309,6 +309,9 @@ __device__ __forceinline__ void mma_f16_ss_n(uint32_t d, const uint64_t* a, cons
 template <int N>
 __device__ __forceinline__ void mma_i8_ss_n(uint32_t d, const uint64_t* a, const uint64_t* b, uint32_t idesc,
                                             uint32_t acc_first);
+template <int N>
+__device__ __forceinline__ void mma_f8_ss_n(uint32_t d, const uint64_t* a, const uint64_t* b, uint32_t idesc,
+                                            uint32_t acc_first);
 // A from TMEM (a[i]: TMEM addresses), B from shared memory, kind::f16
 template <int N>
 __device__ __forceinline__ void mma_f16_ts_n(uint32_t d, const uint32_t* a, const uint64_t* b, uint32_t idesc,
@@ -365,6 +368,20 @@ __device__ __forceinline__ void mma_i8_ss_n<4>(uint32_t d, const uint64_t* a, co
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %2, %6, %9, q;\n\t"
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %3, %7, %9, q;\n\t"
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %4, %8, %9, q;\n\t}"
+      ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(acc_first), "r"(1u));
+}
+// kind::f8f6f4 (E4M3 codes per the instruction descriptor), K = 32 per MMA
+template <>
+__device__ __forceinline__ void mma_f8_ss_n<4>(uint32_t d, const uint64_t* a, const uint64_t* b, uint32_t idesc,
+                                         uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "setp.ne.b32 q, %11, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %5, %9, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %2, %6, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %3, %7, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %4, %8, %9, q;\n\t}"
       ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(acc_first), "r"(1u));
 }
 template <>
@@ -506,6 +523,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major) 
 }
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+// kind::f8f6f4 with E4M3 A and B (format code 0), f32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_f8_e4m3(int M, int N) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 

@@ -1,5 +1,6 @@
 // tm_quant.cu -- per-tile symmetric INT8 quantisation of Q and K
-// (tm_quantize_qk).
+// (tm_quantize_qk), and the FP8 E4M3 codes of the third precision
+// (tm_quantize_qk_fp8).
 //
 // TileMix (Lattice paper page), abstract: the INT8 route computes score tiles
 // from INT8 operands.  Rule implemented here, per (head, tile of `tile` rows of
@@ -12,6 +13,12 @@
 // the codes.  Division is the IEEE round-to-nearest __fdiv_rn and the code
 // conversion is round-to-nearest-even, so the result is bit-identical to the
 // definition.  HBM-bound: bytes per element = 2 (read) + 1 (write).
+//
+// FP8 (the third precision; fp8 scaling page, pytorch-labs float8_experimental
+// #305, for per-axis fp8 scales): s = fl32(amax / 448), 448 being the
+// largest finite E4M3 value; code = E4M3 round-to-nearest-even of
+// fl32(x / s) saturating at +-448, by the hardware conversion
+// cvt.rn.satfinite.e4m3x2.f32; s == 0 gives codes 0.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -23,10 +30,17 @@ namespace {
 
 constexpr int kQuantThreads = 256;
 
-template <int D>
+// two fp32 values to two E4M3 codes (lo in bits 0-7, hi in bits 8-15)
+__device__ __forceinline__ uint32_t e4m3x2_rn_sat(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+template <int D, bool F8>
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_tiles_kernel(const __half* __restrict__ x, int64_t stride_t, int64_t stride_h, int H,
-                          int8_t* __restrict__ codes, float* __restrict__ scales,
+                          uint8_t* __restrict__ codes, float* __restrict__ scales,
                           const int32_t* __restrict__ cu, int64_t L, int tile, DevErr err) {
   constexpr int VPR = D / 8;                       // 16-byte vectors per row
   constexpr int MAXV = 128 * VPR / kQuantThreads;  // vectors per thread at tile = 128
@@ -70,7 +84,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     float a = red[0];
 #pragma unroll
     for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[w]);
-    const float sc = __fdiv_rn(a, 127.0f);
+    const float sc = __fdiv_rn(a, F8 ? 448.0f : 127.0f);
     s_scale = sc;
     scales[(s.tile_base + I) * H + h] = sc;
   }
@@ -84,17 +98,28 @@ __global__ void __launch_bounds__(kQuantThreads)
       const int row = idx / VPR, c = idx % VPR;
       const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
       uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float f = (e & 1) ? __high2float(hv[e >> 1]) : __low2float(hv[e >> 1]);
-        int qv = 0;
+      if (F8) {
         if (sc != 0.f) {
-          qv = __float2int_rn(__fdiv_rn(f, sc));
-          qv = max(-127, min(127, qv));
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const uint32_t pr = e4m3x2_rn_sat(__fdiv_rn(__low2float(hv[e >> 1]), sc),
+                                              __fdiv_rn(__high2float(hv[e >> 1]), sc));
+            packed[e >> 2] |= pr << (8 * (e & 3));
+          }
         }
-        packed[e >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float f = (e & 1) ? __high2float(hv[e >> 1]) : __low2float(hv[e >> 1]);
+          int qv = 0;
+          if (sc != 0.f) {
+            qv = __float2int_rn(__fdiv_rn(f, sc));
+            qv = max(-127, min(127, qv));
+          }
+          packed[e >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
+        }
       }
-      int8_t* dst = codes + (s.start + r0 + row) * code_row_stride + static_cast<int64_t>(h) * D + c * 8;
+      uint8_t* dst = codes + (s.start + r0 + row) * code_row_stride + static_cast<int64_t>(h) * D + c * 8;
       *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
     }
   }
@@ -110,8 +135,9 @@ tm_status check_operand(const tm_tensor* t) {
   return TM_OK;
 }
 
-tm_status launch_quant(const tm_tensor* x, int8_t* codes, float* scales, const int32_t* cu,
-                       int32_t batch, int32_t max_seqlen, int32_t tile, cudaStream_t stream) {
+tm_status launch_quant(const tm_tensor* x, void* codes_ptr, float* scales, const int32_t* cu,
+                       int32_t batch, int32_t max_seqlen, int32_t tile, cudaStream_t stream, bool f8 = false) {
+  uint8_t* codes = static_cast<uint8_t*>(codes_ptr);
   if (codes == nullptr || scales == nullptr) return TM_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(codes) % 16 || reinterpret_cast<uintptr_t>(scales) % 4)
     return TM_ERR_INVALID_ARG;
@@ -123,12 +149,19 @@ tm_status launch_quant(const tm_tensor* x, int8_t* codes, float* scales, const i
   dim3 grid(static_cast<unsigned>(ntile), static_cast<unsigned>(nb), static_cast<unsigned>(x->H));
   DevErr err{device_error_word()};
   const __half* xp = static_cast<const __half*>(x->data);
-  if (x->d == 128)
-    quantize_tiles_kernel<128><<<grid, kQuantThreads, 0, stream>>>(
-        xp, x->stride_t, x->stride_h, static_cast<int>(x->H), codes, scales, cu, x->T, tile, err);
+  const int Hi = static_cast<int>(x->H);
+  if (x->d == 128 && f8)
+    quantize_tiles_kernel<128, true><<<grid, kQuantThreads, 0, stream>>>(xp, x->stride_t, x->stride_h, Hi, codes,
+                                                                          scales, cu, x->T, tile, err);
+  else if (x->d == 128)
+    quantize_tiles_kernel<128, false><<<grid, kQuantThreads, 0, stream>>>(xp, x->stride_t, x->stride_h, Hi, codes,
+                                                                           scales, cu, x->T, tile, err);
+  else if (f8)
+    quantize_tiles_kernel<64, true><<<grid, kQuantThreads, 0, stream>>>(xp, x->stride_t, x->stride_h, Hi, codes,
+                                                                         scales, cu, x->T, tile, err);
   else
-    quantize_tiles_kernel<64><<<grid, kQuantThreads, 0, stream>>>(
-        xp, x->stride_t, x->stride_h, static_cast<int>(x->H), codes, scales, cu, x->T, tile, err);
+    quantize_tiles_kernel<64, false><<<grid, kQuantThreads, 0, stream>>>(xp, x->stride_t, x->stride_h, Hi, codes,
+                                                                          scales, cu, x->T, tile, err);
   return check_cuda(cudaGetLastError());
 }
 
@@ -175,4 +208,24 @@ extern "C" tm_status tm_quantize_qk(const tm_tensor* q, const tm_tensor* k, int8
   st = launch_quant(q, q_codes, q_scales, cu_seqlens, batch, max_seqlen, tile_m, s);
   if (st != TM_OK || k == nullptr) return st;
   return launch_quant(k, k_codes, k_scales, cu_seqlens, batch, max_seqlen, tile_n, s);
+}
+
+extern "C" tm_status tm_quantize_qk_fp8(const tm_tensor* q, const tm_tensor* k, uint8_t* q_codes, float* q_scales,
+                                        uint8_t* k_codes, float* k_scales, const int32_t* cu_seqlens, int32_t batch,
+                                        int32_t max_seqlen, int32_t tile_m, int32_t tile_n, void* stream) {
+  using namespace tmk;
+  if ((tile_m != 64 && tile_m != 128) || (tile_n != 64 && tile_n != 128)) return TM_ERR_UNSUPPORTED;
+  tm_status st = check_operand(q);
+  if (st != TM_OK) return st;
+  if (k != nullptr) {
+    st = check_operand(k);
+    if (st != TM_OK) return st;
+    if (k->d != q->d) return TM_ERR_INVALID_ARG;
+    if (cu_seqlens != nullptr && k->T != q->T) return TM_ERR_INVALID_ARG;
+  }
+  if (cu_seqlens != nullptr && (batch <= 0 || max_seqlen <= 0)) return TM_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  st = launch_quant(q, q_codes, q_scales, cu_seqlens, batch, max_seqlen, tile_m, s, true);
+  if (st != TM_OK || k == nullptr) return st;
+  return launch_quant(k, k_codes, k_scales, cu_seqlens, batch, max_seqlen, tile_n, s, true);
 }

@@ -84,6 +84,8 @@ def _lib():
             "tm_probe_rates": (I32, [ctypes.POINTER(D), I32, P, I64, P]),
             "tm_merge_head_shards": (I32, [P, I64, P, I64, I32, I32, I32, I32, P, P]),
             "tm_set_attn_kernel": (I32, [I32]),
+            "tm_quantize_qk_fp8": (I32, [TP, TP, P, P, P, P, P, I32, I32, I32, I32, P]),
+            "tm_attn_fwd_fp8": (I32, [TP, TP, TP, TP, P, I32, I32, P, P, I64, P, P, P, P, I32, I32, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -212,6 +214,47 @@ def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqle
                             _ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks), _ptr(cu_seqlens), batch,
                             int(max_seqlen or 0), tile_m, tile_n, _stream())
     _check(st, "tm_quantize_qk")
+    return qc, qs, kc, ks
+
+
+def quantize_qk_fp8(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqlen=None,
+                    cu_seqlens_host=None, out=None):
+    """Per-tile FP8 E4M3 codes and fp32 scales of Q and K (the third
+    precision; tm_quantize_qk_fp8): returns (q_codes [Tq,Hq,d] uint8,
+    q_scales [n_qt, Hq] fp32, k_codes, k_scales); the K pair is None when k
+    is None.  out: the same 4-tuple of preallocated tensors."""
+    _cuda(q, "q")
+    _cuda(k, "k")
+    cu_h = _cu_host(cu_seqlens, cu_seqlens_host)
+    batch = 0 if cu_h is None else cu_h.numel() - 1
+    if cu_seqlens is not None and max_seqlen is None:
+        max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0
+    cu_np = None if cu_h is None else cu_h.numpy()
+    nqt = count_tiles(q.shape[0], tile_m, cu_np)
+    if out is not None:
+        qc, qs, kc, ks = out
+        _check_buf(qc, q.shape, torch.uint8, "q_codes")
+        _check_buf(qs, (nqt, q.shape[1]), torch.float32, "q_scales")
+    else:
+        qc = torch.empty(q.shape, dtype=torch.uint8, device=q.device)
+        qs = torch.empty((nqt, q.shape[1]), dtype=torch.float32, device=q.device)
+        kc = ks = None
+    if k is not None:
+        nkt = count_tiles(k.shape[0], tile_n, cu_np)
+        if out is not None:
+            _check_buf(kc, k.shape, torch.uint8, "k_codes")
+            _check_buf(ks, (nkt, k.shape[1]), torch.float32, "k_scales")
+        else:
+            kc = torch.empty(k.shape, dtype=torch.uint8, device=k.device)
+            ks = torch.empty((nkt, k.shape[1]), dtype=torch.float32, device=k.device)
+    else:
+        kc = ks = None
+    qd = _desc(q)
+    kd = _desc(k) if k is not None else None
+    st = _lib().tm_quantize_qk_fp8(ctypes.byref(qd), None if kd is None else ctypes.byref(kd), _ptr(qc), _ptr(qs),
+                                   _ptr(kc), _ptr(ks), _ptr(cu_seqlens), batch, int(max_seqlen or 0), tile_m,
+                                   tile_n, _stream())
+    _check(st, "tm_quantize_qk_fp8")
     return qc, qs, kc, ks
 
 
@@ -390,6 +433,38 @@ def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal
                          _ptr(cu_seqlens), batch, int(max_seqlen or 0), _ptr(bitmask),
                          int(mask_head_stride or 0), tile_m, tile_n, g, int(bool(causal)), _stream())
     _check(st, "tm_attn_fwd")
+    return out
+
+
+def attn_fwd_fp8(q, k, v, *, bitmask_fp8, qf8_quant, kf8_quant, out=None, g=1, causal=False, bitmask=None,
+                 q_quant=None, k_quant=None, cu_seqlens=None, max_seqlen=None, cu_seqlens_host=None):
+    """Attention with the FP8 third precision (tm_attn_fwd_fp8): d = 128,
+    128 x 128 tiles; bitmask_fp8 (int32 view [Hm, n_qt, W], layout of the
+    INT8 bitmask) routes a group to FP8 when its INT8 bit (bitmask, may be
+    None) is clear; qf8_quant / kf8_quant = (codes, scales) from
+    quantize_qk_fp8; q_quant / k_quant the INT8 (codes, scales) when bitmask
+    is given.  Returns out."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (bitmask_fp8, "bitmask_fp8")):
+        _cuda(t, n)
+    if out is None:
+        out = torch.empty_like(q)
+    cu_h = _cu_host(cu_seqlens, cu_seqlens_host)
+    batch = 0 if cu_h is None else cu_h.numel() - 1
+    if cu_seqlens is not None and max_seqlen is None:
+        max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0
+    qd = _desc(q, *(q_quant if q_quant is not None else (None, None)),
+               scale_kind=TM_SCALE_TILE if q_quant is not None else TM_SCALE_NONE)
+    kd = _desc(k, *(k_quant if k_quant is not None else (None, None)),
+               scale_kind=TM_SCALE_TILE if k_quant is not None else TM_SCALE_NONE)
+    vd, od = _desc(v), _desc(out)
+    mhs = 0 if bitmask_fp8.shape[0] == 1 else bitmask_fp8.shape[1] * bitmask_fp8.shape[2]
+    if bitmask is not None and tuple(bitmask.shape) != tuple(bitmask_fp8.shape):
+        raise ValueError("bitmask and bitmask_fp8 must have the same layout")
+    st = _lib().tm_attn_fwd_fp8(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
+                                _ptr(cu_seqlens), batch, int(max_seqlen or 0), _ptr(bitmask), _ptr(bitmask_fp8), mhs,
+                                _ptr(qf8_quant[0]), _ptr(qf8_quant[1]), _ptr(kf8_quant[0]), _ptr(kf8_quant[1]),
+                                g, int(bool(causal)), _stream())
+    _check(st, "tm_attn_fwd_fp8")
     return out
 
 
