@@ -805,6 +805,102 @@ def run_frontier(args):
             "peak": {"bf16_tflops": p16 / 1e12, "source": peak_src}, "points": rows}
 
 
+def run_fp8_table(args):
+    """The FP8 third precision on the routing-sweep inputs: attention time,
+    mix-weighted roofline fraction and output error against the all-FP16
+    output for FP16-only, INT8-only, FP8-only and three-way routing.  Each
+    point's kernel is named; FP8 routes run in the one-tile kernel, so the
+    FP16 and INT8 points are also given there.  E4M3 QK^T runs at the INT8
+    rate, so FP8 pairs take p8 = 2 p16 in the roofline like INT8 pairs.
+    Only the attention launch is timed (median of 20 calls, a 256 MiB buffer
+    written before each)."""
+    from mixed_precision_attention_tm_b200 import ops
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    p16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * 1e12
+    w = inputs.routing_sweep(0.0, seed=args.seed)
+    q, k, v = (x.to(dev) for x in (w.q, w.k, w.v))
+    mk = dict(tile_m=128, tile_n=128, g=w.g, causal=True, Lq=w.Lq, Lk=w.Lk, force_diag=True, force_sink=True)
+    i8 = ops.quantize_qk(q, k)
+    f8 = ops.quantize_qk_fp8(q, k)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(20):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        if ops.get_device_error() != ops.TM_OK:
+            raise RuntimeError("device error in the FP8 report")
+        return float(np.median(ts))
+
+    ref = None
+    rows = []
+
+    def point(name, kernel, p8, pf8):
+        nonlocal ref
+        m8 = None if p8 is None else ops.build_mask(w.hq, p=p8, seed=w.mask_seed, **mk)
+        mf8 = None if pf8 is None else ops.build_mask(w.hq, p=pf8, seed=w.mask_seed + 1, **mk)
+        ops.set_attn_kernel(kernel)
+        try:
+            if mf8 is None:
+                fn = lambda: ops.attn_fwd(q, k, v, out=out, g=w.g, causal=True, bitmask=m8,  # noqa: E731
+                                          q_quant=None if m8 is None else i8[:2],
+                                          k_quant=None if m8 is None else i8[2:])
+            else:
+                fn = lambda: ops.attn_fwd_fp8(q, k, v, out=out, g=w.g, causal=True, bitmask_fp8=mf8,  # noqa: E731
+                                              qf8_quant=f8[:2], kf8_quant=f8[2:], bitmask=m8,
+                                              q_quant=None if m8 is None else i8[:2],
+                                              k_quant=None if m8 is None else i8[2:])
+            ms = timed(fn)
+        finally:
+            ops.set_attn_kernel(ops.ATTN_KERNEL_AUTO)
+        h8 = None if m8 is None else m8.cpu().numpy().view(np.uint32)
+        hf8 = None if mf8 is None else mf8.cpu().numpy().view(np.uint32)
+        nv, e8 = route_stats_of(w, h8)
+        ef8 = 0.0
+        if hf8 is not None:                           # FP8 where the INT8 bit is clear
+            _, ef8 = route_stats_of(w, hf8 if h8 is None else hf8 & ~h8)
+        t_roof = roofline_time(w.d, nv, e8 + ef8, p16, 2.0 * p16)
+        o = out.float()
+        if ref is None:
+            ref = o.clone()
+        diff = (o - ref).abs()
+        rows.append({"point": name, "kernel": {ops.ATTN_KERNEL_AUTO: "auto", ops.ATTN_KERNEL_ONE_TILE: "one-tile",
+                                                ops.ATTN_KERNEL_TWO_TILE: "two-tile"}[kernel],
+                     "int8_group_probability": p8, "fp8_group_probability": pf8,
+                     "realised_int8_fraction": round(e8 / nv, 4), "realised_fp8_fraction": round(ef8 / nv, 4),
+                     "attn_ms": round(ms, 4), "tflops": round(4.0 * w.d * nv / (ms * 1e-3) / 1e12, 1),
+                     "mixed_roofline_frac": round(t_roof / (ms * 1e-3), 3),
+                     "err_max_abs": float(diff.max()), "err_rms": float(diff.pow(2).mean().sqrt())})
+
+    AUTO, ONE = ops.ATTN_KERNEL_AUTO, ops.ATTN_KERNEL_ONE_TILE
+    point("fp16", AUTO, None, None)                   # the error reference
+    point("fp16", ONE, None, None)
+    point("int8", AUTO, 0.75, None)
+    point("int8", ONE, 0.75, None)
+    point("fp8 plane empty", ONE, None, 0.0)          # the FP8 kernel variant with nothing routed to FP8
+    for pf8 in (0.25, 0.5, 0.75, 1.0):
+        point("fp8", ONE, None, pf8)
+    point("int8 + fp8", ONE, 0.5, 0.5)
+    point("int8 + fp8", ONE, 0.75, 1.0)
+    return {"metric": "FP8 third precision: attention time and error by route mix", "unit": "mixed",
+            "n_gpus": 1, "workload": w.name, "config": describe(w),
+            "reference": "all-FP16 output of the automatically chosen kernel on the same inputs",
+            "peak": {"bf16_tflops": p16 / 1e12, "source": peak_src}, "points": rows}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -812,7 +908,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="sweep",
-                    choices=["sweep", "long", "varlen", "prefix", "mlx", "tiny", "mlx_table", "frontier"])
+                    choices=["sweep", "long", "varlen", "prefix", "mlx", "tiny", "mlx_table", "frontier", "fp8_table"])
     ap.add_argument("--p", type=float, default=None,
                     help="INT8 group probability (default: the workload's configuration: 0.75, long context 0.5)")
     ap.add_argument("--seed", type=int, default=0)
@@ -831,9 +927,9 @@ def main():
 
     rank, local_rank, world = dist.world_info()
 
-    if args.workload in ("mlx_table", "frontier"):   # reports, not the contract's bench line
+    if args.workload in ("mlx_table", "frontier", "fp8_table"):   # reports, not the contract's bench line
         if rank == 0:
-            fn = run_mlx_table if args.workload == "mlx_table" else run_frontier
+            fn = {"mlx_table": run_mlx_table, "frontier": run_frontier, "fp8_table": run_fp8_table}[args.workload]
             print(json.dumps(fn(args)), flush=True)
         return
 

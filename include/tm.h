@@ -130,9 +130,9 @@ tm_status tm_quantize_qk_fp8(const tm_tensor* q, const tm_tensor* k, uint8_t* q_
                              int32_t max_seqlen, int32_t tile_m, int32_t tile_n, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Routing bitmask layout (TileMix abstract: "compact bitmasks", one bit per
- * query tile x key-tile group, "each routing bit govern[s] multiple adjacent
- * key tiles").
+ * Routing bitmask layout (TileMix abstract: routing decisions packed into a
+ * bitmask, one bit per query tile x key-tile group, a group being several
+ * neighbouring key tiles).
  *   word  bitmask[h * mask_head_stride + I_glob * W + G / 32], bit G % 32;
  *   G = J / g is the group of key tile J;  bit 1 = INT8, 0 = FP16;
  *   W = tm_mask_words(max Lk, tile_n, g) = ceil(ceil(ceil(Lk/tile_n)/g)/32).

@@ -37,19 +37,18 @@ also listed with its reason in the design notes of this repository):
   (h) GQA: query head h reads KV head h // (Hq / Hkv).
   (j) variable-length batches share one cu_seqlens for Q and K
       (self-attention prefill); query and key tiles restart per sequence.
-      With a separate cu_seqlens_k (prefix-cached prefill, the NEXT-2 item:
-      each sequence's lq new queries attend to lk >= lq keys, prefix first),
-      key rows of sequence b are cu_k[b] .. cu_k[b+1]-1 and causal masking
-      stays bottom-right per sequence (reading (f) with that sequence's Lq,
-      Lk).
+      With a separate cu_seqlens_k (prefix-cached prefill: each sequence's
+      lq new queries attend to lk >= lq keys, prefix first), key rows of
+      sequence b are cu_k[b] .. cu_k[b+1]-1 and causal masking stays
+      bottom-right per sequence (reading (f) with that sequence's Lq, Lk).
   (k) a query row with no visible key outputs 0.
   (m) the mask builder draws an independent Bernoulli(p) per eligible group
       from a counter-based hash (splitmix64); the group holding the query
       tile's last visible key tile ("diagonal") and group 0 ("sink") can be
       forced to FP16.
-  (n) a third precision (the NEXT-3 item; the pages name FP16 and INT8
-      only, and the fp8 scaling page, pytorch-labs float8_experimental #305,
-      gives per-tensor and per-axis fp8 scales): FP8 E4M3 codes with a
+  (p) a third precision (the TileMix abstract names FP16 and INT8 only;
+      the fp8 scaling page, pytorch-labs float8_experimental #305, gives
+      per-tensor and per-axis fp8 scales): FP8 E4M3 codes with a
       symmetric per-tile scale s = fl32(amax / 448) (448 is E4M3's largest
       finite value), code = E4M3 round-to-nearest-even of fl32(x / s),
       saturating at +-448; amax == 0 gives s = 0 and codes 0.  A second bit
@@ -181,7 +180,7 @@ def quantize_tiles(x16, seqs, tile, side):
 
 
 # --------------------------------------------------------------------------
-# FP8 E4M3 (reading (n))
+# FP8 E4M3 (reading (p))
 # --------------------------------------------------------------------------
 
 E4M3_MAX = 448.0
@@ -224,7 +223,7 @@ def e4m3_encode(x):
 
 
 def quantize_tiles_fp8(x16, seqs, tile, side):
-    """Per-(head, tile) FP8 E4M3 quantisation, reading (n): amax = max |x|
+    """Per-(head, tile) FP8 E4M3 quantisation, reading (p): amax = max |x|
     over the tile's rows x d; s = fl32(amax / 448); codes = e4m3_encode(
     fl32(x / s)); amax == 0 gives s = 0 and codes 0.  Returns (codes uint8
     [T, H, d], scales float32 [n_tiles, H]) in the tile order of
@@ -437,7 +436,7 @@ def attention(q, k=None, v=None, *, cu_seqlens=None, causal=False,
     rows: optional iterable of global query rows to evaluate (others are NaN).
     cu_seqlens_k: key offsets per sequence when they differ from cu_seqlens
     (prefix-cached prefill); reading (j).
-    mask_fp8 (reading (n)): a second bit plane in the layout of ``mask``; a
+    mask_fp8 (reading (p)): a second bit plane in the layout of ``mask``; a
     legal group whose INT8 bit is clear and FP8 bit is set takes
     S_ij = sigma * s_q * s_k * (dot product of the E4M3-decoded codes), with
     qf8_quant = (codes, scales[n_qtiles, Hq]) and kf8_quant = (codes,

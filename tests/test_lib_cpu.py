@@ -121,6 +121,48 @@ def test_validation_rejects_before_launch():
                              ctypes.c_uint64(0), 0, 0, 8, None) == ops.TM_ERR_INVALID_ARG
 
 
+def test_fp8_validation_rejects_before_launch():
+    """tm_attn_fwd_fp8 / tm_quantize_qk_fp8 argument checks: every case below
+    returns its status before any CUDA call."""
+    lib = ops._lib()
+    by = ctypes.byref
+    P = ctypes.c_void_p
+    q, k, v, o = _t(d=128), _t(H=1, d=128), _t(H=1, d=128), _t(d=128)
+    ok = P(1 << 20)                                     # an aligned stand-in pointer
+
+    def fwd(q=q, k=k, v=v, o=o, bm8=None, bmf8=ok, qc=ok, qs=ok, kc=ok, ks=ok, g=1):
+        return lib.tm_attn_fwd_fp8(by(q), by(k), by(v), by(o), None, 0, 0, bm8, bmf8, 0, qc, qs, kc, ks, g, 1, None)
+
+    # the FP8 route runs at d = 128 only
+    assert fwd(q=_t(d=64), k=_t(H=1, d=64), v=_t(H=1, d=64), o=_t(d=64)) == ops.TM_ERR_UNSUPPORTED
+    # an INT8 K/V cache is not an FP8 operand
+    kc8 = ops.TmTensor(0, 256, 1, 128, 128, 128, P(1 << 20), P(1 << 21), ops.TM_SCALE_TOKEN)
+    assert fwd(k=kc8, v=kc8) == ops.TM_ERR_UNSUPPORTED
+    # the FP8 plane, codes and scales are required and aligned
+    assert fwd(bmf8=None) == ops.TM_ERR_INVALID_ARG
+    assert fwd(bmf8=P((1 << 20) + 2)) == ops.TM_ERR_INVALID_ARG
+    for name in ("qc", "kc"):
+        assert fwd(**{name: None}) == ops.TM_ERR_INVALID_ARG
+        assert fwd(**{name: P((1 << 20) + 8)}) == ops.TM_ERR_INVALID_ARG
+    for name in ("qs", "ks"):
+        assert fwd(**{name: None}) == ops.TM_ERR_INVALID_ARG
+        assert fwd(**{name: P((1 << 20) + 2)}) == ops.TM_ERR_INVALID_ARG
+    # an INT8 plane needs the INT8 codes on Q and K
+    assert fwd(bm8=ok) == ops.TM_ERR_INVALID_ARG
+    assert fwd(g=0) == ops.TM_ERR_INVALID_ARG
+    # quantiser: tile sizes, null and misaligned outputs
+    assert lib.tm_quantize_qk_fp8(by(q), None, ok, ok, None, None, None, 0, 0, 96, 128, None) == ops.TM_ERR_UNSUPPORTED
+    assert lib.tm_quantize_qk_fp8(by(q), None, None, ok, None, None, None, 0, 0, 128, 128, None) == \
+        ops.TM_ERR_INVALID_ARG
+    assert lib.tm_quantize_qk_fp8(by(q), None, P((1 << 20) + 4), ok, None, None, None, 0, 0, 128, 128, None) == \
+        ops.TM_ERR_INVALID_ARG
+    assert lib.tm_quantize_qk_fp8(by(q), None, ok, P((1 << 20) + 1), None, None, None, 0, 0, 128, 128, None) == \
+        ops.TM_ERR_INVALID_ARG
+    # K of another head width
+    assert lib.tm_quantize_qk_fp8(by(q), by(_t(H=1, d=64)), ok, ok, ok, ok, None, 0, 0, 128, 128, None) == \
+        ops.TM_ERR_INVALID_ARG
+
+
 def test_prefill_plan_buffers_match_library_sizes():
     """The plan preallocates codes, tile scales and the routing mask once; their
     shapes must be the ones the library writes (tile counts per sequence, mask

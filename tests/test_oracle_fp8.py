@@ -1,4 +1,4 @@
-"""Pins of the oracle's FP8 E4M3 third precision (reading (n) of the oracle):
+"""Pins of the oracle's FP8 E4M3 third precision (reading (p) of the oracle):
 the format's published facts, a brute-force check of the encoder's
 rounding, the tile quantiser on cases whose answer is known, and the FP8
 route's wiring on inputs that the format represents exactly."""

@@ -1,9 +1,9 @@
 """Pins of the oracle's routing bitmask: one bit per (query tile, group of g
 key tiles), 1 = INT8, drawn by a counter-based hash.
 
-Source: TileMix (Lattice paper page), abstract -- "compact bitmasks", one
-routing bit governing several adjacent key tiles, all legal tile groups
-routed.  The Bernoulli draw, the forced diagonal/sink groups and the word
+Source: TileMix (Lattice paper page), abstract -- routing decisions packed
+into a bitmask, one bit for several neighbouring key tiles, every legal tile
+group computed.  The Bernoulli draw, the forced diagonal/sink groups and the word
 layout are the readings stated in the oracle's module docstring.
 """
 
