@@ -3,7 +3,13 @@ calls bench.py times: the whole output is computed on the GPU, and sampled
 query rows (tile boundaries plus seeded random rows, every head) are compared
 with the fp64 oracle, which evaluates those rows one by one.  Routing bits,
 INT8 codes and tile scales are compared in full (bit-exact).
+
+With TM_PARITY_REPORT set to a file path, one JSON line per configuration
+(rows compared, max-abs error, bound) is appended to that file.
 """
+
+import json
+import os
 
 import numpy as np
 import pytest
@@ -14,6 +20,23 @@ from gpu_helpers import TOL, max_err, oracle_mask, run_gpu, run_oracle, seqs_of
 from mixed_precision_attention_tm_b200 import inputs
 
 pytestmark = pytest.mark.gpu
+
+_REPORT = []
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _parity_report():
+    yield
+    path = os.environ.get("TM_PARITY_REPORT")
+    if path and _REPORT:
+        with open(path, "a") as f:
+            for r in _REPORT:
+                f.write(json.dumps(r) + "\n")
+
+
+def _record(w, rows, err, exact):
+    _REPORT.append({"workload": w.name, "heads": w.hq, "rows_compared": rows, "max_abs_err": err,
+                    "bound": TOL, "codes_scales_mask": exact})
 
 
 def _sample_rows(seqs, tile, n_random, seed):
@@ -34,6 +57,7 @@ def _check(w, n_random=48):
     assert torch.isfinite(out).all()
     seqs, _ = seqs_of(w)
     mask_u32 = None if m is None else m.numpy().view(np.uint32)
+    exact = "no mask"
     if mask_u32 is not None:
         assert np.array_equal(mask_u32, oracle_mask(w))
         rq = oracle.quantize_tiles(w.q.numpy(), seqs, w.tile_m, "q")
@@ -41,9 +65,11 @@ def _check(w, n_random=48):
         if quant[2] is not None:
             rk = oracle.quantize_tiles(w.k.numpy(), seqs, w.tile_n, "k")
             assert np.array_equal(quant[3].numpy(), rk[1]) and np.array_equal(quant[2].numpy(), rk[0])
+        exact = "bit-exact"
     rows = _sample_rows(seqs, w.tile_m, n_random, 17)
     ref = run_oracle(w, mask_u32, rows=rows)
     err = max_err(out, ref, rows=rows)
+    _record(w, f"{len(rows)} sampled rows x all heads", err, exact)
     assert err <= TOL, f"{w.name}: max abs err {err} over {len(rows)} rows"
 
 
@@ -72,5 +98,9 @@ def test_tiny_config_both_runs():
     for p in (None, 0.5):
         w = inputs.tiny(seed=0, p=p)
         out, m, _ = run_gpu(w)
+        if m is not None:
+            assert np.array_equal(m.numpy().view(np.uint32), oracle_mask(w))
         ref = run_oracle(w, None if m is None else m.numpy().view(np.uint32))
-        assert max_err(out, ref) <= TOL
+        err = max_err(out, ref)
+        _record(w, "all rows", err, "no mask" if m is None else "mask bit-exact")
+        assert err <= TOL
