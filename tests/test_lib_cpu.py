@@ -86,6 +86,23 @@ def test_route_stats_matches_oracle(case):
     assert (nv, e8) == (rnv, re8)
 
 
+@pytest.mark.parametrize("case", MASK_CASES[:5])
+def test_route_stats_of_two_planes_partition_the_pairs(case):
+    """The FP8 pairs of a three-way launch are counted on the plane 'FP8 bit
+    and not INT8 bit': the INT8 count and that count add up to the count of
+    the union plane, and never exceed the visible pairs."""
+    Hq, Lq, Lk, cu, tm, tn, g, causal, p, fd, fs = case
+    kw = dict(tile_m=tm, tile_n=tn, g=g, causal=causal, force_diag=fd, force_sink=fs, Lq=Lq, Lk=Lk,
+              cu_seqlens_host=cu)
+    m8 = ops.build_mask_host(Hq, p=p, seed=3, **kw)
+    mf8 = ops.build_mask_host(Hq, p=0.6, seed=4, **kw)
+    st = dict(Hq=Hq, tile_m=tm, tile_n=tn, g=g, causal=causal, Lq=Lq, Lk=Lk, cu_seqlens_host=cu)
+    nv, e8 = ops.route_stats(m8, **st)
+    _, ef8 = ops.route_stats(mf8 & ~m8, **st)
+    _, eu = ops.route_stats(m8 | mf8, **st)
+    assert e8 + ef8 == eu and eu <= nv
+
+
 def _t(T=256, H=2, d=64, data=1 << 20):
     return ops.TmTensor(data, T, H, d, H * d, d, None, None, 0)
 
