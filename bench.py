@@ -886,6 +886,13 @@ def run_fp8_table(args):
                      "err_max_abs": float(diff.max()), "err_rms": float(diff.pow(2).mean().sqrt())})
 
     AUTO, ONE = ops.ATTN_KERNEL_AUTO, ops.ATTN_KERNEL_ONE_TILE
+    if args.fp8_only is not None:
+        # one FP8-only point (no error reference: its error fields are
+        # against its own output)
+        point("fp8", ONE, None, args.fp8_only)
+        return {"metric": "FP8 third precision: attention time by route mix", "unit": "mixed", "n_gpus": 1,
+                "workload": w.name, "config": describe(w),
+                "peak": {"bf16_tflops": p16 / 1e12, "source": peak_src}, "points": rows}
     point("fp16", AUTO, None, None)                   # the error reference
     point("fp16", ONE, None, None)
     point("int8", AUTO, 0.75, None)
@@ -919,6 +926,8 @@ def main():
     ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
                     help="batch: every rank runs its own seeded problem (weak scaling); heads: one problem "
                          "split by query heads over the ranks, output all-gathered (strong scaling)")
+    ap.add_argument("--fp8-only", type=float, default=None,
+                    help="FP8 report: time only the FP8-only route at this group probability")
     ap.add_argument("--frontier-input", default="channels", choices=["channels", "tokens"],
                     help="frontier report: outlier channels in every token (the routing sweep's inputs) "
                          "or outliers in 0.2%% of the key tokens")
