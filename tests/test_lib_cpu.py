@@ -4,6 +4,8 @@ the oracle, and argument validation rejects bad calls before any launch.
 No GPU compute is called here."""
 
 import ctypes
+import os
+import shutil
 import subprocess
 
 import numpy as np
@@ -25,6 +27,20 @@ def test_library_exports_every_declared_symbol():
     out = subprocess.run(["nm", "-D", "--defined-only", ops.LIB_PATH], capture_output=True, text=True).stdout
     exported = {l.split()[-1] for l in out.splitlines() if l.strip()}
     assert set(names) <= exported
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/tm.h is a C header: it compiles as strict C99 with no CUDA or
+    C++ header on the include path."""
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not found")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "tm.h"\nint main(void) { tm_tensor t; (void)t; return tm_status_string(0) == 0; }\n')
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, "-c", str(src),
+                        "-o", str(tmp_path / "use_header.o")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
 
 
 def test_status_strings_and_version():
