@@ -156,6 +156,22 @@ def test_attention_matches_oracle(name, kw):
     assert err <= TOL, f"{name}: max abs err {err}"
 
 
+def test_long_key_rows_read_routing_words_and_scales_from_global_memory():
+    """Key rows of 2051 tiles at g = 1 need 65 routing words: both kernels keep
+    64 words and the first 256 (two-tile) or 512 (one-tile) key-tile scales in
+    shared memory, and read the rest from global memory."""
+    Lk = 2051 * 128
+    assert ops.mask_words(Lk, 128, 1) > 64
+    w = W(Lq=256, Lk=Lk, hq=2, hkv=1, d=128, causal=True, g=1, p=0.5, fd=True, fs=True)
+    out, m, _ = run_gpu(w)
+    mask_u32 = m.numpy().view(np.uint32)
+    assert np.array_equal(mask_u32, oracle_mask(w))
+    rows = [0, 1, 63, 127, 128, 129, 200, 255]
+    ref = run_oracle(w, mask_u32, rows=rows)
+    err = max_err(out, ref, rows=rows)
+    assert err <= TOL, f"max abs err {err}"
+
+
 # ------------------------------------------------------------------ GPU invariants
 def test_lossless_inputs_route_invisible_on_gpu():
     L, hq, hkv, d = 640, 2, 1, 128
