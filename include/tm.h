@@ -117,8 +117,8 @@ tm_status tm_quantize_qk_varlen(const tm_tensor* q, const tm_tensor* k, int8_t* 
                                 int32_t max_seqlen_k, int32_t tile_m, int32_t tile_n, void* stream);
 
 /* FP8 E4M3 codes of the third precision (the pages name FP16 and INT8; the
- * fp8 scaling page, pytorch-labs float8_experimental #305, describes fp8
- * operands with per-tensor or per-axis scales).  Per (head, tile) as in
+ * "Add rowwise scaling to Float8Inference module" page, Summary, describes
+ * fp8 operands with per-tensor or per-axis scales).  Per (head, tile) as in
  * tm_quantize_qk, with s = fl32(amax / 448) (448: the largest finite E4M3
  * value) and code = E4M3 round-to-nearest-even of fl32(x / s), saturating at
  * +-448 (bit 7 sign, bits 6..3 exponent with bias 7, bits 2..0 mantissa;
@@ -339,8 +339,8 @@ int64_t tm_probe_scratch_bytes(void);
 tm_status tm_probe_rates(double* out, int32_t n_out, void* scratch, int64_t scratch_bytes, void* stream);
 
 /* Attention with the FP8 third precision (the pages route between FP16 and
- * INT8; fp8 scaling page, pytorch-labs float8_experimental #305, for fp8
- * operands with per-axis scales).  As tm_attn_fwd with 128 x 128 tiles and
+ * INT8; fp8 operands with per-axis scales: "Add rowwise scaling to
+ * Float8Inference module" page, Summary).  As tm_attn_fwd with 128 x 128 tiles and
  * d = 128, plus a second routing bit plane `bitmask_fp8` in the layout of
  * `bitmask` (same mask_head_stride): a legal group whose INT8 bit is clear
  * and whose FP8 bit is set computes its scores from the E4M3 codes of

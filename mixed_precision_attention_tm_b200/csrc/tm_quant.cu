@@ -14,8 +14,8 @@
 // conversion is round-to-nearest-even, so the result is bit-identical to the
 // definition.  HBM-bound: bytes per element = 2 (read) + 1 (write).
 //
-// FP8 (the third precision; fp8 scaling page, pytorch-labs float8_experimental
-// #305, for per-axis fp8 scales): s = fl32(amax / 448), 448 being the
+// FP8 (the third precision; per-axis fp8 scales: "Add rowwise scaling to
+// Float8Inference module" page, Summary): s = fl32(amax / 448), 448 being the
 // largest finite E4M3 value; code = E4M3 round-to-nearest-even of
 // fl32(x / s) saturating at +-448, by the hardware conversion
 // cvt.rn.satfinite.e4m3x2.f32; s == 0 gives codes 0.

@@ -47,8 +47,8 @@ also listed with its reason in the design notes of this repository):
       tile's last visible key tile ("diagonal") and group 0 ("sink") can be
       forced to FP16.
   (p) a third precision (the TileMix abstract names FP16 and INT8 only;
-      the fp8 scaling page, pytorch-labs float8_experimental #305, gives
-      per-tensor and per-axis fp8 scales): FP8 E4M3 codes with a
+      the "Add rowwise scaling to Float8Inference module" page, Summary,
+      gives per-tensor and per-axis fp8 scales): FP8 E4M3 codes with a
       symmetric per-tile scale s = fl32(amax / 448) (448 is E4M3's largest
       finite value), code = E4M3 round-to-nearest-even of fl32(x / s),
       saturating at +-448; amax == 0 gives s = 0 and codes 0.  A second bit
