@@ -279,6 +279,8 @@ def run_ours(args, rank, world, local_rank):
     total_ms, attn_ms = dist.max_over_ranks([total_ms, attn_ms], device=dev)
     ms_step = total_ms / K
     value = dist.job_throughput(world, flops, ms_step)
+    if world == 1:
+        w.extra["gpu_out"] = plan.out.cpu()      # the last timed step's output, for the parity sample
 
     # roofline of the attention kernel (dominant launch)
     p16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * 1e12
@@ -590,7 +592,8 @@ def cpu_sample_spec(w, n_pairs):
 
 def oracle_pair(w, seqs, tile, h, prep):
     """Run the oracle on one (query tile, head): all rows of the tile, the
-    head's slice of Q; returns algorithmic FLOPs of the pair."""
+    head's slice of Q; returns the pair's algorithmic FLOPs and the oracle's
+    output rows [rows, d] (fp64)."""
     import oracle
     b, I, r0, rows, ig = tile
     q1 = w.q.numpy()[:, h:h + 1]
@@ -609,11 +612,11 @@ def oracle_pair(w, seqs, tile, h, prep):
         if kw.get("k_quant") is not None:
             kc, ks = kw["k_quant"]
             kw["k_quant"] = (kc[:, hk:hk + 1], ks[:, hk:hk + 1])
-    oracle.attention(q1, k1, v1, rows=range(r0, r0 + rows), **kw)
+    ref = oracle.attention(q1, k1, v1, rows=range(r0, r0 + rows), **kw)[r0:r0 + rows, 0]
     _qs, lq, _ks, lk = seqs[b]
     ii = I * w.tile_m + np.arange(rows)
     lim = np.minimum(lk - 1, ii + lk - lq) if w.causal else np.full(rows, lk - 1)
-    return 4.0 * w.d * float(np.maximum(lim + 1, 0).sum())
+    return 4.0 * w.d * float(np.maximum(lim + 1, 0).sum()), ref
 
 
 def oracle_prep(w, seqs):
@@ -632,26 +635,45 @@ def oracle_prep(w, seqs):
     return prep
 
 
+PARITY_BOUND = 3e-3   # max-abs output error of the parity tests (fp16 output, unit-variance inputs)
+
+
 def cpu_baseline(w, target_s):
     """Time the oracle as it stands on evenly spaced (query tile, head) pairs
-    until about target_s seconds of CPU work have run."""
+    until about target_s seconds of oracle time have run.  When the GPU
+    output of the timed steps is at hand (w.extra["gpu_out"]), the same
+    sampled rows are compared with it (outside the oracle's time).  Returns
+    (cpu_baseline dict, parity dict or None)."""
     cores = len(os.sched_getaffinity(0))
     seqs, _ = cpu_sample_spec(w, 1)
     prep = oracle_prep(w, seqs)            # quantisation and mask: not timed
     n_try = 64
     _, pairs = cpu_sample_spec(w, n_try)
-    flops = 0.0
-    t0 = time.perf_counter()
-    done = 0
+    gpu = w.extra.get("gpu_out")
+    flops, dt, err, n_rows, done = 0.0, 0.0, 0.0, 0, 0
     for tile, h in pairs:
-        flops += oracle_pair(w, seqs, tile, h, prep)
+        t0 = time.perf_counter()
+        f, ref = oracle_pair(w, seqs, tile, h, prep)
+        dt += time.perf_counter() - t0
+        flops += f
         done += 1
-        if time.perf_counter() - t0 > target_s:
+        if gpu is not None:
+            r0, rows = tile[2], tile[3]
+            got = gpu[r0:r0 + rows, h].to(torch.float64).numpy()
+            err = max(err, float(np.abs(got - ref).max()))
+            n_rows += rows
+        if dt > target_s:
             break
-    dt = time.perf_counter() - t0
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+    base = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{done} evenly spaced (query tile, head) pairs of {w.name} (all rows of each tile, "
                       f"fp64 NumPy/BLAS), {dt:.1f} s; quantisation and mask built beforehand, untimed"}
+    parity = None
+    if gpu is not None:
+        parity = {"max_abs_err": err, "bound": PARITY_BOUND, "pass": bool(err <= PARITY_BOUND),
+                  "rows_compared": n_rows,
+                  "sample": "the cpu_baseline pairs: every row of each sampled (query tile, head), the GPU output "
+                            "of the last timed step against the fp64 oracle on the same inputs"}
+    return base, parity
 
 
 def run_reference(args):
@@ -665,7 +687,7 @@ def run_reference(args):
     flops = 0.0
     t0 = time.perf_counter()
     for tile, h in pairs[args.warmup:args.warmup + args.steps]:
-        flops += oracle_pair(w, seqs, tile, h, prep)
+        flops += oracle_pair(w, seqs, tile, h, prep)[0]
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
     line = {
@@ -955,7 +977,9 @@ def main():
     try:
         line, w = (run_sharded if args.shard == "heads" else run_ours)(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+            line["cpu_baseline"], parity = cpu_baseline(w, args.cpu_seconds)
+            if parity is not None:
+                line["parity"] = parity
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
