@@ -47,3 +47,17 @@ def test_visible_pairs_closed_form(Lq, Lk, causal):
         assert metrics.visible_pairs(Lq, Lk, causal) == brute
     n, _ = oracle.route_stats(None, oracle.seq_table(Lq, Lk), 1, 128, 128, 1, causal)
     assert metrics.visible_pairs(Lq, Lk, causal) == n
+
+
+def test_mixed_roofline_closed_forms():
+    """T_roof = 2d E16 / P16 + 2d E8 / P8 + 2d N / P16 with P8 = 2 P16: all-FP16
+    pairs give the FP16 peak, all-INT8 pairs 4/3 of it, and the routing
+    sweep's realised INT8 fraction the bench line's effective peak."""
+    import bench
+    d, n, p16 = 128, 1.0e9, 1673.8e12
+    eff = lambda e8: 4 * d * n / bench.roofline_time(d, n, e8, p16, 2 * p16) / 1e12   # noqa: E731
+    assert abs(eff(0.0) - 1673.8) < 1e-6
+    assert abs(eff(n) - 1673.8 * 4 / 3) < 1e-6
+    f = 0.6801647848642051                      # realised INT8 fraction at p = 0.75
+    assert abs(eff(f * n) - 2 * 1673.8 / (1 + (1 - f) + f / 2)) < 1e-6
+    assert abs(eff(f * n) - 2016.73) < 0.01
