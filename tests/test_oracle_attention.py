@@ -8,7 +8,6 @@ scalar brute force, a library routine (fp64 torch SDPA), a closed form or an
 invariant of the mathematics.
 """
 
-import math
 
 import numpy as np
 import pytest

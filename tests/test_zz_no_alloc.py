@@ -10,7 +10,6 @@ Collected last on purpose: a run that stops at the first failure has already
 run every other test.
 """
 
-import numpy as np
 import pytest
 import torch
 
