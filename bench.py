@@ -126,6 +126,11 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+        return self.summary()
+
+    def summary(self):
+        """Median SM clock, the highest max clock seen and every throttle
+        reason reported active, from the parsed nvidia-smi rows."""
         sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
         mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
         reasons = set()
