@@ -165,6 +165,35 @@ def mask_words(max_lk, tile_n, g):
     return int(_lib().tm_mask_words(int(max_lk), int(tile_n), int(g)))
 
 
+def _need(t, n, dtype, name):
+    """t holds at least n contiguous elements of dtype."""
+    if t is None or t.dtype != dtype or not t.is_contiguous() or t.numel() < n:
+        got = "None" if t is None else f"{tuple(t.shape)} {t.dtype}"
+        raise ValueError(f"{name}: at least {n} contiguous {dtype} elements expected, got {got}")
+
+
+def _check_routing(Tq, Hq, Tk, Hkv, d, tile_m, tile_n, g, maxk, cu_h, ck_h, bitmask, mask_head_stride,
+                   q_quant, k_quant, codes_dtype=torch.int8, what=""):
+    """Sizes of the buffers an attention launch reads (the library receives
+    plain pointers): codes [T, H, d]; tile scales n_tiles x H fp32, tiles
+    counted per sequence; mask words (Hm - 1) x head stride + n_qtiles x W,
+    W = mask_words(longest key row, tile_n, g) as the kernels compute it.
+    ck_h: host key offsets (cu_h when keys share the query offsets), or None
+    when only the device holds them (then the key scales are not counted)."""
+    nqt = count_tiles(Tq, tile_m, None if cu_h is None else cu_h.numpy())
+    if bitmask is not None:
+        rows = nqt * mask_words(maxk, tile_n, g)
+        _need(bitmask, rows + (Hq - 1) * int(mask_head_stride or 0), torch.int32, what + "bitmask")
+    if q_quant is not None:
+        _need(q_quant[0], Tq * Hq * d, codes_dtype, what + "q codes")
+        _need(q_quant[1], nqt * Hq, torch.float32, what + "q scales")
+    if k_quant is not None:
+        _need(k_quant[0], Tk * Hkv * d, codes_dtype, what + "k codes")
+        if ck_h is not None or cu_h is None:
+            nkt = count_tiles(Tk, tile_n, None if ck_h is None else ck_h.numpy())
+            _need(k_quant[1], nkt * Hkv, torch.float32, what + "k scales")
+
+
 # ---------------------------------------------------------------- quantise
 def quantize_qk(q, k=None, *, tile_m=128, tile_n=128, cu_seqlens=None, max_seqlen=None,
                 cu_seqlens_host=None, out=None, cu_seqlens_k=None, max_seqlen_k=None, cu_seqlens_k_host=None):
@@ -404,6 +433,16 @@ def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal
     batch = 0 if cu_h is None else cu_h.numel() - 1
     if cu_seqlens is not None and max_seqlen is None:
         max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0
+    if bitmask is not None and mask_head_stride is None:
+        mask_head_stride = 0 if bitmask.shape[0] == 1 else bitmask.shape[1] * bitmask.shape[2]
+    ck_h = None
+    if cu_seqlens_k is not None and max_seqlen_k is None:
+        ck_h = _cu_host(cu_seqlens_k, None)
+        max_seqlen_k = int((ck_h[1:] - ck_h[:-1]).max()) if batch else 0
+    kshape = (kv_cache[0] if kv_cache is not None else k).shape
+    maxk = (max_seqlen_k if cu_seqlens_k is not None else max_seqlen) if cu_seqlens is not None else kshape[0]
+    _check_routing(q.shape[0], q.shape[1], kshape[0], kshape[1], q.shape[2], tile_m, tile_n, g, maxk or 0, cu_h,
+                   ck_h if cu_seqlens_k is not None else cu_h, bitmask, mask_head_stride, q_quant, k_quant)
     qd = _desc(q, *(q_quant if q_quant is not None else (None, None)),
                scale_kind=TM_SCALE_TILE if q_quant is not None else TM_SCALE_NONE)
     if kv_cache is not None:
@@ -417,12 +456,7 @@ def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal
                    scale_kind=TM_SCALE_TILE if k_quant is not None else TM_SCALE_NONE)
         vd = _desc(v)
     od = _desc(out)
-    if bitmask is not None and mask_head_stride is None:
-        mask_head_stride = 0 if bitmask.shape[0] == 1 else bitmask.shape[1] * bitmask.shape[2]
     if cu_seqlens_k is not None:
-        if max_seqlen_k is None:
-            ck_h = _cu_host(cu_seqlens_k, None)
-            max_seqlen_k = int((ck_h[1:] - ck_h[:-1]).max()) if batch else 0
         st = lib.tm_attn_fwd_varlen(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
                                     _ptr(cu_seqlens), _ptr(cu_seqlens_k), batch, int(max_seqlen or 0),
                                     int(max_seqlen_k or 0), _ptr(bitmask), int(mask_head_stride or 0), tile_m,
@@ -460,6 +494,11 @@ def attn_fwd_fp8(q, k, v, *, bitmask_fp8, qf8_quant, kf8_quant, out=None, g=1, c
     mhs = 0 if bitmask_fp8.shape[0] == 1 else bitmask_fp8.shape[1] * bitmask_fp8.shape[2]
     if bitmask is not None and tuple(bitmask.shape) != tuple(bitmask_fp8.shape):
         raise ValueError("bitmask and bitmask_fp8 must have the same layout")
+    maxk = max_seqlen if cu_seqlens is not None else k.shape[0]
+    _check_routing(q.shape[0], q.shape[1], k.shape[0], k.shape[1], q.shape[2], 128, 128, g, maxk or 0, cu_h, cu_h,
+                   bitmask, mhs, q_quant, k_quant)
+    _check_routing(q.shape[0], q.shape[1], k.shape[0], k.shape[1], q.shape[2], 128, 128, g, maxk or 0, cu_h, cu_h,
+                   bitmask_fp8, mhs, qf8_quant, kf8_quant, codes_dtype=torch.uint8, what="fp8 ")
     st = _lib().tm_attn_fwd_fp8(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
                                 _ptr(cu_seqlens), batch, int(max_seqlen or 0), _ptr(bitmask), _ptr(bitmask_fp8), mhs,
                                 _ptr(qf8_quant[0]), _ptr(qf8_quant[1]), _ptr(kf8_quant[0]), _ptr(kf8_quant[1]),
