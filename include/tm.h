@@ -286,9 +286,14 @@ tm_status tm_attn_fwd_varlen(const tm_tensor* q, const tm_tensor* k, const tm_te
  * data; their codes / scales fields are ignored) and out, as for tm_attn_fwd,
  * and the routing parameters of tm_build_mask (mask_head_stride is implied).
  * No cudaMalloc, cudaFree or other allocating routine is called.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) while that device is current; make that first
- *    call before any stream capture.
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *    in the current device's context, so a reset device or another context
+ *    gets its own address; the lookup allocates nothing.  The first call on a
+ *    device also sets up the library's module there: make it before any
+ *    stream capture.
+ *  - Every argument is checked before the lookup and before any launch, so a
+ *    rejected call leaves the array and out untouched.  The codes / scales
+ *    fields of q, k and v are ignored (v is read as fp16 values).
  *  - All calls share the array and it keeps the last call's contents; every
  *    byte a call reads it first writes, so nothing needs clearing.  Calls
  *    that overlap on the GPU (other streams, other host threads on the same

@@ -16,37 +16,58 @@
 // threads on one device) race on it, so callers serialise them.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "tm_host.h"
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_tm_scratch[TM_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDev = 64;
-unsigned char* g_scratch_dev[kMaxDev] = {};
-std::mutex g_scratch_mu;
-
-// Device address of g_tm_scratch on the current device (looked up once per
-// device; in host code the symbol itself is only a host-side handle).
+// Device address of g_tm_scratch in the current device's context.  In host
+// code the symbol itself is only a host-side handle, so it is resolved here,
+// on every call: the lookup is cheap and allocates nothing, and a cached
+// address would go stale if the caller reset the device or switched
+// contexts between calls.
 tm_status scratch_address(unsigned char** out) {
-  int dev = 0;
-  tm_status st = tmk::check_cuda(cudaGetDevice(&dev));
+  void* p = nullptr;
+  tm_status st = tmk::check_cuda(cudaGetSymbolAddress(&p, g_tm_scratch));
   if (st != TM_OK) return st;
-  if (dev < 0 || dev >= kMaxDev) return TM_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_dev[dev] == nullptr) {
-    void* p = nullptr;
-    st = tmk::check_cuda(cudaGetSymbolAddress(&p, g_tm_scratch));
-    if (st != TM_OK) return st;
-    g_scratch_dev[dev] = static_cast<unsigned char*>(p);
-  }
-  *out = g_scratch_dev[dev];
+  *out = static_cast<unsigned char*>(p);
   return TM_OK;
 }
 
 int64_t align256(int64_t x) { return (x + 255) & ~static_cast<int64_t>(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The checks tm_quantize_qk, tm_build_mask and tm_attn_fwd make on these
+// arguments, made here before anything is launched, so that a rejected call
+// leaves the scratch array and the output untouched.
+tm_status check_fp16(const tm_tensor* t, int64_t d) {
+  if (t == nullptr || t->data == nullptr || !aligned16(t->data)) return TM_ERR_INVALID_ARG;
+  if (t->T < 0 || t->H <= 0 || t->d != d) return TM_ERR_INVALID_ARG;
+  if (t->stride_h < d || (t->stride_h % 8) || (t->stride_t % 8)) return TM_ERR_INVALID_ARG;
+  if (t->stride_t < t->stride_h * (t->H - 1) + d) return TM_ERR_INVALID_ARG;
+  return TM_OK;
+}
+
+tm_status validate(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, const tm_tensor* out,
+                   int32_t tile_m, int32_t tile_n, int32_t g, double p) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return TM_ERR_INVALID_ARG;
+  if ((tile_m != 64 && tile_m != 128) || (tile_n != 64 && tile_n != 128)) return TM_ERR_UNSUPPORTED;
+  if (g < 1 || !(p >= 0.0 && p <= 1.0)) return TM_ERR_INVALID_ARG;
+  const int64_t D = q->d;
+  if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
+  const tm_tensor* ts[4] = {q, k, v, out};
+  for (const tm_tensor* t : ts) {
+    const tm_status st = check_fp16(t, D);
+    if (st != TM_OK) return st;
+  }
+  if (out->T != q->T || out->H != q->H) return TM_ERR_INVALID_ARG;
+  if (k->T != v->T || k->H != v->H) return TM_ERR_INVALID_ARG;
+  if (q->H % k->H != 0 || q->H > 65535) return TM_ERR_INVALID_ARG;
+  if (q->T > 0x7fffffffLL || k->T > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
+  return TM_OK;
+}
 
 }  // namespace
 
@@ -54,14 +75,10 @@ extern "C" tm_status tm_attn_fwd_routed_noalloc(const tm_tensor* q, const tm_ten
                                                 tm_tensor* out, int32_t tile_m, int32_t tile_n, int32_t g,
                                                 int32_t causal, double p, uint64_t seed, int32_t force_diag,
                                                 int32_t force_sink, void* stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return TM_ERR_INVALID_ARG;
-  if (q->data == nullptr || k->data == nullptr || v->data == nullptr || out->data == nullptr)
-    return TM_ERR_INVALID_ARG;
-  if (q->T < 0 || k->T < 0 || q->H <= 0 || k->H <= 0 || g < 1) return TM_ERR_INVALID_ARG;
-  if ((tile_m != 64 && tile_m != 128) || (tile_n != 64 && tile_n != 128)) return TM_ERR_UNSUPPORTED;
-  if (q->d != 64 && q->d != 128) return TM_ERR_UNSUPPORTED;
+  tm_status st = validate(q, k, v, out, tile_m, tile_n, g, p);
+  if (st != TM_OK) return st;
   // Scratch layout (256-byte aligned parts): Q codes, K codes, Q scales,
-  // K scales, routing mask.
+  // K scales, routing mask.  The sizes come from validated shapes.
   const int64_t nqt = (q->T + tile_m - 1) / tile_m;
   const int64_t nkt = (k->T + tile_n - 1) / tile_n;
   const int64_t W = tm_mask_words(k->T, tile_n, g);
@@ -74,7 +91,7 @@ extern "C" tm_status tm_attn_fwd_routed_noalloc(const tm_tensor* q, const tm_ten
   if (total > static_cast<int64_t>(TM_NOALLOC_SCRATCH_BYTES)) return TM_ERR_UNSUPPORTED;
 
   unsigned char* base = nullptr;
-  tm_status st = scratch_address(&base);
+  st = scratch_address(&base);
   if (st != TM_OK) return st;
   int8_t* qc = reinterpret_cast<int8_t*>(base + off_qc);
   int8_t* kc = reinterpret_cast<int8_t*>(base + off_kc);
@@ -82,19 +99,25 @@ extern "C" tm_status tm_attn_fwd_routed_noalloc(const tm_tensor* q, const tm_ten
   float* ks = reinterpret_cast<float*>(base + off_ks);
   uint32_t* mask = reinterpret_cast<uint32_t*>(base + off_m);
 
-  // Every byte read later is written first (all tiles of Q and K, every mask
-  // word of every query-tile row), so nothing needs clearing between calls.
-  st = tm_quantize_qk(q, k, qc, qs, kc, ks, nullptr, 0, 0, tile_m, tile_n, stream);
-  if (st != TM_OK) return st;
-  st = tm_build_mask(mask, static_cast<int32_t>(q->H), nullptr, 0, 0, q->T, k->T, tile_m, tile_n, g, causal, p,
-                     seed, force_diag, force_sink, nqt * W, stream);
-  if (st != TM_OK) return st;
-  tm_tensor qq = *q, kk = *k;
+  // The INT8 fields of q, k and v are the library's here: q and k get the
+  // scratch codes and scales, and v is read as plain fp16 values.
+  tm_tensor qq = *q, kk = *k, vv = *v;
   qq.codes = qc;
   qq.scales = qs;
   qq.scale_kind = TM_SCALE_TILE;
   kk.codes = kc;
   kk.scales = ks;
   kk.scale_kind = TM_SCALE_TILE;
-  return tm_attn_fwd(&qq, &kk, v, out, nullptr, 0, 0, mask, nqt * W, tile_m, tile_n, g, causal, stream);
+  vv.codes = nullptr;
+  vv.scales = nullptr;
+  vv.scale_kind = TM_SCALE_NONE;
+
+  // Every byte read later is written first (all tiles of Q and K, every mask
+  // word of every query-tile row), so nothing needs clearing between calls.
+  st = tm_quantize_qk(&qq, &kk, qc, qs, kc, ks, nullptr, 0, 0, tile_m, tile_n, stream);
+  if (st != TM_OK) return st;
+  st = tm_build_mask(mask, static_cast<int32_t>(q->H), nullptr, 0, 0, q->T, k->T, tile_m, tile_n, g, causal, p,
+                     seed, force_diag, force_sink, nqt * W, stream);
+  if (st != TM_OK) return st;
+  return tm_attn_fwd(&qq, &kk, &vv, out, nullptr, 0, 0, mask, nqt * W, tile_m, tile_n, g, causal, stream);
 }

@@ -73,12 +73,13 @@ def _check(w, n_random=48):
     assert err <= TOL, f"{w.name}: max abs err {err} over {len(rows)} rows"
 
 
-@pytest.mark.parametrize("Lq,Lk,d,hq,hkv,causal", [
-    (4096, 4096, 128, 32, 8, True), (4096, 4096, 64, 16, 2, False), (512, 4096, 128, 32, 8, True),
-    (2048, 2048, 64, 32, 32, True),
-])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Lq,Lk,d,hq,hkv", inputs.MLX_SHAPES)
 def test_mlx_shapes_full_size(Lq, Lk, d, hq, hkv, causal):
-    _check(inputs.mlx_shape(Lq, Lk, d, hq, hkv, causal))
+    """All 48 runs of the MLX-shaped configuration (24 shapes of the MLX PR
+    "Nax Refactor" attention tables, causal and not), each at its own size,
+    through the library's automatic kernel choice as bench.py times them."""
+    _check(inputs.mlx_shape(Lq, Lk, d, hq, hkv, causal), n_random=32)
 
 
 @pytest.mark.parametrize("p", [0.0, 0.75, 1.0])

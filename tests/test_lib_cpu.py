@@ -224,3 +224,45 @@ def test_attn_kernel_choice_rejects_unknown_values():
     assert lib.tm_set_attn_kernel(-1) == ops.TM_ERR_INVALID_ARG
     for c in (ops.ATTN_KERNEL_TWO_TILE, ops.ATTN_KERNEL_ONE_TILE, ops.ATTN_KERNEL_AUTO):
         assert lib.tm_set_attn_kernel(c) == ops.TM_OK
+
+
+def test_noalloc_validates_every_argument_before_any_cuda_call():
+    """tm_attn_fwd_routed_noalloc rejects a bad call before it looks up its
+    scratch array or launches anything: each case below returns its status
+    without a CUDA call.  With no GPU present, a well-formed call gets as far
+    as the first CUDA call (the array's address) and returns TM_ERR_CUDA, which
+    shows the order."""
+    import torch
+    lib = ops._lib()
+    by = ctypes.byref
+    q, k, v, o = _t(d=128, H=4), _t(H=2, d=128), _t(H=2, d=128), _t(d=128, H=4)
+
+    def call(q=q, k=k, v=v, o=o, tm=128, tn=128, g=2, p=0.5):
+        return lib.tm_attn_fwd_routed_noalloc(by(q), by(k), by(v), by(o), tm, tn, g, 1, p, ctypes.c_uint64(1), 1, 1,
+                                              None)
+
+    assert lib.tm_attn_fwd_routed_noalloc(None, by(k), by(v), by(o), 128, 128, 1, 1, 0.5, ctypes.c_uint64(1), 1, 1,
+                                          None) == ops.TM_ERR_INVALID_ARG
+    assert call(tm=96) == ops.TM_ERR_UNSUPPORTED
+    assert call(g=0) == ops.TM_ERR_INVALID_ARG
+    assert call(p=1.5) == ops.TM_ERR_INVALID_ARG
+    assert call(p=float("nan")) == ops.TM_ERR_INVALID_ARG
+    # head width outside {64, 128}, and K / V / out of another head width than Q
+    assert call(q=_t(d=96, H=4), o=_t(d=96, H=4)) == ops.TM_ERR_UNSUPPORTED
+    assert call(k=_t(H=2, d=64)) == ops.TM_ERR_INVALID_ARG
+    assert call(v=_t(H=2, d=64)) == ops.TM_ERR_INVALID_ARG
+    assert call(o=_t(H=4, d=64)) == ops.TM_ERR_INVALID_ARG
+    # Hq not a multiple of Hkv; V's shape differs from K's
+    assert call(k=_t(H=3, d=128), v=_t(H=3, d=128)) == ops.TM_ERR_INVALID_ARG
+    assert call(v=_t(T=255, H=2, d=128)) == ops.TM_ERR_INVALID_ARG
+    assert call(v=_t(H=1, d=128)) == ops.TM_ERR_INVALID_ARG
+    assert call(o=_t(T=128, H=4, d=128)) == ops.TM_ERR_INVALID_ARG
+    # misaligned data and strides
+    assert call(v=ops.TmTensor((1 << 20) + 8, 256, 2, 128, 256, 128, None, None, 0)) == ops.TM_ERR_INVALID_ARG
+    assert call(k=ops.TmTensor(1 << 20, 256, 2, 128, 260, 128, None, None, 0)) == ops.TM_ERR_INVALID_ARG
+    assert call(o=ops.TmTensor(1 << 20, 256, 4, 128, 256, 64, None, None, 0)) == ops.TM_ERR_INVALID_ARG
+    # beyond the fixed array (codes alone: 16384 * 32 * 128 bytes = 64 MiB)
+    big_q = _t(T=16384, H=32, d=128)
+    assert call(q=big_q, o=big_q, k=_t(T=16384, H=8, d=128), v=_t(T=16384, H=8, d=128)) == ops.TM_ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        assert call() == ops.TM_ERR_CUDA

@@ -35,8 +35,9 @@ CALLS = [
 
 
 def test_noalloc_matches_regular_path_on_consecutive_calls():
-    outs = []
-    for (Lq, Lk, hq, hkv, d, tm, tn, g, causal, p, seed, fd, fs) in CALLS:
+    # The first call is the larger one, so the second reuses an array that
+    # still holds longer codes, scales and mask rows from the first.
+    for i, (Lq, Lk, hq, hkv, d, tm, tn, g, causal, p, seed, fd, fs) in enumerate(CALLS):
         q = inputs.randn_f16((Lq, hq, d), seed).cuda()
         k = inputs.randn_f16((Lk, hkv, d), seed + 1).cuda()
         v = inputs.randn_f16((Lk, hkv, d), seed + 2).cuda()
@@ -45,11 +46,25 @@ def test_noalloc_matches_regular_path_on_consecutive_calls():
         ref = _regular(q, k, v, tm, tn, g, causal, p, seed, fd, fs)
         torch.cuda.synchronize()
         assert ops.get_device_error() == ops.TM_OK
-        err = (got.float() - ref.float()).abs().max().item()
-        assert err <= TOL, f"call {len(outs)}: max abs difference {err}"
-        outs.append(got.cpu())
-    # the second call overwrote the shared array; the first result is unaffected
-    assert outs[0].shape != outs[1].shape
+        # the same kernels on the same inputs: the outputs are bit-identical
+        assert torch.equal(got, ref), f"call {i}: max abs difference {(got.float() - ref.float()).abs().max().item()}"
+
+
+def test_noalloc_call_leaves_device_memory_unchanged():
+    Lq, Lk, hq, hkv, d, tm, tn, g, causal, p, seed, fd, fs = CALLS[0]
+    q = inputs.randn_f16((Lq, hq, d), seed).cuda()
+    k = inputs.randn_f16((Lk, hkv, d), seed + 1).cuda()
+    v = inputs.randn_f16((Lk, hkv, d), seed + 2).cuda()
+    out = torch.empty_like(q)
+    kw = dict(out=out, tile_m=tm, tile_n=tn, g=g, causal=causal, p=p, seed=seed, force_diag=fd, force_sink=fs)
+    ops.attn_fwd_routed_noalloc(q, k, v, **kw)   # first call on the device: module and symbol set-up
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    ops.attn_fwd_routed_noalloc(q, k, v, **kw)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
+    assert torch.equal(out, _regular(q, k, v, tm, tn, g, causal, p, seed, fd, fs))
 
 
 def test_noalloc_rejects_problems_beyond_the_array():
