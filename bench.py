@@ -209,6 +209,17 @@ def route_stats_of(w, mask_host):
                            Lq=w.Lq, Lk=w.Lk, cu_seqlens_host=cu, cu_seqlens_k_host=ck)
 
 
+def quant_bytes(plan):
+    """Algorithmic HBM bytes of one quantiser launch: the fp16 operands read
+    once, their int8 codes and fp32 tile scales written once."""
+    n = 0
+    for x, quant in ((plan.q, plan.q_quant), (plan.k, plan.k_quant)):
+        if x is None or quant is None:
+            continue
+        n += x.numel() * 2 + quant[0].numel() + quant[1].numel() * 4
+    return n
+
+
 def roofline_time(d, n_vis, e8, p16, p8):
     """Mix-weighted tensor roofline (seconds): QK^T of FP16 pairs at p16, of
     INT8 pairs at p8, and P.V of every pair at p16 (FLOP/s)."""
@@ -249,6 +260,8 @@ def run_ours(args, rank, world, local_rank):
     K = args.steps
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_qa = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_qb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
     dist.barrier()
@@ -264,7 +277,9 @@ def run_ours(args, rank, world, local_rank):
             flush.zero_()                      # evict the inputs from L2 (outside the step's events)
             st_a[i].record(stream)
         if plan.routed:
+            ev_qa[i].record(stream)
             plan.quantize()
+            ev_qb[i].record(stream)
             plan.mask()
         ev_a[i].record(stream)
         plan.attend()
@@ -279,9 +294,10 @@ def run_ours(args, rank, world, local_rank):
     if flush is not None:
         total_ms = sum(a.elapsed_time(b) for a, b in zip(st_a, st_b))
     attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev_a, ev_b)) / K
+    quant_ms = sum(a.elapsed_time(b) for a, b in zip(ev_qa, ev_qb)) / K if plan.routed else 0.0
     if ops.get_device_error() != ops.TM_OK:
         raise RuntimeError("device error in timed region")
-    total_ms, attn_ms = dist.max_over_ranks([total_ms, attn_ms], device=dev)
+    total_ms, attn_ms, quant_ms = dist.max_over_ranks([total_ms, attn_ms, quant_ms], device=dev)
     ms_step = total_ms / K
     value = dist.job_throughput(world, flops, ms_step)
     if world == 1:
@@ -392,6 +408,19 @@ def run_ours(args, rank, world, local_rank):
     except Exception as exc:                                   # a probe failure must not hide the run
         secondary = {"unavailable": str(exc)}
 
+    # roofline of the quantiser launch (Q and K in one launch): HBM-bound,
+    # 2 bytes read + 1 byte of code written per element, plus the tile scales
+    roofline_quant = None
+    if plan.routed and quant_ms > 0:
+        qbytes = quant_bytes(plan)
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        ach = qbytes / (quant_ms * 1e-3) / 1e9
+        roofline_quant = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                          "traffic": None, "bytes_per_launch": qbytes, "ms_per_launch": quant_ms,
+                          "peak_source": f"{peak_src} copy bandwidth",
+                          "traffic_note": "algorithmic bytes: fp16 Q and K read once, int8 codes and fp32 "
+                                          "tile scales written once"}
+
     launches = plan.launches_per_step * K
     traffic, traffic_note = (None, "traffic captured for the routing-sweep workload only")
     if args.workload == "sweep" and w.p == 0.75:
@@ -416,6 +445,8 @@ def run_ours(args, rank, world, local_rank):
         "attn_ms": attn_ms,
         "mixed_roofline_frac_of_measured": t_roof / (attn_ms * 1e-3),
         "mixed_roofline_frac_of_nominal": t_roof_nom / (attn_ms * 1e-3),
+        "quant_ms": quant_ms,
+        "roofline_quant": roofline_quant,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff, "unit": "TFLOP/s",
                      "frac": achieved / peak_eff, "traffic": traffic, "traffic_note": traffic_note,
                      "peak_source": f"{peak_src} bf16 burst {p16 / 1e12:.1f} TFLOP/s for FP16 pairs, x2 "

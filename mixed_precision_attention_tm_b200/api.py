@@ -97,7 +97,7 @@ class TileMixPrefill:
                 self.bitmask = bitmask
             else:
                 self.bitmask = torch.empty(shape, dtype=torch.int32, device=dev)
-        n_quant = (2 if not int8_cache else 1) if self.routed else 0
+        n_quant = 1 if self.routed else 0          # Q and K are quantised in one launch
         n_mask = 1 if self.routed and not self.external_mask else 0
         self.launches_per_step = 1 + n_quant + n_mask
 

@@ -13,6 +13,10 @@
 //     tile, the tensor pipe runs the other tile's P.V and next QK^T;
 //   * TMEM holds S_A, S_B (128 columns each; P overwrites S in place as fp16)
 //     and the fp32 accumulators O_A, O_B;
+//   * an INT8-routed score tile leaves the tensor core as exact fp32 numbers
+//     (mma_i8_exact_n: a seed MMA, the kind::i8 MMAs, an unseed MMA), so the
+//     softmax handles both routes alike, only the scale differs; the INT8
+//     QK^T takes 6 MMAs of M128 N128 against the FP16 route's 8;
 //   * K / V arrive through a ring of tile-sized shared-memory slots: per key
 //     tile the producer loads the fp16 K tile if either query tile routes it
 //     FP16, the int8 K-code tile if either routes it INT8 (both when they
@@ -96,8 +100,10 @@ struct Cfg2 {
   static constexpr int OFF_Q8 = 2 * Q16_BYTES;
   static constexpr int OFF_SLOT = OFF_Q8 + 2 * Q8_BYTES;
   static constexpr int OFF_BAR = OFF_SLOT + NSLOT * SLOT;
-  static constexpr int BAR_BYTES = 2048;                 // barriers, routing words, key-tile scales
-  static constexpr int KSC_MAX = 256;                    // key tiles whose INT8 scales are staged
+  static constexpr int BAR_BYTES = 2048;                 // barriers, routing words, seed blocks, key-tile scales
+  static constexpr int OFF_SEED = OFF_BAR + 768;         // the INT8 accumulator seed blocks (kSeedBytes)
+  static constexpr int OFF_KSC = OFF_BAR + 1152;
+  static constexpr int KSC_MAX = 224;                    // key tiles whose INT8 scales are staged
   static constexpr int MAXW = 64;                        // routing words per query tile kept in smem
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -115,6 +121,7 @@ struct Cfg2 {
   static constexpr int THREADS = 384;
   static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, CONTROL_REGS = 72;
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(OFF_SEED + kSeedBytes <= OFF_KSC && OFF_KSC + 4 * KSC_MAX <= OFF_BAR + BAR_BYTES, "layout");
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS == THREADS * LAUNCH_REGS,
                 "register split must equal the launch allocation");
   __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
@@ -154,6 +161,7 @@ struct Params2 {
   int kv_chunk;            // KV heads per scheduling chunk (divides Hkv)
   float scale_log2;
   DevErr err;
+  int sched_zero;        // always 0 (see its use in the softmax)
 };
 
 // Routing bit of key tile j (group j / g); row is a shared- or global-memory
@@ -189,7 +197,7 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * C_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * C_COUNT + 4);
   uint32_t* route_words = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 256);   // [2][MAXW]
-  float* ksc = reinterpret_cast<float*>(smem + C::OFF_BAR + 1024);                 // [KSC_MAX]
+  float* ksc = reinterpret_cast<float*>(smem + C::OFF_KSC);                        // [KSC_MAX]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -273,6 +281,10 @@ __global__ void __launch_bounds__(384, 1)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
     tc_fence_before();
+  }
+  if (warp == 10) {
+    seed_blocks_init(reinterpret_cast<uint32_t*>(smem + C::OFF_SEED), lane);
+    fence_async_shared();   // generic-proxy stores, read by tcgen05.mma
   }
   if (warp == 8) {
     if (lane == 0) {
@@ -434,15 +446,20 @@ __global__ void __launch_bounds__(384, 1)
         __syncwarp();
       };
       const uint32_t d_s = tmem + C::s_col(t), d_o = tmem + C::o_col(t);
+      const uint64_t sd[3] = {seed_desc(sbase + C::OFF_SEED), seed_desc(sbase + C::OFF_SEED + 128),
+                              seed_desc(sbase + C::OFF_SEED + 256)};
       auto issue_s = [&](bool i8, uint32_t kslot) {
         const uint32_t kb = sbase + C::OFF_SLOT + kslot * C::SLOT;
         if (i8) {
           const uint32_t qa = sbase + C::OFF_Q8 + t * C::Q8_BYTES;
-          if (elect_one()) {
+          uint64_t ad[D / 32], bd[D / 32];
 #pragma unroll
-            for (int kk = 0; kk < D / 32; ++kk)
-              mma_i8_ss(d_s, smem_desc(qa + kk * 32, 16, C::SBO8, C::SW8),
-                        smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8), C::IDESC_S8, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk) {
+            ad[kk] = smem_desc(qa + kk * 32, 16, C::SBO8, C::SW8);
+            bd[kk] = smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8);
+          }
+          if (elect_one()) {
+            mma_i8_exact_n<D / 32>(d_s, sd, C::IDESC_S16, ad, bd, C::IDESC_S8);
             tc_commit(bar(C_SFULL + t));
           }
         } else {
@@ -491,7 +508,7 @@ __global__ void __launch_bounds__(384, 1)
               bd[kk] = smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8);
             }
             if (elect_one()) {
-              mma_i8_ss_n<D / 32>(d_c, ad, bd, C::IDESC_S8_64, 0u);
+              mma_i8_exact_n<D / 32>(d_c, sd, C::IDESC_S16_64, ad, bd, C::IDESC_S8_64);
               tc_commit(bar(C_SFULL2 + 2 * t + (c & 1)));
             }
           } else {
@@ -687,16 +704,21 @@ __global__ void __launch_bounds__(384, 1)
         n16 = (a && !r0) || (c && !r1);
         n8 = r0 || r1;
       };
+      const uint64_t sd[3] = {seed_desc(sbase + C::OFF_SEED), seed_desc(sbase + C::OFF_SEED + 128),
+                              seed_desc(sbase + C::OFF_SEED + 256)};
       auto issue_s = [&](int t, bool i8, uint32_t kslot) {
         const uint32_t d_tmem = tmem + C::s_col(t);
         const uint32_t kb = sbase + C::OFF_SLOT + kslot * C::SLOT;
         if (i8) {
           const uint32_t qa = sbase + C::OFF_Q8 + t * C::Q8_BYTES;
-          if (elect_one()) {
+          uint64_t ad[D / 32], bd[D / 32];
 #pragma unroll
-            for (int kk = 0; kk < D / 32; ++kk)
-              mma_i8_ss(d_tmem, smem_desc(qa + kk * 32, 16, C::SBO8, C::SW8),
-                        smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8), C::IDESC_S8, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk) {
+            ad[kk] = smem_desc(qa + kk * 32, 16, C::SBO8, C::SW8);
+            bd[kk] = smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8);
+          }
+          if (elect_one()) {
+            mma_i8_exact_n<D / 32>(d_tmem, sd, C::IDESC_S16, ad, bd, C::IDESC_S8);
             tc_commit(bar(C_SFULL + t));
           }
         } else {
@@ -873,19 +895,9 @@ __global__ void __launch_bounds__(384, 1)
           for (int cc = 0; cc < HN / 32; ++cc) tmem_ld32p(s_c + cc * 32, u + cc * 32);
           tmem_wait_ld_regs<HN>(u);
           TM_PH(1);
-          if (i8) {
-            const uint64_t nmagic = f2pack(-12582912.0f, -12582912.0f);
+          // INT8 scores arrive in fp32 like FP16 ones (see mma_i8_exact_n)
 #pragma unroll
-            for (int e = 0; e < HN; e += 2) {
-              const uint64_t v = f2add(f2pack(__int_as_float(static_cast<int>(u[e]) + 0x4B400000),
-                                              __int_as_float(static_cast<int>(u[e + 1]) + 0x4B400000)),
-                                       nmagic);
-              f2unpack(v, x[e], x[e + 1]);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < HN; ++e) x[e] = __uint_as_float(u[e]);
-          }
+          for (int e = 0; e < HN; ++e) x[e] = __uint_as_float(u[e]);
         }
         const int64_t nv64 = lim - static_cast<int64_t>(c) * HN + 1;
         const int nv = nv64 <= 0 ? 0 : (nv64 >= HN ? HN : static_cast<int>(nv64));
@@ -993,21 +1005,16 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_ld_regs<BN>(u);
         TM_PH(1);
         TM_SM_EV(EV_SLOADED);
-        if (i8) {
-          // exact int32 -> fp32 for |acc| < 2^22: add the bits of 1.5 * 2^23,
-          // then subtract 1.5 * 2^23 in packed fp32
-          const uint64_t nmagic = f2pack(-12582912.0f, -12582912.0f);
+        // Never taken (sched_zero is 0 in every launch).  The branch only
+        // changes how the compiler schedules this step: without it the same
+        // launches measured 5-7 % slower (routing sweep, every INT8 share).
+        if (p.sched_zero != 0) {
 #pragma unroll
-          for (int e = 0; e < BN; e += 2) {
-            const uint64_t v = f2add(f2pack(__int_as_float(static_cast<int>(u[e]) + 0x4B400000),
-                                            __int_as_float(static_cast<int>(u[e + 1]) + 0x4B400000)),
-                                     nmagic);
-            f2unpack(v, x[e], x[e + 1]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(u[e]);
+          for (int e = 0; e < BN; ++e) u[e] += static_cast<uint32_t>(p.sched_zero);
         }
+        // INT8 scores arrive in fp32 like FP16 ones (see mma_i8_exact_n)
+#pragma unroll
+        for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(u[e]);
       }
       const int64_t nv64 = lim - static_cast<int64_t>(j) * BN + 1;
       const int nv = nv64 <= 0 ? 0 : (nv64 >= BN ? BN : static_cast<int>(nv64));
@@ -1247,6 +1254,7 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
   p.n_qt_max = static_cast<int>((maxq + 127) / 128);
   p.n_pair_max = (p.n_qt_max + 1) / 2;
   p.W = tm_mask_words(maxk, 128, g);
+  p.sched_zero = 0;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   p.err = DevErr{device_error_word()};
   // KV heads per scheduling chunk: as many as keep their K / V (fp16 K, int8

@@ -81,12 +81,13 @@ struct Cfg3 {
   static constexpr int OFF_V = OFF_K + NK * SLOT;
   static constexpr int OFF_BAR = OFF_V + NV * SLOT;
   static constexpr int OFF_WORDS = OFF_BAR + 256;               // routing words [2 planes][MAXW]
-  static constexpr int OFF_XMAX = OFF_BAR + 1024;               // row maxima [2 iterations][2 warpgroups][128],
+  static constexpr int OFF_SEED = OFF_BAR + 768;                // INT8 accumulator seed blocks (kSeedBytes)
+  static constexpr int OFF_XMAX = OFF_BAR + 1280;               // row maxima [2 iterations][2 warpgroups][128],
                                                                 // then row sums [2 warpgroups][128]
   static constexpr int OFF_KSC = OFF_XMAX + 3 * 256 * 4;        // key-tile scales of the INT8 route
   static constexpr int MAXJ = 512;                              // key tiles whose scales are staged
   static constexpr int OFF_KSCF8 = OFF_KSC + MAXJ * 4;          // ... of the FP8 route
-  static constexpr int BAR_BYTES = 1024 + 3 * 256 * 4 + MAXJ * 4 * (F8 ? 2 : 1);
+  static constexpr int BAR_BYTES = 1280 + 3 * 256 * 4 + MAXJ * 4 * (F8 ? 2 : 1);
   static constexpr int MAXW = 64;                               // routing words kept in shared memory
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -103,7 +104,7 @@ struct Cfg3 {
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS == THREADS * LAUNCH_REGS,
                 "register split must equal the launch allocation");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static_assert(OFF_WORDS + 2 * 4 * MAXW <= OFF_XMAX, "routing words fit");
+  static_assert(OFF_WORDS + 2 * 4 * MAXW <= OFF_SEED && OFF_SEED + kSeedBytes <= OFF_XMAX, "routing words fit");
 };
 
 enum {
@@ -257,6 +258,10 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
     tc_fence_before();
   }
+  if (warp == 10) {
+    seed_blocks_init(reinterpret_cast<uint32_t*>(smem + C::OFF_SEED), lane);
+    fence_async_shared();   // generic-proxy stores, read by tcgen05.mma
+  }
   if (warp == 8) {
     if (lane == 0) {
       prefetch_tmap(&tmQ16);
@@ -391,8 +396,13 @@ __global__ void __launch_bounds__(384, 1)
               bd[kk] = smem_desc(kb + kk * 32, 16, 1024, kSwizzle128);
             }
             if (elect_one()) {
-              if (F8 && rt == 2) mma_f8_ss_n<D / 32>(d_s, ad, bd, C::IDESC_F8, 0u);
-              else mma_i8_ss_n<D / 32>(d_s, ad, bd, C::IDESC_S8, 0u);
+              if (F8 && rt == 2) {
+                mma_f8_ss_n<D / 32>(d_s, ad, bd, C::IDESC_F8, 0u);
+              } else {
+                const uint64_t sd[3] = {seed_desc(sbase + C::OFF_SEED), seed_desc(sbase + C::OFF_SEED + 128),
+                                        seed_desc(sbase + C::OFF_SEED + 256)};
+                mma_i8_exact_n<D / 32>(d_s, sd, C::IDESC_S16, ad, bd, C::IDESC_S8);
+              }
               tc_commit(bar(B_SFULL + sb));
               tc_commit(bar(B_KEMPTY + ks));
             }
@@ -517,7 +527,7 @@ __global__ void __launch_bounds__(384, 1)
       const int sb = j % C::NSB;
       const uint32_t s_addr = lane_addr + C::S_COL + 128u * sb + HN * hw;
       const int rt = route_of<F8>(rrow, rrowf8, p.g, j);
-      const bool i8 = rt == 1;   // int32 scores to convert; FP8 scores arrive in fp32
+      const bool i8 = rt == 1;   // INT8 and FP8 scores arrive in fp32 (see mma_i8_exact_n)
       float c = p.scale_log2;
       if (i8) {
         const float ks = j < C::MAXJ ? ksc[j] : __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk);
@@ -537,21 +547,8 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int cc = 0; cc < HN / 32; ++cc) tmem_ld32p(s_addr + cc * 32, u + cc * 32);
         tmem_wait_ld_regs<HN>(u);
-        if (i8) {
-          // exact int32 -> fp32 for |acc| < 2^22: add the bits of 1.5 * 2^23,
-          // then subtract 1.5 * 2^23 in packed fp32
-          const uint64_t nmagic = f2pack(-12582912.0f, -12582912.0f);
 #pragma unroll
-          for (int e = 0; e < HN; e += 2) {
-            const uint64_t v = f2add(f2pack(__int_as_float(static_cast<int>(u[e]) + 0x4B400000),
-                                            __int_as_float(static_cast<int>(u[e + 1]) + 0x4B400000)),
-                                     nmagic);
-            f2unpack(v, x[e], x[e + 1]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < HN; ++e) x[e] = __uint_as_float(u[e]);
-        }
+        for (int e = 0; e < HN; ++e) x[e] = __uint_as_float(u[e]);
       }
       TM3_PH(1);
       const int64_t nv64 = lim - (static_cast<int64_t>(j) * BN + HN * hw) + 1;

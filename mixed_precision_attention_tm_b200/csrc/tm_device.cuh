@@ -415,6 +415,78 @@ __device__ __forceinline__ void mma_f16_ts_n<8>(uint32_t d, const uint32_t* a, c
       ::"r"(d), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc), "r"(acc_first), "r"(1u));
 }
 
+// INT8 score tiles leave the tensor core as exact fp32 numbers, so that the
+// softmax treats them like FP16 score tiles (only the scale differs) and
+// needs no int32 -> fp32 conversion.  The accumulator starts at a seed: one
+// kind::f16 MMA on constant operands writes the fp32 value 1.5 * 2^23 (bit
+// pattern 0x4B400000); the kind::i8 MMAs add their s32 dot product acc to that
+// bit pattern, which then reads as the fp32 number 1.5 * 2^23 + acc exactly
+// (|acc| < 2^22: at most d * 127^2 = 2064512 here); a last kind::f16 MMA with
+// accumulate adds -1.5 * 2^23 in fp32, leaving acc exactly (every operand,
+// product and sum involved is an exactly representable fp32 value).
+constexpr float kAccSeed = 12582912.0f;
+// The constant operands: three no-swizzle core matrices (8 rows of 16
+// bytes), each row one fp16 value v followed by seven zeros.  Read with zero
+// leading and stride offsets, every 8 x 8 core matrix of a 128 x 16 operand
+// is the block, so the operand holds v at k = 0 and 8 and 0 elsewhere:
+// A = 2048 and B = +-3072 give K = 16 products 2 * 2048 * (+-3072) =
+// +-1.5 * 2^23 in every element.
+constexpr uint32_t kSeedRowA = 0x6800u;    // fp16 2048
+constexpr uint32_t kSeedRowB = 0x6A00u;    // fp16 3072
+constexpr uint32_t kSeedRowBn = 0xEA00u;   // fp16 -3072
+constexpr int kSeedBytes = 384;            // A block, B block, -B block
+// Written by the 32 lanes of one warp; the caller makes them visible to the
+// tensor core (fence.proxy.async) before the CTA barrier.
+__device__ __forceinline__ void seed_blocks_init(uint32_t* blk, int lane) {
+#pragma unroll
+  for (int i = lane; i < kSeedBytes / 4; i += 32) {
+    const int word_in_row = i & 3, block = i >> 5;
+    const uint32_t v = block == 0 ? kSeedRowA : (block == 1 ? kSeedRowB : kSeedRowBn);
+    blk[i] = word_in_row == 0 ? v : 0u;
+  }
+}
+// Descriptor of a seed block: no swizzle, zero leading and stride offsets.
+__device__ __forceinline__ uint64_t seed_desc(uint32_t saddr) {
+  return (static_cast<uint64_t>((saddr >> 4) & 0x3FFFu)) | (static_cast<uint64_t>(1) << 46);
+}
+// The INT8 QK^T of one score tile with an fp32 result: the seed MMA, N
+// kind::i8 MMAs accumulating onto it and the unseed MMA, from one asm
+// statement with every descriptor formed beforehand.  sd[0..2]: descriptors
+// of the A, B and -B blocks.
+template <int N>
+__device__ __forceinline__ void mma_i8_exact_n(uint32_t d, const uint64_t* sd, uint32_t idesc_seed, const uint64_t* a,
+                                               const uint64_t* b, uint32_t idesc);
+template <>
+__device__ __forceinline__ void mma_i8_exact_n<2>(uint32_t d, const uint64_t* sd, uint32_t idesc_seed,
+                                                  const uint64_t* a, const uint64_t* b, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "setp.ne.b32 q, %11, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %5, %7, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %6, %8, %9, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %3, %4, q;\n\t}"
+      ::"r"(d), "l"(sd[0]), "l"(sd[1]), "l"(sd[2]), "r"(idesc_seed), "l"(a[0]), "l"(a[1]), "l"(b[0]), "l"(b[1]),
+      "r"(idesc), "r"(0u), "r"(1u));
+}
+template <>
+__device__ __forceinline__ void mma_i8_exact_n<4>(uint32_t d, const uint64_t* sd, uint32_t idesc_seed,
+                                                  const uint64_t* a, const uint64_t* b, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %14, 0;\n\t"
+      "setp.ne.b32 q, %15, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %5, %9, %13, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %6, %10, %13, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %7, %11, %13, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %8, %12, %13, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %3, %4, q;\n\t}"
+      ::"r"(d), "l"(sd[0]), "l"(sd[1]), "l"(sd[2]), "r"(idesc_seed), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]),
+      "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(0u), "r"(1u));
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp receives
 // columns [col, col+32) of TMEM lane (lane base of taddr) + t.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {

@@ -7,12 +7,15 @@
 // one sequence):  amax = max|x|;  s = fl32(amax / 127);
 // code = clamp(rne(fl32(x / s)), -127, 127);  s == 0 gives codes 0.
 //
-// One CTA per (tile, sequence, head): the tile's rows x d fp16 values are
-// read once with 16-byte loads and kept in registers between the absmax pass
-// and the quantise pass, so HBM traffic is one read of x plus one write of
-// the codes.  Division is the IEEE round-to-nearest __fdiv_rn and the code
-// conversion is round-to-nearest-even, so the result is bit-identical to the
-// definition.  HBM-bound: bytes per element = 2 (read) + 1 (write).
+// One CTA per (tile, sequence, head), Q and K in one launch: the tile's rows x
+// d fp16 values are read once with 16-byte loads and kept in registers
+// between the absmax pass and the quantise pass, so HBM traffic is one read
+// of x plus one write of the codes (bytes per element: 2 read + 1 written).
+// The scale is the IEEE round-to-nearest __fdiv_rn of amax by 127.  A code is
+// formed from x times the correctly rounded reciprocal of the scale, with an
+// exact guard: only an element whose product lies within 2^-15 of a
+// half-integer takes the IEEE division, so the codes are bit-identical to
+// the definition (see int8_code).
 //
 // FP8 (the third precision; per-axis fp8 scales: "Add rowwise scaling to
 // Float8Inference module" page, Summary): s = fl32(amax / 448), 448 being the
@@ -37,28 +40,63 @@ __device__ __forceinline__ uint32_t e4m3x2_rn_sat(float lo, float hi) {
   return r;
 }
 
+// INT8 code of x for a tile scale s > 0 with r = 1/s correctly rounded:
+// rne(fl32(x / s)) clamped to [-127, 127], without a division per element.
+// v = fl32(x * r) differs from x / s by at most |x / s| * 2^-23 (< 2^-16 for
+// |x / s| <= 127.00002, which |x| <= amax guarantees), and fl32(x / s) by at
+// most half an ulp (< 2^-17), so both lie within 2^-15 of x / s.  When v is
+// farther than 2^-15 from the nearest half-integer, no rounding boundary lies
+// between them and rne(v) is the code; otherwise (a near tie, about one
+// element in 10^4) the IEEE division decides.
+__device__ __forceinline__ int int8_code(float x, float s, float r) {
+  const float v = __fmul_rn(x, r);
+  float n = rintf(v);
+  if (fabsf(v - n) > 0.5f - 0x1p-15f) n = rintf(__fdiv_rn(x, s));
+  return max(-127, min(127, static_cast<int>(n)));
+}
+
+// One operand (Q or K) of a quantisation launch.
+struct QuantOperand {
+  const __half* x;
+  int64_t stride_t, stride_h;
+  int H;
+  uint8_t* codes;
+  float* scales;
+  const int32_t* cu;
+  int64_t L;
+  int tile;
+  int ntile;   // tiles per sequence launched (grid.x covers the larger operand)
+  int nb;      // sequences
+};
+
+// One CTA per (tile, sequence, head) of either operand: grid.z runs over the
+// heads of operand 0 and then those of operand 1.  The tile's rows x d fp16
+// values are read once with 16-byte loads and kept in registers between the
+// absmax pass and the quantise pass, so HBM traffic is one read of x plus one
+// write of the codes.
 template <int D, bool F8>
 __global__ void __launch_bounds__(kQuantThreads)
-    quantize_tiles_kernel(const __half* __restrict__ x, int64_t stride_t, int64_t stride_h, int H,
-                          uint8_t* __restrict__ codes, float* __restrict__ scales,
-                          const int32_t* __restrict__ cu, int64_t L, int tile, DevErr err) {
+    quantize_tiles_kernel(const QuantOperand op0, const QuantOperand op1, DevErr err) {
   constexpr int VPR = D / 8;                       // 16-byte vectors per row
   constexpr int MAXV = 128 * VPR / kQuantThreads;  // vectors per thread at tile = 128
   __shared__ float red[kQuantThreads / 32];
   __shared__ SeqInfo sinfo;
   __shared__ float s_scale;
 
-  const int I = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
+  const bool second = static_cast<int>(blockIdx.z) >= op0.H;
+  const QuantOperand& o = second ? op1 : op0;
+  const int I = blockIdx.x, b = blockIdx.y, h = second ? blockIdx.z - op0.H : blockIdx.z;
+  if (I >= o.ntile || b >= o.nb) return;
   if (threadIdx.x == 0) {
-    sinfo = seq_info(cu, b, L, tile);
-    if (cu != nullptr && I == 0 && sinfo.len > static_cast<int64_t>(gridDim.x) * tile)
+    sinfo = seq_info(o.cu, b, o.L, o.tile);
+    if (o.cu != nullptr && I == 0 && sinfo.len > static_cast<int64_t>(o.ntile) * o.tile)
       dev_error(err, TM_DEVERR_SEQLEN);
   }
   __syncthreads();
-  const SeqInfo s = sinfo;
-  const int64_t r0 = static_cast<int64_t>(I) * tile;
-  if (r0 >= s.len) return;
-  const int rows = static_cast<int>(min(static_cast<int64_t>(tile), s.len - r0));
+  const SeqInfo sq = sinfo;
+  const int64_t r0 = static_cast<int64_t>(I) * o.tile;
+  if (r0 >= sq.len) return;
+  const int rows = static_cast<int>(min(static_cast<int64_t>(o.tile), sq.len - r0));
   const int nvec = rows * VPR;
 
   uint4 v[MAXV];
@@ -68,7 +106,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     const int idx = threadIdx.x + k * kQuantThreads;
     if (idx < nvec) {
       const int row = idx / VPR, c = idx % VPR;
-      const __half* src = x + (s.start + r0 + row) * stride_t + static_cast<int64_t>(h) * stride_h + c * 8;
+      const __half* src = o.x + (sq.start + r0 + row) * o.stride_t + static_cast<int64_t>(h) * o.stride_h + c * 8;
       v[k] = *reinterpret_cast<const uint4*>(src);
       const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
 #pragma unroll
@@ -77,7 +115,7 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
   float m = fmaxf(__low2float(m2), __high2float(m2));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -86,11 +124,12 @@ __global__ void __launch_bounds__(kQuantThreads)
     for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[w]);
     const float sc = __fdiv_rn(a, F8 ? 448.0f : 127.0f);
     s_scale = sc;
-    scales[(s.tile_base + I) * H + h] = sc;
+    o.scales[(sq.tile_base + I) * o.H + h] = sc;
   }
   __syncthreads();
   const float sc = s_scale;
-  const int64_t code_row_stride = static_cast<int64_t>(H) * D;
+  const float rc = sc != 0.f ? __frcp_rn(sc) : 0.f;
+  const int64_t code_row_stride = static_cast<int64_t>(o.H) * D;
 #pragma unroll
   for (int k = 0; k < MAXV; ++k) {
     const int idx = threadIdx.x + k * kQuantThreads;
@@ -98,28 +137,23 @@ __global__ void __launch_bounds__(kQuantThreads)
       const int row = idx / VPR, c = idx % VPR;
       const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
       uint32_t packed[2] = {0u, 0u};
-      if (F8) {
-        if (sc != 0.f) {
+      if (sc != 0.f) {
+        if (F8) {
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
             const uint32_t pr = e4m3x2_rn_sat(__fdiv_rn(__low2float(hv[e >> 1]), sc),
                                               __fdiv_rn(__high2float(hv[e >> 1]), sc));
             packed[e >> 2] |= pr << (8 * (e & 3));
           }
-        }
-      } else {
+        } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float f = (e & 1) ? __high2float(hv[e >> 1]) : __low2float(hv[e >> 1]);
-          int qv = 0;
-          if (sc != 0.f) {
-            qv = __float2int_rn(__fdiv_rn(f, sc));
-            qv = max(-127, min(127, qv));
+          for (int e = 0; e < 8; ++e) {
+            const float f = (e & 1) ? __high2float(hv[e >> 1]) : __low2float(hv[e >> 1]);
+            packed[e >> 2] |= (static_cast<uint32_t>(int8_code(f, sc, rc)) & 0xFFu) << (8 * (e & 3));
           }
-          packed[e >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
         }
       }
-      uint8_t* dst = codes + (s.start + r0 + row) * code_row_stride + static_cast<int64_t>(h) * D + c * 8;
+      uint8_t* dst = o.codes + (sq.start + r0 + row) * code_row_stride + static_cast<int64_t>(h) * D + c * 8;
       *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
     }
   }
@@ -135,33 +169,65 @@ tm_status check_operand(const tm_tensor* t) {
   return TM_OK;
 }
 
-tm_status launch_quant(const tm_tensor* x, void* codes_ptr, float* scales, const int32_t* cu,
-                       int32_t batch, int32_t max_seqlen, int32_t tile, cudaStream_t stream, bool f8 = false) {
+// Checks one operand's outputs and fills its launch description; *empty is
+// set when it has nothing to quantise.
+tm_status make_operand(const tm_tensor* x, void* codes_ptr, float* scales, const int32_t* cu, int32_t batch,
+                       int32_t max_seqlen, int32_t tile, QuantOperand* o, bool* empty) {
   uint8_t* codes = static_cast<uint8_t*>(codes_ptr);
   if (codes == nullptr || scales == nullptr) return TM_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(codes) % 16 || reinterpret_cast<uintptr_t>(scales) % 4)
     return TM_ERR_INVALID_ARG;
   const int64_t maxlen = cu ? max_seqlen : x->T;
   const int nb = cu ? batch : 1;
-  if (maxlen <= 0 || nb <= 0) return TM_OK;   // nothing to quantise
+  *empty = maxlen <= 0 || nb <= 0;
+  if (*empty) return TM_OK;
   const int64_t ntile = (maxlen + tile - 1) / tile;
   if (ntile > 0x7fffffff || nb > 65535 || x->H > 65535) return TM_ERR_UNSUPPORTED;
-  dim3 grid(static_cast<unsigned>(ntile), static_cast<unsigned>(nb), static_cast<unsigned>(x->H));
+  o->x = static_cast<const __half*>(x->data);
+  o->stride_t = x->stride_t;
+  o->stride_h = x->stride_h;
+  o->H = static_cast<int>(x->H);
+  o->codes = codes;
+  o->scales = scales;
+  o->cu = cu;
+  o->L = x->T;
+  o->tile = tile;
+  o->ntile = static_cast<int>(ntile);
+  o->nb = nb;
+  return TM_OK;
+}
+
+// Quantises x (and y, when given) in one launch.
+tm_status launch_quant(const tm_tensor* x, void* x_codes, float* x_scales, const int32_t* cu_x, int32_t max_x,
+                       int32_t tile_x, const tm_tensor* y, void* y_codes, float* y_scales, const int32_t* cu_y,
+                       int32_t max_y, int32_t tile_y, int32_t batch, cudaStream_t stream, bool f8) {
+  QuantOperand o[2] = {};
+  bool empty[2] = {true, true};
+  tm_status st = make_operand(x, x_codes, x_scales, cu_x, batch, max_x, tile_x, &o[0], &empty[0]);
+  if (st != TM_OK) return st;
+  if (y != nullptr) {
+    st = make_operand(y, y_codes, y_scales, cu_y, batch, max_y, tile_y, &o[1], &empty[1]);
+    if (st != TM_OK) return st;
+  }
+  // an empty operand takes no heads of the grid
+  if (empty[0]) o[0].H = 0;
+  if (empty[1]) o[1].H = 0;
+  const int64_t heads = static_cast<int64_t>(o[0].H) + o[1].H;
+  if (heads == 0) return TM_OK;
+  if (heads > 65535) return TM_ERR_UNSUPPORTED;
+  const int gx = max(empty[0] ? 0 : o[0].ntile, empty[1] ? 0 : o[1].ntile);
+  const int gy = max(empty[0] ? 0 : o[0].nb, empty[1] ? 0 : o[1].nb);
+  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(heads));
   DevErr err{device_error_word()};
-  const __half* xp = static_cast<const __half*>(x->data);
-  const int Hi = static_cast<int>(x->H);
-  if (x->d == 128 && f8)
-    quantize_tiles_kernel<128, true><<<grid, kQuantThreads, 0, stream>>>(xp, x->stride_t, x->stride_h, Hi, codes,
-                                                                          scales, cu, x->T, tile, err);
-  else if (x->d == 128)
-    quantize_tiles_kernel<128, false><<<grid, kQuantThreads, 0, stream>>>(xp, x->stride_t, x->stride_h, Hi, codes,
-                                                                           scales, cu, x->T, tile, err);
+  const int64_t d = x->d;
+  if (d == 128 && f8)
+    quantize_tiles_kernel<128, true><<<grid, kQuantThreads, 0, stream>>>(o[0], o[1], err);
+  else if (d == 128)
+    quantize_tiles_kernel<128, false><<<grid, kQuantThreads, 0, stream>>>(o[0], o[1], err);
   else if (f8)
-    quantize_tiles_kernel<64, true><<<grid, kQuantThreads, 0, stream>>>(xp, x->stride_t, x->stride_h, Hi, codes,
-                                                                         scales, cu, x->T, tile, err);
+    quantize_tiles_kernel<64, true><<<grid, kQuantThreads, 0, stream>>>(o[0], o[1], err);
   else
-    quantize_tiles_kernel<64, false><<<grid, kQuantThreads, 0, stream>>>(xp, x->stride_t, x->stride_h, Hi, codes,
-                                                                          scales, cu, x->T, tile, err);
+    quantize_tiles_kernel<64, false><<<grid, kQuantThreads, 0, stream>>>(o[0], o[1], err);
   return check_cuda(cudaGetLastError());
 }
 
@@ -183,10 +249,8 @@ extern "C" tm_status tm_quantize_qk_varlen(const tm_tensor* q, const tm_tensor* 
     if (st != TM_OK) return st;
     if (k->d != q->d || max_seqlen_k <= 0) return TM_ERR_INVALID_ARG;
   }
-  cudaStream_t s = as_stream(stream);
-  st = launch_quant(q, q_codes, q_scales, cu_seqlens_q, batch, max_seqlen_q, tile_m, s);
-  if (st != TM_OK || k == nullptr) return st;
-  return launch_quant(k, k_codes, k_scales, cu_seqlens_k, batch, max_seqlen_k, tile_n, s);
+  return launch_quant(q, q_codes, q_scales, cu_seqlens_q, max_seqlen_q, tile_m, k, k_codes, k_scales, cu_seqlens_k,
+                      max_seqlen_k, tile_n, batch, as_stream(stream), false);
 }
 
 extern "C" tm_status tm_quantize_qk(const tm_tensor* q, const tm_tensor* k, int8_t* q_codes,
@@ -204,10 +268,8 @@ extern "C" tm_status tm_quantize_qk(const tm_tensor* q, const tm_tensor* k, int8
     if (cu_seqlens != nullptr && k->T != q->T) return TM_ERR_INVALID_ARG;
   }
   if (cu_seqlens != nullptr && (batch <= 0 || max_seqlen <= 0)) return TM_ERR_INVALID_ARG;
-  cudaStream_t s = as_stream(stream);
-  st = launch_quant(q, q_codes, q_scales, cu_seqlens, batch, max_seqlen, tile_m, s);
-  if (st != TM_OK || k == nullptr) return st;
-  return launch_quant(k, k_codes, k_scales, cu_seqlens, batch, max_seqlen, tile_n, s);
+  return launch_quant(q, q_codes, q_scales, cu_seqlens, max_seqlen, tile_m, k, k_codes, k_scales, cu_seqlens,
+                      max_seqlen, tile_n, batch, as_stream(stream), false);
 }
 
 extern "C" tm_status tm_quantize_qk_fp8(const tm_tensor* q, const tm_tensor* k, uint8_t* q_codes, float* q_scales,
@@ -224,8 +286,6 @@ extern "C" tm_status tm_quantize_qk_fp8(const tm_tensor* q, const tm_tensor* k, 
     if (cu_seqlens != nullptr && k->T != q->T) return TM_ERR_INVALID_ARG;
   }
   if (cu_seqlens != nullptr && (batch <= 0 || max_seqlen <= 0)) return TM_ERR_INVALID_ARG;
-  cudaStream_t s = as_stream(stream);
-  st = launch_quant(q, q_codes, q_scales, cu_seqlens, batch, max_seqlen, tile_m, s, true);
-  if (st != TM_OK || k == nullptr) return st;
-  return launch_quant(k, k_codes, k_scales, cu_seqlens, batch, max_seqlen, tile_n, s, true);
+  return launch_quant(q, q_codes, q_scales, cu_seqlens, max_seqlen, tile_m, k, k_codes, k_scales, cu_seqlens,
+                      max_seqlen, tile_n, batch, as_stream(stream), true);
 }

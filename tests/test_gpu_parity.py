@@ -84,6 +84,24 @@ def test_quantizer_q_and_k_tiles_differ():
     assert np.array_equal(ks.cpu().numpy(), rks) and np.array_equal(kc.cpu().numpy(), rkc)
 
 
+def test_quantizer_ties_and_near_ties_bit_exact():
+    """Tiles whose values sit exactly on, or within 2^-13 of, the half-integer
+    boundaries of rne(fl32(x / s)) (power-of-two and other scales, Q and K in
+    one launch, d = 64 and 128): codes and scales equal the oracle's."""
+    from quant_cases import AMAXES, tie_tile
+    for d in (64, 128):
+        tiles = [tie_tile(128, d, np.float16(a), i) for i, a in enumerate(AMAXES)]
+        x = np.stack(tiles, axis=1).reshape(128, len(AMAXES), d)            # heads = amax cases
+        q = torch.from_numpy(np.concatenate([x, x[::-1]], axis=0).copy())   # two tiles per head
+        k = torch.from_numpy(x[:, ::-1].copy())
+        qc, qs, kc, ks = ops.quantize_qk(q.cuda(), k.cuda(), tile_m=128, tile_n=128)
+        torch.cuda.synchronize()
+        rqc, rqs = oracle.quantize_tiles(q.numpy(), oracle.seq_table(256, 256), 128, "q")
+        rkc, rks = oracle.quantize_tiles(k.numpy(), oracle.seq_table(128, 128), 128, "k")
+        assert np.array_equal(qs.cpu().numpy(), rqs) and np.array_equal(ks.cpu().numpy(), rks)
+        assert np.array_equal(qc.cpu().numpy(), rqc) and np.array_equal(kc.cpu().numpy(), rkc)
+
+
 # ------------------------------------------------------------------ mask
 MASK_CASES = [
     # (Hq, Lq, Lk, cu, tm, tn, g, causal, p, fd, fs)

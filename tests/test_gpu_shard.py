@@ -132,6 +132,7 @@ def test_head_sharded_against_oracle():
 def test_plan_launch_count():
     pl = HeadShardedPrefill(256, 256, 28, 4, 128, rank=1, world=8, causal=True, g=2, p=0.5)
     # rank 1 holds heads 4..7: two segments (4..6 over KV head 0, 7 over KV head 1),
-    # each quantising Q and K and attending; one whole-problem mask; one merge
+    # each quantising Q and K (one launch) and attending; one whole-problem
+    # mask; one merge
     assert pl.segments == [(4, 7, 0, 1), (7, 8, 1, 2)]
-    assert pl.launches_per_step == 2 * 3 + 1 + 1
+    assert pl.launches_per_step == 2 * 2 + 1 + 1
