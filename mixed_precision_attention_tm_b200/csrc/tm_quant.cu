@@ -55,43 +55,6 @@ __device__ __forceinline__ int int8_code(float x, float s, float r) {
   return max(-127, min(127, static_cast<int>(n)));
 }
 
-// The eight INT8 codes of one 16-byte vector of fp16 values, packed into two
-// words, by the rule of int8_code without conversion instructions: for
-// |v| < 2^22, t = fl32(v + 1.5 * 2^23) rounds v to the nearest integer, ties
-// to even (the float spacing there is 1), t - 1.5 * 2^23 is that integer
-// exactly, and the bits of t minus 0x4B400000 are it as an int32.  |v| is at
-// most 127.00002 (|x| <= amax), so the integer is in [-127, 127] and needs no
-// clamp.  If any of the eight products lies within 2^-15 of a half-integer,
-// all eight take int8_code (a vote per warp).
-__device__ __forceinline__ uint2 int8_codes8(const __half2* hv, float s, float r) {
-  const uint64_t r2 = f2pack(r, r);
-  const uint64_t m2 = f2pack(12582912.0f, 12582912.0f), nm2 = f2pack(-12582912.0f, -12582912.0f);
-  const float lim = 0.5f - 0x1p-15f;
-  int c[8];
-  bool near = false;
-#pragma unroll
-  for (int e = 0; e < 8; e += 2) {
-    const float2 f = __half22float2(hv[e >> 1]);
-    const uint64_t v2 = f2mul(f2pack(f.x, f.y), r2);
-    const uint64_t t2 = f2add(v2, m2);
-    const uint64_t d2 = f2add(v2, f2add(t2, nm2));   // v - rne(v), exact
-    float t0, t1, d0, d1;
-    f2unpack(t2, t0, t1);
-    f2unpack(d2, d0, d1);
-    near |= fabsf(d0) > lim || fabsf(d1) > lim;
-    c[e] = __float_as_int(t0) - 0x4B400000;
-    c[e + 1] = __float_as_int(t1) - 0x4B400000;
-  }
-  if (__any_sync(__activemask(), near)) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      c[e] = int8_code((e & 1) ? __high2float(hv[e >> 1]) : __low2float(hv[e >> 1]), s, r);
-  }
-  const uint32_t w0 = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
-  const uint32_t w1 = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410);
-  return make_uint2(w0, w1);
-}
-
 // One operand (Q or K) of a quantisation launch.
 struct QuantOperand {
   const __half* x;
@@ -112,7 +75,7 @@ struct QuantOperand {
 // absmax pass and the quantise pass, so HBM traffic is one read of x plus one
 // write of the codes.
 template <int D, bool F8>
-__global__ void __launch_bounds__(kQuantThreads, 3)
+__global__ void __launch_bounds__(kQuantThreads)
     quantize_tiles_kernel(const QuantOperand op0, const QuantOperand op1, DevErr err) {
   constexpr int VPR = D / 8;                       // 16-byte vectors per row
   constexpr int MAXV = 128 * VPR / kQuantThreads;  // vectors per thread at tile = 128
@@ -183,9 +146,11 @@ __global__ void __launch_bounds__(kQuantThreads, 3)
             packed[e >> 2] |= pr << (8 * (e & 3));
           }
         } else {
-          const uint2 w = int8_codes8(hv, sc, rc);
-          packed[0] = w.x;
-          packed[1] = w.y;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float f = (e & 1) ? __high2float(hv[e >> 1]) : __low2float(hv[e >> 1]);
+            packed[e >> 2] |= (static_cast<uint32_t>(int8_code(f, sc, rc)) & 0xFFu) << (8 * (e & 3));
+          }
         }
       }
       uint8_t* dst = o.codes + (sq.start + r0 + row) * code_row_stride + static_cast<int64_t>(h) * D + c * 8;

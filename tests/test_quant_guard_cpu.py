@@ -2,7 +2,7 @@
 one IEEE division per element (tm_quant.cu, int8_code): with r the correctly
 rounded reciprocal of the tile scale s, code = rne(fl32(x * r)) unless that
 product lies within 2^-15 of a half-integer, where fl32(x / s) decides.  The
-rule (with the kernel's magic-number rounding) is emulated here in numpy float32 and compared, over every fp16 value of
+rule is emulated here in numpy float32 and compared, over every fp16 value of
 a tile's range and over constructed near-ties, with the oracle's codes (one
 IEEE fp32 division per element).  GPU parity tests compare the kernel itself."""
 
@@ -14,23 +14,18 @@ from quant_cases import AMAXES, all_f16_up_to, near_tie_values
 
 
 def _guarded_codes(x16, s):
-    """The kernel's rule: v = fl32(x * r); t = fl32(v + 1.5 * 2^23) (round to
-    nearest even for |v| < 2^22); code = bits(t) - 0x4B400000; when
-    |v - (t - 1.5 * 2^23)| > 1/2 - 2^-15 the IEEE quotient decides."""
+    """The kernel's rule: v = fl32(x * r); code = rne(v) unless
+    |v - rne(v)| > 1/2 - 2^-15, where the IEEE quotient fl32(x / s) decides."""
     x = x16.astype(np.float32)
     s = np.float32(s)
     r = np.float32(np.float64(1.0) / np.float64(s))       # RN(1/s): exact 1/s rounded once
     v = (x * r).astype(np.float32)
-    magic = np.float32(1.5 * 2.0 ** 23)
-    t = (v + magic).astype(np.float32)
-    n = (t - magic).astype(np.float32)
-    code = t.view(np.int32) - np.int32(0x4B400000)
-    assert np.array_equal(code, n.astype(np.int32))       # the bits of t are the integer
+    n = np.rint(v)
     near = np.abs((v - n).astype(np.float32)) > np.float32(0.5 - 2.0 ** -15)
     exact = np.rint((x.astype(np.float64) / np.float64(s)).astype(np.float32))   # fl32(x / s)
-    code = np.where(near, np.clip(exact, -127, 127).astype(np.int32), code)
-    assert code.min() >= -127 and code.max() <= 127           # no clamp needed off the fallback
-    return code.astype(np.int8), int(near.sum())
+    n = np.where(near, exact, n)
+    assert np.abs(n).max() <= 127                              # no clamp needed off the fallback
+    return np.clip(n, -127, 127).astype(np.int8), int(near.sum())
 
 
 @pytest.mark.parametrize("amax", AMAXES)
