@@ -604,6 +604,12 @@ tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor*
     if (k->T != v->T || k->H != v->H || k->d != D || v->d != D || k->T < 0) return TM_ERR_INVALID_ARG;
     if (shared && k->T != q->T) return TM_ERR_INVALID_ARG;
     if (D != 128 || tile_n != 128) return TM_ERR_UNSUPPORTED;
+    // 128-row query tiles: two per CTA, unless that leaves SMs idle or the
+    // one-tile kernel is chosen (tm_set_attn_kernel)
+    const int64_t n_qt = ((cu_seqlens ? max_seqlen : q->T) + 127) / 128;
+    if (tile_m == 128 && !use_one_tile_kernel(n_qt, cu_seqlens ? batch : 1, q->H, true, causal != 0))
+      return launch_attn_pair_cache(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask,
+                                    mask_head_stride, g, causal, as_stream(stream));
     return launch_attn_cache(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
                              tile_m, g, causal, as_stream(stream));
   }

@@ -46,12 +46,14 @@
 #include "tm_device.cuh"
 #include "tm_host.h"
 
-#ifdef TM_TRACE
+#if defined(TM_TRACE) || defined(TM_TIMEOUT_INFO)
 extern "C" int tm_debug_timeout_read(unsigned int* host) {
   if (cudaMemcpyFromSymbol(host, tmk::g_tm_timeout_info, sizeof(tmk::g_tm_timeout_info)) != cudaSuccess) return -1;
   static const unsigned int zero[5] = {0, 0, 0, 0, 0};
   return cudaMemcpyToSymbol(tmk::g_tm_timeout_info, zero, sizeof(zero)) == cudaSuccess ? 0 : -1;
 }
+#endif
+#ifdef TM_TRACE
 extern "C" int tm_debug_trace_read(unsigned long long* host, unsigned int block) {
   if (host == nullptr) {
     static unsigned long long zero[TM_TRACE_ROLES][TM_TRACE_EVENTS];
@@ -88,7 +90,12 @@ enum : unsigned {
   EV_HW_P_END = 43
 };
 
-template <int D>
+// CACHE: K / V come from an INT8 cache (codes + fp16 scale per token and KV
+// head): a dequantisation warpgroup (warps 12-15) writes the fp16 K tiles of
+// FP16-routed key tiles and every fp16 V tile into the ring, the producer
+// brings the int8 K code tiles of INT8-routed ones, and the softmax applies
+// the per-token key scales of INT8 tiles per column.
+template <int D, bool CACHE = false>
 struct Cfg2 {
   static constexpr int BM = 128, BN = 128;
   static constexpr int SLOT = BN * D * 2;                // one fp16 K or V tile
@@ -101,10 +108,16 @@ struct Cfg2 {
   static constexpr int OFF_SLOT = OFF_Q8 + 2 * Q8_BYTES;
   static constexpr int OFF_BAR = OFF_SLOT + NSLOT * SLOT;
   static constexpr int BAR_BYTES = 2048;                 // barriers, routing words, seed blocks, key-tile scales
-  static constexpr int OFF_SEED = OFF_BAR + 768;         // the INT8 accumulator seed blocks (kSeedBytes)
+  // Without CACHE: routing words [2][64] at +256, seed blocks at +768,
+  // INT8 key-tile scales at +1152.  With CACHE: routing words [2][32] at
+  // +256, the extra barriers at +512, seed blocks at +640, two stages of
+  // per-token key scales (128 fp32 each) at +1024.
+  static constexpr int OFF_SEED = OFF_BAR + (CACHE ? 640 : 768);   // the INT8 accumulator seed blocks (kSeedBytes)
   static constexpr int OFF_KSC = OFF_BAR + 1152;
-  static constexpr int KSC_MAX = 224;                    // key tiles whose INT8 scales are staged
-  static constexpr int MAXW = 64;                        // routing words per query tile kept in smem
+  static constexpr int KSC_MAX = CACHE ? 0 : 224;        // key tiles whose INT8 scales are staged
+  static constexpr int OFF_CBAR = OFF_BAR + 512;         // CACHE: key-scale stage barriers
+  static constexpr int OFF_KST = OFF_BAR + 1024;         // CACHE: key-scale stages [2][128] fp32
+  static constexpr int MAXW = CACHE ? 32 : 64;           // routing words per query tile kept in smem
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S16 = idesc_f16(BM, BN, false);
@@ -114,15 +127,22 @@ struct Cfg2 {
   static constexpr uint32_t IDESC_PV = idesc_f16(BM, D, true);
   static constexpr uint32_t SW8 = (D == 128) ? kSwizzle128 : kSwizzle64;
   static constexpr uint32_t SBO8 = (D == 128) ? 1024u : 512u;
-  // 8 softmax warps + (producer, MMA issuer, 2 idle) warps.  Launch: 168
-  // registers per thread (3 warps per SM sub-partition); the softmax
-  // warpgroups then take 216 and the control warpgroup keeps 72:
-  // 2 * 128 * 216 + 128 * 72 = 384 * 168.
-  static constexpr int THREADS = 384;
-  static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, CONTROL_REGS = 72;
+  // 8 softmax warps + (producer, MMA issuers, wait helper) warps, and with
+  // CACHE the 4 dequantisation warps.  Launch: 168 registers per thread (3
+  // warps per SM sub-partition); the softmax warpgroups then take 216 and the
+  // control warpgroup keeps 72: 2 * 128 * 216 + 128 * 72 = 384 * 168.  With
+  // CACHE: 128 at launch (4 warps per sub-partition), softmax 208, control
+  // 48, dequantisation 48: 2 * 128 * 208 + 128 * 48 + 128 * 48 = 512 * 128.
+  static constexpr int THREADS = CACHE ? 512 : 384;
+  static constexpr int LAUNCH_REGS = CACHE ? 128 : 168, SOFTMAX_REGS = CACHE ? 208 : 216;
+  static constexpr int CONTROL_REGS = CACHE ? 48 : 72, DEQ_REGS = CACHE ? 48 : 0;
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static_assert(OFF_SEED + kSeedBytes <= OFF_KSC && OFF_KSC + 4 * KSC_MAX <= OFF_BAR + BAR_BYTES, "layout");
-  static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS == THREADS * LAUNCH_REGS,
+  static_assert(CACHE ? (OFF_BAR + 256 + 4 * 2 * MAXW <= OFF_CBAR && OFF_CBAR + 8 * 10 <= OFF_SEED &&
+                         OFF_SEED + kSeedBytes <= OFF_KST &&
+                         OFF_KST + 2 * 128 * 4 <= OFF_BAR + BAR_BYTES)
+                      : (OFF_SEED + kSeedBytes <= OFF_KSC && OFF_KSC + 4 * KSC_MAX <= OFF_BAR + BAR_BYTES),
+                "layout");
+  static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS + 128 * DEQ_REGS == THREADS * LAUNCH_REGS,
                 "register split must equal the launch allocation");
   __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
   __host__ __device__ static constexpr uint32_t o_col(int t) { return 256u + D * t; }
@@ -143,7 +163,12 @@ enum {
 //   NB_P + t:  softmax warpgroup t (128, arrive) -> issuer t (32, sync): P_t stored
 //   NB_KV + t: wait helper (32) <-> issuer t (32): operands landed
 //   NB_START: softmax A (128, arrive) -> issuer B (32, sync), once: P_A(0) stored
-enum : int { NB_P = 1, NB_KV = 3, NB_START = 5 };
+//   NB_DEQ:    the four dequantisation warps (128, CACHE): a tile is written
+enum : int { NB_P = 1, NB_KV = 3, NB_START = 5, NB_DEQ = 6 };
+// CACHE barriers (at OFF_CBAR): key-scale stage s written (count 128), and
+// read by query tile t (count 4: one arrival per softmax warp); the code
+// tile of a ring slot's next fp16 tile landed (count 1, TMA bytes).
+enum { CB_KSFULL = 0, CB_KSEMPTY = 2, CB_CFULL = 6, CB_COUNT = 10 };
 
 struct Params2 {
   __half* out;
@@ -162,6 +187,9 @@ struct Params2 {
   float scale_log2;
   DevErr err;
   int sched_zero;        // always 0 (see its use in the softmax)
+  // CACHE: fp16 scales [T, Hkv] of the K and V cache (the codes come by TMA)
+  const __half* k_tok_scale;
+  const __half* v_tok_scale;
 };
 
 // Routing bit of key tile j (group j / g); row is a shared- or global-memory
@@ -180,12 +208,56 @@ struct TileInfo {
   const uint32_t* mrow;
 };
 
-template <int D, int EMU, bool DUAL, bool CH>
-__global__ void __launch_bounds__(384, 1)
+// Row r of an fp16 K or V tile of the INT8 cache, converted in place: the
+// slot's upper half holds the int8 code tile as the TMA wrote it (128-byte
+// rows, 16-byte chunk c of row r at chunk c ^ (r & 7)); the fp16 tile takes
+// the whole slot in the layout the TMA writes for fp16 tiles (two 64-column
+// slabs of 128-byte rows, the same chunk swizzle).  Each value is
+// fp16_rn(code * scale).  Row r's output in the upper slab covers exactly
+// row r's codes, which this thread has read by then, and no other thread
+// reads them, so the conversion is race-free in place.  Codes become fp16
+// without integer-to-float conversions: XOR 0x80 turns a code x into the
+// byte x + 128, which placed under the fp16 exponent byte 0x64 reads as
+// 1024 + x + 128 exactly (ulp 1); subtracting 1152 gives x exactly, and one
+// fp16 multiply by the fp16 scale rounds the exact product once.
+__device__ __forceinline__ void dequant_row_inplace(uint8_t* slot, int r, __half scale, int half_bytes) {
+  const int sw = r & 7;
+  const __half2 bias = __float2half2_rn(1152.0f);
+  const __half2 s2 = __half2half2(scale);
+  const uint8_t* codes = slot + half_bytes + r * 128;
+  // A rolled loop over the row's eight 16-byte code chunks (small code: this
+  // role shares the SM's instruction cache with the softmax and control
+  // roles).  Chunk c goes to slab c / 4, chunks 2 (c % 4) and 2 (c % 4) + 1;
+  // in slab 1 these overlay code chunks 2 (c - 4) and 2 (c - 4) + 1, which
+  // are chunk c itself or ones read in earlier iterations.
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {
+    const uint4 rw = *reinterpret_cast<const uint4*>(codes + ((c ^ sw) << 4));
+    const uint32_t w[4] = {rw.x ^ 0x80808080u, rw.y ^ 0x80808080u, rw.z ^ 0x80808080u, rw.w ^ 0x80808080u};
+    uint32_t hq[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t lo = __byte_perm(w[q], 0x64646464u, 0x4140u);   // bytes b0, 0x64, b1, 0x64
+      uint32_t hi = __byte_perm(w[q], 0x64646464u, 0x4342u);   // bytes b2, 0x64, b3, 0x64
+      __half2 vlo = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&lo), bias), s2);
+      __half2 vhi = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&hi), bias), s2);
+      hq[2 * q] = *reinterpret_cast<uint32_t*>(&vlo);
+      hq[2 * q + 1] = *reinterpret_cast<uint32_t*>(&vhi);
+    }
+    uint8_t* row = slot + (c >> 2) * half_bytes + r * 128;
+    const int c0 = 2 * (c & 3);
+    *reinterpret_cast<uint4*>(row + ((c0 ^ sw) << 4)) = make_uint4(hq[0], hq[1], hq[2], hq[3]);
+    *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ sw) << 4)) = make_uint4(hq[4], hq[5], hq[6], hq[7]);
+  }
+}
+
+template <int D, int EMU, bool DUAL, bool CH, bool CACHE>
+__global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmQ8,
                      const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmK8,
                      const __grid_constant__ CUtensorMap tmV16, const Params2 p) {
-  using C = Cfg2<D>;
+  using C = Cfg2<D, CACHE>;
+  static_assert(!CACHE || (DUAL && !CH && D == 128), "the INT8 cache runs in the two-issuer mode, d = 128");
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -198,6 +270,8 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * C_COUNT + 4);
   uint32_t* route_words = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 256);   // [2][MAXW]
   float* ksc = reinterpret_cast<float*>(smem + C::OFF_KSC);                        // [KSC_MAX]
+  auto cbar = [&](int i) -> uint32_t { return sbase + C::OFF_CBAR + 8u * static_cast<uint32_t>(i); };
+  float* kst = reinterpret_cast<float*>(smem + C::OFF_KST);                        // CACHE: [2][128]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -274,6 +348,14 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(C_FULL + s), 1);
       mbar_init(bar(C_EMPTY + s), DUAL ? 2 : 1);
     }
+    if (CACHE) {
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(cbar(CB_KSFULL + s), 128);
+        mbar_init(cbar(CB_KSEMPTY + 2 * s), 4);
+        mbar_init(cbar(CB_KSEMPTY + 2 * s + 1), 4);
+      }
+      for (int s = 0; s < C::NSLOT; ++s) mbar_init(cbar(CB_CFULL + s), 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -298,7 +380,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int w = lane; w < p.W; w += 32) route_words[t * C::MAXW + w] = __ldg(ti[t].mrow + w);
     // the INT8 route's key-tile scales (shared by both query tiles), so that
     // no softmax step waits on a global load for them
-    if (ti[0].mrow != nullptr || ti[1].mrow != nullptr) {
+    if (!CACHE && (ti[0].mrow != nullptr || ti[1].mrow != nullptr)) {
       const int nst = nJ < C::KSC_MAX ? nJ : C::KSC_MAX;
       for (int j = lane; j < nst; j += 32) ksc[j] = __ldg(p.k_scales + (skq.tile_base + j) * p.Hkv + hk);
     }
@@ -316,7 +398,63 @@ __global__ void __launch_bounds__(384, 1)
     n8 = r0 || r1;
   };
 
-  if (warp >= 8) {
+  if (CACHE && warp >= 12) {
+    // ======================= dequantisation (CACHE; one key row per thread) ====
+    // Walks the ring positions of every key tile in the producer's order
+    // ([fp16 K], [int8 K codes], fp16 V): writes the fp16 K tile of a key
+    // tile that either query tile routes FP16, and every fp16 V tile, from
+    // the cache's codes and per-token scales; the int8 K tiles are the
+    // producer's.  Also stages the key tile's per-token K scales for the
+    // softmax of INT8 tiles (two stages).  A wait that times out only
+    // records the failure: the warps still write and signal every tile, so
+    // nothing waits on them forever.
+    regs_dec<C::DEQ_REGS>();
+    const int r = threadIdx.x - 384;   // key row within the tile
+    if (nJ > 0) {
+      uint32_t n = 0;
+      uint32_t cpar = 0;   // bit s: parity of slot s's next code-barrier phase
+      // this row's K and V token scales, loaded one key tile ahead
+      auto scales_of = [&](int jj, __half& k_s, __half& v_s) {
+        const int64_t kr = static_cast<int64_t>(jj) * BN + r;   // key row within the sequence
+        const bool in = jj < nJ && kr < Lk;
+        const int64_t tok = kstart + kr;
+        k_s = in ? p.k_tok_scale[tok * p.Hkv + hk] : __float2half(0.f);
+        v_s = in ? p.v_tok_scale[tok * p.Hkv + hk] : __float2half(0.f);
+      };
+      __half ksh_next, vsh_next;
+      scales_of(0, ksh_next, vsh_next);
+      for (int j = 0; j < nJ; ++j) {
+        bool r0, r1, n16, n8;
+        needs(j, r0, r1, n16, n8);
+        const __half ksh = ksh_next, vsh = vsh_next;
+        scales_of(j + 1, ksh_next, vsh_next);
+        const int s = j & 1;
+        if (j >= 2) {   // stage s was key tile j - 2's: both tiles have read it
+          if (j - 2 < nJA) mbar_wait_warp(cbar(CB_KSEMPTY + 2 * s), ((j - 2) >> 1) & 1, p.err, abort_flag);
+          if (j - 2 < nJB) mbar_wait_warp(cbar(CB_KSEMPTY + 2 * s + 1), ((j - 2) >> 1) & 1, p.err, abort_flag);
+        }
+        kst[s * 128 + r] = __half2float(ksh);
+        mbar_arrive(cbar(CB_KSFULL + s));
+        // An fp16 tile: wait for its code tile, convert it in place (rows
+        // past the key sequence get scale 0, so they read as zeros), then
+        // hand the slot to the MMA side.  The slot itself was acquired by
+        // the producer (its release barrier), which the code barrier orders.
+        auto convert = [&](__half scale) {
+          const uint32_t slot = n % C::NSLOT;
+          ++n;
+          mbar_wait_warp(cbar(CB_CFULL + slot), (cpar >> slot) & 1u, p.err, abort_flag);
+          cpar ^= 1u << slot;
+          dequant_row_inplace(smem + C::OFF_SLOT + slot * C::SLOT, r, scale, C::HALF);
+          fence_async_shared();   // generic-proxy stores, read by tcgen05.mma
+          named_bar_sync(NB_DEQ, 128);
+          if (r == 0) mbar_arrive(bar(C_FULL + slot));
+        };
+        if (n16) convert(ksh);
+        if (n8) ++n;   // the producer's int8 K tile
+        convert(vsh);
+      }
+    }
+  } else if (warp >= 8) {
    regs_dec<C::CONTROL_REGS>();
    if (warp == 8) {
     // ======================= TMA producer =======================
@@ -366,6 +504,30 @@ __global__ void __launch_bounds__(384, 1)
         needs(j, r0, r1, n16, n8);
         const int32_t krow = static_cast<int32_t>(kstart + static_cast<int64_t>(j) * BN);
         uint32_t s;
+        if (CACHE) {
+          // Ring positions of this key tile: [fp16 K], [int8 K codes], fp16 V.
+          // For an fp16 tile the producer brings the int8 code tile into the
+          // upper half of the slot (signalled on the slot's code barrier);
+          // the dequantisation warps turn it into the fp16 tile in place and
+          // signal the slot's full barrier.  An int8 K tile lands at the
+          // slot's start as usual.  (tmV16 holds the V codes' map here.)
+          if (n16) {
+            if (!(ok = acquire(s))) break;
+            mbar_arrive_expect_tx(cbar(CB_CFULL + s), BN * D);
+            tma_load_3d_hint(sbase + C::OFF_SLOT + s * C::SLOT + C::SLOT / 2, &tmK8, cbar(CB_CFULL + s), 0, hk,
+                             krow, pol_kv);
+          }
+          if (n8) {
+            if (!(ok = acquire(s))) break;
+            mbar_arrive_expect_tx(bar(C_FULL + s), BN * D);
+            tma_load_3d_hint(sbase + C::OFF_SLOT + s * C::SLOT, &tmK8, bar(C_FULL + s), 0, hk, krow, pol_kv);
+          }
+          if (!(ok = acquire(s))) break;
+          mbar_arrive_expect_tx(cbar(CB_CFULL + s), BN * D);
+          tma_load_3d_hint(sbase + C::OFF_SLOT + s * C::SLOT + C::SLOT / 2, &tmV16, cbar(CB_CFULL + s), 0, hk, krow,
+                           pol_kv);
+          continue;
+        }
         if (n16) {
           if (!(ok = acquire(s))) break;
           mbar_arrive_expect_tx(bar(C_FULL + s), C::SLOT);
@@ -584,6 +746,7 @@ __global__ void __launch_bounds__(384, 1)
           if (n8) take(s8);
           take(sv);
           kv_handoff();   // K tiles of j (and V of j-1) landed
+          if (CACHE) tc_fence_after();   // tiles the dequantisation warps wrote
           // P.V of the previous key tile first (S_t(j) overwrites P_t(j-1))
           if (j > 0) issue_pv(j - 1, v_prev);
           if (tracer) TM_TRACE_EV(3, EV_K_READY);
@@ -600,6 +763,7 @@ __global__ void __launch_bounds__(384, 1)
           v_prev = sv;
         }
         kv_handoff();   // V of the last key tile landed
+        if (CACHE) tc_fence_after();
         issue_pv(nJt - 1, v_prev);
       }
       if (elect_one()) tc_commit(bar(C_DRAIN + t));
@@ -987,8 +1151,12 @@ __global__ void __launch_bounds__(384, 1)
       const bool i8 = route8(rrow[t], p.g, j);
       float c = p.scale_log2;
       if (i8) {
-        const float ks = j < C::KSC_MAX ? ksc[j] : __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk);
-        c = fmaxf(c8_row * ks, 1e-30f);
+        if (CACHE) {
+          c = fmaxf(c8_row, 1e-30f);   // the per-token key scales multiply the scores per column below
+        } else {
+          const float ks = j < C::KSC_MAX ? ksc[j] : __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk);
+          c = fmaxf(c8_row * ks, 1e-30f);
+        }
       }
       // No early exit: the issuer expects one P handoff per key tile, so a
       // failed wait only marks the launch failed and the loop runs on.
@@ -1015,6 +1183,29 @@ __global__ void __launch_bounds__(384, 1)
         // INT8 scores arrive in fp32 like FP16 ones (see mma_i8_exact_n)
 #pragma unroll
         for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(u[e]);
+      }
+      if constexpr (CACHE) {
+        // INT8 cache: the score of key column e is acc * s_k[e] * s_q * sigma;
+        // s_k of this key tile's tokens is staged in stage j & 1
+        const int ks_stage = j & 1;
+        // Every key tile waits for its stage, FP16 ones too: a warp must not
+        // release stage j & 1 for key tile j before the dequantisation warps
+        // have written it, or that barrier would run two phases ahead of
+        // their wait for key tile j - 2.
+        if (!mbar_wait(cbar(CB_KSFULL + ks_stage), (j >> 1) & 1, p.err, abort_flag)) ok = false;
+        if (i8) {
+          const float2* ks2 = reinterpret_cast<const float2*>(kst + ks_stage * 128);
+#pragma unroll
+          for (int e = 0; e < BN; e += 2) {
+            const float2 kk = ks2[e >> 1];
+            f2unpack(f2mul(f2pack(x[e], x[e + 1]), f2pack(kk.x, kk.y)), x[e], x[e + 1]);
+            // eight scale pairs in flight at most (keeps them out of the
+            // registers the scores need)
+            if ((e & 15) == 14) asm volatile("" ::: "memory");
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(cbar(CB_KSEMPTY + 2 * ks_stage + t));   // this warp is done with the stage
       }
       const int64_t nv64 = lim - static_cast<int64_t>(j) * BN + 1;
       const int nv = nv64 <= 0 ? 0 : (nv64 >= BN ? BN : static_cast<int>(nv64));
@@ -1161,13 +1352,13 @@ std::mutex g_mu2;
 // One-time kernel attributes; the warpgroup register split assumes exactly
 // LAUNCH_REGS per thread at launch (any other allocation could leave
 // setmaxnreg.inc waiting), so a build that differs is refused.
-template <int D, bool DUAL, bool CH>
+template <int D, bool DUAL, bool CH, bool CACHE = false>
 tm_status prepare_pair_kernel() {
-  using C = Cfg2<D>;
+  using C = Cfg2<D, CACHE>;
   static bool attr_done = false;
   std::lock_guard<std::mutex> lk(g_mu2);
   if (attr_done) return TM_OK;
-  auto kern = attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, DUAL, CH>;
+  auto kern = attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, DUAL, CH, CACHE>;
   cudaFuncAttributes fa;
   tm_status st = check_cuda(cudaFuncGetAttributes(&fa, kern));
   if (st != TM_OK) return st;
@@ -1231,7 +1422,7 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
     mQ8 = mQ16;
     mK8 = mK16;
   }
-  Params2 p;
+  Params2 p = {};
   p.out = static_cast<__half*>(out->data);
   p.out_st = out->stride_t;
   p.out_sh = out->stride_h;
@@ -1272,18 +1463,100 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
   if (grid == 0) return TM_OK;
   if (grid > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
   if (chunked)
-    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, true>
+    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, true, false>
         <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   else if (dual)
-    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, false>
+    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, false, false>
         <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   else
-    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, false, false>
+    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, false, false, false>
         <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   return check_cuda(cudaGetLastError());
 }
 
+// The INT8 K / V cache on the two-query-tile kernel (d = 128, 128-row query
+// tiles, 128-key tiles): k and v carry codes [T, Hkv, 128] and fp16 scales
+// [T, Hkv]; the routing bitmask and Q's INT8 codes and tile scales as for
+// launch_pair.
+tm_status launch_pair_cache(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                            const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
+                            const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
+                            cudaStream_t stream) {
+  constexpr int D = 128;
+  using C = Cfg2<D, true>;
+  tm_status st = prepare_pair_kernel<D, true, false, true>();
+  if (st != TM_OK) return st;
+  CUtensorMap mQ16, mQ8, mK8, mV8;
+  Params2 p = {};
+  st = encode_thd_map(&mQ16, q->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q->T, q->H, D, q->stride_t, q->stride_h,
+                      64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TM_OK) return st;
+  st = encode_thd_map(&mK8, k->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k->T, k->H, D, k->H * D, D, D, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TM_OK) return st;
+  st = encode_thd_map(&mV8, v->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, v->T, v->H, D, v->H * D, D, D, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TM_OK) return st;
+  if (bitmask != nullptr) {
+    st = encode_thd_map(&mQ8, q->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q->T, q->H, D, q->H * D, D, D, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TM_OK) return st;
+  } else {
+    mQ8 = mQ16;
+  }
+  p.out = static_cast<__half*>(out->data);
+  p.out_st = out->stride_t;
+  p.out_sh = out->stride_h;
+  p.q_scales = static_cast<const float*>(q->scales);
+  p.k_scales = nullptr;
+  p.bitmask = bitmask;
+  p.mask_hs = mask_hs;
+  p.cu = cu;
+  p.cu_k = cu ? (cu_k ? cu_k : cu) : nullptr;
+  p.Lq = q->T;
+  p.Lk = k->T;
+  p.Hq = static_cast<int>(q->H);
+  p.Hkv = static_cast<int>(k->H);
+  p.g = g;
+  p.causal = causal ? 1 : 0;
+  p.batch = cu ? batch : 1;
+  const int64_t maxq = cu ? max_q : q->T;
+  const int64_t maxk = cu ? max_k : k->T;
+  p.max_lk = maxk;
+  p.n_qt_max = static_cast<int>((maxq + 127) / 128);
+  p.n_pair_max = (p.n_qt_max + 1) / 2;
+  p.W = tm_mask_words(maxk, 128, g);
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
+  p.err = DevErr{device_error_word()};
+  p.sched_zero = 0;
+  p.k_tok_scale = static_cast<const __half*>(k->scales);
+  p.v_tok_scale = static_cast<const __half*>(v->scales);
+  // KV heads per scheduling chunk, as in launch_pair, from the cache's bytes
+  // per key row (codes of K and V)
+  {
+    const double kv_bytes = static_cast<double>(maxk) * D * 2;
+    int c = static_cast<int>(40.0e6 / (kv_bytes > 1.0 ? kv_bytes : 1.0));
+    c = c < 1 ? 1 : (c > p.Hkv ? p.Hkv : c);
+    while (c < p.Hkv && static_cast<int64_t>(c) * (p.Hq / p.Hkv) * p.batch * p.n_pair_max < 2 * 148) ++c;
+    while (p.Hkv % c) ++c;
+    p.kv_chunk = c;
+  }
+  const int64_t grid = static_cast<int64_t>(p.n_pair_max) * p.batch * p.Hq;
+  if (grid == 0) return TM_OK;
+  if (grid > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
+  attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, false, true>
+      <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mQ16, mK8, mV8, p);
+  return check_cuda(cudaGetLastError());
+}
+
 }  // namespace
+
+tm_status launch_attn_pair_cache(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                                 const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q,
+                                 int32_t max_k, const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
+                                 cudaStream_t stream) {
+  return launch_pair_cache(q, k, v, out, cu, cu_k, batch, max_q, max_k, bitmask, mask_hs, g, causal, stream);
+}
 
 tm_status launch_attn_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                            const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,

@@ -34,7 +34,15 @@ tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_ten
                             const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
                             cudaStream_t stream, const Fp8Route* f8 = nullptr);
 
-// INT8 K/V cache (codes + per-token fp16 scales), d = 128, 128-key tiles.
+// INT8 K/V cache on the two-query-tile kernel: d = 128, 128-row query tiles
+// and 128-key tiles; a dequantisation warpgroup writes the fp16 tiles.
+tm_status launch_attn_pair_cache(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                                 const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q,
+                                 int32_t max_k, const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
+                                 cudaStream_t stream);
+
+// INT8 K/V cache (codes + per-token fp16 scales), d = 128, 128-key tiles, one
+// query tile per CTA.
 tm_status launch_attn_cache(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                             const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
                             const uint32_t* bitmask, int64_t mask_hs, int32_t tile_m, int32_t g,

@@ -104,9 +104,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Waits until the phase with the given parity has completed.  Gives up (and
 // reports) after limit_ns of global time, or early when *abort becomes
 // non-zero.
-#ifdef TM_TRACE
-// First timed-out wait of a launch (TM_TRACE builds): block, barrier offset
-// within the block's shared window, parity, thread.
+#if defined(TM_TRACE) || defined(TM_TIMEOUT_INFO)
+// First timed-out wait of a launch (TM_TRACE or TM_TIMEOUT_INFO builds):
+// block, barrier offset within the block's shared window, parity, thread.
 static __device__ unsigned int g_tm_timeout_info[5];
 #endif
 __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, const DevErr& err,
@@ -117,7 +117,7 @@ __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, c
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (global_ns() - t0 > limit_ns) {
-#ifdef TM_TRACE
+#if defined(TM_TRACE) || defined(TM_TIMEOUT_INFO)
       if (atomicCAS(&g_tm_timeout_info[0], 0u, 1u) == 0u) {
         g_tm_timeout_info[1] = blockIdx.x;
         g_tm_timeout_info[2] = bar;
