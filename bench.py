@@ -867,8 +867,9 @@ def run_fp8_table(args):
     """The FP8 third precision on the routing-sweep inputs: attention time,
     mix-weighted roofline fraction and output error against the all-FP16
     output for FP16-only, INT8-only, FP8-only and three-way routing.  Each
-    point's kernel is named; FP8 routes run in the one-tile kernel, so the
-    FP16 and INT8 points are also given there.  E4M3 QK^T runs at the INT8
+    point's kernel is named: FP8 / FP16 routing runs in the two-tile kernel
+    (auto) and in the one-tile kernel; three-way routing in the one-tile
+    kernel.  E4M3 QK^T runs at the INT8
     rate, so FP8 pairs take p8 = 2 p16 in the roofline like INT8 pairs.
     Only the attention launch is timed (median of 20 calls, a 256 MiB buffer
     written before each)."""
@@ -947,7 +948,7 @@ def run_fp8_table(args):
     if args.fp8_only is not None:
         # one FP8-only point (no error reference: its error fields are
         # against its own output)
-        point("fp8", ONE, None, args.fp8_only)
+        point("fp8", AUTO, None, args.fp8_only)
         return {"metric": "FP8 third precision: attention time by route mix", "unit": "mixed", "n_gpus": 1,
                 "workload": w.name, "config": describe(w),
                 "peak": {"bf16_tflops": p16 / 1e12, "source": peak_src}, "points": rows}
@@ -955,10 +956,13 @@ def run_fp8_table(args):
     point("fp16", ONE, None, None)
     point("int8", AUTO, 0.75, None)
     point("int8", ONE, 0.75, None)
-    point("fp8 plane empty", ONE, None, 0.0)          # the FP8 kernel variant with nothing routed to FP8
+    point("fp8 plane empty", AUTO, None, 0.0)         # the two-tile kernel's FP8 variant, nothing routed to FP8
+    for pf8 in (0.25, 0.5, 0.75, 1.0):
+        point("fp8", AUTO, None, pf8)                 # FP8 and FP16 only: the two-tile kernel
+    point("fp8 plane empty", ONE, None, 0.0)          # the one-tile kernel's FP8 variant
     for pf8 in (0.25, 0.5, 0.75, 1.0):
         point("fp8", ONE, None, pf8)
-    point("int8 + fp8", ONE, 0.5, 0.5)
+    point("int8 + fp8", ONE, 0.5, 0.5)                # three-way routing: the one-tile kernel
     point("int8 + fp8", ONE, 0.75, 1.0)
     return {"metric": "FP8 third precision: attention time and error by route mix", "unit": "mixed",
             "n_gpus": 1, "workload": w.name, "config": describe(w),

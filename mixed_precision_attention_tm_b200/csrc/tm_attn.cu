@@ -625,9 +625,25 @@ tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor*
       return TM_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);
-  if (f8 != nullptr)
+  if (f8 != nullptr) {
+    // FP8 and FP16 only (no INT8 plane): the two-query-tile kernel with its
+    // 8-bit route in E4M3, unless that leaves SMs idle or the one-tile
+    // kernel is chosen; three-way routing runs on the one-tile kernel
+    const int64_t n_qt = ((cu_seqlens ? max_seqlen : q->T) + 127) / 128;
+    if (bitmask == nullptr && !use_one_tile_kernel(n_qt, cu_seqlens ? batch : 1, q->H, true, causal != 0)) {
+      tm_tensor qq = *q, kk = *k;
+      qq.codes = reinterpret_cast<const int8_t*>(f8->q_codes);
+      qq.scales = f8->q_scales;
+      qq.scale_kind = TM_SCALE_TILE;
+      kk.codes = reinterpret_cast<const int8_t*>(f8->k_codes);
+      kk.scales = f8->k_scales;
+      kk.scale_kind = TM_SCALE_TILE;
+      return launch_attn_pair_fp8(&qq, &kk, v, out, cu_seqlens, batch, max_seqlen, f8->bitmask, mask_head_stride,
+                                  g, causal, s);
+    }
     return launch_attn_split(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride, g,
                              causal, s, f8);
+  }
   if (tile_m == 128 && tile_n == 128) {
     const int64_t n_qt = ((cu_seqlens ? max_seqlen : q->T) + 127) / 128;
     if (D == 128 && (TM_SPLIT_KERNEL == 2 ||

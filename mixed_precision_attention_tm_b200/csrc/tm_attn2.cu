@@ -122,6 +122,7 @@ struct Cfg2 {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S16 = idesc_f16(BM, BN, false);
   static constexpr uint32_t IDESC_S8 = idesc_i8(BM, BN);
+  static constexpr uint32_t IDESC_F8 = idesc_f8_e4m3(BM, BN);           // the FP8 route (F8 launches)
   static constexpr uint32_t IDESC_S16_64 = idesc_f16(BM, 64, false);   // chunked mode: 64-key chunks
   static constexpr uint32_t IDESC_S8_64 = idesc_i8(BM, 64);
   static constexpr uint32_t IDESC_PV = idesc_f16(BM, D, true);
@@ -251,13 +252,18 @@ __device__ __forceinline__ void dequant_row_inplace(uint8_t* slot, int r, __half
   }
 }
 
-template <int D, int EMU, bool DUAL, bool CH, bool CACHE>
+// F8: the 8-bit route is FP8 E4M3 instead of INT8 (a launch with an FP8 bit
+// plane and no INT8 plane): the Q8 / K8 maps, tile scales and bitmask are the
+// FP8 ones, and the route's QK^T is four kind::f8f6f4 MMAs with an fp32
+// result (no seed).  Everything else is the INT8 route's.
+template <int D, int EMU, bool DUAL, bool CH, bool CACHE, bool F8 = false>
 __global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmQ8,
                      const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmK8,
                      const __grid_constant__ CUtensorMap tmV16, const Params2 p) {
   using C = Cfg2<D, CACHE>;
   static_assert(!CACHE || (DUAL && !CH && D == 128), "the INT8 cache runs in the two-issuer mode, d = 128");
+  static_assert(!F8 || (!CACHE && !CH && D == 128), "the FP8 route: d = 128, fp16 K / V, routed launches");
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -621,7 +627,8 @@ __global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
             bd[kk] = smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8);
           }
           if (elect_one()) {
-            mma_i8_exact_n<D / 32>(d_s, sd, C::IDESC_S16, ad, bd, C::IDESC_S8);
+            if constexpr (F8) mma_f8_ss_n<D / 32>(d_s, ad, bd, C::IDESC_F8, 0u);
+            else mma_i8_exact_n<D / 32>(d_s, sd, C::IDESC_S16, ad, bd, C::IDESC_S8);
             tc_commit(bar(C_SFULL + t));
           }
         } else {
@@ -882,7 +889,8 @@ __global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
             bd[kk] = smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8);
           }
           if (elect_one()) {
-            mma_i8_exact_n<D / 32>(d_tmem, sd, C::IDESC_S16, ad, bd, C::IDESC_S8);
+            if constexpr (F8) mma_f8_ss_n<D / 32>(d_tmem, ad, bd, C::IDESC_F8, 0u);
+            else mma_i8_exact_n<D / 32>(d_tmem, sd, C::IDESC_S16, ad, bd, C::IDESC_S8);
             tc_commit(bar(C_SFULL + t));
           }
         } else {
@@ -1352,13 +1360,13 @@ std::mutex g_mu2;
 // One-time kernel attributes; the warpgroup register split assumes exactly
 // LAUNCH_REGS per thread at launch (any other allocation could leave
 // setmaxnreg.inc waiting), so a build that differs is refused.
-template <int D, bool DUAL, bool CH, bool CACHE = false>
+template <int D, bool DUAL, bool CH, bool CACHE = false, bool F8 = false>
 tm_status prepare_pair_kernel() {
   using C = Cfg2<D, CACHE>;
   static bool attr_done = false;
   std::lock_guard<std::mutex> lk(g_mu2);
   if (attr_done) return TM_OK;
-  auto kern = attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, DUAL, CH, CACHE>;
+  auto kern = attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, DUAL, CH, CACHE, F8>;
   cudaFuncAttributes fa;
   tm_status st = check_cuda(cudaFuncGetAttributes(&fa, kern));
   if (st != TM_OK) return st;
@@ -1388,7 +1396,9 @@ constexpr int64_t kDualIssuerKeyTiles = 64;
 #define TM_PAIR_CHUNKED 1
 #endif
 
-template <int D>
+// F8: q / k carry the FP8 E4M3 codes and tile scales in their codes / scales
+// fields and bitmask is the FP8 bit plane (d = 128).
+template <int D, bool F8 = false>
 tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                       const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
                       const uint32_t* bitmask,
@@ -1396,9 +1406,10 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
   using C = Cfg2<D>;
   const int64_t maxk_tiles = ((cu ? max_k : k->T) + 127) / 128;
   const bool dual = maxk_tiles >= kDualIssuerKeyTiles;
-  const bool chunked = dual && D == 128 && TM_PAIR_CHUNKED && bitmask == nullptr;
+  const bool chunked = !F8 && dual && D == 128 && TM_PAIR_CHUNKED && bitmask == nullptr;
   tm_status st = chunked ? prepare_pair_kernel<D, true, true>()
-                         : (dual ? prepare_pair_kernel<D, true, false>() : prepare_pair_kernel<D, false, false>());
+                         : (dual ? prepare_pair_kernel<D, true, false, false, F8>()
+                                 : prepare_pair_kernel<D, false, false, false, F8>());
   if (st != TM_OK) return st;
   CUtensorMap mQ16, mQ8, mK16, mK8, mV16;
   st = encode_thd_map(&mQ16, q->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q->T, q->H, D, q->stride_t,
@@ -1466,10 +1477,10 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
     attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, true, false>
         <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   else if (dual)
-    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, false, false>
+    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, false, false, F8>
         <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   else
-    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, false, false, false>
+    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, false, false, false, F8>
         <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   return check_cuda(cudaGetLastError());
 }
@@ -1556,6 +1567,14 @@ tm_status launch_attn_pair_cache(const tm_tensor* q, const tm_tensor* k, const t
                                  int32_t max_k, const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
                                  cudaStream_t stream) {
   return launch_pair_cache(q, k, v, out, cu, cu_k, batch, max_q, max_k, bitmask, mask_hs, g, causal, stream);
+}
+
+tm_status launch_attn_pair_fp8(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                               const int32_t* cu, int32_t batch, int32_t max_q, const uint32_t* bitmask_fp8,
+                               int64_t mask_hs, int32_t g, int32_t causal, cudaStream_t stream) {
+  if (q->d != 128) return TM_ERR_UNSUPPORTED;
+  return launch_pair<128, true>(q, k, v, out, cu, nullptr, batch, max_q, max_q, bitmask_fp8, mask_hs, g, causal,
+                                stream);
 }
 
 tm_status launch_attn_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,

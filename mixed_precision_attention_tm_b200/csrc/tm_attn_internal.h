@@ -16,6 +16,13 @@ tm_status launch_attn_pair(const tm_tensor* q, const tm_tensor* k, const tm_tens
                            const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
                            cudaStream_t stream);
 
+// The FP8 route on the two-query-tile kernel, for launches without an INT8
+// plane: q / k carry the FP8 E4M3 codes and tile scales in their codes /
+// scales fields; bitmask_fp8 is the FP8 bit plane (d = 128, 128 x 128 tiles).
+tm_status launch_attn_pair_fp8(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                               const int32_t* cu, int32_t batch, int32_t max_q, const uint32_t* bitmask_fp8,
+                               int64_t mask_hs, int32_t g, int32_t causal, cudaStream_t stream);
+
 // The FP8 third precision: a second routing bit plane (layout of the INT8
 // bitmask) and the E4M3 codes and tile scales of Q and K.
 struct Fp8Route {

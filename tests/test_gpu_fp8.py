@@ -92,8 +92,18 @@ def _run(L, hq, hkv, causal, g, p8, pf8, cu=None, seed=0, qk=None):
     return out.cpu(), ref, omf8, om8
 
 
+@pytest.fixture(params=[ops.ATTN_KERNEL_TWO_TILE, ops.ATTN_KERNEL_ONE_TILE], ids=["two_tile", "one_tile"])
+def attn_kernel(request):
+    """FP8 launches without an INT8 plane run on either d = 128 kernel (the
+    two-tile kernel with its 8-bit route in E4M3, or the one-tile kernel);
+    three-way launches always take the one-tile kernel."""
+    ops.set_attn_kernel(request.param)
+    yield request.param
+    ops.set_attn_kernel(ops.ATTN_KERNEL_AUTO)
+
+
 @pytest.mark.parametrize("case", FP8_CASES, ids=[c[0] for c in FP8_CASES])
-def test_fp8_routed_attention_matches_oracle(case):
+def test_fp8_routed_attention_matches_oracle(case, attn_kernel):
     name, L, hq, hkv, causal, g, p8, pf8 = case
     cu = None
     if isinstance(L, list):
@@ -107,7 +117,7 @@ def test_fp8_routed_attention_matches_oracle(case):
     assert err <= TOL, f"{name}: max abs err {err}"
 
 
-def test_fp8_route_on_exact_inputs_matches_fp16():
+def test_fp8_route_on_exact_inputs_matches_fp16(attn_kernel):
     """Q, K whose values are E4M3 values x 2^-4 with every tile reaching
     448 x 2^-4: each tile scale is 2^-4, the codes are exact and the FP8 route
     computes the FP16 route's scores; the two outputs agree up to the fp32
