@@ -325,7 +325,7 @@ def build_mask(Hq, seqs, tile_m, tile_n, g, causal, p, seed,
 
 
 def build_mask_scale_policy(Hq, Hkv, seqs, tile_m, tile_n, g, causal, q_scales, k_scales, tau,
-                            force_diag=False, force_sink=False, words=None):
+                            force_diag=False, force_sink=False, words=None, k_token_scales=None):
     """Content-driven routing bitmask from the tile quantisation scales,
     uint32 [Hq, n_qtiles, W] in the layout of ``build_mask``.
 
@@ -343,8 +343,22 @@ def build_mask_scale_policy(Hq, Hkv, seqs, tile_m, tile_n, g, causal, q_scales, 
     forcing are those of ``build_mask``.  tau = +inf routes every eligible
     group INT8; tau < 0 none.
     q_scales: fp32 [n_qtiles, Hq]; k_scales: fp32 [n_ktiles, Hkv], global
-    tile order of ``tile_table``.
+    tile order of ``tile_table``.  The sequences may have their own key
+    offsets (``seq_table`` with ``cu_seqlens_k``): key tiles, legality and
+    causality then follow each sequence's (Lq, Lk).
+
+    k_token_scales (instead of k_scales): fp16 [Tk, Hkv], one scale per key
+    token, as an INT8 cache carries.  The FP16 route then reads the fp16 view
+    k^ = fp16(c_k * s_k) and the INT8 route s_q * s_k * (c_q . c_k), so per
+    score the two differ by at most about d * s_q * s_k * (127/2 + 127^2 / 2^11)
+    (half a step of Q rounding times |c_k| <= 127, plus the fp16 rounding of
+    the dequantised key), again proportional to s_q * s_k.  mk is then the
+    largest fp32 value of s_k over the key tokens of the group's visible key
+    tiles: rows [G*g*tile_n, min(min((G+1)*g, nj)*tile_n, Lk)) of the
+    sequence's keys.
     """
+    if (k_scales is None) == (k_token_scales is None):
+        raise ValueError("give k_scales (per key tile) or k_token_scales (per key token)")
     qt = tile_table(seqs, tile_m, "q")
     kt = tile_table(seqs, tile_n, "k")
     kbase = {}
@@ -354,7 +368,10 @@ def build_mask_scale_policy(Hq, Hkv, seqs, tile_m, tile_n, g, causal, q_scales, 
     if words is None:
         words = mask_words(max([s[3] for s in seqs] + [1]), tile_n, g)
     q_scales = np.asarray(q_scales, dtype=np.float32)
-    k_scales = np.asarray(k_scales, dtype=np.float32)
+    if k_scales is not None:
+        k_scales = np.asarray(k_scales, dtype=np.float32)
+    else:
+        k_tok = np.asarray(k_token_scales, dtype=np.float16).astype(np.float32)
     tau = np.float32(tau)
     grp = Hq // Hkv
     out = np.zeros((Hq, len(qt), words), dtype=np.uint32)
@@ -371,8 +388,13 @@ def build_mask_scale_policy(Hq, Hkv, seqs, tile_m, tile_n, g, causal, q_scales, 
             for G in range(ng):
                 if (force_sink and G == 0) or (force_diag and G == gdiag):
                     continue
-                js = range(G * g, min((G + 1) * g, nj))
-                mk = max(k_scales[kbase[b] + j, hk] for j in js)
+                j1 = min((G + 1) * g, nj)
+                if k_scales is not None:
+                    mk = max(k_scales[kbase[b] + j, hk] for j in range(G * g, j1))
+                else:
+                    k0 = seqs[b][2]
+                    r_end = min(j1 * tile_n, seqs[b][3])
+                    mk = max(k_tok[k0 + r, hk] for r in range(G * g * tile_n, r_end))
                 if np.float32(sq * mk) <= tau:
                     out[h, ig, G // 32] |= np.uint32(1 << (G % 32))
     return out
