@@ -202,6 +202,46 @@ tm_status tm_build_mask_scale_policy(uint32_t* bitmask, int32_t Hq, int32_t Hkv,
                                      const float* k_scales, float tau, int32_t force_diag, int32_t force_sink,
                                      int64_t mask_head_stride, void* stream);
 
+/* tm_build_mask_scale_policy with separate key offsets (prefix-cached
+ * prefill): sequence b has lq = cu_q[b+1] - cu_q[b] queries and lk =
+ * cu_k[b+1] - cu_k[b] keys, bottom-right causal; key tiles are numbered per
+ * key sequence (k_scales: device fp32 [sum_b ceil(lk_b / tile_n), Hkv], as
+ * tm_quantize_qk writes them with key offsets, or as tm_key_tile_scales
+ * writes them from an INT8 cache); W = tm_mask_words(max_seqlen_k, tile_n, g).
+ * A key sequence longer than max_seqlen_k is reported by tm_get_device_error
+ * (TM_ERR_INVALID_ARG) and its rows are not written.  TM_ERR_INVALID_ARG for
+ * a null cu_seqlens_q / cu_seqlens_k, max_seqlen_k <= 0 or the conditions of
+ * tm_build_mask_scale_policy. */
+tm_status tm_build_mask_scale_policy_varlen(uint32_t* bitmask, int32_t Hq, int32_t Hkv,
+                                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                            int32_t batch, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                            int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal,
+                                            const float* q_scales, const float* k_scales, float tau,
+                                            int32_t force_diag, int32_t force_sink, int64_t mask_head_stride,
+                                            void* stream);
+
+/* Key-tile statistic of the scale policy for an INT8 cache, whose keys carry
+ * one fp16 scale per token and kv head.  For the cache the FP16 route reads
+ * k^ = fp16(c_k * s_k) and the INT8 route s_q * s_k * (c_q . c_k), so a score's
+ * two values differ by at most about d * s_q * s_k * (127/2 + 127^2 / 2^11):
+ * again s_q times the key's scale.  This writes, per key tile J and kv head
+ * hk, the largest token scale over the tile's tokens, as fp32 (exact); fed to
+ * tm_build_mask_scale_policy(_varlen) as k_scales, each group's statistic is
+ * then the largest token scale over its visible key tiles' tokens.
+ *   k_tile_scales: device fp32 [n_ktiles, Hkv] (out), key tiles numbered per
+ *                  sequence in order, each sequence starting a new tile.
+ *   k_token_scales: device fp16 [Tk, Hkv], contiguous (the cache's K scales),
+ *                  finite and >= 0.
+ *   cu_seqlens_k: device int32 [batch+1] key offsets, or NULL for one
+ *                  sequence of Lk keys; max_seqlen_k bounds the key lengths
+ *                  (a longer sequence is reported by tm_get_device_error and
+ *                  not written).
+ * TM_ERR_INVALID_ARG for null or misaligned pointers, Hkv <= 0, tile_n <= 0,
+ * batch <= 0 with offsets, negative lengths. */
+tm_status tm_key_tile_scales(float* k_tile_scales, const void* k_token_scales, int32_t Hkv,
+                             const int32_t* cu_seqlens_k, int32_t batch, int32_t max_seqlen_k, int64_t Lk,
+                             int32_t tile_n, void* stream);
+
 /* Same bits computed on the host (bitmask_host and cu_seqlens_host are host
  * pointers), written with mask_head_stride = n_qtiles * W; bit-identical to
  * tm_build_mask. */

@@ -25,8 +25,9 @@ class TileMixPrefill:
                  tau=None, cu_seqlens_k=None, out=None, bitmask=None, device="cuda"):
         """p: Bernoulli INT8 probability per eligible group (seeded mask);
         tau: instead of p, the content-driven policy (INT8 iff the tile
-        scales' score-error bound s_q * s_k is at most tau).  Neither: all
-        FP16.  cu_seqlens_k: key offsets per sequence when they differ from
+        scales' score-error bound s_q * s_k is at most tau; with the INT8
+        cache s_k is the largest per-token key scale of the group's tiles).
+        Neither: all FP16.  cu_seqlens_k: key offsets per sequence when they differ from
         cu_seqlens (prefix-cached prefill: Lq = total new queries, Lk = total
         keys).  out: an fp16 [Lq, hq, d] device tensor to write the output
         into (heads contiguous; rows may be strided) instead of a new one.
@@ -39,8 +40,6 @@ class TileMixPrefill:
             raise ValueError("give either p (random routing) or tau (scale policy), not both")
         if bitmask is not None and (p is not None or tau is not None):
             raise ValueError("a caller-written bitmask replaces p and tau")
-        if tau is not None and int8_cache:
-            raise ValueError("the scale policy needs tile scales of K; the INT8 cache has per-token scales")
         self.p, self.seed, self.force_diag, self.force_sink = p, seed, force_diag, force_sink
         self.tau = tau
         self.int8_cache = int8_cache
@@ -51,8 +50,6 @@ class TileMixPrefill:
         self.max_seqlen = None if cu_h is None else int((cu_h[1:] - cu_h[:-1]).max())
         if cu_seqlens_k is not None and cu_seqlens is None:
             raise ValueError("cu_seqlens_k needs cu_seqlens")
-        if cu_seqlens_k is not None and tau is not None:
-            raise ValueError("the scale policy takes shared query / key offsets")
         self.cu_k = None if cu_seqlens_k is None else cu_seqlens_k.to(self.device, torch.int32)
         self.ck_h = None if cu_seqlens_k is None else cu_seqlens_k.to("cpu", torch.int32).contiguous()
         self.max_seqlen_k = None if self.ck_h is None else int((self.ck_h[1:] - self.ck_h[:-1]).max())
@@ -77,18 +74,21 @@ class TileMixPrefill:
             self.out = torch.empty((Lq, hq, d), dtype=torch.float16, device=dev)
         self.external_mask = bitmask is not None
         self.routed = p is not None or tau is not None or self.external_mask
-        self.q_quant = self.k_quant = self.bitmask = None
+        self.q_quant = self.k_quant = self.bitmask = self.k_tile_sc = None
         if self.routed:
             # codes, tile scales and the routing mask: allocated once, rewritten every step
             cu_np = None if cu_h is None else cu_h.numpy()
             nqt = ops.count_tiles(Lq, tile_m, cu_np)
             self.q_quant = (torch.empty((Lq, hq, d), dtype=torch.int8, device=dev),
                             torch.empty((nqt, hq), dtype=torch.float32, device=dev))
+            ck_np = cu_np if self.ck_h is None else self.ck_h.numpy()
+            nkt = ops.count_tiles(Lk, tile_n, ck_np)
             if not int8_cache:
-                ck_np = cu_np if self.ck_h is None else self.ck_h.numpy()
-                nkt = ops.count_tiles(Lk, tile_n, ck_np)
                 self.k_quant = (torch.empty((Lk, hkv, d), dtype=torch.int8, device=dev),
                                 torch.empty((nkt, hkv), dtype=torch.float32, device=dev))
+            elif tau is not None:
+                # the policy's key statistic from the cache's per-token scales
+                self.k_tile_sc = torch.empty((nkt, hkv), dtype=torch.float32, device=dev)
             maxk = Lk if cu_h is None else (self.max_seqlen if self.ck_h is None else self.max_seqlen_k)
             shape = (hq, nqt, ops.mask_words(maxk, tile_n, g))
             if self.external_mask:
@@ -99,6 +99,7 @@ class TileMixPrefill:
                 self.bitmask = torch.empty(shape, dtype=torch.int32, device=dev)
         n_quant = 1 if self.routed else 0          # Q and K are quantised in one launch
         n_mask = 1 if self.routed and not self.external_mask else 0
+        n_mask += 1 if self.k_tile_sc is not None else 0
         self.launches_per_step = 1 + n_quant + n_mask
 
     # -- inputs -----------------------------------------------------------
@@ -133,11 +134,18 @@ class TileMixPrefill:
     def mask(self):
         Lq, Lk = self.shape[0], self.shape[1]
         if self.tau is not None:
-            ops.build_mask_scale_policy(self.q_quant[1], self.k_quant[1], self.shape[2], self.shape[3],
+            k_sc = self.k_quant[1] if self.k_tile_sc is None else self.k_tile_sc
+            if self.k_tile_sc is not None:
+                shared = self.cu_k is None
+                ops.key_tile_scales(self.ks, tile_n=self.tile_n, cu_seqlens_k=self.cu if shared else self.cu_k,
+                                    max_seqlen_k=self.max_seqlen if shared else self.max_seqlen_k,
+                                    cu_seqlens_k_host=self.cu_h if shared else self.ck_h, out=k_sc)
+            ops.build_mask_scale_policy(self.q_quant[1], k_sc, self.shape[2], self.shape[3],
                                         tile_m=self.tile_m, tile_n=self.tile_n, g=self.g, causal=self.causal,
                                         tau=self.tau, force_diag=self.force_diag, force_sink=self.force_sink,
                                         Lq=Lq, Lk=Lk, cu_seqlens=self.cu, max_seqlen=self.max_seqlen,
-                                        cu_seqlens_host=self.cu_h, out=self.bitmask)
+                                        cu_seqlens_host=self.cu_h, out=self.bitmask, cu_seqlens_k=self.cu_k,
+                                        max_seqlen_k=self.max_seqlen_k, cu_seqlens_k_host=self.ck_h)
             return
         ops.build_mask(self.shape[2], tile_m=self.tile_m, tile_n=self.tile_n, g=self.g,
                        causal=self.causal, p=self.p, seed=self.seed, force_diag=self.force_diag,

@@ -1,5 +1,6 @@
-// tm_mask.cu -- routing bitmask (tm_build_mask, tm_build_mask_host) and
-// routing statistics (tm_route_stats).
+// tm_mask.cu -- routing bitmask (tm_build_mask, tm_build_mask_host), the
+// content-driven scale policy (tm_build_mask_scale_policy(_varlen),
+// tm_key_tile_scales) and routing statistics (tm_route_stats).
 //
 // TileMix (Lattice paper page), abstract: routing decisions are packed into
 // compact bitmasks, one bit per query tile x group of g adjacent key tiles,
@@ -133,22 +134,58 @@ __device__ inline uint32_t policy_word(const PolicyArgs& a, int h, int64_t ig, i
   return word;
 }
 
+// cu_k: key offsets when they differ from the query offsets (prefix-cached
+// prefill); key tiles are then numbered per key sequence.
 __global__ void build_mask_policy_kernel(uint32_t* __restrict__ bm, int64_t head_stride,
-                                         const int32_t* __restrict__ cu, int64_t Lq, int64_t Lk,
-                                         PolicyArgs a, const float* __restrict__ qs,
-                                         const float* __restrict__ ks, DevErr err) {
+                                         const int32_t* __restrict__ cu, const int32_t* __restrict__ cu_k,
+                                         int64_t Lq, int64_t Lk, int64_t max_lk, PolicyArgs a,
+                                         const float* __restrict__ qs, const float* __restrict__ ks,
+                                         DevErr err) {
   const int I = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
   SeqInfo s = seq_info(cu, b, Lq, a.tile_m);
   const int64_t lq = s.len;
-  const int64_t lk = cu ? s.len : Lk;
+  const SeqInfo sk = seq_info(cu_k ? cu_k : cu, b, Lk, a.tile_n);
+  const int64_t lk = cu_k ? sk.len : (cu ? s.len : Lk);
+  if (cu_k != nullptr && lk > max_lk) {   // the row of W words was sized for max_lk
+    if (I == 0 && threadIdx.x == 0) dev_error(err, TM_DEVERR_SEQLEN);
+    return;
+  }
   if (cu != nullptr && I == 0 && threadIdx.x == 0 &&
       lq > static_cast<int64_t>(gridDim.x) * a.tile_m)
     dev_error(err, TM_DEVERR_SEQLEN);
   if (static_cast<int64_t>(I) * a.tile_m >= lq) return;
-  const int64_t kbase = seq_info(cu, b, Lk, a.tile_n).tile_base;
+  const int64_t kbase = sk.tile_base;
   const int64_t ig = s.tile_base + I;
   uint32_t* row = bm + static_cast<int64_t>(h) * head_stride + ig * a.W;
   for (int w = threadIdx.x; w < a.W; w += blockDim.x) row[w] = policy_word(a, h, ig, I, lq, lk, kbase, qs, ks, w);
+}
+
+// Per-token key scales (the fp16 scales of an INT8 cache, [T, Hkv]) reduced
+// to one fp32 value per key tile and kv head: the largest scale over the
+// tile's tokens.  The scale policy's group statistic is then the largest of
+// these over the group's visible key tiles, which equals the largest token
+// scale over those tiles' tokens (max is exact and associative).  One block
+// of kKeyScaleWarps warps per (key tile, sequence); each warp takes a head.
+constexpr int kKeyScaleWarps = 8;
+
+__global__ void __launch_bounds__(32 * kKeyScaleWarps)
+key_tile_scale_kernel(float* __restrict__ out, const __half* __restrict__ tok, int Hkv,
+                      const int32_t* __restrict__ cu_k, int64_t Lk, int64_t max_lk, int tile_n, DevErr err) {
+  const int J = blockIdx.x, b = blockIdx.y;
+  const SeqInfo s = seq_info(cu_k, b, Lk, tile_n);
+  if (cu_k != nullptr && J == 0 && threadIdx.x == 0 && s.len > max_lk) dev_error(err, TM_DEVERR_SEQLEN);
+  if (cu_k != nullptr && s.len > max_lk) return;
+  const int64_t r0 = static_cast<int64_t>(J) * tile_n;
+  if (r0 >= s.len) return;
+  const int64_t rows = (s.len - r0) < tile_n ? (s.len - r0) : tile_n;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int h = warp; h < Hkv; h += kKeyScaleWarps) {
+    float m = -INFINITY;
+    for (int64_t r = lane; r < rows; r += 32)
+      m = fmaxf(m, __half2float(tok[(s.start + r0 + r) * Hkv + h]));
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) out[(s.tile_base + J) * Hkv + h] = m;
+  }
 }
 
 tm_status check_mask_args(int32_t Hq, int32_t tile_m, int32_t tile_n, int32_t g, double p) {
@@ -210,11 +247,12 @@ tm_status tm_build_mask_varlen(uint32_t* bitmask, int32_t Hq, const int32_t* cu_
                          tile_n, g, causal, p, seed, force_diag, force_sink, mask_head_stride, stream);
 }
 
-tm_status tm_build_mask_scale_policy(uint32_t* bitmask, int32_t Hq, int32_t Hkv, const int32_t* cu_seqlens,
-                                     int32_t batch, int32_t max_seqlen, int64_t Lq, int64_t Lk, int32_t tile_m,
-                                     int32_t tile_n, int32_t g, int32_t causal, const float* q_scales,
-                                     const float* k_scales, float tau, int32_t force_diag, int32_t force_sink,
-                                     int64_t mask_head_stride, void* stream) {
+static tm_status scale_policy_impl(uint32_t* bitmask, int32_t Hq, int32_t Hkv, const int32_t* cu_seqlens,
+                                   const int32_t* cu_k, int32_t batch, int32_t max_seqlen, int32_t max_k,
+                                   int64_t Lq, int64_t Lk, int32_t tile_m, int32_t tile_n, int32_t g,
+                                   int32_t causal, const float* q_scales, const float* k_scales, float tau,
+                                   int32_t force_diag, int32_t force_sink, int64_t mask_head_stride,
+                                   void* stream) {
   using namespace tmk;
   tm_status st = check_mask_args(Hq, tile_m, tile_n, g, 0.5);
   if (st != TM_OK) return st;
@@ -223,7 +261,8 @@ tm_status tm_build_mask_scale_policy(uint32_t* bitmask, int32_t Hq, int32_t Hkv,
   if (bitmask == nullptr || reinterpret_cast<uintptr_t>(bitmask) % 4) return TM_ERR_INVALID_ARG;
   if (q_scales == nullptr || k_scales == nullptr) return TM_ERR_INVALID_ARG;
   const int64_t maxq = cu_seqlens ? max_seqlen : Lq;
-  const int64_t maxk = cu_seqlens ? max_seqlen : Lk;
+  const int64_t maxk = cu_seqlens ? (cu_k ? max_k : max_seqlen) : Lk;
+  if (cu_k != nullptr && (cu_seqlens == nullptr || max_k <= 0)) return TM_ERR_INVALID_ARG;
   if (cu_seqlens != nullptr && (batch <= 0 || max_seqlen <= 0)) return TM_ERR_INVALID_ARG;
   if (maxq < 0 || maxk < 0) return TM_ERR_INVALID_ARG;
   PolicyArgs a{Hq, Hkv, tile_m, tile_n, g, causal ? 1 : 0, tau, force_diag ? 1 : 0, force_sink ? 1 : 0,
@@ -236,8 +275,52 @@ tm_status tm_build_mask_scale_policy(uint32_t* bitmask, int32_t Hq, int32_t Hkv,
   if (nqt_max > 0x7fffffff || nb > 65535 || Hq > 65535) return TM_ERR_UNSUPPORTED;
   dim3 grid(static_cast<unsigned>(nqt_max), static_cast<unsigned>(nb), static_cast<unsigned>(Hq));
   DevErr err{device_error_word()};
-  build_mask_policy_kernel<<<grid, 32, 0, as_stream(stream)>>>(bitmask, mask_head_stride, cu_seqlens, Lq, Lk, a,
-                                                               q_scales, k_scales, err);
+  build_mask_policy_kernel<<<grid, 32, 0, as_stream(stream)>>>(bitmask, mask_head_stride, cu_seqlens, cu_k, Lq,
+                                                               Lk, maxk, a, q_scales, k_scales, err);
+  return check_cuda(cudaGetLastError());
+}
+
+tm_status tm_build_mask_scale_policy(uint32_t* bitmask, int32_t Hq, int32_t Hkv, const int32_t* cu_seqlens,
+                                     int32_t batch, int32_t max_seqlen, int64_t Lq, int64_t Lk, int32_t tile_m,
+                                     int32_t tile_n, int32_t g, int32_t causal, const float* q_scales,
+                                     const float* k_scales, float tau, int32_t force_diag, int32_t force_sink,
+                                     int64_t mask_head_stride, void* stream) {
+  return scale_policy_impl(bitmask, Hq, Hkv, cu_seqlens, nullptr, batch, max_seqlen, 0, Lq, Lk, tile_m, tile_n, g,
+                           causal, q_scales, k_scales, tau, force_diag, force_sink, mask_head_stride, stream);
+}
+
+tm_status tm_build_mask_scale_policy_varlen(uint32_t* bitmask, int32_t Hq, int32_t Hkv,
+                                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                            int32_t batch, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                            int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal,
+                                            const float* q_scales, const float* k_scales, float tau,
+                                            int32_t force_diag, int32_t force_sink, int64_t mask_head_stride,
+                                            void* stream) {
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return TM_ERR_INVALID_ARG;
+  return scale_policy_impl(bitmask, Hq, Hkv, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q, max_seqlen_k, 0, 0,
+                           tile_m, tile_n, g, causal, q_scales, k_scales, tau, force_diag, force_sink,
+                           mask_head_stride, stream);
+}
+
+tm_status tm_key_tile_scales(float* k_tile_scales, const void* k_token_scales, int32_t Hkv,
+                             const int32_t* cu_seqlens_k, int32_t batch, int32_t max_seqlen_k, int64_t Lk,
+                             int32_t tile_n, void* stream) {
+  using namespace tmk;
+  if (k_tile_scales == nullptr || k_token_scales == nullptr) return TM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(k_tile_scales) % 4 || reinterpret_cast<uintptr_t>(k_token_scales) % 2)
+    return TM_ERR_INVALID_ARG;
+  if (Hkv <= 0 || tile_n <= 0) return TM_ERR_INVALID_ARG;
+  if (cu_seqlens_k != nullptr && (batch <= 0 || max_seqlen_k < 0)) return TM_ERR_INVALID_ARG;
+  const int64_t maxk = cu_seqlens_k ? max_seqlen_k : Lk;
+  if (maxk < 0) return TM_ERR_INVALID_ARG;
+  const int64_t nkt_max = (maxk + tile_n - 1) / tile_n;
+  if (nkt_max == 0) return TM_OK;
+  const int nb = cu_seqlens_k ? batch : 1;
+  if (nkt_max > 0x7fffffff || nb > 65535) return TM_ERR_UNSUPPORTED;
+  dim3 grid(static_cast<unsigned>(nkt_max), static_cast<unsigned>(nb));
+  DevErr err{device_error_word()};
+  key_tile_scale_kernel<<<grid, 32 * kKeyScaleWarps, 0, as_stream(stream)>>>(
+      k_tile_scales, static_cast<const __half*>(k_token_scales), Hkv, cu_seqlens_k, Lk, maxk, tile_n, err);
   return check_cuda(cudaGetLastError());
 }
 

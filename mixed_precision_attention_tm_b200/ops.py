@@ -65,6 +65,9 @@ def _lib():
             "tm_build_mask_host": (I32, [P, I32, P, I32, I64, I64, I32, I32, I32, I32, D, U64, I32, I32]),
             "tm_build_mask_scale_policy": (I32, [P, I32, I32, P, I32, I32, I64, I64, I32, I32, I32, I32, P, P,
                                                  ctypes.c_float, I32, I32, I64, P]),
+            "tm_build_mask_scale_policy_varlen": (I32, [P, I32, I32, P, P, I32, I32, I32, I32, I32, I32, I32,
+                                                        P, P, ctypes.c_float, I32, I32, I64, P]),
+            "tm_key_tile_scales": (I32, [P, P, I32, P, I32, I32, I64, I32, P]),
             "tm_route_stats": (I32, [P, I64, I32, P, I32, I64, I64, I32, I32, I32, I32,
                                      ctypes.POINTER(D), ctypes.POINTER(D)]),
             "tm_attn_fwd": (I32, [TP, TP, TP, TP, P, I32, I32, P, I64, I32, I32, I32, I32, P]),
@@ -334,21 +337,30 @@ def build_mask(Hq, *, tile_m, tile_n, g, causal, p, seed, force_diag=False, forc
 
 def build_mask_scale_policy(q_scales, k_scales, Hq, Hkv, *, tile_m, tile_n, g, causal, tau, force_diag=False,
                             force_sink=False, Lq=None, Lk=None, cu_seqlens=None, max_seqlen=None,
-                            cu_seqlens_host=None, out=None):
+                            cu_seqlens_host=None, out=None, cu_seqlens_k=None, max_seqlen_k=None,
+                            cu_seqlens_k_host=None):
     """Content-driven routing bitmask (int32 view [Hq, n_qt, W]): group G of
     query tile I goes INT8 iff s_q[I] * max s_k over its visible key tiles
     <= tau (see tm_build_mask_scale_policy).  q_scales / k_scales: the device
-    tile scales from quantize_qk."""
+    tile scales from quantize_qk, or k_scales from key_tile_scales for an INT8
+    cache.  cu_seqlens_k: key offsets when they differ from cu_seqlens."""
     _cuda(q_scales, "q_scales")
     _cuda(k_scales, "k_scales")
     lib = _lib()
     cu_h = _cu_host(cu_seqlens, cu_seqlens_host)
     batch = 0 if cu_h is None else cu_h.numel() - 1
+    if cu_seqlens_k is not None and cu_h is None:
+        raise ValueError("cu_seqlens_k needs cu_seqlens")
     if cu_h is not None:
         maxk = int((cu_h[1:] - cu_h[:-1]).max()) if batch else 0
         if max_seqlen is None:
             max_seqlen = maxk
         nqt = count_tiles(None, tile_m, cu_h.numpy())
+        if cu_seqlens_k is not None:
+            ck_h = _cu_host(cu_seqlens_k, cu_seqlens_k_host)
+            if max_seqlen_k is None:
+                max_seqlen_k = int((ck_h[1:] - ck_h[:-1]).max()) if batch else 0
+            maxk = max_seqlen_k
     else:
         maxk = Lk
         nqt = count_tiles(Lq, tile_m)
@@ -357,11 +369,46 @@ def build_mask_scale_policy(q_scales, k_scales, Hq, Hkv, *, tile_m, tile_n, g, c
         out = torch.empty((Hq, nqt, W), dtype=torch.int32, device=q_scales.device)
     else:
         _check_buf(out, (Hq, nqt, W), torch.int32, "bitmask")
+    if cu_seqlens_k is not None:
+        st = lib.tm_build_mask_scale_policy_varlen(
+            _ptr(out), Hq, Hkv, _ptr(cu_seqlens), _ptr(cu_seqlens_k), batch, int(max_seqlen or 0),
+            int(max_seqlen_k or 0), tile_m, tile_n, g, int(bool(causal)), _ptr(q_scales), _ptr(k_scales),
+            float(tau), int(bool(force_diag)), int(bool(force_sink)), nqt * W, _stream())
+        _check(st, "tm_build_mask_scale_policy_varlen")
+        return out
     st = lib.tm_build_mask_scale_policy(_ptr(out), Hq, Hkv, _ptr(cu_seqlens), batch, int(max_seqlen or 0),
                                         int(Lq or 0), int(Lk or 0), tile_m, tile_n, g, int(bool(causal)),
                                         _ptr(q_scales), _ptr(k_scales), float(tau), int(bool(force_diag)),
                                         int(bool(force_sink)), nqt * W, _stream())
     _check(st, "tm_build_mask_scale_policy")
+    return out
+
+
+def key_tile_scales(k_token_scales, *, tile_n, cu_seqlens_k=None, max_seqlen_k=None, cu_seqlens_k_host=None,
+                    out=None):
+    """Largest per-token key scale of every key tile and kv head (fp32
+    [n_ktiles, Hkv]) from an INT8 cache's fp16 scales [Tk, Hkv]: the k_scales
+    of the scale policy for that cache (see tm_key_tile_scales)."""
+    _cuda(k_token_scales, "k_token_scales")
+    if k_token_scales.dtype != torch.float16 or k_token_scales.dim() != 2 or not k_token_scales.is_contiguous():
+        raise ValueError("k_token_scales: contiguous fp16 [Tk, Hkv]")
+    Tk, Hkv = k_token_scales.shape
+    lib = _lib()
+    ck_h = _cu_host(cu_seqlens_k, cu_seqlens_k_host)
+    batch = 0 if ck_h is None else ck_h.numel() - 1
+    if ck_h is not None:
+        if max_seqlen_k is None:
+            max_seqlen_k = int((ck_h[1:] - ck_h[:-1]).max()) if batch else 0
+        nkt = count_tiles(None, tile_n, ck_h.numpy())
+    else:
+        nkt = count_tiles(Tk, tile_n)
+    if out is None:
+        out = torch.empty((nkt, Hkv), dtype=torch.float32, device=k_token_scales.device)
+    else:
+        _check_buf(out, (nkt, Hkv), torch.float32, "k_tile_scales")
+    st = lib.tm_key_tile_scales(_ptr(out), _ptr(k_token_scales), Hkv, _ptr(cu_seqlens_k), batch,
+                                int(max_seqlen_k or 0), int(Tk), tile_n, _stream())
+    _check(st, "tm_key_tile_scales")
     return out
 
 

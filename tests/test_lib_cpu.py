@@ -266,3 +266,34 @@ def test_noalloc_validates_every_argument_before_any_cuda_call():
     assert call(q=big_q, o=big_q, k=_t(T=16384, H=8, d=128), v=_t(T=16384, H=8, d=128)) == ops.TM_ERR_UNSUPPORTED
     if not torch.cuda.is_available():
         assert call() == ops.TM_ERR_CUDA
+
+
+def test_policy_entries_validate_before_launch():
+    """tm_build_mask_scale_policy_varlen and tm_key_tile_scales return their
+    status for bad arguments before any CUDA call."""
+    lib = ops._lib()
+    P = ctypes.c_void_p
+    bm, cu, ck, sc = P(1 << 20), P(2 << 20), P(3 << 20), P(4 << 20)
+    inf = ctypes.c_float(float("inf"))
+    pol = lib.tm_build_mask_scale_policy_varlen
+    # missing key offsets, missing query offsets
+    assert pol(bm, 4, 2, cu, None, 2, 64, 64, 128, 128, 1, 1, sc, sc, inf, 0, 0, 8, None) == ops.TM_ERR_INVALID_ARG
+    assert pol(bm, 4, 2, None, ck, 2, 64, 64, 128, 128, 1, 1, sc, sc, inf, 0, 0, 8, None) == ops.TM_ERR_INVALID_ARG
+    # Hq not a multiple of Hkv, NaN tau, null scales, max_seqlen_k <= 0, batch <= 0
+    assert pol(bm, 3, 2, cu, ck, 2, 64, 64, 128, 128, 1, 1, sc, sc, inf, 0, 0, 8, None) == ops.TM_ERR_INVALID_ARG
+    assert pol(bm, 4, 2, cu, ck, 2, 64, 64, 128, 128, 1, 1, sc, sc, ctypes.c_float(float("nan")), 0, 0, 8,
+               None) == ops.TM_ERR_INVALID_ARG
+    assert pol(bm, 4, 2, cu, ck, 2, 64, 64, 128, 128, 1, 1, None, sc, inf, 0, 0, 8, None) == ops.TM_ERR_INVALID_ARG
+    assert pol(bm, 4, 2, cu, ck, 2, 64, 0, 128, 128, 1, 1, sc, sc, inf, 0, 0, 8, None) == ops.TM_ERR_INVALID_ARG
+    assert pol(bm, 4, 2, cu, ck, 0, 64, 64, 128, 128, 1, 1, sc, sc, inf, 0, 0, 8, None) == ops.TM_ERR_INVALID_ARG
+    kts = lib.tm_key_tile_scales
+    # null output / input, misaligned output, Hkv <= 0, tile_n <= 0, offsets without batch, negative length
+    assert kts(None, sc, 2, None, 0, 0, 256, 128, None) == ops.TM_ERR_INVALID_ARG
+    assert kts(sc, None, 2, None, 0, 0, 256, 128, None) == ops.TM_ERR_INVALID_ARG
+    assert kts(P((4 << 20) + 2), sc, 2, None, 0, 0, 256, 128, None) == ops.TM_ERR_INVALID_ARG
+    assert kts(sc, sc, 0, None, 0, 0, 256, 128, None) == ops.TM_ERR_INVALID_ARG
+    assert kts(sc, sc, 2, None, 0, 0, 256, 0, None) == ops.TM_ERR_INVALID_ARG
+    assert kts(sc, sc, 2, ck, 0, 256, 0, 128, None) == ops.TM_ERR_INVALID_ARG
+    assert kts(sc, sc, 2, None, 0, 0, -1, 128, None) == ops.TM_ERR_INVALID_ARG
+    # nothing to do: no launch, TM_OK
+    assert kts(sc, sc, 2, None, 0, 0, 0, 128, None) == ops.TM_OK
