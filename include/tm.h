@@ -310,6 +310,40 @@ tm_status tm_attn_fwd_varlen(const tm_tensor* q, const tm_tensor* k, const tm_te
                              void* stream);
 
 /* ---------------------------------------------------------------------------
+ * tm_attn_fwd_cache_ws -- tm_attn_fwd / tm_attn_fwd_varlen over an INT8 K/V
+ * cache, with the cache expanded once per call into a caller-owned workspace.
+ *
+ * TileMix (Lattice paper page, abstract) supports INT8 K/V caches; the
+ * FP16-routed groups and P.V read the cache's fp16 view fp16(code * scale)
+ * and the INT8-routed groups its K codes with the scale of each key.  Every
+ * K / V tile of a KV head is read by every query tile of the Hq / Hkv query
+ * heads of its group, so this call first writes the fp16 view of K and V
+ * (and the per-token K scales as fp32, one row of 128 per key tile) into `workspace`
+ * with one HBM-bound pass, then runs the attention on that view.  Results
+ * equal tm_attn_fwd's over the same cache (same scores, same softmax).
+ *   k, v: the INT8 cache (data NULL, codes [Tk, Hkv, 128] dense int8 +
+ *         TM_SCALE_TOKEN fp16 scales [Tk, Hkv] dense), as for tm_attn_fwd.
+ *   cu_seqlens_q: NULL for one sequence (Lq = q->T, Lk = k->T); else the
+ *         query offsets, with cu_seqlens_k the key offsets or NULL (keys use
+ *         the query offsets); max_seqlen_q / max_seqlen_k as for
+ *         tm_attn_fwd_varlen.
+ *   workspace: device memory of at least tm_cache_workspace_bytes(Tk, Hkv,
+ *         batch) bytes (batch = 0 without cu_seqlens_q), 256-byte aligned,
+ *         owned by the caller; overwritten by each call and free again once
+ *         the call's work on `stream` has finished.
+ * 128 x 128 tiles, d = 128.  tile_m = 64 runs tm_attn_fwd's in-kernel
+ * conversion and leaves the workspace untouched.  TM_ERR_INVALID_ARG for a
+ * null or short workspace, k / v that are not a cache, or the conditions of
+ * tm_attn_fwd(_varlen).
+ * ------------------------------------------------------------------------- */
+int64_t tm_cache_workspace_bytes(int64_t Tk, int32_t Hkv, int32_t batch);
+tm_status tm_attn_fwd_cache_ws(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch,
+                               int32_t max_seqlen_q, int32_t max_seqlen_k, const uint32_t* bitmask,
+                               int64_t mask_head_stride, int32_t tile_m, int32_t tile_n, int32_t g, int32_t causal,
+                               void* workspace, int64_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * tm_attn_fwd_routed_noalloc -- the routed prefill step for callers that
  * cannot allocate device memory.  (Library addition; it has no counterpart
  * in the paper.)

@@ -61,6 +61,12 @@ class TileMixPrefill:
             self.vc = torch.empty((Lk, hkv, d), dtype=torch.int8, device=dev)
             self.ks = torch.empty((Lk, hkv), dtype=torch.float16, device=dev)
             self.vs = torch.empty((Lk, hkv), dtype=torch.float16, device=dev)
+            # the cache's fp16 view and per-token K scales by key tile, written
+            # once per step (tm_attn_fwd_cache_ws; 128 x 128 tiles, d = 128)
+            self.cache_ws = None
+            if tile_m == 128 and tile_n == 128 and d == 128:
+                nb = 0 if cu_h is None else cu_h.numel() - 1
+                self.cache_ws = torch.empty(ops.cache_workspace_bytes(Lk, hkv, nb), dtype=torch.uint8, device=dev)
         else:
             self.k = torch.empty((Lk, hkv, d), dtype=torch.float16, device=dev)
             self.v = torch.empty((Lk, hkv, d), dtype=torch.float16, device=dev)
@@ -100,6 +106,7 @@ class TileMixPrefill:
         n_quant = 1 if self.routed else 0          # Q and K are quantised in one launch
         n_mask = 1 if self.routed and not self.external_mask else 0
         n_mask += 1 if self.k_tile_sc is not None else 0
+        n_mask += 1 if int8_cache and self.cache_ws is not None else 0   # the cache expansion
         self.launches_per_step = 1 + n_quant + n_mask
 
     # -- inputs -----------------------------------------------------------
@@ -162,7 +169,8 @@ class TileMixPrefill:
                             q_quant=self.q_quant if self.routed else None,
                             k_quant=self.k_quant if self.routed else None, kv_cache=kv,
                             cu_seqlens=self.cu, max_seqlen=self.max_seqlen, cu_seqlens_host=self.cu_h,
-                            cu_seqlens_k=self.cu_k, max_seqlen_k=self.max_seqlen_k)
+                            cu_seqlens_k=self.cu_k, max_seqlen_k=self.max_seqlen_k,
+                            cache_workspace=self.cache_ws if self.int8_cache else None)
 
     def run(self):
         """One prefill step on the resident inputs; returns the device output."""

@@ -20,7 +20,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtm.so")
-SOURCES = ["tm_api.cu", "tm_quant.cu", "tm_mask.cu", "tm_attn.cu", "tm_attn2.cu", "tm_attn3.cu", "tm_attn_cache.cu", "tm_noalloc.cu", "tm_probe.cu",
+SOURCES = ["tm_api.cu", "tm_quant.cu", "tm_mask.cu", "tm_attn.cu", "tm_attn2.cu", "tm_attn3.cu", "tm_attn_cache.cu", "tm_cache_expand.cu", "tm_noalloc.cu", "tm_probe.cu",
            "tm_shard.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -560,7 +560,8 @@ namespace {
 tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                         const int32_t* cu_seqlens, const int32_t* cu_k, int32_t batch, int32_t max_seqlen,
                         int32_t max_k, const uint32_t* bitmask, int64_t mask_head_stride, int32_t tile_m,
-                        int32_t tile_n, int32_t g, int32_t causal, void* stream, const Fp8Route* f8 = nullptr) {
+                        int32_t tile_n, int32_t g, int32_t causal, void* stream, const Fp8Route* f8 = nullptr,
+                        void* cache_ws = nullptr, int64_t cache_ws_bytes = 0) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return TM_ERR_INVALID_ARG;
   const int64_t D = q->d;
   if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
@@ -604,6 +605,35 @@ tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor*
     if (k->T != v->T || k->H != v->H || k->d != D || v->d != D || k->T < 0) return TM_ERR_INVALID_ARG;
     if (shared && k->T != q->T) return TM_ERR_INVALID_ARG;
     if (D != 128 || tile_n != 128) return TM_ERR_UNSUPPORTED;
+    if (cache_ws != nullptr && tile_m == 128) {
+      // The cache expanded once into the caller's workspace (its fp16 view
+      // and per-token K scales by key tile), then attention over the fp16
+      // view: all-FP16 launches as for fp16 K / V, routed launches on the
+      // two-query-tile kernel with the INT8 route's scales per key token.
+      const CacheWsLayout L = cache_ws_layout(k->T, static_cast<int32_t>(k->H), cu_seqlens ? batch : 0);
+      if (cache_ws_bytes < L.bytes || (reinterpret_cast<uintptr_t>(cache_ws) & 255u)) return TM_ERR_INVALID_ARG;
+      const int32_t* key_cu = cu_seqlens ? (cu_k ? cu_k : cu_seqlens) : nullptr;
+      cudaStream_t s = as_stream(stream);
+      st = launch_cache_expand(k, v, key_cu, batch, max_k, cache_ws, L, s);
+      if (st != TM_OK) return st;
+      uint8_t* ws = static_cast<uint8_t*>(cache_ws);
+      tm_tensor kk = *k, vv = *v;
+      kk.data = ws + L.off_k16;
+      vv.data = ws + L.off_v16;
+      kk.stride_t = vv.stride_t = k->H * 128;
+      kk.stride_h = vv.stride_h = 128;
+      kk.scales = vv.scales = nullptr;
+      kk.scale_kind = vv.scale_kind = TM_SCALE_NONE;
+      vv.codes = nullptr;
+      if (bitmask == nullptr) {
+        kk.codes = nullptr;
+        return attn_fwd_impl(q, &kk, &vv, out, cu_seqlens, cu_k, batch, max_seqlen, cu_k ? max_k : 0, nullptr,
+                             mask_head_stride, tile_m, tile_n, g, causal, stream);
+      }
+      return launch_attn_pair_toks(q, &kk, &vv, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask,
+                                   mask_head_stride, g, causal, reinterpret_cast<const float*>(ws + L.off_kst),
+                                   L.kst_tiles, s);
+    }
     // 128-row query tiles: two per CTA, unless that leaves SMs idle or the
     // one-tile kernel is chosen (tm_set_attn_kernel)
     const int64_t n_qt = ((cu_seqlens ? max_seqlen : q->T) + 127) / 128;
@@ -689,6 +719,21 @@ extern "C" tm_status tm_attn_fwd_varlen(const tm_tensor* q, const tm_tensor* k, 
   if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return TM_ERR_INVALID_ARG;
   return tmk::attn_fwd_impl(q, k, v, out, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q, max_seqlen_k, bitmask,
                             mask_head_stride, tile_m, tile_n, g, causal, stream);
+}
+
+extern "C" tm_status tm_attn_fwd_cache_ws(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v,
+                                          tm_tensor* out, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                          int32_t batch, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                          const uint32_t* bitmask, int64_t mask_head_stride, int32_t tile_m,
+                                          int32_t tile_n, int32_t g, int32_t causal, void* workspace,
+                                          int64_t workspace_bytes, void* stream) {
+  if (k == nullptr || v == nullptr || k->scale_kind != TM_SCALE_TOKEN || v->scale_kind != TM_SCALE_TOKEN)
+    return TM_ERR_INVALID_ARG;
+  if (workspace == nullptr) return TM_ERR_INVALID_ARG;
+  if (cu_seqlens_k != nullptr && cu_seqlens_q == nullptr) return TM_ERR_INVALID_ARG;
+  return tmk::attn_fwd_impl(q, k, v, out, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q,
+                            cu_seqlens_k ? max_seqlen_k : 0, bitmask, mask_head_stride, tile_m, tile_n, g, causal,
+                            stream, nullptr, workspace, workspace_bytes);
 }
 
 extern "C" tm_status tm_attn_fwd_fp8(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,

@@ -95,7 +95,7 @@ enum : unsigned {
 // FP16-routed key tiles and every fp16 V tile into the ring, the producer
 // brings the int8 K code tiles of INT8-routed ones, and the softmax applies
 // the per-token key scales of INT8 tiles per column.
-template <int D, bool CACHE = false>
+template <int D, bool CACHE = false, bool TOKS = false>
 struct Cfg2 {
   static constexpr int BM = 128, BN = 128;
   static constexpr int SLOT = BN * D * 2;                // one fp16 K or V tile
@@ -112,12 +112,16 @@ struct Cfg2 {
   // INT8 key-tile scales at +1152.  With CACHE: routing words [2][32] at
   // +256, the extra barriers at +512, seed blocks at +640, two stages of
   // per-token key scales (128 fp32 each) at +1024.
-  static constexpr int OFF_SEED = OFF_BAR + (CACHE ? 640 : 768);   // the INT8 accumulator seed blocks (kSeedBytes)
+  static constexpr int OFF_SEED = OFF_BAR + (CACHE ? 640 : (TOKS ? 512 : 768));   // INT8 accumulator seed blocks
   static constexpr int OFF_KSC = OFF_BAR + 1152;
   static constexpr int KSC_MAX = CACHE ? 0 : 224;        // key tiles whose INT8 scales are staged
   static constexpr int OFF_CBAR = OFF_BAR + 512;         // CACHE: key-scale stage barriers
   static constexpr int OFF_KST = OFF_BAR + 1024;         // CACHE: key-scale stages [2][128] fp32
-  static constexpr int MAXW = CACHE ? 32 : 64;           // routing words per query tile kept in smem
+  static constexpr int MAXW = (CACHE || TOKS) ? 32 : 64;  // routing words per query tile kept in smem
+  // TOKS (per-token key scales; fp16 K / V): routing words [2][32] at +256,
+  // seed blocks at +512, and one row of 128 fp32 key scales per softmax
+  // warpgroup at +896, which that warpgroup writes and reads.
+  static constexpr int OFF_KSTT = OFF_BAR + 896;
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S16 = idesc_f16(BM, BN, false);
@@ -134,15 +138,20 @@ struct Cfg2 {
   // control warpgroup keeps 72: 2 * 128 * 216 + 128 * 72 = 384 * 168.  With
   // CACHE: 128 at launch (4 warps per sub-partition), softmax 208, control
   // 48, dequantisation 48: 2 * 128 * 208 + 128 * 48 + 128 * 48 = 512 * 128.
+  // TOKS: softmax 224 (its per-column key-scale multiply), control 56:
+  // 2 * 128 * 224 + 128 * 56 = 384 * 168.
   static constexpr int THREADS = CACHE ? 512 : 384;
-  static constexpr int LAUNCH_REGS = CACHE ? 128 : 168, SOFTMAX_REGS = CACHE ? 208 : 216;
-  static constexpr int CONTROL_REGS = CACHE ? 48 : 72, DEQ_REGS = CACHE ? 48 : 0;
+  static constexpr int LAUNCH_REGS = CACHE ? 128 : 168, SOFTMAX_REGS = CACHE ? 208 : (TOKS ? 224 : 216);
+  static constexpr int CONTROL_REGS = CACHE ? 48 : (TOKS ? 56 : 72), DEQ_REGS = CACHE ? 48 : 0;
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(CACHE ? (OFF_BAR + 256 + 4 * 2 * MAXW <= OFF_CBAR && OFF_CBAR + 8 * 10 <= OFF_SEED &&
                          OFF_SEED + kSeedBytes <= OFF_KST &&
                          OFF_KST + 2 * 128 * 4 <= OFF_BAR + BAR_BYTES)
                       : (OFF_SEED + kSeedBytes <= OFF_KSC && OFF_KSC + 4 * KSC_MAX <= OFF_BAR + BAR_BYTES),
                 "layout");
+  static_assert(!TOKS || (OFF_BAR + 256 + 4 * 2 * MAXW <= OFF_SEED && OFF_SEED + kSeedBytes <= OFF_KSTT &&
+                          OFF_KSTT + 2 * 512 <= OFF_BAR + BAR_BYTES),
+                "per-token key-scale rows");
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS + 128 * DEQ_REGS == THREADS * LAUNCH_REGS,
                 "register split must equal the launch allocation");
   __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
@@ -165,7 +174,8 @@ enum {
 //   NB_KV + t: wait helper (32) <-> issuer t (32): operands landed
 //   NB_START: softmax A (128, arrive) -> issuer B (32, sync), once: P_A(0) stored
 //   NB_DEQ:    the four dequantisation warps (128, CACHE): a tile is written
-enum : int { NB_P = 1, NB_KV = 3, NB_START = 5, NB_DEQ = 6 };
+//   NB_KST + t: softmax warpgroup t (128, TOKS): its key-scale row written / read
+enum : int { NB_P = 1, NB_KV = 3, NB_START = 5, NB_DEQ = 6, NB_KST = 7 };
 // CACHE barriers (at OFF_CBAR): key-scale stage s written (count 128), and
 // read by query tile t (count 4: one arrival per softmax warp); the code
 // tile of a ring slot's next fp16 tile landed (count 1, TMA bytes).
@@ -191,6 +201,10 @@ struct Params2 {
   // CACHE: fp16 scales [T, Hkv] of the K and V cache (the codes come by TMA)
   const __half* k_tok_scale;
   const __half* v_tok_scale;
+  // TOKS: per-token K scales laid out [Hkv][kst_tiles][128] fp32 by key tile
+  // (tiles numbered per key sequence, rows past a sequence's end hold 0)
+  const float* kst_ws;
+  int64_t kst_tiles;
 };
 
 // Routing bit of key tile j (group j / g); row is a shared- or global-memory
@@ -256,14 +270,15 @@ __device__ __forceinline__ void dequant_row_inplace(uint8_t* slot, int r, __half
 // plane and no INT8 plane): the Q8 / K8 maps, tile scales and bitmask are the
 // FP8 ones, and the route's QK^T is four kind::f8f6f4 MMAs with an fp32
 // result (no seed).  Everything else is the INT8 route's.
-template <int D, int EMU, bool DUAL, bool CH, bool CACHE, bool F8 = false>
+template <int D, int EMU, bool DUAL, bool CH, bool CACHE, bool F8 = false, bool TOKS = false>
 __global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmQ8,
                      const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmK8,
                      const __grid_constant__ CUtensorMap tmV16, const Params2 p) {
-  using C = Cfg2<D, CACHE>;
+  using C = Cfg2<D, CACHE, TOKS>;
   static_assert(!CACHE || (DUAL && !CH && D == 128), "the INT8 cache runs in the two-issuer mode, d = 128");
   static_assert(!F8 || (!CACHE && !CH && D == 128), "the FP8 route: d = 128, fp16 K / V, routed launches");
+  static_assert(!TOKS || (!CACHE && !CH && !F8 && D == 128), "per-token key scales: d = 128, routed launches");
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -278,6 +293,7 @@ __global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
   float* ksc = reinterpret_cast<float*>(smem + C::OFF_KSC);                        // [KSC_MAX]
   auto cbar = [&](int i) -> uint32_t { return sbase + C::OFF_CBAR + 8u * static_cast<uint32_t>(i); };
   float* kst = reinterpret_cast<float*>(smem + C::OFF_KST);                        // CACHE: [2][128]
+  float* kstt = reinterpret_cast<float*>(smem + C::OFF_KSTT);                      // TOKS: [2][128]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -386,7 +402,7 @@ __global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
           for (int w = lane; w < p.W; w += 32) route_words[t * C::MAXW + w] = __ldg(ti[t].mrow + w);
     // the INT8 route's key-tile scales (shared by both query tiles), so that
     // no softmax step waits on a global load for them
-    if (!CACHE && (ti[0].mrow != nullptr || ti[1].mrow != nullptr)) {
+    if (!CACHE && !TOKS && (ti[0].mrow != nullptr || ti[1].mrow != nullptr)) {
       const int nst = nJ < C::KSC_MAX ? nJ : C::KSC_MAX;
       for (int j = lane; j < nst; j += 32) ksc[j] = __ldg(p.k_scales + (skq.tile_base + j) * p.Hkv + hk);
     }
@@ -1034,6 +1050,16 @@ __global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
     const SeqInfo sk = seq_info(p.cu_k, b, p.Lk, BN);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    // TOKS: this warpgroup's row of key scales and the next key tile's scale
+    // of column r (loaded one key tile ahead)
+    float* kst_row = kstt + 128 * t;
+    const float* kst_src = TOKS ? p.kst_ws + (static_cast<int64_t>(hk) * p.kst_tiles + sk.tile_base) * 128 + r
+                                : nullptr;
+    float kst_next = 0.f;
+    if (TOKS) {
+      if (T.nJ > 0) kst_row[r] = __ldg(kst_src);
+      if (T.nJ > 1) kst_next = __ldg(kst_src + 128);
+    }
     TM_TRACE_DECL
 #ifndef TM_TRACE_WARP
 #define TM_TRACE_WARP 0
@@ -1159,7 +1185,7 @@ __global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
       const bool i8 = route8(rrow[t], p.g, j);
       float c = p.scale_log2;
       if (i8) {
-        if (CACHE) {
+        if (CACHE || TOKS) {
           c = fmaxf(c8_row, 1e-30f);   // the per-token key scales multiply the scores per column below
         } else {
           const float ks = j < C::KSC_MAX ? ksc[j] : __ldg(p.k_scales + (sk.tile_base + j) * p.Hkv + hk);
@@ -1214,6 +1240,26 @@ __global__ void __launch_bounds__(Cfg2<D, CACHE>::THREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(cbar(CB_KSEMPTY + 2 * ks_stage + t));   // this warp is done with the stage
+      }
+      if constexpr (TOKS) {
+        // Per-token K scales of key tile j, in this warpgroup's row: thread r
+        // wrote scale r during the previous key tile (or before the loop);
+        // the first barrier makes the row visible, the second lets thread r
+        // overwrite its entry with key tile j + 1's scale once every thread
+        // has read the row.  Both run for every key tile, FP16 ones too.
+        named_bar_sync(NB_KST + t, 128);
+        if (i8) {
+          const float4* kp = reinterpret_cast<const float4*>(kst_row);
+#pragma unroll
+          for (int e = 0; e < BN; e += 4) {
+            const float4 kk = kp[e >> 2];
+            f2unpack(f2mul(f2pack(x[e], x[e + 1]), f2pack(kk.x, kk.y)), x[e], x[e + 1]);
+            f2unpack(f2mul(f2pack(x[e + 2], x[e + 3]), f2pack(kk.z, kk.w)), x[e + 2], x[e + 3]);
+          }
+        }
+        named_bar_sync(NB_KST + t, 128);
+        kst_row[r] = kst_next;
+        kst_next = (j + 2 < T.nJ) ? __ldg(kst_src + (j + 2) * 128) : 0.f;
       }
       const int64_t nv64 = lim - static_cast<int64_t>(j) * BN + 1;
       const int nv = nv64 <= 0 ? 0 : (nv64 >= BN ? BN : static_cast<int>(nv64));
@@ -1360,13 +1406,13 @@ std::mutex g_mu2;
 // One-time kernel attributes; the warpgroup register split assumes exactly
 // LAUNCH_REGS per thread at launch (any other allocation could leave
 // setmaxnreg.inc waiting), so a build that differs is refused.
-template <int D, bool DUAL, bool CH, bool CACHE = false, bool F8 = false>
+template <int D, bool DUAL, bool CH, bool CACHE = false, bool F8 = false, bool TOKS = false>
 tm_status prepare_pair_kernel() {
-  using C = Cfg2<D, CACHE>;
+  using C = Cfg2<D, CACHE, TOKS>;
   static bool attr_done = false;
   std::lock_guard<std::mutex> lk(g_mu2);
   if (attr_done) return TM_OK;
-  auto kern = attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, DUAL, CH, CACHE, F8>;
+  auto kern = attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, DUAL, CH, CACHE, F8, TOKS>;
   cudaFuncAttributes fa;
   tm_status st = check_cuda(cudaFuncGetAttributes(&fa, kern));
   if (st != TM_OK) return st;
@@ -1397,19 +1443,23 @@ constexpr int64_t kDualIssuerKeyTiles = 64;
 #endif
 
 // F8: q / k carry the FP8 E4M3 codes and tile scales in their codes / scales
-// fields and bitmask is the FP8 bit plane (d = 128).
-template <int D, bool F8 = false>
+// fields and bitmask is the FP8 bit plane (d = 128).  TOKS: k carries the
+// INT8 cache's K codes (its scales field unused), k / v the cache's fp16 view,
+// and the INT8 route's key scales are per token, from kst_ws laid out
+// [Hkv][kst_tiles][128] fp32 (d = 128, bitmask non-null).
+template <int D, bool F8 = false, bool TOKS = false>
 tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                       const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
                       const uint32_t* bitmask,
-                      int64_t mask_hs, int32_t g, int32_t causal, cudaStream_t stream) {
+                      int64_t mask_hs, int32_t g, int32_t causal, cudaStream_t stream,
+                      const float* kst_ws = nullptr, int64_t kst_tiles = 0) {
   using C = Cfg2<D>;
   const int64_t maxk_tiles = ((cu ? max_k : k->T) + 127) / 128;
   const bool dual = maxk_tiles >= kDualIssuerKeyTiles;
-  const bool chunked = !F8 && dual && D == 128 && TM_PAIR_CHUNKED && bitmask == nullptr;
+  const bool chunked = !F8 && !TOKS && dual && D == 128 && TM_PAIR_CHUNKED && bitmask == nullptr;
   tm_status st = chunked ? prepare_pair_kernel<D, true, true>()
-                         : (dual ? prepare_pair_kernel<D, true, false, false, F8>()
-                                 : prepare_pair_kernel<D, false, false, false, F8>());
+                         : (dual ? prepare_pair_kernel<D, true, false, false, F8, TOKS>()
+                                 : prepare_pair_kernel<D, false, false, false, F8, TOKS>());
   if (st != TM_OK) return st;
   CUtensorMap mQ16, mQ8, mK16, mK8, mV16;
   st = encode_thd_map(&mQ16, q->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q->T, q->H, D, q->stride_t,
@@ -1459,6 +1509,8 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
   p.sched_zero = 0;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   p.err = DevErr{device_error_word()};
+  p.kst_ws = kst_ws;
+  p.kst_tiles = kst_tiles;
   // KV heads per scheduling chunk: as many as keep their K / V (fp16 K, int8
   // K, fp16 V) within ~40 MB of L2, widened until a chunk fills two waves of
   // 148 CTAs; always a divisor of Hkv.
@@ -1477,10 +1529,10 @@ tm_status launch_pair(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v
     attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, true, false>
         <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   else if (dual)
-    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, false, false, F8>
+    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, true, false, false, F8, TOKS>
         <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   else
-    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, false, false, false, F8>
+    attn_pair_kernel<D, TM_EXP2_EMU_PAIRS, false, false, false, F8, TOKS>
         <<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16, p);
   return check_cuda(cudaGetLastError());
 }
@@ -1567,6 +1619,15 @@ tm_status launch_attn_pair_cache(const tm_tensor* q, const tm_tensor* k, const t
                                  int32_t max_k, const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
                                  cudaStream_t stream) {
   return launch_pair_cache(q, k, v, out, cu, cu_k, batch, max_q, max_k, bitmask, mask_hs, g, causal, stream);
+}
+
+tm_status launch_attn_pair_toks(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                                const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
+                                const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
+                                const float* kst_ws, int64_t kst_tiles, cudaStream_t stream) {
+  if (q->d != 128 || bitmask == nullptr || kst_ws == nullptr) return TM_ERR_UNSUPPORTED;
+  return launch_pair<128, false, true>(q, k, v, out, cu, cu_k, batch, max_q, max_k, bitmask, mask_hs, g, causal,
+                                       stream, kst_ws, kst_tiles);
 }
 
 tm_status launch_attn_pair_fp8(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,

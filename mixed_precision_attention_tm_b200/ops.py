@@ -68,6 +68,9 @@ def _lib():
             "tm_build_mask_scale_policy_varlen": (I32, [P, I32, I32, P, P, I32, I32, I32, I32, I32, I32, I32,
                                                         P, P, ctypes.c_float, I32, I32, I64, P]),
             "tm_key_tile_scales": (I32, [P, P, I32, P, I32, I32, I64, I32, P]),
+            "tm_cache_workspace_bytes": (I64, [I64, I32, I32]),
+            "tm_attn_fwd_cache_ws": (I32, [TP, TP, TP, TP, P, P, I32, I32, I32, P, I64, I32, I32, I32, I32, P, I64,
+                                           P]),
             "tm_route_stats": (I32, [P, I64, I32, P, I32, I64, I64, I32, I32, I32, I32,
                                      ctypes.POINTER(D), ctypes.POINTER(D)]),
             "tm_attn_fwd": (I32, [TP, TP, TP, TP, P, I32, I32, P, I64, I32, I32, I32, I32, P]),
@@ -467,11 +470,15 @@ def route_stats(mask_host, *, Hq, tile_m, tile_n, g, causal, Lq=None, Lk=None, c
 # ---------------------------------------------------------------- attention
 def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal=False,
              bitmask=None, mask_head_stride=None, q_quant=None, k_quant=None, kv_cache=None,
-             cu_seqlens=None, max_seqlen=None, cu_seqlens_host=None, cu_seqlens_k=None, max_seqlen_k=None):
+             cu_seqlens=None, max_seqlen=None, cu_seqlens_host=None, cu_seqlens_k=None, max_seqlen_k=None,
+             cache_workspace=None):
     """Fused tile-routed attention.  q: fp16 [Tq,Hq,d]; k, v: fp16 [Tk,Hkv,d]
     (or kv_cache = (k_codes, k_scale16, v_codes, v_scale16)); bitmask: int32
     view [Hm, n_qt, W] (Hm = Hq or 1) or None (all FP16); q_quant / k_quant:
-    (codes, scales) from quantize_qk, needed with a bitmask.  Returns out."""
+    (codes, scales) from quantize_qk, needed with a bitmask.
+    cache_workspace: with kv_cache, a uint8 device tensor of at least
+    cache_workspace_bytes(...) bytes; the cache is then expanded into it once
+    and read from there (tm_attn_fwd_cache_ws).  Returns out."""
     _cuda(q, "q")
     lib = _lib()
     if out is None:
@@ -503,6 +510,21 @@ def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal
                    scale_kind=TM_SCALE_TILE if k_quant is not None else TM_SCALE_NONE)
         vd = _desc(v)
     od = _desc(out)
+    if cache_workspace is not None:
+        if kv_cache is None:
+            raise ValueError("cache_workspace is for an INT8 K/V cache")
+        _cuda(cache_workspace, "cache_workspace")
+        need = cache_workspace_bytes(kshape[0], kshape[1], batch)
+        if cache_workspace.dtype != torch.uint8 or cache_workspace.numel() < need \
+                or not cache_workspace.is_contiguous():
+            raise ValueError(f"cache_workspace: contiguous uint8 of at least {need} bytes expected")
+        st = lib.tm_attn_fwd_cache_ws(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
+                                      _ptr(cu_seqlens), _ptr(cu_seqlens_k), batch, int(max_seqlen or 0),
+                                      int(max_seqlen_k or 0), _ptr(bitmask), int(mask_head_stride or 0), tile_m,
+                                      tile_n, g, int(bool(causal)), _ptr(cache_workspace),
+                                      int(cache_workspace.numel()), _stream())
+        _check(st, "tm_attn_fwd_cache_ws")
+        return out
     if cu_seqlens_k is not None:
         st = lib.tm_attn_fwd_varlen(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
                                     _ptr(cu_seqlens), _ptr(cu_seqlens_k), batch, int(max_seqlen or 0),
@@ -515,6 +537,15 @@ def attn_fwd(q, k=None, v=None, *, out=None, tile_m=128, tile_n=128, g=1, causal
                          int(mask_head_stride or 0), tile_m, tile_n, g, int(bool(causal)), _stream())
     _check(st, "tm_attn_fwd")
     return out
+
+
+def cache_workspace_bytes(Tk, Hkv, batch=0):
+    """Bytes of the workspace tm_attn_fwd_cache_ws needs for a cache of Tk
+    tokens and Hkv heads (batch: sequences, 0 for one without offsets)."""
+    n = int(_lib().tm_cache_workspace_bytes(int(Tk), int(Hkv), int(batch)))
+    if n < 0:
+        raise ValueError("bad cache shape")
+    return n
 
 
 def attn_fwd_fp8(q, k, v, *, bitmask_fp8, qf8_quant, kf8_quant, out=None, g=1, causal=False, bitmask=None,

@@ -14,7 +14,8 @@ import torch
 from mixed_precision_attention_tm_b200 import inputs, ops
 
 DEVICE_CALLS = ("tm_quantize_qk", "tm_quantize_qk_varlen", "tm_quantize_qk_fp8", "tm_build_mask",
-                "tm_build_mask_varlen", "tm_build_mask_scale_policy", "tm_attn_fwd", "tm_attn_fwd_varlen",
+                "tm_build_mask_varlen", "tm_build_mask_scale_policy", "tm_build_mask_scale_policy_varlen",
+                "tm_key_tile_scales", "tm_attn_fwd", "tm_attn_fwd_varlen", "tm_attn_fwd_cache_ws",
                 "tm_attn_fwd_fp8", "tm_merge_head_shards")
 
 
@@ -170,4 +171,4 @@ def test_plans_pass_the_checks(host_lib, plan):
                                         **{x: y for x, y in common.items() if x != "cu_seqlens_k"})
                 sp.load(q, k, v, kv)
                 sp.run_local()
-    assert "tm_attn_fwd" in host_lib.calls or "tm_attn_fwd_varlen" in host_lib.calls
+    assert any(c in host_lib.calls for c in ("tm_attn_fwd", "tm_attn_fwd_varlen", "tm_attn_fwd_cache_ws"))

@@ -17,7 +17,7 @@ import torch
 
 import oracle
 from gpu_helpers import TOL, max_err, oracle_mask, run_gpu, run_oracle, seqs_of
-from mixed_precision_attention_tm_b200 import inputs
+from mixed_precision_attention_tm_b200 import inputs, ops
 
 pytestmark = pytest.mark.gpu
 
@@ -89,6 +89,43 @@ def test_routing_sweep_full_size(p):
 
 def test_varlen_int8_cache_full_size():
     _check(inputs.varlen_int8_cache(), n_random=64)
+
+
+def _check_plan(w, n_random=48):
+    """Full size through the prefill plan exactly as bench.py builds and times
+    it (for an INT8 cache: the cache expanded into the plan's workspace)."""
+    from mixed_precision_attention_tm_b200.api import TileMixPrefill
+    pl = TileMixPrefill(w.Lq, w.Lk, w.hq, w.hkv, w.d, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g,
+                        p=w.p, seed=w.mask_seed, force_diag=w.force_diag, force_sink=w.force_sink,
+                        cu_seqlens=w.cu_seqlens, int8_cache=w.kv_cache is not None, cu_seqlens_k=w.cu_seqlens_k)
+    pl.load(w.q, w.k, w.v, w.kv_cache)
+    out = pl.run().cpu()
+    torch.cuda.synchronize()
+    assert ops.get_device_error() == ops.TM_OK
+    assert torch.isfinite(out).all()
+    cu = None if w.cu_seqlens is None else w.cu_seqlens.tolist()
+    ck = None if w.cu_seqlens_k is None else w.cu_seqlens_k.tolist()
+    seqs = oracle.seq_table(w.Lq, w.Lk, cu, ck)
+    mask_u32 = pl.bitmask.cpu().numpy().view(np.uint32)
+    assert np.array_equal(mask_u32, oracle.build_mask(w.hq, seqs, w.tile_m, w.tile_n, w.g, w.causal, w.p,
+                                                      w.mask_seed, w.force_diag, w.force_sink))
+    rq = oracle.quantize_tiles(w.q.numpy(), seqs, w.tile_m, "q")
+    assert np.array_equal(pl.q_quant[1].cpu().numpy(), rq[1]) and np.array_equal(pl.q_quant[0].cpu().numpy(), rq[0])
+    rows = _sample_rows(seqs, w.tile_m, n_random, 17)
+    ref = oracle.attention(w.q.numpy(), kv_cache=tuple(t.numpy() for t in w.kv_cache), cu_seqlens=cu,
+                           cu_seqlens_k=ck, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n, g=w.g,
+                           mask=mask_u32, q_quant=rq, rows=rows)
+    err = max_err(out, ref, rows=rows)
+    _record(w, f"{len(rows)} sampled rows x all heads (plan, cache workspace)", err, "bit-exact")
+    assert err <= TOL, f"{w.name}: max abs err {err} over {len(rows)} rows"
+
+
+def test_varlen_int8_cache_full_size_through_the_plan():
+    _check_plan(inputs.varlen_int8_cache(), n_random=64)
+
+
+def test_prefix_int8_cache_full_size_through_the_plan():
+    _check_plan(inputs.prefix_int8_cache(), n_random=64)
 
 
 def test_long_context_full_size():

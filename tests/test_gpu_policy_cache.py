@@ -172,7 +172,7 @@ def test_cache_policy_plan_matches_direct_calls():
     pl.load(q, kv_cache=(kc, ks16, vc, vs16))
     out = pl.run().clone()
     torch.cuda.synchronize()
-    assert pl.launches_per_step == 4
+    assert pl.launches_per_step == 5   # quantise Q, key statistic, mask, cache expansion, attention
     cq, ck = torch.tensor(cu_q).cuda(), torch.tensor(cu_k).cuda()
     qc, qs, _, _ = ops.quantize_qk(q.cuda(), None, cu_seqlens=cq)
     kstat = ops.key_tile_scales(ks16.cuda(), tile_n=128, cu_seqlens_k=ck)
@@ -180,6 +180,7 @@ def test_cache_policy_plan_matches_direct_calls():
                                     cu_seqlens=cq, cu_seqlens_k=ck)
     assert torch.equal(pl.bitmask, m)
     kv = tuple(t.cuda() for t in (kc, ks16, vc, vs16))
+    ws = torch.empty_like(pl.cache_ws)
     direct = ops.attn_fwd(q.cuda(), None, None, g=2, causal=True, bitmask=m, q_quant=(qc, qs), kv_cache=kv,
-                          cu_seqlens=cq, cu_seqlens_k=ck)
+                          cu_seqlens=cq, cu_seqlens_k=ck, cache_workspace=ws)
     assert torch.equal(out, direct)

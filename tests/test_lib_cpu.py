@@ -213,7 +213,9 @@ def test_prefill_plan_buffers_match_library_sizes():
     assert pl.k_quant[0].shape == (T, 2, 128) and pl.k_quant[1].shape == (nkt, 2)
     assert pl.bitmask.shape == (8, nqt, oracle.mask_words(max(lens), 128, 2))
     cache = TileMixPrefill(T, T, 8, 2, 128, p=0.5, cu_seqlens=cu, int8_cache=True, device="cpu")
-    assert cache.k_quant is None and cache.launches_per_step == 3
+    # quantise Q, build the mask, expand the cache into the workspace, attend
+    assert cache.k_quant is None and cache.launches_per_step == 4
+    assert cache.cache_ws.numel() == ops.cache_workspace_bytes(T, 2, len(lens))
     plain = TileMixPrefill(256, 256, 8, 2, 128, device="cpu")
     assert plain.bitmask is None and plain.launches_per_step == 1
 
@@ -297,3 +299,22 @@ def test_policy_entries_validate_before_launch():
     assert kts(sc, sc, 2, None, 0, 0, -1, 128, None) == ops.TM_ERR_INVALID_ARG
     # nothing to do: no launch, TM_OK
     assert kts(sc, sc, 2, None, 0, 0, 0, 128, None) == ops.TM_OK
+
+
+def test_cache_workspace_entry_validates_before_launch():
+    """tm_attn_fwd_cache_ws: a null or short workspace, or K / V that are not
+    an INT8 cache, return TM_ERR_INVALID_ARG before any CUDA call."""
+    lib = ops._lib()
+    by = ctypes.byref
+    q, o = _t(d=128), _t(d=128)
+    kc = ops.TmTensor(None, 256, 1, 128, 128, 128, 2 << 20, 3 << 20, ops.TM_SCALE_TOKEN)
+    need = lib.tm_cache_workspace_bytes(256, 1, 0)
+    assert need >= 2 * 256 * 128 * 2 + 2 * 128 * 4
+    P = ctypes.c_void_p
+    call = lambda k, ws, nbytes: lib.tm_attn_fwd_cache_ws(by(q), by(k), by(k), by(o), None, None, 0, 0, 0, None, 0,
+                                                          128, 128, 1, 1, ws, nbytes, None)
+    assert call(kc, None, need) == ops.TM_ERR_INVALID_ARG
+    assert call(kc, P(4 << 20), need - 256) == ops.TM_ERR_INVALID_ARG
+    assert call(kc, P((4 << 20) + 16), need) == ops.TM_ERR_INVALID_ARG      # not 256-byte aligned
+    assert call(_t(H=1, d=128), P(4 << 20), need) == ops.TM_ERR_INVALID_ARG  # fp16 K / V, not a cache
+    assert lib.tm_cache_workspace_bytes(-1, 1, 0) < 0 and lib.tm_cache_workspace_bytes(10, 0, 0) < 0
