@@ -42,30 +42,33 @@ sys.path.insert(0, ROOT)
 from mixed_precision_attention_tm_b200 import dist, inputs  # noqa: E402
 
 PROFILE = os.path.join(ROOT, "profiles", "attn_pair_routing_sweep.md")
+PROFILE_CACHE = os.path.join(ROOT, "profiles", "attn_pair_toks_varlen_int8_cache.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "mixed_precision_attention_tm_b200", "csrc", f)
                   for f in ("tm_attn2.cu", "tm_device.cuh")]
+CACHE_SOURCES = KERNEL_SOURCES + [os.path.join(ROOT, "mixed_precision_attention_tm_b200", "csrc",
+                                               "tm_cache_expand.cu")]
 
 
-def kernel_source_hash():
+def kernel_source_hash(sources=None):
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in (sources or KERNEL_SOURCES):
         with open(f, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
+def profiled_traffic(profile=PROFILE, sources=None):
     """DRAM bytes per attention launch from the committed ncu summary, or
     None when the kernel sources changed since that capture."""
-    if not os.path.exists(PROFILE):
+    if not os.path.exists(profile):
         return None, "no committed capture"
     fields = {}
-    for line in open(PROFILE):
+    for line in open(profile):
         if line.startswith("- ") and ":" in line:
             k, v = line[2:].split(":", 1)
             fields[k.strip().strip("`")] = v.strip().strip("`")
-    if fields.get("kernel_source_sha256") != kernel_source_hash():
+    if fields.get("kernel_source_sha256") != kernel_source_hash(sources):
         return None, "kernel changed since the committed capture"
     try:
         return float(fields["dram_bytes_per_launch"]), fields.get("workload", "")
@@ -422,9 +425,11 @@ def run_ours(args, rank, world, local_rank):
                                           "tile scales written once"}
 
     launches = plan.launches_per_step * K
-    traffic, traffic_note = (None, "traffic captured for the routing-sweep workload only")
+    traffic, traffic_note = (None, "traffic captured for the routing-sweep and INT8-cache workloads only")
     if args.workload == "sweep" and w.p == 0.75:
         traffic, traffic_note = profiled_traffic()
+    elif args.workload == "varlen" and w.p == 0.75:
+        traffic, traffic_note = profiled_traffic(PROFILE_CACHE, CACHE_SOURCES)
     line = {
         "metric": "prefill attention TFLOPS (tile-routed FP16/INT8 QK^T, FP16 P.V)",
         "value": value,
@@ -443,6 +448,9 @@ def run_ours(args, rank, world, local_rank):
         "realised_int8_fraction": e8 / n_vis,
         "visible_pairs": n_vis,
         "attn_ms": attn_ms,
+        "attn_launches": ("cache expansion + attention (the INT8 cache's fp16 view written once into the plan's "
+                          "workspace, then the attention kernel); the roofline charges both"
+                          if getattr(plan, "cache_ws", None) is not None else "attention kernel"),
         "mixed_roofline_frac_of_measured": t_roof / (attn_ms * 1e-3),
         "mixed_roofline_frac_of_nominal": t_roof_nom / (attn_ms * 1e-3),
         "quant_ms": quant_ms,
