@@ -406,7 +406,10 @@ def run_ours(args, rank, world, local_rank):
             "mma_f16_tflops_back_to_back": 2.0 * 128 * 128 * 16 / rates["mma_f16_m128n128k16_cycles"]
                                            * sms * f_hz / 1e12,
             "note": "exp: one exp2 per visible pair; the kernels evaluate 3 of every 8 on the FMA pipe "
-                    "(mufu_share); conversion: one int32->fp32 per INT8-routed pair",
+                    "(mufu_share); conversion: the floor one int32->fp32 per INT8-routed pair would set "
+                    "in the softmax -- the two-tile and one-tile kernels take INT8 scores from the "
+                    "tensor core already in fp32 (exact seed / unseed MMAs) and pay none of it; the "
+                    "64-row kernel and the in-kernel INT8-cache conversion kernel still convert",
         }
     except Exception as exc:                                   # a probe failure must not hide the run
         secondary = {"unavailable": str(exc)}
