@@ -676,9 +676,9 @@ tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor*
   }
   if (tile_m == 128 && tile_n == 128) {
     const int64_t n_qt = ((cu_seqlens ? max_seqlen : q->T) + 127) / 128;
-    if (D == 128 && (TM_SPLIT_KERNEL == 2 ||
-                     (TM_SPLIT_KERNEL == 1 && use_one_tile_kernel(n_qt, cu_seqlens ? batch : 1, q->H,
-                                                                  bitmask != nullptr, causal != 0))))
+    if (TM_SPLIT_KERNEL == 2 ||
+        (TM_SPLIT_KERNEL == 1 && use_one_tile_kernel(n_qt, cu_seqlens ? batch : 1, q->H, bitmask != nullptr,
+                                                     causal != 0)))
       return launch_attn_split(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
                                g, causal, s);
     return launch_attn_pair(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,

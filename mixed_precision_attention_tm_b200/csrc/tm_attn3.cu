@@ -65,11 +65,14 @@ extern "C" int tm_debug_trace_read_split(unsigned long long* host, unsigned int 
 namespace tmk {
 namespace {
 
-template <bool F8>
+template <int D_, bool F8>
 struct Cfg3 {
-  static constexpr int D = 128, BM = 128, BN = 128, HN = 64;   // HN: keys per softmax warpgroup
-  static constexpr int SLOT = BN * D * 2;                       // one fp16 K or V tile (32 KB)
-  static constexpr int NK = F8 ? 2 : 3, NV = 2;                 // K and V ring slots
+  static constexpr int D = D_, BM = 128, BN = 128, HN = 64;     // HN: keys per softmax warpgroup
+  static constexpr int ON = D / 2;                              // O columns per softmax warpgroup
+  static constexpr int SLOT = BN * D * 2;                       // one fp16 K or V tile (32 KB; 16 KB at d = 64)
+  // K and V ring slots: at d = 64 the tiles are half as large and both
+  // rings twice as deep
+  static constexpr int NK = F8 ? 2 : (D == 64 ? 4 : 3), NV = D == 64 ? 4 : 2;
   static constexpr int NSB = 3;                                 // score buffers in TMEM
   static constexpr int Q16_BYTES = BM * D * 2;
   static constexpr int Q8_BYTES = BM * D;
@@ -97,6 +100,10 @@ struct Cfg3 {
   static constexpr uint32_t IDESC_S8 = idesc_i8(BM, BN);
   static constexpr uint32_t IDESC_F8 = idesc_f8_e4m3(BM, BN);
   static constexpr uint32_t IDESC_PV = idesc_f16(BM, D, true);
+  // INT8 / E4M3 code tiles: one D-byte row per key (128-byte swizzle at
+  // d = 128, 64-byte at d = 64)
+  static constexpr uint32_t SW8 = (D == 128) ? kSwizzle128 : kSwizzle64;
+  static constexpr uint32_t SBO8 = (D == 128) ? 1024u : 512u;
   // 8 softmax warps + K producer, issuer, wait helper, V producer.  The
   // register split is the two-tile kernel's: 2 * 128 * 216 + 128 * 72 = 384 * 168.
   static constexpr int THREADS = 384;
@@ -104,6 +111,9 @@ struct Cfg3 {
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS == THREADS * LAUNCH_REGS,
                 "register split must equal the launch allocation");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(D == 64 || D == 128, "head dimension");
+  static_assert(!F8 || D == 128, "the FP8 route is built for d = 128");
+  static_assert(NK <= 4 && NV <= 4, "ring barriers");
   static_assert(OFF_WORDS + 2 * 4 * MAXW <= OFF_SEED && OFF_SEED + kSeedBytes <= OFF_XMAX, "routing words fit");
 };
 
@@ -112,12 +122,12 @@ enum {
   B_SFULL = 1,   // +NSB: S(j) in buffer j mod 3 completed
   B_ODONE = 4,   // +2: P.V(j) completed (barrier j mod 2)
   B_DRAIN = 6,   // every MMA of the CTA completed (one phase)
-  B_KFULL = 7,   // +NK
-  B_KEMPTY = 10, // +NK
-  B_VFULL = 13,  // +NV
-  B_VEMPTY = 15, // +NV
-  B_PREADY = 17, // +NSB: P(j) of buffer j mod 3 stored (one arrival per softmax warp)
-  B_COUNT = 20
+  B_KFULL = 7,   // +NK (<= 4)
+  B_KEMPTY = 11, // +NK
+  B_VFULL = 15,  // +NV (<= 4)
+  B_VEMPTY = 19, // +NV
+  B_PREADY = 23, // +NSB: P(j) of buffer j mod 3 stored (one arrival per softmax warp)
+  B_COUNT = 26
 };
 // Named barriers (0 is __syncthreads):
 //   NB_KV:  wait helper (32) <-> issuer (32): operands (and P) ready
@@ -167,14 +177,14 @@ __device__ __forceinline__ int route_of(const uint32_t* row8, const uint32_t* ro
   return 0;
 }
 
-template <int EMU, bool F8>
+template <int D, int EMU, bool F8>
 __global__ void __launch_bounds__(384, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmQ8,
                       const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmK8,
                       const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmQF8,
                       const __grid_constant__ CUtensorMap tmKF8, const Params3 p) {
-  using C = Cfg3<F8>;
-  constexpr int D = C::D, BN = C::BN, HN = C::HN;
+  using C = Cfg3<D, F8>;
+  constexpr int BN = C::BN, HN = C::HN, ON = C::ON;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
@@ -392,8 +402,8 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t qa = sbase + (rt == 1 ? C::OFF_Q8 : C::OFF_QF8);
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk) {
-              ad[kk] = smem_desc(qa + kk * 32, 16, 1024, kSwizzle128);
-              bd[kk] = smem_desc(kb + kk * 32, 16, 1024, kSwizzle128);
+              ad[kk] = smem_desc(qa + kk * 32, 16, C::SBO8, C::SW8);
+              bd[kk] = smem_desc(kb + kk * 32, 16, C::SBO8, C::SW8);
             }
             if (elect_one()) {
               if (F8 && rt == 2) {
@@ -511,7 +521,7 @@ __global__ void __launch_bounds__(384, 1)
     const int hw = warp >> 2;
     const int r = threadIdx.x & 127;                 // row in the tile = TMEM lane
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t o_addr = lane_addr + C::O_COL + HN * hw;   // this warpgroup's half of O's columns
+    const uint32_t o_addr = lane_addr + C::O_COL + ON * hw;   // this warpgroup's half of O's columns
     const bool row_ok = r < rows;
     const int64_t i_row = r0 + r;
     int64_t lim = -1;
@@ -609,20 +619,20 @@ __global__ void __launch_bounds__(384, 1)
           if (!mbar_wait(bar(B_ODONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.err, abort_flag)) ok = false;
           tc_fence_after();
           __syncwarp();
-          uint32_t o[HN];
+          uint32_t o[ON];
 #pragma unroll
-          for (int cc = 0; cc < HN / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
-          tmem_wait_ld_regs<HN>(o);
+          for (int cc = 0; cc < ON / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
+          tmem_wait_ld_regs<ON>(o);
           const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
-          for (int e = 0; e < HN; e += 2) {
+          for (int e = 0; e < ON; e += 2) {
             float o0, o1;
             f2unpack(f2mul(f2pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), o0, o1);
             o[e] = __float_as_uint(o0);
             o[e + 1] = __float_as_uint(o1);
           }
 #pragma unroll
-          for (int cc = 0; cc < HN / 32; ++cc) tmem_st32p(o_addr + cc * 32, o + cc * 32);
+          for (int cc = 0; cc < ON / 32; ++cc) tmem_st32p(o_addr + cc * 32, o + cc * 32);
         }
       }
       tmem_wait_st();
@@ -652,19 +662,19 @@ __global__ void __launch_bounds__(384, 1)
     const float lsum = xs[r] + xs[128 + r];
     const float inv = (m_used != -INFINITY && lsum > 0.f) ? 1.f / lsum : 0.f;
     __syncwarp();
-    uint32_t o[HN];
+    uint32_t o[ON];
     if (__all_sync(0xffffffffu, have_o)) {
 #pragma unroll
-      for (int cc = 0; cc < HN / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
-      tmem_wait_ld_regs<HN>(o);
+      for (int cc = 0; cc < ON / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
+      tmem_wait_ld_regs<ON>(o);
     } else {
 #pragma unroll
-      for (int e = 0; e < HN; ++e) o[e] = 0u;
+      for (int e = 0; e < ON; ++e) o[e] = 0u;
     }
     if (row_ok) {
-      __half* orow = p.out + (row0 + r) * p.out_st + static_cast<int64_t>(h) * p.out_sh + HN * hw;
+      __half* orow = p.out + (row0 + r) * p.out_st + static_cast<int64_t>(h) * p.out_sh + ON * hw;
 #pragma unroll
-      for (int cc = 0; cc < HN / 8; ++cc) {
+      for (int cc = 0; cc < ON / 8; ++cc) {
         uint4 pkt;
         pkt.x = pack_half2(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv);
         pkt.y = pack_half2(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv);
@@ -693,32 +703,30 @@ std::mutex g_mu3;
 
 // One-time kernel attributes; the warpgroup register split assumes exactly
 // LAUNCH_REGS per thread at launch, so a build that differs is refused.
-template <bool F8>
+template <int D, bool F8>
 tm_status prepare_split_kernel() {
   static bool attr_done = false;
   std::lock_guard<std::mutex> lk(g_mu3);
   if (attr_done) return TM_OK;
-  auto kern = attn_split_kernel<TM_EXP2_EMU_PAIRS, F8>;
+  auto kern = attn_split_kernel<D, TM_EXP2_EMU_PAIRS, F8>;
   cudaFuncAttributes fa;
   tm_status st = check_cuda(cudaFuncGetAttributes(&fa, kern));
   if (st != TM_OK) return st;
-  if (fa.numRegs != Cfg3<F8>::LAUNCH_REGS) return TM_ERR_UNSUPPORTED;
-  st = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg3<F8>::SMEM_BYTES));
+  if (fa.numRegs != Cfg3<D, F8>::LAUNCH_REGS) return TM_ERR_UNSUPPORTED;
+  st = check_cuda(
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg3<D, F8>::SMEM_BYTES));
   if (st != TM_OK) return st;
   attr_done = true;
   return TM_OK;
 }
 
-}  // namespace
-
-tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
-                            const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
-                            const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
-                            cudaStream_t stream, const Fp8Route* f8) {
-  constexpr int D = 128;
-  if (q->d != D) return TM_ERR_UNSUPPORTED;
-  const bool use_f8 = f8 != nullptr && f8->bitmask != nullptr;
-  tm_status st = use_f8 ? prepare_split_kernel<true>() : prepare_split_kernel<false>();
+template <int D>
+tm_status launch_split(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                       const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
+                       const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
+                       cudaStream_t stream, const Fp8Route* f8) {
+  const bool use_f8 = D == 128 && f8 != nullptr && f8->bitmask != nullptr;
+  tm_status st = use_f8 ? prepare_split_kernel<128, true>() : prepare_split_kernel<D, false>();
   if (st != TM_OK) return st;
   CUtensorMap mQ16, mQ8, mK16, mK8, mV16, mQF8, mKF8;
   st = encode_thd_map(&mQ16, q->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, q->T, q->H, D, q->stride_t,
@@ -730,12 +738,13 @@ tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_ten
   st = encode_thd_map(&mV16, v->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, v->T, v->H, D, v->stride_t,
                       v->stride_h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != TM_OK) return st;
+  const CUtensorMapSwizzle swz8 = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if (bitmask != nullptr) {
     st = encode_thd_map(&mQ8, q->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q->T, q->H, D, q->H * D, D, D, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+                        swz8);
     if (st != TM_OK) return st;
     st = encode_thd_map(&mK8, k->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k->T, k->H, D, k->H * D, D, D, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+                        swz8);
     if (st != TM_OK) return st;
   } else {
     mQ8 = mQ16;
@@ -794,14 +803,28 @@ tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_ten
   if (grid == 0) return TM_OK;
   if (grid > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
   if (use_f8)
-    attn_split_kernel<TM_EXP2_EMU_PAIRS, true><<<static_cast<unsigned>(grid), Cfg3<true>::THREADS,
-                                                 Cfg3<true>::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16,
-                                                                                   mQF8, mKF8, p);
+    attn_split_kernel<128, TM_EXP2_EMU_PAIRS, true><<<static_cast<unsigned>(grid), Cfg3<128, true>::THREADS,
+                                                      Cfg3<128, true>::SMEM_BYTES, stream>>>(
+        mQ16, mQ8, mK16, mK8, mV16, mQF8, mKF8, p);
   else
-    attn_split_kernel<TM_EXP2_EMU_PAIRS, false><<<static_cast<unsigned>(grid), Cfg3<false>::THREADS,
-                                                  Cfg3<false>::SMEM_BYTES, stream>>>(mQ16, mQ8, mK16, mK8, mV16,
-                                                                                     mQF8, mKF8, p);
+    attn_split_kernel<D, TM_EXP2_EMU_PAIRS, false><<<static_cast<unsigned>(grid), Cfg3<D, false>::THREADS,
+                                                    Cfg3<D, false>::SMEM_BYTES, stream>>>(
+        mQ16, mQ8, mK16, mK8, mV16, mQF8, mKF8, p);
   return check_cuda(cudaGetLastError());
+}
+
+}  // namespace
+
+tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
+                            const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
+                            const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,
+                            cudaStream_t stream, const Fp8Route* f8) {
+  const bool use_f8 = f8 != nullptr && f8->bitmask != nullptr;
+  if (q->d == 128)
+    return launch_split<128>(q, k, v, out, cu, cu_k, batch, max_q, max_k, bitmask, mask_hs, g, causal, stream, f8);
+  if (q->d == 64 && !use_f8)
+    return launch_split<64>(q, k, v, out, cu, cu_k, batch, max_q, max_k, bitmask, mask_hs, g, causal, stream, f8);
+  return TM_ERR_UNSUPPORTED;
 }
 
 }  // namespace tmk
