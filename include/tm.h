@@ -94,7 +94,8 @@ typedef struct {
  * dense [Tq, Hq, d]; q_scales: fp32 [n_qtiles, Hq].  Same for k with tile_n
  * into k_codes [Tk, Hkv, d] / k_scales [n_ktiles, Hkv]; k may be NULL (Q only;
  * used with an INT8 K/V cache).  Code rows outside every sequence are not
- * written.  tile_m, tile_n in {64, 128}.
+ * written.  tile_m, tile_n in {64, 128}.  A sequence of more than 65535
+ * tiles (over 8.3 M rows at 128-row tiles) returns TM_ERR_UNSUPPORTED.
  * Results are bit-identical to the definition above (no contraction of the
  * division, round-to-nearest-even conversion).
  * ------------------------------------------------------------------------- */

@@ -12,10 +12,11 @@
 // between the absmax pass and the quantise pass, so HBM traffic is one read
 // of x plus one write of the codes (bytes per element: 2 read + 1 written).
 // The scale is the IEEE round-to-nearest __fdiv_rn of amax by 127.  A code is
-// formed from x times the correctly rounded reciprocal of the scale, with an
-// exact guard: only an element whose product lies within 2^-15 of a
-// half-integer takes the IEEE division, so the codes are bit-identical to
-// the definition (see int8_code).
+// formed from x times the correctly rounded reciprocal of the scale, rounded
+// by the packed fp32 add of 1.5 * 2^23, with an exact guard: only a vector
+// holding a product within 2^-15 of a half-integer takes the IEEE division,
+// so the codes are bit-identical to the definition (see int8_code and
+// int8_codes8).
 //
 // FP8 (the third precision; per-axis fp8 scales: "Add rowwise scaling to
 // Float8Inference module" page, Summary): s = fl32(amax / 448), 448 being the
@@ -69,13 +70,52 @@ struct QuantOperand {
   int nb;      // sequences
 };
 
-// One CTA per (tile, sequence, head) of either operand: grid.z runs over the
-// heads of operand 0 and then those of operand 1.  The tile's rows x d fp16
+// INT8 codes of 8 fp16 values (one 16-byte vector) for a tile scale s > 0
+// with r = 1/s correctly rounded, packed little-endian into two words.  Pairs
+// of values go through the packed fp32 pipe: v = fl32(x * r); rne(v) by
+// adding and subtracting 1.5 * 2^23 (exact for |v| < 2^22, so the sum's low
+// byte is the two's-complement code and no float-to-int conversion runs);
+// the same near-tie guard as int8_code, taken per vector when any of its
+// eight values is within 2^-15 of a half-integer.
+__device__ __forceinline__ void int8_codes8(const __half2* hv, float s, float r, uint32_t& w0, uint32_t& w1) {
+  const uint64_t r2 = f2pack(r, r);
+  const uint64_t mg = f2pack(12582912.0f, 12582912.0f), nmg = f2pack(-12582912.0f, -12582912.0f);
+  uint32_t tb[8];
+  float dmax = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(hv[e]);
+    const uint64_t v2 = f2mul(f2pack(f.x, f.y), r2);
+    const uint64_t t2 = f2add(v2, mg);
+    const uint64_t n2 = f2add(t2, nmg);
+    float v0, v1, n0, n1, t0, t1;
+    f2unpack(v2, v0, v1);
+    f2unpack(n2, n0, n1);
+    f2unpack(t2, t0, t1);
+    dmax = fmaxf(dmax, fmaxf(fabsf(v0 - n0), fabsf(v1 - n1)));
+    tb[2 * e] = __float_as_uint(t0);
+    tb[2 * e + 1] = __float_as_uint(t1);
+  }
+  if (dmax > 0.5f - 0x1p-15f) {   // a near tie: the IEEE division decides every value of the vector
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x = (e & 1) ? __high2float(hv[e >> 1]) : __low2float(hv[e >> 1]);
+      tb[e] = static_cast<uint32_t>(int8_code(x, s, r));
+    }
+  }
+  w0 = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
+  w1 = __byte_perm(__byte_perm(tb[4], tb[5], 0x0040), __byte_perm(tb[6], tb[7], 0x0040), 0x5410);
+}
+
+// One CTA per (head, tile, sequence) of either operand: grid.x runs over the
+// heads of operand 0 and then those of operand 1 (heads fastest, so that the
+// CTAs running at once read and write whole token rows of Q and K, all heads
+// side by side).  The tile's rows x d fp16
 // values are read once with 16-byte loads and kept in registers between the
 // absmax pass and the quantise pass, so HBM traffic is one read of x plus one
 // write of the codes.
 template <int D, bool F8>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 4)
     quantize_tiles_kernel(const QuantOperand op0, const QuantOperand op1, DevErr err) {
   constexpr int VPR = D / 8;                       // 16-byte vectors per row
   constexpr int MAXV = 128 * VPR / kQuantThreads;  // vectors per thread at tile = 128
@@ -83,9 +123,9 @@ __global__ void __launch_bounds__(kQuantThreads)
   __shared__ SeqInfo sinfo;
   __shared__ float s_scale;
 
-  const bool second = static_cast<int>(blockIdx.z) >= op0.H;
+  const bool second = static_cast<int>(blockIdx.x) >= op0.H;
   const QuantOperand& o = second ? op1 : op0;
-  const int I = blockIdx.x, b = blockIdx.y, h = second ? blockIdx.z - op0.H : blockIdx.z;
+  const int I = blockIdx.y, b = blockIdx.z, h = second ? blockIdx.x - op0.H : blockIdx.x;
   if (I >= o.ntile || b >= o.nb) return;
   if (threadIdx.x == 0) {
     sinfo = seq_info(o.cu, b, o.L, o.tile);
@@ -146,11 +186,7 @@ __global__ void __launch_bounds__(kQuantThreads)
             packed[e >> 2] |= pr << (8 * (e & 3));
           }
         } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float f = (e & 1) ? __high2float(hv[e >> 1]) : __low2float(hv[e >> 1]);
-            packed[e >> 2] |= (static_cast<uint32_t>(int8_code(f, sc, rc)) & 0xFFu) << (8 * (e & 3));
-          }
+          int8_codes8(hv, sc, rc, packed[0], packed[1]);
         }
       }
       uint8_t* dst = o.codes + (sq.start + r0 + row) * code_row_stride + static_cast<int64_t>(h) * D + c * 8;
@@ -217,7 +253,8 @@ tm_status launch_quant(const tm_tensor* x, void* x_codes, float* x_scales, const
   if (heads > 65535) return TM_ERR_UNSUPPORTED;
   const int gx = max(empty[0] ? 0 : o[0].ntile, empty[1] ? 0 : o[1].ntile);
   const int gy = max(empty[0] ? 0 : o[0].nb, empty[1] ? 0 : o[1].nb);
-  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(heads));
+  if (gx > 65535) return TM_ERR_UNSUPPORTED;   // tiles per sequence on grid.y
+  dim3 grid(static_cast<unsigned>(heads), static_cast<unsigned>(gx), static_cast<unsigned>(gy));
   DevErr err{device_error_word()};
   const int64_t d = x->d;
   if (d == 128 && f8)
