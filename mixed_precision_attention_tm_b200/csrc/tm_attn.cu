@@ -63,9 +63,15 @@ int device_sms() {
 // already balance their waves by running the longest query tiles first).
 std::atomic<int> g_attn_kernel{0};   // tm_set_attn_kernel
 
-bool use_one_tile_kernel(int64_t n_qt, int64_t batch, int64_t hq, bool routed, bool causal) {
+bool use_one_tile_kernel(int64_t n_qt, int64_t batch, int64_t hq, bool routed, bool causal, int64_t d = 128) {
   const int choice = g_attn_kernel.load(std::memory_order_relaxed);
   if (choice != 0) return choice == 2;
+  // At d = 64 a tile's MMAs are half as long while its softmax costs the
+  // same, so the two-tile kernel's chain (softmax, P.V, next QK^T) leaves
+  // the softmax waiting; the one-tile kernel's three score buffers keep it
+  // busy.  Measured on the 24 MLX-shaped d = 64 runs: equal or faster on 21
+  // (up to 1.8x), at most 7 % slower on 3.
+  if (d == 64) return true;
   const int64_t sms = device_sms();
   const int64_t pair_ctas = (n_qt + 1) / 2 * batch * hq, one_ctas = n_qt * batch * hq;
   if (pair_ctas < sms) return true;
@@ -678,7 +684,7 @@ tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor*
     const int64_t n_qt = ((cu_seqlens ? max_seqlen : q->T) + 127) / 128;
     if (TM_SPLIT_KERNEL == 2 ||
         (TM_SPLIT_KERNEL == 1 && use_one_tile_kernel(n_qt, cu_seqlens ? batch : 1, q->H, bitmask != nullptr,
-                                                     causal != 0)))
+                                                     causal != 0, D)))
       return launch_attn_split(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
                                g, causal, s);
     return launch_attn_pair(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
