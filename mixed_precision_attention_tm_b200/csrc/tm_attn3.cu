@@ -1,5 +1,5 @@
 // tm_attn3.cu -- fused tile-routed attention, one 128-row query tile per CTA
-// with three score buffers in TMEM (d = 128, 128-key tiles).
+// with three score buffers in TMEM (d = 128 or 64, 128-key tiles).
 //
 // TileMix (Lattice paper page), abstract: score tiles routed per group of g
 // key tiles to an FP16 or an INT8 QK^T, both feeding one online-softmax state.
@@ -10,19 +10,30 @@
 // its probabilities P share TMEM columns, a query tile runs the chain
 //     softmax(j) -> P.V(j) -> QK^T(j+1) -> softmax(j+1)
 // and pays that latency once per key tile.  Here the 512 TMEM columns hold
-// the fp32 accumulator O (128 columns) and three score buffers, so the tensor
-// pipe computes QK^T(j+1) and QK^T(j+2) ahead while the softmax works on S(j):
+// the fp32 accumulator O (128 columns; two of 64 at d = 64) and three score
+// buffers, so the tensor pipe computes QK^T(j+1) and QK^T(j+2) ahead while
+// the softmax works on S(j):
 //
-//   * S(j) goes to buffer j mod 3.  The keys of each score tile are split
-//     between two softmax warpgroups (one query row per thread): warpgroup h
-//     (warps 4h .. 4h+3) owns keys [64h, 64h+64).  The two exchange their
-//     row maxima of the tile through shared memory, so both rescale against
-//     one running max m (raised lazily, kLazyRescaleLog2), each sums its
-//     half of the row sum, and each rescales its half of O's columns;
-//   * each warpgroup overwrites the first half of its 64 score columns with
-//     its P as fp16; once both have, P.V(j) is one group of eight MMAs into
-//     O, and QK^T(j+3) follows it into the same buffer (the tensor pipe runs
-//     them in order);
+//   * S(j) goes to buffer j mod 3.  At d = 128 the keys of each score tile
+//     are split between two softmax warpgroups (one query row per thread):
+//     warpgroup h (warps 4h .. 4h+3) owns keys [64h, 64h+64).  The two
+//     exchange their row maxima of the tile through shared memory, so both
+//     rescale against one running max m (raised lazily, kLazyRescaleLog2),
+//     each sums its half of the row sum, and each rescales its half of O's
+//     columns;
+//   * at d = 64 (dual stream) warpgroup h instead takes whole score tiles,
+//     those with j mod 2 == h, and keeps its own running max, row sum and O
+//     (O of warpgroup h in TMEM columns [64h, 64h+64)); the epilogue merges
+//     the two streams.  No maxima are exchanged per tile and the two
+//     warpgroups do not run in lockstep: while one waits for its next
+//     scores, the other computes, so the MUFU / FMA pipes stay busy.  (At
+//     d = 128 two O accumulators and three score buffers would need 640 of
+//     the 512 TMEM columns.)
+//   * each warpgroup overwrites the first half of its score columns with
+//     its P as fp16; once the tile's P is complete, P.V(j) is one group of
+//     eight MMAs into O (dual stream: into the O of warpgroup j mod 2), and
+//     QK^T(j+3) follows it into the same buffer (the tensor pipe runs them
+//     in order);
 //   * K and V reach shared memory through two rings of 32 KB slots (three K
 //     slots holding the int8 or the fp16 K tile by route, two V slots), each
 //     slot released by a tcgen05.commit once the MMAs reading it completed,
@@ -67,8 +78,15 @@ namespace {
 
 template <int D_, bool F8>
 struct Cfg3 {
-  static constexpr int D = D_, BM = 128, BN = 128, HN = 64;     // HN: keys per softmax warpgroup
-  static constexpr int ON = D / 2;                              // O columns per softmax warpgroup
+  // DS (dual stream, d = 64): warpgroup h takes the whole key tiles j with
+  // j mod 2 == h, each warpgroup with its own running max, row sum and O
+  // (two 64-column accumulators), merged in the epilogue.  At d = 128 two O
+  // accumulators and three score buffers would need 640 TMEM columns.
+  static constexpr bool DS = D_ == 64;
+  static constexpr int D = D_, BM = 128, BN = 128;
+  static constexpr int HN = DS ? 128 : 64;                      // keys per softmax warpgroup and tile
+  static constexpr int ON = DS ? D : D / 2;                     // O columns each softmax warpgroup rescales
+  static constexpr int EN = D / 2;                              // output columns each softmax warpgroup writes
   static constexpr int SLOT = BN * D * 2;                       // one fp16 K or V tile (32 KB; 16 KB at d = 64)
   // K and V ring slots: at d = 64 the tiles are half as large and both
   // rings twice as deep
@@ -94,7 +112,7 @@ struct Cfg3 {
   static constexpr int MAXW = 64;                               // routing words kept in shared memory
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t O_COL = 0;
+  static constexpr uint32_t O_COL = 0;                          // d = 128: one O; DS: O of warpgroup h at 64 h
   static constexpr uint32_t S_COL = 128;                        // + 128 buffer
   static constexpr uint32_t IDESC_S16 = idesc_f16(BM, BN, false);
   static constexpr uint32_t IDESC_S8 = idesc_i8(BM, BN);
@@ -184,7 +202,7 @@ __global__ void __launch_bounds__(384, 1)
                       const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmQF8,
                       const __grid_constant__ CUtensorMap tmKF8, const Params3 p) {
   using C = Cfg3<D, F8>;
-  constexpr int BN = C::BN, HN = C::HN, ON = C::ON;
+  constexpr int BN = C::BN, HN = C::HN, ON = C::ON, EN = C::EN;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
@@ -259,7 +277,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_VEMPTY + s), 1);
     }
-    for (int i = 0; i < C::NSB; ++i) mbar_init(bar(B_PREADY + i), 8);
+    for (int i = 0; i < C::NSB; ++i) mbar_init(bar(B_PREADY + i), C::DS ? 4 : 8);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -440,13 +458,18 @@ __global__ void __launch_bounds__(384, 1)
           uint64_t bd[8];
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            // keys 16kk .. 16kk+15: P of warpgroup kk / 4 at its columns
-            at[kk] = d_s + (kk >> 2) * HN + (kk & 3) * 8;
+            // keys 16kk .. 16kk+15: DS, P of the tile's warpgroup in its first
+            // 64 columns; otherwise P of warpgroup kk / 4 at its columns
+            at[kk] = C::DS ? d_s + kk * 8 : d_s + (kk >> 2) * HN + (kk & 3) * 8;
             bd[kk] = smem_desc(vb + kk * 2048, C::HALF, 1024, kSwizzle128);
           }
+          // DS: P.V(j) accumulates into the O of warpgroup j mod 2, which its
+          // first tile (j < 2) initialises
+          const uint32_t d_o = tmem + C::O_COL + (C::DS ? static_cast<uint32_t>(D * (j & 1)) : 0u);
+          const uint32_t acc = (C::DS ? j > 1 : j > 0) ? 1u : 0u;
           tc_fence_after();   // orders the softmax warps' TMEM stores of P before the MMAs read it
           if (elect_one()) {
-            mma_f16_ts_n<8>(tmem + C::O_COL, at, bd, C::IDESC_PV, j > 0 ? 1u : 0u);
+            mma_f16_ts_n<8>(d_o, at, bd, C::IDESC_PV, acc);
             tc_commit(bar(B_ODONE + (j & 1)));
             tc_commit(bar(B_VEMPTY + vs));
           }
@@ -521,7 +544,7 @@ __global__ void __launch_bounds__(384, 1)
     const int hw = warp >> 2;
     const int r = threadIdx.x & 127;                 // row in the tile = TMEM lane
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t o_addr = lane_addr + C::O_COL + ON * hw;   // this warpgroup's half of O's columns
+    const uint32_t o_addr = lane_addr + C::O_COL + ON * hw;   // this warpgroup's O (DS) or half of O's columns
     const bool row_ok = r < rows;
     const int64_t i_row = r0 + r;
     int64_t lim = -1;
@@ -533,9 +556,12 @@ __global__ void __launch_bounds__(384, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     TM3_PH_DECL
-    for (int j = 0; j < nJ; ++j) {
+    // DS: this warpgroup's key tiles are j = hw, hw + 2, ...; otherwise every
+    // key tile, keys [64 hw, 64 hw + 64)
+    const int key_off = C::DS ? 0 : HN * hw;
+    for (int j = C::DS ? hw : 0; j < nJ; j += C::DS ? 2 : 1) {
       const int sb = j % C::NSB;
-      const uint32_t s_addr = lane_addr + C::S_COL + 128u * sb + HN * hw;
+      const uint32_t s_addr = lane_addr + C::S_COL + 128u * sb + key_off;
       const int rt = route_of<F8>(rrow, rrowf8, p.g, j);
       const bool i8 = rt == 1;   // INT8 and FP8 scores arrive in fp32 (see mma_i8_exact_n)
       float c = p.scale_log2;
@@ -561,19 +587,25 @@ __global__ void __launch_bounds__(384, 1)
         for (int e = 0; e < HN; ++e) x[e] = __uint_as_float(u[e]);
       }
       TM3_PH(1);
-      const int64_t nv64 = lim - (static_cast<int64_t>(j) * BN + HN * hw) + 1;
+      const int64_t nv64 = lim - (static_cast<int64_t>(j) * BN + key_off) + 1;
       const int nv = nv64 <= 0 ? 0 : (nv64 >= HN ? HN : static_cast<int>(nv64));
       if (!__all_sync(0xffffffffu, nv == HN)) {
 #pragma unroll
         for (int e = 0; e < HN; ++e) x[e] = (e < nv) ? x[e] : -INFINITY;
       }
-      // row max of the tile in log2 units, over both warpgroups' keys
+      // row max of the tile in log2 units (-inf when no key is visible); but
+      // in DS, over both warpgroups' keys
       {
-        float* xm = xmax + (j & 1) * 256;
-        xm[hw * 128 + r] = row_max<HN>(x) * c;   // -inf when no key of this half is visible
-        __syncwarp();
-        named_bar_sync(NB_MAX, 256);
-        const float mt = fmaxf(xm[r], xm[128 + r]);
+        float mt;
+        if constexpr (C::DS) {
+          mt = row_max<HN>(x) * c;
+        } else {
+          float* xm = xmax + (j & 1) * 256;
+          xm[hw * 128 + r] = row_max<HN>(x) * c;   // -inf when no key of this half is visible
+          __syncwarp();
+          named_bar_sync(NB_MAX, 256);
+          mt = fmaxf(xm[r], xm[128 + r]);
+        }
         float alpha = 1.f;
         if (mt > m_used + kLazyRescaleLog2) {
           alpha = ex2_approx(m_used - mt);
@@ -608,15 +640,20 @@ __global__ void __launch_bounds__(384, 1)
         }
         TM3_PH(3);
         __syncwarp();
-        tmem_st32p(s_addr, pk);   // P_hw(j) over the first 32 columns of this warpgroup's scores
-        // This warpgroup's half of O is rescaled only when a row of this warp
-        // raised the running max.  Then P.V(j-1) must have completed: S(j)
-        // was issued after P.V(j-3) and has completed, so of the barrier
-        // P.V(j-1) commits to (j-1 mod 2) the previous phase, P.V(j-3), is
-        // done and the next, P.V(j+1), cannot be: the parity wait is
-        // unambiguous.
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          if (!mbar_wait(bar(B_ODONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.err, abort_flag)) ok = false;
+        // P_hw(j) over the first HN / 2 columns of this warpgroup's scores
+#pragma unroll
+        for (int cc = 0; cc < HN / 64; ++cc) tmem_st32p(s_addr + cc * 32, pk + cc * 32);
+        // This warpgroup's O columns are rescaled only when a row of this warp
+        // raised the running max.  Then the previous P.V into them, P.V(jp)
+        // with jp = j - 2 (DS) or j - 1, must have completed.  It commits to
+        // barrier jp mod 2, whose phases are P.V(jp mod 2), P.V(jp mod 2 + 2),
+        // ...  S(j) was issued after P.V(j-3) and has completed, so P.V(jp-2)
+        // is done; P.V(jp+2) cannot be, as the issuer takes P(jp+2) (DS: P(j);
+        // otherwise P(j+1)) only after this warpgroup signals it at the end of
+        // this step or a later one: the parity wait is unambiguous.
+        const int jp = j - (C::DS ? 2 : 1);
+        if (jp >= 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (!mbar_wait(bar(B_ODONE + (jp & 1)), (jp >> 1) & 1, p.err, abort_flag)) ok = false;
           tc_fence_after();
           __syncwarp();
           uint32_t o[ON];
@@ -649,7 +686,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     __syncwarp();
 #endif
-    // ---- epilogue: row sum over both warpgroups, this warpgroup's columns of O
+    // ---- epilogue: row sums over both warpgroups (DS: and the two streams'
+    // maxima), then this warpgroup's EN output columns
     bool have_o = false;
     if (ok && nJ > 0) {
       have_o = mbar_wait(bar(B_DRAIN), 0, p.err, abort_flag);
@@ -657,24 +695,56 @@ __global__ void __launch_bounds__(384, 1)
     }
     float* xs = xmax + 512;   // past both iterations' maxima
     xs[hw * 128 + r] = l;
+    if constexpr (C::DS) xmax[hw * 128 + r] = m_used;
     __syncwarp();
     named_bar_sync(NB_EPI, 256);
-    const float lsum = xs[r] + xs[128 + r];
-    const float inv = (m_used != -INFINITY && lsum > 0.f) ? 1.f / lsum : 0.f;
+    // DS: stream w contributes a_w * O_w and a_w * l_w with a_w = 2^(m_w - m),
+    // m the larger running max; a stream without a visible key (m_w = -inf)
+    // contributes nothing
+    float a0 = 1.f, a1 = 0.f, inv;
+    if constexpr (C::DS) {
+      const float m0 = xmax[r], m1 = xmax[128 + r];
+      const float mm = fmaxf(m0, m1);
+      a0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
+      a1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
+      const float lsum = xs[r] * a0 + xs[128 + r] * a1;
+      inv = (mm != -INFINITY && lsum > 0.f) ? 1.f / lsum : 0.f;
+    } else {
+      const float lsum = xs[r] + xs[128 + r];
+      inv = (m_used != -INFINITY && lsum > 0.f) ? 1.f / lsum : 0.f;
+    }
     __syncwarp();
-    uint32_t o[ON];
+    const uint32_t e_addr = lane_addr + C::O_COL + EN * hw;
+    uint32_t o[EN];
     if (__all_sync(0xffffffffu, have_o)) {
 #pragma unroll
-      for (int cc = 0; cc < ON / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
-      tmem_wait_ld_regs<ON>(o);
+      for (int cc = 0; cc < EN / 32; ++cc) tmem_ld32p(e_addr + cc * 32, o + cc * 32);
+      if constexpr (C::DS) {
+        // the same columns of stream 1's O (written only when nJ > 1)
+        uint32_t o1[EN];
+        if (nJ > 1) {
+#pragma unroll
+          for (int cc = 0; cc < EN / 32; ++cc) tmem_ld32p(e_addr + D + cc * 32, o1 + cc * 32);
+          tmem_wait_ld_regs<EN>(o1);
+        } else {
+#pragma unroll
+          for (int e = 0; e < EN; ++e) o1[e] = 0u;
+        }
+        tmem_wait_ld_regs<EN>(o);
+#pragma unroll
+        for (int e = 0; e < EN; ++e)
+          o[e] = __float_as_uint(__uint_as_float(o[e]) * a0 + __uint_as_float(o1[e]) * a1);
+      } else {
+        tmem_wait_ld_regs<EN>(o);
+      }
     } else {
 #pragma unroll
-      for (int e = 0; e < ON; ++e) o[e] = 0u;
+      for (int e = 0; e < EN; ++e) o[e] = 0u;
     }
     if (row_ok) {
-      __half* orow = p.out + (row0 + r) * p.out_st + static_cast<int64_t>(h) * p.out_sh + ON * hw;
+      __half* orow = p.out + (row0 + r) * p.out_st + static_cast<int64_t>(h) * p.out_sh + EN * hw;
 #pragma unroll
-      for (int cc = 0; cc < ON / 8; ++cc) {
+      for (int cc = 0; cc < EN / 8; ++cc) {
         uint4 pkt;
         pkt.x = pack_half2(__uint_as_float(o[8 * cc + 0]) * inv, __uint_as_float(o[8 * cc + 1]) * inv);
         pkt.y = pack_half2(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv);
