@@ -68,13 +68,19 @@ bool use_one_tile_kernel(int64_t n_qt, int64_t batch, int64_t hq, bool routed, b
   if (choice != 0) return choice == 2;
   // At d = 64 a tile's MMAs are half as long while its softmax costs the
   // same, so the two-tile kernel's chain (softmax, P.V, next QK^T) leaves
-  // the softmax waiting; the one-tile kernel's three score buffers keep it
-  // busy.  Measured on the 24 MLX-shaped d = 64 runs: equal or faster on 21
-  // (up to 1.8x), at most 7 % slower on 3.
+  // the softmax waiting; the one-tile kernel's three score buffers and its
+  // two independent softmax streams keep it busy.  Measured on the 24
+  // MLX-shaped d = 64 runs: equal on one (1024^2, 32 heads, non-causal),
+  // faster on the rest (up to 2.2x).
   if (d == 64) return true;
   const int64_t sms = device_sms();
   const int64_t pair_ctas = (n_qt + 1) / 2 * batch * hq, one_ctas = n_qt * batch * hq;
-  if (pair_ctas < sms) return true;
+  // Fewer two-tile CTAs than SMs: the one-tile kernel, except for all-FP16
+  // non-causal launches where the two-tile kernel still fills >= 80 % of the
+  // SMs in one wave and the one-tile kernel would need a second (1024^2,
+  // 32 heads: 0.032 against 0.035 ms; 2048^2, 16 heads: even).
+  if (pair_ctas < sms)
+    return routed || causal || 5 * pair_ctas < 4 * sms || one_ctas <= sms;
   if (routed || causal) return false;
   auto fill = [&](int64_t ctas) { return static_cast<double>(ctas) / (((ctas + sms - 1) / sms) * sms); };
   return fill(one_ctas) > 1.1 * fill(pair_ctas);

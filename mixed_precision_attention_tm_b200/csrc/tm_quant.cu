@@ -8,7 +8,7 @@
 // code = clamp(rne(fl32(x / s)), -127, 127);  s == 0 gives codes 0.
 //
 // One CTA per (tile, sequence, head), Q and K in one launch: the tile's rows x
-// d fp16 values are read once with 16-byte loads and kept in registers
+// d fp16 values arrive in shared memory by one TMA copy and stay there
 // between the absmax pass and the quantise pass, so HBM traffic is one read
 // of x plus one write of the codes (bytes per element: 2 read + 1 written).
 // The scale is the IEEE round-to-nearest __fdiv_rn of amax by 127.  A code is
@@ -26,6 +26,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "tm_device.cuh"
 #include "tm_host.h"
 
@@ -33,6 +35,7 @@ namespace tmk {
 namespace {
 
 constexpr int kQuantThreads = 256;
+constexpr int kQuantCtasPerSm = 6;
 
 // two fp32 values to two E4M3 codes (lo in bits 0-7, hi in bits 8-15)
 __device__ __forceinline__ uint32_t e4m3x2_rn_sat(float lo, float hi) {
@@ -110,45 +113,54 @@ __device__ __forceinline__ void int8_codes8(const __half2* hv, float s, float r,
 // One CTA per (head, tile, sequence) of either operand: grid.x runs over the
 // heads of operand 0 and then those of operand 1 (heads fastest, so that the
 // CTAs running at once read and write whole token rows of Q and K, all heads
-// side by side).  The tile's rows x d fp16
-// values are read once with 16-byte loads and kept in registers between the
-// absmax pass and the quantise pass, so HBM traffic is one read of x plus one
-// write of the codes.
+// side by side).  One thread brings the tile's rows x d fp16 values into
+// shared memory with a single TMA copy (rows past the tensor's end arrive as
+// zeros and are not used); the absmax pass and the quantise pass then read
+// them from there, so HBM traffic is one read of x plus one write of the
+// codes.  With the tile in shared memory rather than in registers, six CTAs
+// fit on an SM, and their copies keep 192 KB per SM in flight.
 template <int D, bool F8>
-__global__ void __launch_bounds__(kQuantThreads, 4)
-    quantize_tiles_kernel(const QuantOperand op0, const QuantOperand op1, DevErr err) {
+__global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm)
+    quantize_tiles_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+                          const QuantOperand op0, const QuantOperand op1, DevErr err) {
   constexpr int VPR = D / 8;                       // 16-byte vectors per row
   constexpr int MAXV = 128 * VPR / kQuantThreads;  // vectors per thread at tile = 128
+  extern __shared__ uint8_t quant_smem_raw[];   // tile rows x D fp16, row-major, from a 128-byte boundary
   __shared__ float red[kQuantThreads / 32];
-  __shared__ SeqInfo sinfo;
-  __shared__ float s_scale;
+  __shared__ __align__(8) uint64_t full_bar;
+  uint8_t* tile_smem = quant_smem_raw + ((128u - (smem_u32(quant_smem_raw) & 127u)) & 127u);
 
   const bool second = static_cast<int>(blockIdx.x) >= op0.H;
   const QuantOperand& o = second ? op1 : op0;
   const int I = blockIdx.y, b = blockIdx.z, h = second ? blockIdx.x - op0.H : blockIdx.x;
   if (I >= o.ntile || b >= o.nb) return;
-  if (threadIdx.x == 0) {
-    sinfo = seq_info(o.cu, b, o.L, o.tile);
-    if (o.cu != nullptr && I == 0 && sinfo.len > static_cast<int64_t>(o.ntile) * o.tile)
-      dev_error(err, TM_DEVERR_SEQLEN);
-  }
-  __syncthreads();
-  const SeqInfo sq = sinfo;
+  // every thread reads the same offsets (broadcast loads)
+  const SeqInfo sq = seq_info(o.cu, b, o.L, o.tile);
+  if (threadIdx.x == 0 && o.cu != nullptr && I == 0 && sq.len > static_cast<int64_t>(o.ntile) * o.tile)
+    dev_error(err, TM_DEVERR_SEQLEN);
   const int64_t r0 = static_cast<int64_t>(I) * o.tile;
   if (r0 >= sq.len) return;
   const int rows = static_cast<int>(min(static_cast<int64_t>(o.tile), sq.len - r0));
   const int nvec = rows * VPR;
+  const uint32_t bar = smem_u32(&full_bar);
+  const uint32_t dst = smem_u32(tile_smem);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(o.tile) * D * 2);
+    tma_load_3d(dst, second ? &tm1 : &tm0, bar, 0, h, static_cast<int32_t>(sq.start + r0));
+  }
+  __syncthreads();   // the barrier is initialised before any thread waits on it
+  volatile int never = 0;
+  mbar_wait_warp(bar, 0, err, &never);
 
-  uint4 v[MAXV];
   __half2 m2 = __float2half2_rn(0.f);
 #pragma unroll
   for (int k = 0; k < MAXV; ++k) {
     const int idx = threadIdx.x + k * kQuantThreads;
     if (idx < nvec) {
-      const int row = idx / VPR, c = idx % VPR;
-      const __half* src = o.x + (sq.start + r0 + row) * o.stride_t + static_cast<int64_t>(h) * o.stride_h + c * 8;
-      v[k] = *reinterpret_cast<const uint4*>(src);
-      const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
+      const uint4 v = *reinterpret_cast<const uint4*>(tile_smem + idx * 16);
+      const __half2* hv = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
       for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(hv[e]));
     }
@@ -158,16 +170,12 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float a = red[0];
+  // every thread forms the tile's scale from the warp maxima (one barrier)
+  float a = red[0];
 #pragma unroll
-    for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[w]);
-    const float sc = __fdiv_rn(a, F8 ? 448.0f : 127.0f);
-    s_scale = sc;
-    o.scales[(sq.tile_base + I) * o.H + h] = sc;
-  }
-  __syncthreads();
-  const float sc = s_scale;
+  for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[w]);
+  const float sc = __fdiv_rn(a, F8 ? 448.0f : 127.0f);
+  if (threadIdx.x == 0) o.scales[(sq.tile_base + I) * o.H + h] = sc;
   const float rc = sc != 0.f ? __frcp_rn(sc) : 0.f;
   const int64_t code_row_stride = static_cast<int64_t>(o.H) * D;
 #pragma unroll
@@ -175,7 +183,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     const int idx = threadIdx.x + k * kQuantThreads;
     if (idx < nvec) {
       const int row = idx / VPR, c = idx % VPR;
-      const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
+      const uint4 v = *reinterpret_cast<const uint4*>(tile_smem + idx * 16);
+      const __half2* hv = reinterpret_cast<const __half2*>(&v);
       uint32_t packed[2] = {0u, 0u};
       if (sc != 0.f) {
         if (F8) {
@@ -189,10 +198,32 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
           int8_codes8(hv, sc, rc, packed[0], packed[1]);
         }
       }
-      uint8_t* dst = o.codes + (sq.start + r0 + row) * code_row_stride + static_cast<int64_t>(h) * D + c * 8;
-      *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+      uint8_t* dst_codes = o.codes + (sq.start + r0 + row) * code_row_stride + static_cast<int64_t>(h) * D + c * 8;
+      *reinterpret_cast<uint2*>(dst_codes) = make_uint2(packed[0], packed[1]);
     }
   }
+}
+
+// Asks once for the largest shared-memory carveout, so that kQuantCtasPerSm
+// CTAs with their staged tiles fit on an SM (a hint; the launch is correct
+// with any carveout).
+std::once_flag g_quant_attr_once;
+tm_status g_quant_attr_status = TM_OK;
+tm_status prepare_quant_kernels() {
+  std::call_once(g_quant_attr_once, [] {
+    const int carve = cudaSharedmemCarveoutMaxShared;
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(quantize_tiles_kernel<128, false>, cudaFuncAttributePreferredSharedMemoryCarveout, carve);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(quantize_tiles_kernel<128, true>, cudaFuncAttributePreferredSharedMemoryCarveout, carve);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(quantize_tiles_kernel<64, false>, cudaFuncAttributePreferredSharedMemoryCarveout, carve);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(quantize_tiles_kernel<64, true>, cudaFuncAttributePreferredSharedMemoryCarveout, carve);
+    g_quant_attr_status = check_cuda(e);
+  });
+  return g_quant_attr_status;
 }
 
 tm_status check_operand(const tm_tensor* t) {
@@ -257,14 +288,30 @@ tm_status launch_quant(const tm_tensor* x, void* x_codes, float* x_scales, const
   dim3 grid(static_cast<unsigned>(heads), static_cast<unsigned>(gx), static_cast<unsigned>(gy));
   DevErr err{device_error_word()};
   const int64_t d = x->d;
+  // one TMA map per operand: box of one tile (tile rows x d), no swizzle
+  CUtensorMap map[2];
+  const tm_tensor* src[2] = {x, y};
+  for (int i = 0; i < 2; ++i) {
+    if (empty[i]) continue;
+    st = encode_thd_map(&map[i], src[i]->data, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, src[i]->T, src[i]->H, d,
+                        src[i]->stride_t, src[i]->stride_h, static_cast<int>(d), o[i].tile,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != TM_OK) return st;
+  }
+  if (empty[0]) map[0] = map[1];
+  if (empty[1]) map[1] = map[0];
+  // the larger operand tile, plus room to align it to 128 bytes (TMA destination)
+  const size_t smem = static_cast<size_t>(max(empty[0] ? 0 : o[0].tile, empty[1] ? 0 : o[1].tile)) * d * 2 + 128;
+  st = prepare_quant_kernels();
+  if (st != TM_OK) return st;
   if (d == 128 && f8)
-    quantize_tiles_kernel<128, true><<<grid, kQuantThreads, 0, stream>>>(o[0], o[1], err);
+    quantize_tiles_kernel<128, true><<<grid, kQuantThreads, smem, stream>>>(map[0], map[1], o[0], o[1], err);
   else if (d == 128)
-    quantize_tiles_kernel<128, false><<<grid, kQuantThreads, 0, stream>>>(o[0], o[1], err);
+    quantize_tiles_kernel<128, false><<<grid, kQuantThreads, smem, stream>>>(map[0], map[1], o[0], o[1], err);
   else if (f8)
-    quantize_tiles_kernel<64, true><<<grid, kQuantThreads, 0, stream>>>(o[0], o[1], err);
+    quantize_tiles_kernel<64, true><<<grid, kQuantThreads, smem, stream>>>(map[0], map[1], o[0], o[1], err);
   else
-    quantize_tiles_kernel<64, false><<<grid, kQuantThreads, 0, stream>>>(o[0], o[1], err);
+    quantize_tiles_kernel<64, false><<<grid, kQuantThreads, smem, stream>>>(map[0], map[1], o[0], o[1], err);
   return check_cuda(cudaGetLastError());
 }
 
