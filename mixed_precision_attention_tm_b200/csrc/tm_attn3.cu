@@ -768,6 +768,15 @@ __global__ void __launch_bounds__(384, 1)
 #ifndef TM_EXP2_EMU_PAIRS
 #define TM_EXP2_EMU_PAIRS 3       // exp2 pairs (of every 8) evaluated on the FMA pipe
 #endif
+// At d = 64 (dual stream) the FMA pipe also carries both streams' row sums
+// and packing with half the MMA time per tile to hide them: 2 of 8 pairs on
+// the FMA pipe measured 1-3 % faster than 3 on the MLX-shaped d = 64 runs and
+// on a routed L = 16384 launch, 4 of 8 5 % slower.
+#ifndef TM_EXP2_EMU_PAIRS_D64
+#define TM_EXP2_EMU_PAIRS_D64 2
+#endif
+template <int D>
+constexpr int kEmuPairs = D == 64 ? TM_EXP2_EMU_PAIRS_D64 : TM_EXP2_EMU_PAIRS;
 
 std::mutex g_mu3;
 
@@ -778,7 +787,7 @@ tm_status prepare_split_kernel() {
   static bool attr_done = false;
   std::lock_guard<std::mutex> lk(g_mu3);
   if (attr_done) return TM_OK;
-  auto kern = attn_split_kernel<D, TM_EXP2_EMU_PAIRS, F8>;
+  auto kern = attn_split_kernel<D, kEmuPairs<D>, F8>;
   cudaFuncAttributes fa;
   tm_status st = check_cuda(cudaFuncGetAttributes(&fa, kern));
   if (st != TM_OK) return st;
@@ -873,11 +882,11 @@ tm_status launch_split(const tm_tensor* q, const tm_tensor* k, const tm_tensor* 
   if (grid == 0) return TM_OK;
   if (grid > 0x7fffffffLL) return TM_ERR_UNSUPPORTED;
   if (use_f8)
-    attn_split_kernel<128, TM_EXP2_EMU_PAIRS, true><<<static_cast<unsigned>(grid), Cfg3<128, true>::THREADS,
+    attn_split_kernel<128, kEmuPairs<128>, true><<<static_cast<unsigned>(grid), Cfg3<128, true>::THREADS,
                                                       Cfg3<128, true>::SMEM_BYTES, stream>>>(
         mQ16, mQ8, mK16, mK8, mV16, mQF8, mKF8, p);
   else
-    attn_split_kernel<D, TM_EXP2_EMU_PAIRS, false><<<static_cast<unsigned>(grid), Cfg3<D, false>::THREADS,
+    attn_split_kernel<D, kEmuPairs<D>, false><<<static_cast<unsigned>(grid), Cfg3<D, false>::THREADS,
                                                     Cfg3<D, false>::SMEM_BYTES, stream>>>(
         mQ16, mQ8, mK16, mK8, mV16, mQF8, mKF8, p);
   return check_cuda(cudaGetLastError());
