@@ -83,6 +83,7 @@ struct QuantOperand {
 __device__ __forceinline__ void int8_codes8(const __half2* hv, float s, float r, uint32_t& w0, uint32_t& w1) {
   const uint64_t r2 = f2pack(r, r);
   const uint64_t mg = f2pack(12582912.0f, 12582912.0f), nmg = f2pack(-12582912.0f, -12582912.0f);
+  const uint64_t neg1 = f2pack(-1.0f, -1.0f);
   uint32_t tb[8];
   float dmax = 0.f;
 #pragma unroll
@@ -91,11 +92,13 @@ __device__ __forceinline__ void int8_codes8(const __half2* hv, float s, float r,
     const uint64_t v2 = f2mul(f2pack(f.x, f.y), r2);
     const uint64_t t2 = f2add(v2, mg);
     const uint64_t n2 = f2add(t2, nmg);
-    float v0, v1, n0, n1, t0, t1;
-    f2unpack(v2, v0, v1);
-    f2unpack(n2, n0, n1);
+    // v - n for both lanes in one packed FMA (exact: |v - n| <= 1/2 and
+    // both are multiples of ulp(v), so the single rounding changes nothing)
+    const uint64_t d2 = f2fma(n2, neg1, v2);
+    float d0, d1, t0, t1;
+    f2unpack(d2, d0, d1);
     f2unpack(t2, t0, t1);
-    dmax = fmaxf(dmax, fmaxf(fabsf(v0 - n0), fabsf(v1 - n1)));
+    dmax = fmax3(dmax, fabsf(d0), fabsf(d1));
     tb[2 * e] = __float_as_uint(t0);
     tb[2 * e + 1] = __float_as_uint(t1);
   }
