@@ -439,16 +439,20 @@ tm_status tm_attn_fwd_fp8(const tm_tensor* q, const tm_tensor* k, const tm_tenso
                           const float* q_fp8_scales, const uint8_t* k_fp8_codes, const float* k_fp8_scales,
                           int32_t g, int32_t causal, void* stream);
 
-/* Kernel choice for d = 128 attention with 128 x 128 tiles (tm_attn_fwd,
- * tm_attn_fwd_varlen; fp16 K / V).  Two kernels compute the same result: one
- * holding two 128-row query tiles per CTA (faster per tile once INT8 tiles
- * are routed) and one holding a single query tile per CTA with three score
- * buffers in tensor memory (twice as many CTAs).  choice: 0 automatic (the
- * default: the one-tile kernel when the two-tile kernel would launch fewer
- * CTAs than the GPU has SMs, or for an all-FP16 launch without a causal
- * mask whose last wave it fills clearly better), 1 always the two-tile
- * kernel, 2 always the one-tile kernel.  Process-wide; TM_ERR_INVALID_ARG for
- * any other value. */
+/* Kernel choice for attention with 128 x 128 tiles (tm_attn_fwd,
+ * tm_attn_fwd_varlen; fp16 K / V; d = 64 or 128).  Two kernels compute the
+ * same result: one holding two 128-row query tiles per CTA (faster per tile
+ * once INT8 tiles are routed at d = 128) and one holding a single query tile
+ * per CTA with three score buffers in tensor memory (twice as many CTAs; at
+ * d = 64 its two softmax warpgroups run independent streams over alternate
+ * key tiles).  choice: 0 automatic (the default: at d = 64 the one-tile
+ * kernel; at d = 128 the one-tile kernel when the two-tile kernel would
+ * launch fewer CTAs than the GPU has SMs, except for an all-FP16 launch
+ * without a causal mask that the two-tile kernel still spreads over at
+ * least 80 % of the SMs in one wave, and for an all-FP16 launch without a
+ * causal mask whose last wave it fills clearly better), 1 always the
+ * two-tile kernel, 2 always the one-tile kernel.  Process-wide;
+ * TM_ERR_INVALID_ARG for any other value. */
 tm_status tm_set_attn_kernel(int32_t choice);
 
 /* Head-sharded prefill: reassembly of the output after the all-gather.

@@ -34,9 +34,10 @@ struct Fp8Route {
   const float* k_scales;
 };
 
-// One 128-row query tile per CTA with three score buffers in TMEM and the
-// keys of each score tile split between two softmax warpgroups (d = 128).
-// f8: the FP8 route (null or a null bitmask: FP16 / INT8 only).
+// One 128-row query tile per CTA with three score buffers in TMEM: at d = 128
+// the keys of each score tile are split between two softmax warpgroups, at
+// d = 64 the warpgroups take alternate key tiles (two softmax streams).
+// f8: the FP8 route, d = 128 only (null or a null bitmask: FP16 / INT8 only).
 tm_status launch_attn_split(const tm_tensor* q, const tm_tensor* k, const tm_tensor* v, tm_tensor* out,
                             const int32_t* cu, const int32_t* cu_k, int32_t batch, int32_t max_q, int32_t max_k,
                             const uint32_t* bitmask, int64_t mask_hs, int32_t g, int32_t causal,

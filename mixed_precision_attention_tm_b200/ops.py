@@ -607,9 +607,9 @@ ATTN_KERNEL_AUTO, ATTN_KERNEL_TWO_TILE, ATTN_KERNEL_ONE_TILE = 0, 1, 2
 
 
 def set_attn_kernel(choice):
-    """Kernel for d = 128, 128 x 128-tile attention (tm_set_attn_kernel):
-    ATTN_KERNEL_AUTO (default), ATTN_KERNEL_TWO_TILE or ATTN_KERNEL_ONE_TILE.
-    Process-wide."""
+    """Kernel for 128 x 128-tile attention with fp16 K / V, d = 64 or 128
+    (tm_set_attn_kernel): ATTN_KERNEL_AUTO (default), ATTN_KERNEL_TWO_TILE or
+    ATTN_KERNEL_ONE_TILE.  Process-wide."""
     _check(_lib().tm_set_attn_kernel(int(choice)), "tm_set_attn_kernel")
 
 
