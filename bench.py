@@ -41,12 +41,17 @@ sys.path.insert(0, ROOT)
 
 from mixed_precision_attention_tm_b200 import dist, inputs  # noqa: E402
 
-PROFILE = os.path.join(ROOT, "profiles", "attn_pair_routing_sweep.md")
+# ncu summaries of the kernel each workload's attention runs: the routing
+# sweep's routed launches run the one-query-tile kernel (tm_attn3.cu), the
+# INT8-cache workload the two-query-tile kernel on the expanded cache
+# (tm_attn2.cu) after the expansion (tm_cache_expand.cu).  A summary records
+# the hash of those sources; a changed kernel reports no traffic.
+PROFILE = os.path.join(ROOT, "profiles", "attn_split_routing_sweep.md")
 PROFILE_CACHE = os.path.join(ROOT, "profiles", "attn_pair_toks_varlen_int8_cache.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "mixed_precision_attention_tm_b200", "csrc", f)
-                  for f in ("tm_attn2.cu", "tm_device.cuh")]
-CACHE_SOURCES = KERNEL_SOURCES + [os.path.join(ROOT, "mixed_precision_attention_tm_b200", "csrc",
-                                               "tm_cache_expand.cu")]
+                  for f in ("tm_attn3.cu", "tm_device.cuh")]
+CACHE_SOURCES = [os.path.join(ROOT, "mixed_precision_attention_tm_b200", "csrc", f)
+                 for f in ("tm_attn2.cu", "tm_device.cuh", "tm_cache_expand.cu")]
 
 
 def kernel_source_hash(sources=None):

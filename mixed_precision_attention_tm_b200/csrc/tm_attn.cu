@@ -86,6 +86,23 @@ bool use_one_tile_kernel(int64_t n_qt, int64_t batch, int64_t hq, bool routed, b
   return fill(one_ctas) > 1.1 * fill(pair_ctas);
 }
 
+// The choice for fp16 K / V without the FP8 route, where the one-tile
+// kernel runs its ping-pong softmax at d = 128 (tm_attn3.cu): measured on
+// B200 it beats the two-tile kernel on routed launches (routing sweep,
+// L = 16384: 2.03 / 2.05 / 2.01 ms against 2.13 / 2.21 / 2.08 ms at INT8
+// group probability 0 / 0.75 / 1) and on all-FP16 rows of fewer than 64 key
+// tiles (4096^2 32 heads non-causal 0.261 against 0.305 ms, causal 0.159
+// against 0.163; 2048^2 and 1024^2 equal or faster).  All-FP16 rows of 64 or
+// more key tiles keep the rule above: there the two-tile kernel's chunked
+// mode is faster (routing-sweep shape without a mask: 2.08 against 2.21 ms).
+bool use_one_tile_kernel_fp16(int64_t n_qt, int64_t n_kt, int64_t batch, int64_t hq, bool routed, bool causal,
+                              int64_t d) {
+  const int choice = g_attn_kernel.load(std::memory_order_relaxed);
+  if (choice != 0) return choice == 2;
+  if (d == 128 && (routed || n_kt < 64)) return true;
+  return use_one_tile_kernel(n_qt, batch, hq, routed, causal, d);
+}
+
 }  // namespace
 }  // namespace tmk
 
@@ -688,9 +705,10 @@ tm_status attn_fwd_impl(const tm_tensor* q, const tm_tensor* k, const tm_tensor*
   }
   if (tile_m == 128 && tile_n == 128) {
     const int64_t n_qt = ((cu_seqlens ? max_seqlen : q->T) + 127) / 128;
+    const int64_t n_kt = ((cu_seqlens ? max_k : k->T) + 127) / 128;
     if (TM_SPLIT_KERNEL == 2 ||
-        (TM_SPLIT_KERNEL == 1 && use_one_tile_kernel(n_qt, cu_seqlens ? batch : 1, q->H, bitmask != nullptr,
-                                                     causal != 0, D)))
+        (TM_SPLIT_KERNEL == 1 && use_one_tile_kernel_fp16(n_qt, n_kt, cu_seqlens ? batch : 1, q->H,
+                                                          bitmask != nullptr, causal != 0, D)))
       return launch_attn_split(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,
                                g, causal, s);
     return launch_attn_pair(q, k, v, out, cu_seqlens, cu_k, batch, max_seqlen, max_k, bitmask, mask_head_stride,

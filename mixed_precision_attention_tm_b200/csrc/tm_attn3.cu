@@ -83,9 +83,17 @@ struct Cfg3 {
   // (two 64-column accumulators), merged in the epilogue.  At d = 128 two O
   // accumulators and three score buffers would need 640 TMEM columns.
   static constexpr bool DS = D_ == 64;
+  // PP (ping-pong, d = 128 without the FP8 route): warpgroup h also takes
+  // the whole key tiles with j mod 2 == h, but both accumulate into one O.
+  // The running max is handed from tile to tile in key order: before its
+  // exponentials, tile j's warpgroup waits until tile j-1's P is stored and
+  // takes that tile's reference max (raising it lazily, as one stream
+  // would), so every P.V adds into O against one reference.
+  static constexpr bool PP = D_ == 128 && !F8;
+  static constexpr bool ALT = DS || PP;                         // warpgroups take alternate key tiles
   static constexpr int D = D_, BM = 128, BN = 128;
-  static constexpr int HN = DS ? 128 : 64;                      // keys per softmax warpgroup and tile
-  static constexpr int ON = DS ? D : D / 2;                     // O columns each softmax warpgroup rescales
+  static constexpr int HN = ALT ? 128 : 64;                     // keys per softmax warpgroup and tile
+  static constexpr int ON = ALT ? D : D / 2;                    // O columns a softmax warpgroup rescales
   static constexpr int EN = D / 2;                              // output columns each softmax warpgroup writes
   static constexpr int SLOT = BN * D * 2;                       // one fp16 K or V tile (32 KB; 16 KB at d = 64)
   // K and V ring slots: at d = 64 the tiles are half as large and both
@@ -277,7 +285,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_VEMPTY + s), 1);
     }
-    for (int i = 0; i < C::NSB; ++i) mbar_init(bar(B_PREADY + i), C::DS ? 4 : 8);
+    for (int i = 0; i < C::NSB; ++i) mbar_init(bar(B_PREADY + i), C::ALT ? 4 : 8);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -458,9 +466,9 @@ __global__ void __launch_bounds__(384, 1)
           uint64_t bd[8];
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            // keys 16kk .. 16kk+15: DS, P of the tile's warpgroup in its first
-            // 64 columns; otherwise P of warpgroup kk / 4 at its columns
-            at[kk] = C::DS ? d_s + kk * 8 : d_s + (kk >> 2) * HN + (kk & 3) * 8;
+            // keys 16kk .. 16kk+15: DS / PP, P of the tile's warpgroup in its
+            // first 64 columns; otherwise P of warpgroup kk / 4 at its columns
+            at[kk] = C::ALT ? d_s + kk * 8 : d_s + (kk >> 2) * HN + (kk & 3) * 8;
             bd[kk] = smem_desc(vb + kk * 2048, C::HALF, 1024, kSwizzle128);
           }
           // DS: P.V(j) accumulates into the O of warpgroup j mod 2, which its
@@ -544,7 +552,10 @@ __global__ void __launch_bounds__(384, 1)
     const int hw = warp >> 2;
     const int r = threadIdx.x & 127;                 // row in the tile = TMEM lane
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t o_addr = lane_addr + C::O_COL + ON * hw;   // this warpgroup's O (DS) or half of O's columns
+    // the O columns this warpgroup rescales: its own O (DS), all of O (PP),
+    // or its half of O's columns
+    const uint32_t o_addr = lane_addr + C::O_COL + (C::PP ? 0u : static_cast<uint32_t>(ON * hw));
+    float* mpub = xmax;   // PP: reference max of the last stored tile, per row
     const bool row_ok = r < rows;
     const int64_t i_row = r0 + r;
     int64_t lim = -1;
@@ -556,10 +567,10 @@ __global__ void __launch_bounds__(384, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     TM3_PH_DECL
-    // DS: this warpgroup's key tiles are j = hw, hw + 2, ...; otherwise every
-    // key tile, keys [64 hw, 64 hw + 64)
-    const int key_off = C::DS ? 0 : HN * hw;
-    for (int j = C::DS ? hw : 0; j < nJ; j += C::DS ? 2 : 1) {
+    // DS / PP: this warpgroup's key tiles are j = hw, hw + 2, ...; otherwise
+    // every key tile, keys [64 hw, 64 hw + 64)
+    const int key_off = C::ALT ? 0 : HN * hw;
+    for (int j = C::ALT ? hw : 0; j < nJ; j += C::ALT ? 2 : 1) {
       const int sb = j % C::NSB;
       const uint32_t s_addr = lane_addr + C::S_COL + 128u * sb + key_off;
       const int rt = route_of<F8>(rrow, rrowf8, p.g, j);
@@ -593,11 +604,11 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int e = 0; e < HN; ++e) x[e] = (e < nv) ? x[e] : -INFINITY;
       }
-      // row max of the tile in log2 units (-inf when no key is visible); but
-      // in DS, over both warpgroups' keys
+      // row max of the tile in log2 units (-inf when no key is visible); with
+      // the keys split between the warpgroups, over both halves
       {
         float mt;
-        if constexpr (C::DS) {
+        if constexpr (C::ALT) {
           mt = row_max<HN>(x) * c;
         } else {
           float* xm = xmax + (j & 1) * 256;
@@ -606,11 +617,34 @@ __global__ void __launch_bounds__(384, 1)
           named_bar_sync(NB_MAX, 256);
           mt = fmaxf(xm[r], xm[128 + r]);
         }
-        float alpha = 1.f;
-        if (mt > m_used + kLazyRescaleLog2) {
-          alpha = ex2_approx(m_used - mt);
-          m_used = mt;
+        // m_prev: the reference the previous tile of this stream used.  PP:
+        // the previous tile (j-1) belongs to the other warpgroup; wait until
+        // its P is stored (it published its reference before signalling).
+        // The barrier's next phase, P(j+2), is this warpgroup's own and its
+        // previous one, P(j-4), completed before S(j) could be issued, so
+        // the parity wait is unambiguous.
+        float m_prev = m_used;
+        if constexpr (C::PP) {
+          m_prev = -INFINITY;
+          if (j > 0) {
+            const int jq = j - 1;
+            if (!mbar_wait(bar(B_PREADY + jq % C::NSB), (jq / C::NSB) & 1, p.err, abort_flag)) ok = false;
+            m_prev = mpub[r];
+          }
         }
+        float alpha = 1.f;   // O's factor
+        float m_new = m_prev;
+        if (mt > m_prev + kLazyRescaleLog2) {
+          alpha = ex2_approx(m_prev - mt);
+          m_new = mt;
+        }
+        // this warpgroup's row sum was accumulated against m_used (PP: the
+        // reference of its own previous tile, which the other stream's tile
+        // may have raised since)
+        float alpha_l = alpha;
+        if constexpr (C::PP) alpha_l = (m_used == m_new) ? 1.f : ex2_approx(m_used - m_new);
+        m_used = m_new;
+        if constexpr (C::PP) mpub[r] = m_new;   // read by the other warpgroup once P(j) is signalled
                 TM3_PH(2);
         const float msub = (m_used == -INFINITY) ? 0.f : m_used;
         const uint64_t c2 = f2pack(c, c);
@@ -631,21 +665,31 @@ __global__ void __launch_bounds__(384, 1)
           }
           acc2[(e >> 1) & 3] = f2add(acc2[(e >> 1) & 3], f2pack(p0, p1));
           pk[e >> 1] = pack_half2(p0, p1);
+          // PP: each 32 columns of P go to TMEM as soon as they are complete
+          // (their scores were read into registers already), so that fewer
+          // registers stay live through the loop
+          if (C::PP && (e & 63) == 62) {
+            __syncwarp();
+            tmem_st32p(s_addr + (e >> 6) * 32, pk + (e >> 6) * 32);
+          }
         }
         {
           const uint64_t s2 = f2add(f2add(acc2[0], acc2[1]), f2add(acc2[2], acc2[3]));
           float s0, s1;
           f2unpack(s2, s0, s1);
-          l = l * alpha + (s0 + s1);
+          l = l * alpha_l + (s0 + s1);
         }
         TM3_PH(3);
         __syncwarp();
         // P_hw(j) over the first HN / 2 columns of this warpgroup's scores
+        if constexpr (!C::PP) {
 #pragma unroll
-        for (int cc = 0; cc < HN / 64; ++cc) tmem_st32p(s_addr + cc * 32, pk + cc * 32);
+          for (int cc = 0; cc < HN / 64; ++cc) tmem_st32p(s_addr + cc * 32, pk + cc * 32);
+        }
         // This warpgroup's O columns are rescaled only when a row of this warp
         // raised the running max.  Then the previous P.V into them, P.V(jp)
-        // with jp = j - 2 (DS) or j - 1, must have completed.  It commits to
+        // with jp = j - 2 (DS) or j - 1 (PP and the split keys), must have
+        // completed.  It commits to
         // barrier jp mod 2, whose phases are P.V(jp mod 2), P.V(jp mod 2 + 2),
         // ...  S(j) was issued after P.V(j-3) and has completed, so P.V(jp-2)
         // is done; P.V(jp+2) cannot be, as the issuer takes P(jp+2) (DS: P(j);
@@ -656,20 +700,24 @@ __global__ void __launch_bounds__(384, 1)
           if (!mbar_wait(bar(B_ODONE + (jp & 1)), (jp >> 1) & 1, p.err, abort_flag)) ok = false;
           tc_fence_after();
           __syncwarp();
-          uint32_t o[ON];
-#pragma unroll
-          for (int cc = 0; cc < ON / 32; ++cc) tmem_ld32p(o_addr + cc * 32, o + cc * 32);
-          tmem_wait_ld_regs<ON>(o);
           const uint64_t a2 = f2pack(alpha, alpha);
+          // 64 columns at a time (PP rescales all 128 of O)
 #pragma unroll
-          for (int e = 0; e < ON; e += 2) {
-            float o0, o1;
-            f2unpack(f2mul(f2pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), o0, o1);
-            o[e] = __float_as_uint(o0);
-            o[e + 1] = __float_as_uint(o1);
+          for (int oc = 0; oc < ON; oc += 64) {
+            uint32_t o[64];
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) tmem_ld32p(o_addr + oc + cc * 32, o + cc * 32);
+            tmem_wait_ld_regs<64>(o);
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+              float o0, o1;
+              f2unpack(f2mul(f2pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), o0, o1);
+              o[e] = __float_as_uint(o0);
+              o[e + 1] = __float_as_uint(o1);
+            }
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) tmem_st32p(o_addr + oc + cc * 32, o + cc * 32);
           }
-#pragma unroll
-          for (int cc = 0; cc < ON / 32; ++cc) tmem_st32p(o_addr + cc * 32, o + cc * 32);
         }
       }
       tmem_wait_st();
@@ -694,19 +742,23 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
     }
     float* xs = xmax + 512;   // past both iterations' maxima
+    float* xm_epi = xmax + (C::PP ? 256 : 0);   // PP: clear of the published maxima
     xs[hw * 128 + r] = l;
-    if constexpr (C::DS) xmax[hw * 128 + r] = m_used;
+    if constexpr (C::ALT) xm_epi[hw * 128 + r] = m_used;
     __syncwarp();
     named_bar_sync(NB_EPI, 256);
     // DS: stream w contributes a_w * O_w and a_w * l_w with a_w = 2^(m_w - m),
     // m the larger running max; a stream without a visible key (m_w = -inf)
-    // contributes nothing
+    // contributes nothing.  PP: O already holds every tile against the last
+    // tile's reference m (the larger of the two); each warpgroup's row sum
+    // l_w is against the reference of its own last tile, so it enters as
+    // a_w * l_w alike.
     float a0 = 1.f, a1 = 0.f, inv;
-    if constexpr (C::DS) {
-      const float m0 = xmax[r], m1 = xmax[128 + r];
+    if constexpr (C::ALT) {
+      const float m0 = xm_epi[r], m1 = xm_epi[128 + r];
       const float mm = fmaxf(m0, m1);
-      a0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
-      a1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
+      a0 = m0 == -INFINITY ? 0.f : (m0 == mm ? 1.f : ex2_approx(m0 - mm));
+      a1 = m1 == -INFINITY ? 0.f : (m1 == mm ? 1.f : ex2_approx(m1 - mm));
       const float lsum = xs[r] * a0 + xs[128 + r] * a1;
       inv = (mm != -INFINITY && lsum > 0.f) ? 1.f / lsum : 0.f;
     } else {
