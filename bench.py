@@ -252,6 +252,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
+    ops.set_attn_kernel({"auto": ops.ATTN_KERNEL_AUTO, "two": ops.ATTN_KERNEL_TWO_TILE,
+                         "one": ops.ATTN_KERNEL_ONE_TILE}[args.attn_kernel])
     w = make_workload(args.workload, args.p, seed=dist.rank_seed(args.seed, rank))
     plan = TileMixPrefill(w.Lq, w.Lk, w.hq, w.hkv, w.d, causal=w.causal, tile_m=w.tile_m, tile_n=w.tile_n,
                           g=w.g, p=w.p, seed=w.mask_seed, force_diag=w.force_diag, force_sink=w.force_sink,
@@ -484,6 +486,8 @@ def run_ours(args, rank, world, local_rank):
         line["e2e"] = e2e
     if sweep is not None:
         line["sweep"] = sweep
+    if args.attn_kernel != "auto":
+        line["config"]["attn_kernel"] = args.attn_kernel
     return line, w
 
 
@@ -1015,6 +1019,9 @@ def main():
                          "split by query heads over the ranks, output all-gathered (strong scaling)")
     ap.add_argument("--fp8-only", type=float, default=None,
                     help="FP8 report: time only the FP8-only route at this group probability")
+    ap.add_argument("--attn-kernel", default="auto", choices=["auto", "two", "one"],
+                    help="128 x 128-tile attention kernel: the library's automatic choice (default), the "
+                         "two-query-tile or the one-query-tile kernel (tm_set_attn_kernel)")
     ap.add_argument("--frontier-input", default="channels", choices=["channels", "tokens"],
                     help="frontier report: outlier channels in every token (the routing sweep's inputs) "
                          "or outliers in 0.2%% of the key tokens")
