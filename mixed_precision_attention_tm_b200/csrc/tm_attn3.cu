@@ -14,24 +14,34 @@
 // buffers, so the tensor pipe computes QK^T(j+1) and QK^T(j+2) ahead while
 // the softmax works on S(j):
 //
-//   * S(j) goes to buffer j mod 3.  At d = 128 the keys of each score tile
-//     are split between two softmax warpgroups (one query row per thread):
-//     warpgroup h (warps 4h .. 4h+3) owns keys [64h, 64h+64).  The two
-//     exchange their row maxima of the tile through shared memory, so both
-//     rescale against one running max m (raised lazily, kLazyRescaleLog2),
-//     each sums its half of the row sum, and each rescales its half of O's
-//     columns;
-//   * at d = 64 (dual stream) warpgroup h instead takes whole score tiles,
-//     those with j mod 2 == h, and keeps its own running max, row sum and O
-//     (O of warpgroup h in TMEM columns [64h, 64h+64)); the epilogue merges
-//     the two streams.  No maxima are exchanged per tile and the two
-//     warpgroups do not run in lockstep: while one waits for its next
-//     scores, the other computes, so the MUFU / FMA pipes stay busy.  (At
+//   * S(j) goes to buffer j mod 3.  Two softmax warpgroups (one query row
+//     per thread, warpgroup h = warps 4h .. 4h+3) take alternate score
+//     tiles, those with j mod 2 == h, in one of two forms:
+//   * at d = 128 (ping-pong) both accumulate into one O (128 columns).  The
+//     running max m (raised lazily, kLazyRescaleLog2) is handed from tile to
+//     tile in key order: after loading S(j) and its row maxima, tile j's
+//     warpgroup waits until P(j-1) is stored, reads the m that tile j-1
+//     published in shared memory, raises it if tile j needs it (rescaling O
+//     once P.V(j-1) has completed) and publishes its own.  So the two
+//     warpgroups' exponentials alternate while one's loads and maxima
+//     overlap the other's exponentials, and every P.V adds into O against
+//     the reference a single stream would hold.  Each warpgroup keeps its
+//     row sum against the reference of its own last tile; the epilogue
+//     brings both to the final one;
+//   * at d = 64 (dual stream) each warpgroup keeps its own running max, row
+//     sum and O (O of warpgroup h in TMEM columns [64h, 64h+64)) and never
+//     waits for the other; the epilogue merges the two streams.  (At
 //     d = 128 two O accumulators and three score buffers would need 640 of
 //     the 512 TMEM columns.)
+//   * with the FP8 route (three-way routing, d = 128) the keys of each score
+//     tile are instead split between the warpgroups (warpgroup h owns keys
+//     [64h, 64h+64)); they exchange the tile's row maxima through shared
+//     memory, so both rescale against one running max, each sums its half
+//     of the row sum and rescales its half of O's columns;
 //   * each warpgroup overwrites the first half of its score columns with
-//     its P as fp16; once the tile's P is complete, P.V(j) is one group of
-//     eight MMAs into O (dual stream: into the O of warpgroup j mod 2), and
+//     its P as fp16 (ping-pong: 32 columns at a time, as they are computed);
+//     once the tile's P is complete, P.V(j) is one group of eight MMAs into
+//     O (dual stream: into the O of warpgroup j mod 2), and
 //     QK^T(j+3) follows it into the same buffer (the tensor pipe runs them
 //     in order);
 //   * K and V reach shared memory through two rings of 32 KB slots (three K
@@ -39,8 +49,8 @@
 //     slot released by a tcgen05.commit once the MMAs reading it completed,
 //     so K prefetch never waits for a P.V;
 //   * the softmax arithmetic is the same as in the two-tile kernel (packed
-//     fp32 pairs; 3 of every 8 exp2 pairs as a degree-3 minimax polynomial on
-//     the FMA pipe, the rest on MUFU.ex2).
+//     fp32 pairs; 3 of every 8 exp2 pairs -- 2 at d = 64 -- as a degree-3
+//     minimax polynomial on the FMA pipe, the rest on MUFU.ex2).
 // Every mbarrier wait is bounded (tm_device.cuh).
 #include <cuda.h>
 #include <cuda_fp16.h>
