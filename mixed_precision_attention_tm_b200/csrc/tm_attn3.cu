@@ -744,8 +744,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     __syncwarp();
 #endif
-    // ---- epilogue: row sums over both warpgroups (DS: and the two streams'
-    // maxima), then this warpgroup's EN output columns
+    // ---- epilogue: row sums over both warpgroups (DS / PP: with each
+    // warpgroup's reference max), then this warpgroup's EN output columns
     bool have_o = false;
     if (ok && nJ > 0) {
       have_o = mbar_wait(bar(B_DRAIN), 0, p.err, abort_flag);
