@@ -455,6 +455,19 @@ tm_status tm_attn_fwd_fp8(const tm_tensor* q, const tm_tensor* k, const tm_tenso
  * TM_ERR_INVALID_ARG for any other value. */
 tm_status tm_set_attn_kernel(int32_t choice);
 
+/* Which of the two kernels above tm_attn_fwd / tm_attn_fwd_varlen would run
+ * for a launch with 128 x 128 tiles, fp16 K / V and no FP8 route (the pages
+ * have no counterpart; a query for callers tuning their shapes).  max_q /
+ * max_k: the longest query / key sequence; batch: sequences (1 without
+ * offsets); hq: query heads; d: 64 or 128; routed: non-zero when a routing
+ * bitmask is given; causal: non-zero for the bottom-right causal mask;
+ * sm_count: the GPU's SM count, or 0 for the current device's (the only
+ * case that queries the device).  Returns 1 for the two-query-tile kernel,
+ * 2 for the one-query-tile kernel (honouring tm_set_attn_kernel), 0 for
+ * invalid arguments.  Host-only: launches nothing. */
+int32_t tm_attn_kernel_choice(int64_t max_q, int64_t max_k, int32_t batch, int32_t hq, int32_t d, int32_t routed,
+                              int32_t causal, int32_t sm_count);
+
 /* Head-sharded prefill: reassembly of the output after the all-gather.
  * The pages do not speak of more than one GPU.  Every step of the method
  * (TileMix abstract: per-tile quantisation, routing bits, scores, shared

@@ -54,16 +54,22 @@ int device_sms() {
   return sms;
 }
 
-// Measured on B200 (a table of all-FP16 MLX-shaped launches and the routing
-// sweep): per tile the two-tile kernel is as fast as the one-tile kernel on
-// FP16 tiles and faster once INT8 tiles are routed, but it has half as many
-// CTAs.  The one-tile kernel is taken when the two-tile kernel would leave
-// SMs idle (fewer CTAs than SMs), and for all-FP16 launches without a causal
-// mask when its CTAs fill their last wave clearly better (causal launches
-// already balance their waves by running the longest query tiles first).
+// The choice between a two-query-tile kernel and its one-query-tile
+// counterpart for the INT8-cache and FP8 launches and for all-FP16 rows of
+// 64 or more key tiles (the fp16 path below takes the one-tile kernel's
+// ping-pong form everywhere else).  Measured on B200 (a table of all-FP16
+// MLX-shaped launches and the routing sweep): per tile the two-tile kernels
+// are as fast as those one-tile ones on FP16 tiles and faster once INT8
+// tiles are routed, but they have half as many CTAs.  The one-tile kernel is
+// taken when the two-tile kernel would leave SMs idle (fewer CTAs than SMs),
+// and for all-FP16 launches without a causal mask when its CTAs fill their
+// last wave clearly better (causal launches already balance their waves by
+// running the longest query tiles first).  sms: the GPU's SM count (0: the
+// current device's).
 std::atomic<int> g_attn_kernel{0};   // tm_set_attn_kernel
 
-bool use_one_tile_kernel(int64_t n_qt, int64_t batch, int64_t hq, bool routed, bool causal, int64_t d = 128) {
+bool use_one_tile_kernel(int64_t n_qt, int64_t batch, int64_t hq, bool routed, bool causal, int64_t d = 128,
+                         int64_t sms = 0) {
   const int choice = g_attn_kernel.load(std::memory_order_relaxed);
   if (choice != 0) return choice == 2;
   // At d = 64 a tile's MMAs are half as long while its softmax costs the
@@ -73,7 +79,7 @@ bool use_one_tile_kernel(int64_t n_qt, int64_t batch, int64_t hq, bool routed, b
   // MLX-shaped d = 64 runs: equal on one (1024^2, 32 heads, non-causal),
   // faster on the rest (up to 2.2x).
   if (d == 64) return true;
-  const int64_t sms = device_sms();
+  if (sms <= 0) sms = device_sms();
   const int64_t pair_ctas = (n_qt + 1) / 2 * batch * hq, one_ctas = n_qt * batch * hq;
   // Fewer two-tile CTAs than SMs: the one-tile kernel, except for all-FP16
   // non-causal launches where the two-tile kernel still fills >= 80 % of the
@@ -96,11 +102,11 @@ bool use_one_tile_kernel(int64_t n_qt, int64_t batch, int64_t hq, bool routed, b
 // more key tiles keep the rule above: there the two-tile kernel's chunked
 // mode is faster (routing-sweep shape without a mask: 2.08 against 2.21 ms).
 bool use_one_tile_kernel_fp16(int64_t n_qt, int64_t n_kt, int64_t batch, int64_t hq, bool routed, bool causal,
-                              int64_t d) {
+                              int64_t d, int64_t sms = 0) {
   const int choice = g_attn_kernel.load(std::memory_order_relaxed);
   if (choice != 0) return choice == 2;
   if (d == 128 && (routed || n_kt < 64)) return true;
-  return use_one_tile_kernel(n_qt, batch, hq, routed, causal, d);
+  return use_one_tile_kernel(n_qt, batch, hq, routed, causal, d, sms);
 }
 
 }  // namespace
@@ -110,6 +116,13 @@ extern "C" tm_status tm_set_attn_kernel(int32_t choice) {
   if (choice < 0 || choice > 2) return TM_ERR_INVALID_ARG;
   tmk::g_attn_kernel.store(choice, std::memory_order_relaxed);
   return TM_OK;
+}
+
+extern "C" int32_t tm_attn_kernel_choice(int64_t max_q, int64_t max_k, int32_t batch, int32_t hq, int32_t d,
+                                         int32_t routed, int32_t causal, int32_t sm_count) {
+  if (max_q <= 0 || max_k <= 0 || batch <= 0 || hq <= 0 || (d != 64 && d != 128) || sm_count < 0) return 0;
+  const int64_t n_qt = (max_q + 127) / 128, n_kt = (max_k + 127) / 128;
+  return tmk::use_one_tile_kernel_fp16(n_qt, n_kt, batch, hq, routed != 0, causal != 0, d, sm_count) ? 2 : 1;
 }
 #include "tm_device.cuh"
 #include "tm_host.h"

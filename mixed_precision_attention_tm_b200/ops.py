@@ -90,6 +90,7 @@ def _lib():
             "tm_probe_rates": (I32, [ctypes.POINTER(D), I32, P, I64, P]),
             "tm_merge_head_shards": (I32, [P, I64, P, I64, I32, I32, I32, I32, P, P]),
             "tm_set_attn_kernel": (I32, [I32]),
+            "tm_attn_kernel_choice": (I32, [I64, I64, I32, I32, I32, I32, I32, I32]),
             "tm_quantize_qk_fp8": (I32, [TP, TP, P, P, P, P, P, I32, I32, I32, I32, P]),
             "tm_attn_fwd_fp8": (I32, [TP, TP, TP, TP, P, I32, I32, P, P, I64, P, P, P, P, I32, I32, P]),
         }
@@ -611,6 +612,17 @@ def set_attn_kernel(choice):
     (tm_set_attn_kernel): ATTN_KERNEL_AUTO (default), ATTN_KERNEL_TWO_TILE or
     ATTN_KERNEL_ONE_TILE.  Process-wide."""
     _check(_lib().tm_set_attn_kernel(int(choice)), "tm_set_attn_kernel")
+
+
+def attn_kernel_choice(max_q, max_k, hq, d, *, batch=1, routed=False, causal=True, sm_count=0):
+    """Kernel tm_attn_fwd would run for 128 x 128 tiles with fp16 K / V
+    (tm_attn_kernel_choice): ATTN_KERNEL_TWO_TILE or ATTN_KERNEL_ONE_TILE.
+    sm_count 0 queries the current device."""
+    r = int(_lib().tm_attn_kernel_choice(int(max_q), int(max_k), int(batch), int(hq), int(d), int(bool(routed)),
+                                         int(bool(causal)), int(sm_count)))
+    if r == 0:
+        raise ValueError("tm_attn_kernel_choice: invalid arguments")
+    return r
 
 
 def merge_head_shards(out, gathered, head_start):

@@ -228,6 +228,50 @@ def test_attn_kernel_choice_rejects_unknown_values():
         assert lib.tm_set_attn_kernel(c) == ops.TM_OK
 
 
+def test_kernel_choice_follows_the_documented_rule():
+    """tm_attn_kernel_choice (host-only with an explicit SM count) returns the
+    kernel tm_attn_fwd would launch, by the rule include/tm.h states: d = 64
+    and routed d = 128 launches take the one-query-tile kernel, as do
+    all-FP16 rows of fewer than 64 key tiles; longer all-FP16 rows keep the
+    two-query-tile kernel unless it leaves SMs idle or fills its last wave
+    clearly worse; tm_set_attn_kernel overrides."""
+    one, two = ops.ATTN_KERNEL_ONE_TILE, ops.ATTN_KERNEL_TWO_TILE
+    ch = ops.attn_kernel_choice
+    sms = 148
+    try:
+        ops.set_attn_kernel(ops.ATTN_KERNEL_AUTO)
+        # d = 64: the dual-stream one-tile kernel, whatever the shape
+        for L, h, causal in ((1024, 32, False), (16384, 32, True), (65536, 8, False)):
+            assert ch(L, L, h, 64, causal=causal, sm_count=sms) == one
+        # d = 128 routed: the ping-pong one-tile kernel at every length
+        for L in (640, 16384, 65536):
+            assert ch(L, L, 32, 128, routed=True, sm_count=sms) == one
+        # d = 128 all-FP16 rows under 64 key tiles (8191 keys: 64 tiles minus one key)
+        assert ch(4096, 4096, 32, 128, causal=True, sm_count=sms) == one
+        assert ch(512, 8064, 32, 128, causal=False, sm_count=sms) == one
+        # 64 key tiles or more, causal, enough CTAs: the two-tile kernel (chunked)
+        assert ch(16384, 16384, 32, 128, causal=True, sm_count=sms) == two
+        assert ch(8192, 8192, 32, 128, causal=True, sm_count=sms) == two
+        # ... unless its CTAs leave SMs idle: 8192 rows, 2 heads = 64 two-tile CTAs
+        assert ch(8192, 8192, 2, 128, causal=True, sm_count=sms) == one
+        # non-causal long rows: the kernel whose last wave is fuller (32 heads x 64
+        # query tiles: 1024 pair CTAs fill 7 waves 0.99, 2048 one-tile CTAs 14 waves 0.99)
+        assert ch(8192, 8192, 32, 128, causal=False, sm_count=sms) == two
+        # the SM count enters the rule: 64 two-tile CTAs fill a 64-SM part
+        assert ch(8192, 8192, 2, 128, causal=True, sm_count=64) == two
+        # overrides
+        ops.set_attn_kernel(ops.ATTN_KERNEL_TWO_TILE)
+        assert ch(4096, 4096, 32, 64, sm_count=sms) == two
+        ops.set_attn_kernel(ops.ATTN_KERNEL_ONE_TILE)
+        assert ch(16384, 16384, 32, 128, sm_count=sms) == one
+    finally:
+        ops.set_attn_kernel(ops.ATTN_KERNEL_AUTO)
+    lib = ops._lib()
+    for bad in ((0, 1, 1, 8, 128, 0, 1, sms), (1, 1, 1, 8, 96, 0, 1, sms), (1, 1, 0, 8, 128, 0, 1, sms),
+                (1, 1, 1, 8, 128, 0, 1, -1)):
+        assert lib.tm_attn_kernel_choice(*bad) == 0, bad
+
+
 def test_noalloc_validates_every_argument_before_any_cuda_call():
     """tm_attn_fwd_routed_noalloc rejects a bad call before it looks up its
     scratch array or launches anything: each case below returns its status
