@@ -488,6 +488,11 @@ def run_ours(args, rank, world, local_rank):
         line["sweep"] = sweep
     if args.attn_kernel != "auto":
         line["config"]["attn_kernel"] = args.attn_kernel
+    if w.kv_cache is None and w.cu_seqlens is None and w.tile_m == 128 and w.tile_n == 128:
+        # which 128 x 128-tile kernel the step's attention ran (tm_attn_kernel_choice)
+        kc = ops.attn_kernel_choice(w.Lq, w.Lk, w.hq, w.d, routed=plan.routed, causal=w.causal)
+        line["attn_kernel"] = {ops.ATTN_KERNEL_TWO_TILE: "two query tiles per CTA",
+                               ops.ATTN_KERNEL_ONE_TILE: "one query tile per CTA"}[kc]
     return line, w
 
 
