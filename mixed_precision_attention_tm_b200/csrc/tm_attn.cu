@@ -28,9 +28,10 @@
 
 #include <mutex>
 
-// Which d = 128, 128 x 128-tile launches take the kernel with one query tile
-// per CTA and three score buffers (tm_attn3.cu) instead of the two-tile
-// kernel (tm_attn2.cu): 0 none, 1 by use_one_tile_kernel below, 2 all.
+// Which 128 x 128-tile launches with fp16 K / V take the kernel with one
+// query tile per CTA and three score buffers (tm_attn3.cu) instead of the
+// two-tile kernel (tm_attn2.cu): 0 none, 1 by use_one_tile_kernel_fp16
+// below, 2 all.
 #ifndef TM_SPLIT_KERNEL
 #define TM_SPLIT_KERNEL 1
 #endif
